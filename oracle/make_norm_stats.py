@@ -1,0 +1,88 @@
+"""Writes the per-feature input standardisation of every atomic network.
+
+    python -m oracle.make_norm_stats [workload ...]
+
+Part of the weight recipe, not of the model: the paper's trained weights are
+not available, and random Xavier weights applied to raw embedded densities
+(values up to ~1e3 with a spread of a few percent) would saturate tanh and
+leave the forces near zero.  So each network sees (rho - shift) / scale,
+with shift = mean(rho^t_f) and scale = std(rho^t_f) + 1e-3 mean|rho^t_f|
++ 1e-6, measured per layer t, per element of the centre atom and per
+feature f on the workload's own seeded structure.  Layer t's statistics are
+measured with the networks of layers < t already standardised.
+
+Only the oracle and the seeded input generators run here; the output file
+molecular_dynamics_b200/data/norm_<workload>.json is read by
+molecular_dynamics_b200.synth.weight_blob.
+"""
+from __future__ import annotations
+
+import json
+import os
+import sys
+import time
+
+import numpy as np
+
+import oracle
+from molecular_dynamics_b200 import presets, synth
+
+OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "molecular_dynamics_b200", "data")
+
+
+def measure(p, verbose=True):
+    pos, types, box = synth.make_structure(p)
+    n = len(pos)
+    t0 = time.time()
+    if n <= 20000:
+        pairs = oracle.pairs_brute(pos, box, p.r_cut, p.skin)
+    else:
+        pairs = oracle.pairs_cells(pos, box, p.r_cut, p.skin)
+    depth = p.stats_depth
+    ne, D = p.n_elements, p.D
+    shift = np.zeros((depth, ne, D))
+    scale = np.ones((depth, ne, D))
+    sat = []
+    for t in range(depth):
+        T = t + 1
+        blob = synth.weight_blob(p, T=T, norm=(shift[:t], scale[:t]), use_stored_norm=False)
+        model = oracle.Model.from_preset(p, blob, T=T)
+        res = oracle.energy_forces(model, pos, types, box, pairs, forces=False, intermediates=True)
+        rho = res.rho[t]
+        for e in range(ne):
+            sel = types == e
+            r = rho[sel]
+            mu = r.mean(0)
+            sd = r.std(0) + 1e-3 * np.abs(r).mean(0) + 1e-6
+            shift[t, e] = np.float32(mu)
+            scale[t, e] = np.float32(sd)
+            # diagnostic: fraction of first-layer pre-activations beyond |3|
+            layer = t if t < p.T - 1 else synth.ENERGY_LAYER
+            raw = synth.raw_network(p, layer, e)
+            z = ((r - shift[t, e]) / scale[t, e]) @ raw["W1"].T + raw["b1"]
+            sat.append(float((np.abs(z) > 3).mean()))
+        if verbose:
+            print(f"  {p.key} layer {t}: {time.time() - t0:.1f}s, saturated fraction {sat[-1]:.3f}", flush=True)
+    return shift, scale, sat
+
+
+def main(keys):
+    os.makedirs(OUT, exist_ok=True)
+    for k in keys:
+        p = presets.get(k)
+        shift, scale, sat = measure(p)
+        out = {
+            "workload": k,
+            "recipe": "shift = mean(rho^t_f), scale = std(rho^t_f) + 1e-3 mean|rho^t_f| + 1e-6, per layer t, "
+                      "element of the centre atom and feature f, on the workload's seeded structure",
+            "shift": shift.tolist(),
+            "scale": scale.tolist(),
+            "saturated_fraction": sat,
+        }
+        with open(os.path.join(OUT, f"norm_{k}.json"), "w") as f:
+            json.dump(out, f)
+        print(f"wrote norm_{k}.json  max saturated fraction {max(sat):.3f}")
+
+
+if __name__ == "__main__":
+    main(sys.argv[1:] or list(presets.ORDER))
