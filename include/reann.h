@@ -1,0 +1,242 @@
+/*
+ * reann.h -- C ABI of libreann.so, a B200 (sm_100a) implementation of the
+ * energy+force evaluation of the REANN message-passing neural-network
+ * potential and of velocity-Verlet MD driven by it.
+ *
+ * The operations follow "Efficient Parallelization of Message Passing
+ * Neural Network Potentials for Large-Scale Molecular Dynamics" (Xia and
+ * Jiang):
+ *   - embedded atom density, section "REANN Architecture", Eq. 1;
+ *   - message (orbital-coefficient) update by per-element atomic networks,
+ *     Eq. 2; atomic energies from the last layer's density (Eq. 3 input);
+ *   - forces by the chain rule through every layer, Eqs. 3-5, evaluated as
+ *     vector-Jacobian products (section "Parallelization Algorithm");
+ *   - one neighbour list built once and reused by all T layers (same
+ *     section, Fig. 2), with a Verlet skin (section "Introduction");
+ *   - the local/ghost-atom spatial decomposition with a per-layer ghost
+ *     refresh (Fig. 3a, Fig. 4), as a single-GPU checking mode.
+ *
+ * Conventions shared by every entry point:
+ *   units     A, eV, fs, amu; forces eV/A; velocities A/fs.
+ *   box       orthorhombic, fully periodic, edges box[3] (A), each at least
+ *             2 (r_cut + skin).
+ *   arrays    per-atom vectors are row-major [n][3] in the caller's atom
+ *             order.  Any array pointer may point to device memory or to
+ *             host memory (pinned or pageable); the library detects which
+ *             with cudaPointerGetAttributes and copies host arrays through
+ *             its own device buffers on the given stream.  The caller owns
+ *             every array it passes; the library owns the context and all
+ *             workspaces.
+ *   streams   work is enqueued on the caller's stream; calls that return a
+ *             host value (energy, statistics, counters) synchronise it.
+ *   errors    every call returns a reann_status; reann_last_error() gives a
+ *             message.  Conditions found on the device (neighbour capacity,
+ *             skin violation, non-finite values) are recorded in a status
+ *             word that the next synchronising call reads.  No call aborts
+ *             or traps the device.
+ *   threads   a context is not thread-safe; use one context per thread.
+ */
+#ifndef REANN_H
+#define REANN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct reann_ctx reann_ctx; /* opaque */
+typedef void *reann_stream;         /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    REANN_OK = 0,
+    REANN_ERR_ARG = 1,       /* invalid argument or configuration */
+    REANN_ERR_BOX = 2,       /* box edge <= 0 or < 2 (r_cut + skin) */
+    REANN_ERR_CAPACITY = 3,  /* a fixed-size buffer would overflow */
+    REANN_ERR_NONFINITE = 4, /* NaN/Inf in positions, energy or forces */
+    REANN_ERR_SKIN = 5,      /* an atom moved more than skin/2 since the list was built */
+    REANN_ERR_STATE = 6,     /* call out of order, e.g. forces before a neighbour list */
+    REANN_ERR_CUDA = 7,      /* a CUDA runtime call failed */
+    REANN_ERR_TIMEOUT = 8,   /* a bounded device wait gave up */
+    REANN_ERR_UNSUPPORTED = 9
+} reann_status;
+
+/*
+ * Model hyperparameters (section "REANN Architecture").  D = n_radial *
+ * (l_max + 1) features per atom: feature (n, l) sits at index
+ * l * n_radial + n.  Radial primitive n has centre mu_n = r_cut n /
+ * (n_radial - 1) and width alpha; the cutoff function is
+ * (cos(pi r / r_cut) + 1) / 2 for r < r_cut.
+ */
+typedef struct {
+    int32_t n_elements;    /* 1..8 */
+    int32_t T;             /* message-passing layers, 1..8 */
+    int32_t n_radial;      /* N_phi: 8 or 10 */
+    int32_t l_max;         /* L: 2 */
+    int32_t hidden[2];     /* atomic-network hidden widths: 64 or 128 each */
+    double r_cut;          /* A */
+    double skin;           /* A; the list radius is r_cut + skin */
+    double alpha;          /* A^-2 */
+    int32_t mlp_precision; /* 0 = fp32 networks; 1 = bf16 tensor-core GEMMs, fp32 accumulate */
+    int32_t dd_grid[3];    /* {0,0,0} = monolithic; else subdomains per axis (checking mode) */
+} reann_config;
+
+/*
+ * Weight blob (float32, read once by reann_create):
+ *   C0[n_elements][D]                      initial coefficients c^0 per element
+ *   for t = 0..T-2, for e = 0..n_elements-1: coefficient network M^t_e (rho^t -> c^{t+1}), n_out = D
+ *   for e = 0..n_elements-1:                 energy network N_e (rho^{T-1} -> E_i), n_out = 1
+ * and each network is
+ *   shift[D], scale[D], W1[H1][D], b1[H1], W2[H2][H1], b2[H2], W3[n_out][H2], b3[n_out]
+ * evaluating y = W3 tanh(W2 tanh(W1 ((x - shift) / scale) + b1) + b2) + b3.
+ */
+
+typedef struct {
+    double e_pot;       /* potential energy after the last step, eV */
+    double e_kin;       /* kinetic energy after the last step, eV */
+    double e_pot0;      /* potential energy at entry, eV */
+    double e_kin0;      /* kinetic energy at entry, eV */
+    int64_t rebuilds;   /* neighbour-list rebuilds during the call */
+    int64_t steps;      /* steps completed */
+} reann_md_stats;
+
+typedef struct {
+    int64_t n_atoms;
+    int64_t nnz;                 /* neighbour-list entries (ordered pairs within r_cut + skin) */
+    int64_t capacity;            /* allocated neighbour-list entries */
+    int64_t max_row;             /* longest neighbour row */
+    int64_t active_pairs;        /* ordered pairs within r_cut at the last evaluation */
+    int64_t builds;              /* neighbour-list builds since creation */
+    int64_t evaluations;         /* energy+force evaluations since creation */
+    int64_t ghost_slots;         /* domain-decomposed mode: ghost atoms over all subdomains */
+    int64_t ghost_bytes_fwd;     /* domain-decomposed mode: bytes gathered per layer, forward */
+    int64_t ghost_bytes_bwd;     /* domain-decomposed mode: bytes reduced per layer, backward */
+    int64_t kernel_launches;     /* kernels this context has launched since creation */
+    int32_t cells[3];            /* cell grid of the neighbour search */
+    int32_t reserved;
+} reann_counters;
+
+/* Kernel groups timed by reann_profile / reann_profile_read. */
+typedef enum {
+    REANN_K_ACTIVE = 0,      /* compaction of the pairs within r_cut */
+    REANN_K_DENSITY = 1,     /* orbital + density forward, one launch per layer (Eq. 1) */
+    REANN_K_MLP_FWD = 2,     /* coefficient networks, forward (Eq. 2) */
+    REANN_K_MLP_ENERGY = 3,  /* energy network, forward + input gradient */
+    REANN_K_EDGE_BWD = 4,    /* edge VJP + force gather, one launch per layer (Eqs. 3-4) */
+    REANN_K_MLP_BWD = 5,     /* coefficient networks, input gradient (Eq. 5) */
+    REANN_K_ENERGY_SUM = 6,  /* energy reduction */
+    REANN_K_INTEGRATE = 7,   /* velocity-Verlet kicks and drift */
+    REANN_K_NEIGHBORS = 8,   /* binning + neighbour list build (all kernels of one build) */
+    REANN_K_OTHER = 9,       /* gathers, scatters, checks */
+    REANN_K_COUNT = 10
+} reann_kernel_group;
+
+/*
+ * Creates a context on CUDA device `device` and uploads the weights.
+ * weights: host float32 blob of nbytes bytes laid out as above (nbytes
+ * must match the configuration exactly).  On success *out receives the
+ * context.  Errors: REANN_ERR_ARG (bad configuration or blob size),
+ * REANN_ERR_UNSUPPORTED (a hyperparameter outside the compiled set),
+ * REANN_ERR_CUDA.
+ */
+reann_status reann_create(const reann_config *cfg, const void *weights, size_t nbytes, int device, reann_ctx **out);
+
+/* Frees the context and every workspace.  NULL is accepted. */
+reann_status reann_destroy(reann_ctx *ctx);
+
+/*
+ * Builds the neighbour list (section "Parallelization Algorithm": built once,
+ * reused by every layer) for n atoms.
+ * pos: float32 [n][3] positions (A), any image; types: int32 [n] element
+ * indices in [0, n_elements); box: host double[3].
+ * Atoms are binned into cells at least r_cut + skin wide by a counting sort
+ * on (element, cell), and the list holds every ordered pair (i, j), i != j,
+ * whose minimum-image distance satisfies (dx*dx + dy*dy) + dz*dz <
+ * (r_cut + skin)^2, evaluated in fp64 without fused multiply-add.  Rows
+ * are sorted.  Allocates workspaces for n atoms (the only call besides
+ * reann_create that allocates).  Synchronises the stream once to size the
+ * list.  Errors: REANN_ERR_ARG, REANN_ERR_BOX, REANN_ERR_NONFINITE,
+ * REANN_ERR_CAPACITY (more than 2^31-1 entries), REANN_ERR_CUDA.
+ */
+reann_status reann_build_neighbors(reann_ctx *ctx, int64_t n, const float *pos, const int32_t *types,
+                                   const double box[3], reann_stream stream);
+
+/*
+ * One energy+force evaluation (Eqs. 1-5) at positions pos (float32 [n][3],
+ * same atoms and types as the last reann_build_neighbors).
+ * energy: host double*, receives E = sum_i E_i (eV), may be NULL.
+ * forces: float32 [n][3] (eV/A), may be NULL.
+ * atom_energy: float32 [n] (eV), may be NULL.
+ * Does not allocate.  Synchronises the stream (to return the energy and
+ * the device status).  Errors: REANN_ERR_STATE (no list), REANN_ERR_SKIN
+ * (an atom moved more than skin/2 since the list was built: rebuild and
+ * call again; outputs are then not valid), REANN_ERR_NONFINITE,
+ * REANN_ERR_CUDA.
+ */
+reann_status reann_energy_forces(reann_ctx *ctx, const float *pos, double *energy, float *forces,
+                                 float *atom_energy, reann_stream stream);
+
+/*
+ * nsteps of velocity Verlet with time step dt_fs:
+ *   v += F/m dt/2;  x += v dt;  wrap x into [0, L);  rebuild the list when
+ *   an atom has moved more than skin/2 since the last build;  F = -dE/dx;
+ *   v += F/m dt/2.
+ * The acceleration unit is 1 eV/(A amu) = 1/103.6426965 A/fs^2.
+ * x: double [n][3] (A) and v: double [n][3] (A/fs), updated in place.
+ * mass_amu: host double[n_elements].  stats (host, may be NULL) receives
+ * energies and counts.  Forces are evaluated once per step on the float32
+ * rounding of x, plus once at entry -- unless the call continues the
+ * previous one (x and v bitwise equal to what the previous reann_md_step
+ * on this context returned, same dt and masses, no other call in between),
+ * in which case the resident state, list and forces are reused and the
+ * trajectory is identical to one longer call.  Requires a prior
+ * reann_build_neighbors for the same atoms and types (positions may have
+ * moved; the list is rebuilt at entry).  Allocates only if the neighbour
+ * list outgrows its capacity.  Synchronises the stream once per step (to
+ * read the rebuild flag) and at the end.  Errors: as reann_energy_forces.
+ */
+reann_status reann_md_step(reann_ctx *ctx, int32_t nsteps, double dt_fs, double *x, double *v,
+                           const double *mass_amu, reann_md_stats *stats, reann_stream stream);
+
+/* Copies the counters of the context into *out (host).  Synchronises nothing. */
+reann_status reann_get_counters(const reann_ctx *ctx, reann_counters *out);
+
+/* Message of the last error on this context (or of the last failed create when ctx is NULL). */
+const char *reann_last_error(const reann_ctx *ctx);
+
+/*
+ * Diagnostics (parity tests).  Copies the current neighbour list in the
+ * caller's atom order: row[n+1] (int64) and col[nnz] (int32), rows sorted
+ * by caller index.  Host or device pointers; cap is col's length.
+ * Synchronises the stream.  Errors: REANN_ERR_STATE, REANN_ERR_CAPACITY.
+ */
+reann_status reann_get_neighbors(reann_ctx *ctx, int64_t *row, int32_t *col, int64_t cap, reann_stream stream);
+
+/*
+ * Diagnostics (parity tests).  After reann_energy_forces, copies layer t's
+ * per-atom embedded density rho^t (float32 [n][D]) and coefficients c^t
+ * (float32 [n][D]) in the caller's atom order.  Either pointer may be NULL.
+ * Synchronises the stream.  Errors: REANN_ERR_STATE, REANN_ERR_ARG.
+ */
+reann_status reann_get_features(reann_ctx *ctx, int32_t t, float *rho, float *coef, reann_stream stream);
+
+/*
+ * Diagnostics (measurement).  enable != 0 starts timing every kernel launch
+ * of this context with a CUDA event pair recorded on the launching stream,
+ * and clears the accumulated times; enable == 0 stops it.  Timing adds two
+ * event records per launch and never synchronises by itself; the times are
+ * collected at the synchronisations the other calls already make.
+ */
+reann_status reann_profile(reann_ctx *ctx, int32_t enable);
+
+/*
+ * Accumulated device time (ms) and launch count of one kernel group since
+ * the last reann_profile(ctx, 1).  Errors: REANN_ERR_ARG.
+ */
+reann_status reann_profile_read(const reann_ctx *ctx, int32_t group, double *ms, int64_t *launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* REANN_H */

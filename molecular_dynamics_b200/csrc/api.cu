@@ -1,0 +1,653 @@
+// C ABI entry points of libreann.so (declared in include/reann.h).
+//
+// Orchestration of one energy+force evaluation, following "Efficient
+// Parallelization of Message Passing Neural Network Potentials for
+// Large-Scale Molecular Dynamics":
+//   forward  (section "REANN Architecture", Eqs. 1-2)
+//     t = 0 .. T-1:  A^t, rho^t from c^t (c^0 = element table)   [edge.cu]
+//                    c^{t+1} = M^t(rho^t) for t < T-1            [mlp.cu]
+//     E_i = N(rho^{T-1}) and G^{T-1} = dE/dA^{T-1}                [mlp.cu]
+//   backward (section "Parallelization Algorithm", Eqs. 3-5)
+//     t = T-1 .. 0:  F += edge VJP, dE/dc^t                      [edge.cu]
+//                    G^{t-1} from M^{t-1}'s VJP (Eq. 5)          [mlp.cu]
+//   E = sum_i E_i (deterministic fp64 tree)                      [md.cu]
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace reann;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+reann_status fail(reann_ctx *c, reann_status st, const std::string &msg) {
+    if (c) c->last_error = msg;
+    else g_create_error = msg;
+    return st;
+}
+
+reann_status cuda_fail(reann_ctx *c, cudaError_t e, const char *where) {
+    cudaGetLastError();
+    return fail(c, REANN_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(call)                                              \
+    do {                                                      \
+        cudaError_t _e = (call);                              \
+        if (_e != cudaSuccess) return cuda_fail(c, _e, #call); \
+    } while (0)
+
+bool is_device_ptr(const void *p) {
+    if (!p) return false;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+template <class T>
+cudaError_t dalloc(T **p, size_t count) {
+    if (*p) {
+        cudaFree(*p);
+        *p = nullptr;
+    }
+    if (count == 0) count = 1;
+    return cudaMalloc((void **)p, sizeof(T) * count);
+}
+
+template <class T>
+void dfree(T *&p) {
+    if (p) cudaFree(p);
+    p = nullptr;
+}
+
+int64_t net_size(const reann_ctx *c, int n_out) {
+    return 2LL * c->D + (int64_t)c->H1 * c->D + c->H1 + (int64_t)c->H2 * c->H1 + c->H2 + (int64_t)n_out * c->H2 + n_out;
+}
+
+NetOffsets bind_net(const reann_ctx *c, int64_t &off, int n_out) {
+    NetOffsets o;
+    o.n_out = n_out;
+    o.shift = off; off += c->D;
+    o.scale = off; off += c->D;
+    o.W1 = off; off += (int64_t)c->H1 * c->D;
+    o.b1 = off; off += c->H1;
+    o.W2 = off; off += (int64_t)c->H2 * c->H1;
+    o.b2 = off; off += c->H2;
+    o.W3 = off; off += (int64_t)n_out * c->H2;
+    o.b3 = off; off += n_out;
+    return o;
+}
+
+void free_atoms(reann_ctx *c) {
+    dfree(c->d_key); dfree(c->d_perm); dfree(c->d_perm_tmp); dfree(c->d_inv); dfree(c->d_types_caller);
+    dfree(c->d_pos); dfree(c->d_pos_build); dfree(c->d_row); dfree(c->d_cnt); dfree(c->d_act_cnt);
+    dfree(c->d_A); dfree(c->d_rho); dfree(c->d_coef); dfree(c->d_G); dfree(c->d_dc); dfree(c->d_Ei);
+    dfree(c->d_F); dfree(c->d_Epart); dfree(c->d_stage_f); dfree(c->d_stage_i); dfree(c->d_stage_x);
+    dfree(c->d_stage_v); dfree(c->d_stage_e); dfree(c->d_x); dfree(c->d_v); dfree(c->d_diag);
+    dfree(c->d_last_x); dfree(c->d_last_v);
+    c->md_valid = false;
+    c->n_alloc = 0;
+}
+
+reann_status ensure_atoms(reann_ctx *c, int64_t n) {
+    if (n <= c->n_alloc && c->d_row) return REANN_OK;
+    free_atoms(c);
+    size_t N = (size_t)n;
+    CK(dalloc(&c->d_key, N));
+    CK(dalloc(&c->d_perm, N));
+    CK(dalloc(&c->d_perm_tmp, N));
+    CK(dalloc(&c->d_inv, N));
+    CK(dalloc(&c->d_types_caller, N));
+    CK(dalloc(&c->d_pos, N));
+    CK(dalloc(&c->d_pos_build, N));
+    CK(dalloc(&c->d_row, N + 1));
+    CK(dalloc(&c->d_cnt, N));
+    CK(dalloc(&c->d_act_cnt, N));
+    CK(dalloc(&c->d_A, (size_t)c->T * N * c->NA));
+    CK(dalloc(&c->d_rho, (size_t)c->T * N * c->D));
+    CK(dalloc(&c->d_coef, (size_t)c->T * N * c->D));
+    CK(dalloc(&c->d_G, N * c->NA));
+    CK(dalloc(&c->d_dc, N * c->D));
+    CK(dalloc(&c->d_Ei, N));
+    CK(dalloc(&c->d_F, 3 * N));
+    CK(dalloc(&c->d_Epart, N / 256 + 2));
+    CK(dalloc(&c->d_stage_f, 3 * N));
+    CK(dalloc(&c->d_stage_i, N));
+    CK(dalloc(&c->d_stage_x, 3 * N));
+    CK(dalloc(&c->d_stage_v, 3 * N));
+    CK(dalloc(&c->d_stage_e, N));
+    CK(dalloc(&c->d_x, 3 * N));
+    CK(dalloc(&c->d_v, 3 * N));
+    CK(dalloc(&c->d_diag, N * (size_t)std::max(c->D, c->NA)));
+    CK(dalloc(&c->d_last_x, 3 * N));
+    CK(dalloc(&c->d_last_v, 3 * N));
+    c->n_alloc = n;
+    return REANN_OK;
+}
+
+reann_status ensure_scan_tmp(reann_ctx *c, int64_t n) {
+    size_t need = scan_tmp_bytes(n);
+    if (need <= c->scan_tmp_size) return REANN_OK;
+    if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
+    c->d_scan_tmp = nullptr;
+    CK(cudaMalloc(&c->d_scan_tmp, need));
+    c->scan_tmp_size = need;
+    return REANN_OK;
+}
+
+reann_status ensure_bins(reann_ctx *c) {
+    if (c->nbins <= c->nbins_alloc) return REANN_OK;
+    CK(dalloc(&c->d_bin_count, (size_t)c->nbins + 1));
+    CK(dalloc(&c->d_bin_start, (size_t)c->nbins + 1));
+    CK(dalloc(&c->d_bin_fill, (size_t)c->nbins + 1));
+    c->nbins_alloc = c->nbins;
+    return REANN_OK;
+}
+
+reann_status ensure_capacity(reann_ctx *c, int64_t nnz) {
+    if (nnz <= c->cap && c->d_col) return REANN_OK;
+    int64_t cap = nnz + nnz / 5 + 1024;
+    if (cap > INT32_MAX) cap = INT32_MAX;
+    CK(dalloc(&c->d_col, (size_t)cap));
+    CK(dalloc(&c->d_act_col, (size_t)cap));
+    c->cap = cap;
+    return REANN_OK;
+}
+
+cudaError_t sync_stream(reann_ctx *c, cudaStream_t s) {
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) prof_harvest(c);
+    return e;
+}
+
+// status word -> API status
+reann_status check_status(reann_ctx *c, int st) {
+    if (st & ST_BADTYPE) return fail(c, REANN_ERR_ARG, "atom type outside [0, n_elements)");
+    if (st & ST_NONFINITE) return fail(c, REANN_ERR_NONFINITE, "non-finite position, energy or force");
+    if (st & ST_CAPACITY) return fail(c, REANN_ERR_CAPACITY, "neighbour capacity exceeded");
+    if (st & ST_TIMEOUT) return fail(c, REANN_ERR_TIMEOUT, "a bounded device wait gave up");
+    if (st & ST_SKIN) return fail(c, REANN_ERR_SKIN, "an atom moved more than skin/2 since the neighbour list was built");
+    return REANN_OK;
+}
+
+// Binning + CSR for the caller-order float positions/types already on the
+// device.  Reads nnz back (one synchronisation) and grows the list if needed.
+reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s) {
+    CK(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
+    CK(launch_build(c, d_pos_caller, d_types_caller, s));
+    CK(cudaMemcpyAsync(c->h_i64, c->d_i64, sizeof(int64_t) * 3, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    // element segment starts: bin_start[e * ncell]
+    for (int e = 0; e <= c->ne; ++e)
+        CK(cudaMemcpyAsync(c->h_seg + e, c->d_bin_start + (int64_t)e * c->ncell, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CK(sync_stream(c, s));
+    reann_status st = check_status(c, *c->h_status & ~ST_SKIN);
+    if (st) return st;
+    int64_t nnz = c->h_i64[1];
+    if (nnz > INT32_MAX) return fail(c, REANN_ERR_CAPACITY, "neighbour list exceeds 2^31-1 entries");
+    if ((st = ensure_capacity(c, nnz))) return st;
+    CK(launch_fill(c, s));
+    c->nnz = nnz;
+    c->max_row = c->h_i64[2];
+    // tile table of the atomic networks: element segments cut into 32-row tiles
+    std::vector<int4> tiles;
+    for (int e = 0; e < c->ne; ++e)
+        for (int r = c->h_seg[e]; r < c->h_seg[e + 1]; r += 32)
+            tiles.push_back(make_int4(e, r, std::min(32, c->h_seg[e + 1] - r), 0));
+    bool same = (int)tiles.size() == c->n_tiles && c->elem_start.size() == (size_t)c->ne + 1 &&
+                std::equal(c->elem_start.begin(), c->elem_start.end(), c->h_seg);
+    if (!same) {
+        if ((int)tiles.size() > c->n_tiles_alloc) {
+            CK(dalloc(&c->d_tiles, tiles.size()));
+            c->n_tiles_alloc = (int)tiles.size();
+        }
+        if (!tiles.empty())
+            CK(cudaMemcpyAsync(c->d_tiles, tiles.data(), sizeof(int4) * tiles.size(), cudaMemcpyHostToDevice, s));
+        CK(sync_stream(c, s));
+        c->n_tiles = (int)tiles.size();
+        c->elem_start.assign(c->h_seg, c->h_seg + c->ne + 1);
+    }
+    c->have_list = true;
+    c->counters.builds++;
+    return REANN_OK;
+}
+
+// One energy+force evaluation on the internal positions d_pos.
+reann_status run_ef(reann_ctx *c, cudaStream_t s) {
+    CK(launch_active(c, s));
+    for (int t = 0; t < c->T; ++t) {
+        CK(launch_density_fwd(c, t, s));
+        if (t + 1 < c->T) CK(launch_mlp_coef_fwd(c, t, s));
+    }
+    CK(launch_mlp_energy(c, s));
+    for (int t = c->T - 1; t >= 0; --t) {
+        CK(launch_edge_bwd(c, t, t != c->T - 1, s));
+        if (t >= 1) CK(launch_mlp_coef_bwd(c, t, s));
+    }
+    CK(launch_energy_sum(c, s));
+    c->counters.evaluations++;
+    c->have_eval = true;
+    return REANN_OK;
+}
+
+void fill_counters(reann_ctx *c) {
+    c->counters.n_atoms = c->n;
+    c->counters.nnz = c->nnz;
+    c->counters.capacity = c->cap;
+    c->counters.max_row = c->max_row;
+    for (int a = 0; a < 3; ++a) c->counters.cells[a] = c->m[a];
+}
+
+}  // namespace
+
+namespace reann {
+
+LaunchScope::LaunchScope(reann_ctx *c_, int g, cudaStream_t s_, int kernels) : c(c_), group(g), s(s_) {
+    c->counters.kernel_launches += kernels;
+    if (!c->prof) return;
+    for (cudaEvent_t *ev : {&a, &b}) {
+        if (!c->prof_pool.empty()) {
+            *ev = c->prof_pool.back();
+            c->prof_pool.pop_back();
+        } else if (cudaEventCreate(ev) != cudaSuccess) {
+            cudaGetLastError();
+            *ev = nullptr;
+        }
+    }
+    if (a && b) cudaEventRecord(a, s);
+}
+
+LaunchScope::~LaunchScope() {
+    if (!a || !b) {
+        if (a) c->prof_pool.push_back(a);
+        if (b) c->prof_pool.push_back(b);
+        return;
+    }
+    cudaEventRecord(b, s);
+    c->prof_pending.push_back({group, a, b});
+}
+
+void prof_harvest(reann_ctx *c) {
+    for (auto &r : c->prof_pending) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+            c->prof_ms[r.group] += ms;
+            c->prof_n[r.group] += 1;
+        } else {
+            cudaGetLastError();
+        }
+        c->prof_pool.push_back(r.a);
+        c->prof_pool.push_back(r.b);
+    }
+    c->prof_pending.clear();
+}
+
+}  // namespace reann
+
+// ---------------------------------------------------------------------------
+
+extern "C" reann_status reann_create(const reann_config *cfg, const void *weights, size_t nbytes, int device,
+                                     reann_ctx **out) {
+    if (!cfg || !weights || !out) return fail(nullptr, REANN_ERR_ARG, "null argument");
+    *out = nullptr;
+    if (cfg->n_elements < 1 || cfg->n_elements > MAX_ELEMENTS || cfg->T < 1 || cfg->T > MAX_T ||
+        !(cfg->r_cut > 0) || !(cfg->skin >= 0) || !(cfg->alpha > 0) || !std::isfinite(cfg->r_cut) ||
+        !std::isfinite(cfg->skin) || cfg->mlp_precision < 0 || cfg->mlp_precision > 1)
+        return fail(nullptr, REANN_ERR_ARG, "invalid configuration");
+    if (cfg->mlp_precision == 1)
+        return fail(nullptr, REANN_ERR_UNSUPPORTED, "bf16 tensor-core networks are not built yet");
+    if (cfg->l_max != 2 || (cfg->n_radial != 8 && cfg->n_radial != 10) ||
+        (cfg->hidden[0] != 64 && cfg->hidden[0] != 128) || (cfg->hidden[1] != 64 && cfg->hidden[1] != 128))
+        return fail(nullptr, REANN_ERR_UNSUPPORTED, "supported: l_max 2, n_radial 8 or 10, hidden widths 64 or 128");
+    for (int a = 0; a < 3; ++a)
+        if (cfg->dd_grid[a] != 0) return fail(nullptr, REANN_ERR_UNSUPPORTED, "domain-decomposed mode is not built");
+    reann_ctx *c = new reann_ctx();
+    c->cfg = *cfg;
+    c->device = device;
+    c->NP = cfg->n_radial;
+    c->D = c->NP * (cfg->l_max + 1);
+    c->NA = c->NP * NT;
+    c->T = cfg->T;
+    c->ne = cfg->n_elements;
+    c->H1 = cfg->hidden[0];
+    c->H2 = cfg->hidden[1];
+    int64_t expect = (int64_t)c->ne * c->D + (int64_t)(c->T - 1) * c->ne * net_size(c, c->D) + (int64_t)c->ne * net_size(c, 1);
+    if ((int64_t)nbytes != expect * (int64_t)sizeof(float)) {
+        delete c;
+        return fail(nullptr, REANN_ERR_ARG, "weight blob size does not match the configuration (expected " +
+                                                std::to_string(expect * sizeof(float)) + " bytes)");
+    }
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+        cudaGetLastError();
+        delete c;
+        return fail(nullptr, REANN_ERR_CUDA, "no such CUDA device");
+    }
+    DeviceGuard guard(device);
+    int64_t off = (int64_t)c->ne * c->D;
+    for (int t = 0; t + 1 < c->T; ++t)
+        for (int e = 0; e < c->ne; ++e) c->coef_nets.push_back(bind_net(c, off, c->D));
+    for (int e = 0; e < c->ne; ++e) c->energy_nets.push_back(bind_net(c, off, 1));
+    c->n_w = expect;
+    c->h_C0.assign((const float *)weights, (const float *)weights + (size_t)c->ne * c->D);
+    cudaError_t e;
+    cudaDeviceProp prop;
+    if ((e = cudaGetDeviceProperties(&prop, device)) ||
+        (e = cudaMalloc(&c->d_w, nbytes)) ||
+        (e = cudaMemcpy(c->d_w, weights, nbytes, cudaMemcpyHostToDevice)) ||
+        (e = cudaMalloc(&c->d_status, sizeof(int) * 4)) ||
+        (e = cudaMemset(c->d_status, 0, sizeof(int) * 4)) ||
+        (e = cudaMalloc(&c->d_i64, sizeof(int64_t) * 8)) ||
+        (e = cudaMemset(c->d_i64, 0, sizeof(int64_t) * 8)) ||
+        (e = cudaMalloc(&c->d_E, sizeof(double) * 4)) ||
+        (e = cudaMallocHost(&c->h_status, sizeof(int) * 4)) ||
+        (e = cudaMallocHost(&c->h_i64, sizeof(int64_t) * 8)) ||
+        (e = cudaMallocHost(&c->h_E, sizeof(double) * 4)) ||
+        (e = cudaMallocHost(&c->h_seg, sizeof(int) * (MAX_ELEMENTS + 1)))) {
+        std::string msg = std::string("CUDA initialisation failed: ") + cudaGetErrorString(e);
+        cudaGetLastError();
+        reann_destroy(c);
+        return fail(nullptr, REANN_ERR_CUDA, msg);
+    }
+    c->sm_count = prop.multiProcessorCount;
+    *out = c;
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_destroy(reann_ctx *c) {
+    if (!c) return REANN_OK;
+    DeviceGuard guard(c->device);
+    free_atoms(c);
+    dfree(c->d_w); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
+    dfree(c->d_act_col); dfree(c->d_tiles); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
+    if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
+    if (c->h_status) cudaFreeHost(c->h_status);
+    if (c->h_i64) cudaFreeHost(c->h_i64);
+    if (c->h_E) cudaFreeHost(c->h_E);
+    if (c->h_seg) cudaFreeHost(c->h_seg);
+    for (auto &r : c->prof_pending) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (auto ev : c->prof_pool) cudaEventDestroy(ev);
+    delete c;
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_build_neighbors(reann_ctx *c, int64_t n, const float *pos, const int32_t *types,
+                                              const double box[3], reann_stream stream) {
+    if (!c) return REANN_ERR_ARG;
+    if (n < 0 || (n > 0 && (!pos || !types)) || !box) return fail(c, REANN_ERR_ARG, "invalid arguments");
+    if (n >= INT32_MAX) return fail(c, REANN_ERR_CAPACITY, "too many atoms");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    double rl = c->cfg.r_cut + c->cfg.skin;
+    for (int a = 0; a < 3; ++a)
+        if (!(box[a] > 0) || !std::isfinite(box[a]) || box[a] < 2.0 * rl)
+            return fail(c, REANN_ERR_BOX, "box edge must be finite and at least 2 (r_cut + skin)");
+    reann_status st;
+    if ((st = ensure_atoms(c, n))) return st;
+    c->n = n;
+    c->have_list = c->have_eval = false;
+    c->md_valid = false;
+    int ncell = 1;
+    for (int a = 0; a < 3; ++a) {
+        c->box[a] = box[a];
+        c->m[a] = std::max(1, (int)std::floor(box[a] / rl));
+        ncell *= c->m[a];
+    }
+    c->ncell = ncell;
+    c->nbins = ncell * c->ne;
+    if ((st = ensure_bins(c))) return st;
+    if ((st = ensure_scan_tmp(c, std::max<int64_t>(n, c->nbins)))) return st;
+    const float *d_pos = pos;
+    if (n > 0 && !is_device_ptr(pos)) {
+        CK(cudaMemcpyAsync(c->d_stage_f, pos, sizeof(float) * 3 * n, cudaMemcpyHostToDevice, s));
+        d_pos = c->d_stage_f;
+    }
+    if (n > 0) CK(cudaMemcpyAsync(c->d_types_caller, types, sizeof(int) * n, cudaMemcpyDefault, s));
+    if ((st = build_internal(c, d_pos, c->d_types_caller, s))) return st;
+    CK(sync_stream(c, s));
+    fill_counters(c);
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_energy_forces(reann_ctx *c, const float *pos, double *energy, float *forces,
+                                            float *atom_energy, reann_stream stream) {
+    if (!c) return REANN_ERR_ARG;
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if (c->n > 0 && !pos) return fail(c, REANN_ERR_ARG, "null positions");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n;
+    c->md_valid = false;
+    CK(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
+    if (n > 0) {
+        const float *d_pos = pos;
+        if (!is_device_ptr(pos)) {
+            CK(cudaMemcpyAsync(c->d_stage_f, pos, sizeof(float) * 3 * n, cudaMemcpyHostToDevice, s));
+            d_pos = c->d_stage_f;
+        }
+        CK(launch_pos_from_caller(c, d_pos, s));
+        CK(launch_skin_check(c, c->d_status, s));
+    }
+    reann_status st = run_ef(c, s);
+    if (st) return st;
+    bool f_dev = forces && is_device_ptr(forces), e_dev = atom_energy && is_device_ptr(atom_energy);
+    float *fo = forces ? (f_dev ? forces : c->d_stage_f) : nullptr;
+    float *eo = atom_energy ? (e_dev ? atom_energy : c->d_stage_e) : nullptr;
+    CK(launch_scatter_outputs(c, fo, eo, s));
+    if (forces && !f_dev && n > 0)
+        CK(cudaMemcpyAsync(forces, c->d_stage_f, sizeof(float) * 3 * n, cudaMemcpyDeviceToHost, s));
+    if (atom_energy && !e_dev && n > 0)
+        CK(cudaMemcpyAsync(atom_energy, c->d_stage_e, sizeof(float) * n, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_E, c->d_E, sizeof(double), cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_i64 + 3, c->d_i64 + 3, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+    CK(sync_stream(c, s));
+    c->counters.active_pairs = c->h_i64[3];
+    fill_counters(c);
+    if (energy) *energy = c->h_E[0];
+    return check_status(c, *c->h_status);
+}
+
+extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v,
+                                      const double *mass_amu, reann_md_stats *stats, reann_stream stream) {
+    if (!c) return REANN_ERR_ARG;
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if (nsteps < 0 || !std::isfinite(dt_fs) || !mass_amu || (c->n > 0 && (!x || !v)))
+        return fail(c, REANN_ERR_ARG, "invalid arguments");
+    double inv_mass[MAX_ELEMENTS], mass[MAX_ELEMENTS];
+    for (int e = 0; e < c->ne; ++e) {
+        if (!(mass_amu[e] > 0) || !std::isfinite(mass_amu[e])) return fail(c, REANN_ERR_ARG, "masses must be positive");
+        mass[e] = mass_amu[e];
+        inv_mass[e] = 1.0 / mass_amu[e];
+    }
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n;
+    const size_t bytes3 = sizeof(double) * 3 * (size_t)n;
+    bool x_dev = is_device_ptr(x), v_dev = is_device_ptr(v);
+    reann_status st;
+    int64_t rebuilds = 0;
+    int32_t done = 0;
+    bool resume = false;
+    if (n > 0) {
+        CK(cudaMemcpyAsync(c->d_stage_x, x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
+        CK(cudaMemcpyAsync(c->d_stage_v, v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
+        if (c->md_valid) {
+            // a continuation: the caller passes back exactly the state the last
+            // call returned, so the resident internal state and forces are reused
+            CK(cudaMemsetAsync(c->d_status + 2, 0, sizeof(int), s));
+            CK(launch_md_compare(c, c->d_stage_x, c->d_stage_v, c->d_status + 2, s));
+            CK(cudaMemcpyAsync(c->h_status + 2, c->d_status + 2, sizeof(int), cudaMemcpyDeviceToHost, s));
+            CK(sync_stream(c, s));
+            resume = c->h_status[2] == 0 && c->md_dt == dt_fs &&
+                     std::equal(mass, mass + c->ne, c->md_mass);
+        }
+    }
+    c->md_valid = false;
+    CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
+    if (!resume) {
+        if (n > 0) {
+            // caller-order state (wrapped into the box) -> list -> internal order
+            CK(launch_wrap_state(c, c->d_stage_x, c->d_stage_f, s));
+            if ((st = build_internal(c, c->d_stage_f, c->d_types_caller, s))) return st;
+            CK(launch_md_gather(c, c->d_stage_x, c->d_stage_v, s));
+        }
+        CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
+        if ((st = run_ef(c, s))) return st;
+    }
+    CK(launch_kinetic(c, mass, c->d_E + 1, s));
+    CK(cudaMemcpyAsync(c->h_E + 2, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
+    for (int32_t step = 0; step < nsteps; ++step) {
+        CK(launch_md_kick_drift(c, dt_fs, inv_mass, c->d_status + 1, s));
+        CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int) * 2, cudaMemcpyDeviceToHost, s));
+        CK(sync_stream(c, s));
+        if ((st = check_status(c, c->h_status[0]))) return st;
+        if (c->h_status[1]) {
+            CK(launch_md_scatter(c, c->d_stage_x, c->d_stage_v, c->d_stage_f, s));
+            if ((st = build_internal(c, c->d_stage_f, c->d_types_caller, s))) return st;
+            CK(launch_md_gather(c, c->d_stage_x, c->d_stage_v, s));
+            CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
+            ++rebuilds;
+        }
+        if ((st = run_ef(c, s))) return st;
+        CK(launch_md_kick(c, dt_fs, inv_mass, s));
+        ++done;
+    }
+    CK(launch_kinetic(c, mass, c->d_E + 1, s));
+    CK(cudaMemcpyAsync(c->h_E, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
+    if (n > 0) {
+        // final state in caller order: kept for continuation checks, then copied out
+        CK(launch_md_scatter(c, c->d_last_x, c->d_last_v, nullptr, s));
+        CK(cudaMemcpyAsync(x, c->d_last_x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, s));
+        CK(cudaMemcpyAsync(v, c->d_last_v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, s));
+    }
+    CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CK(sync_stream(c, s));
+    c->md_valid = (c->h_status[0] & ~ST_SKIN) == 0;
+    c->md_dt = dt_fs;
+    std::copy(mass, mass + c->ne, c->md_mass);
+    fill_counters(c);
+    if (stats) {
+        stats->e_pot = c->h_E[0];
+        stats->e_kin = c->h_E[1];
+        stats->e_pot0 = c->h_E[2];
+        stats->e_kin0 = c->h_E[3];
+        stats->rebuilds = rebuilds;
+        stats->steps = done;
+    }
+    return check_status(c, c->h_status[0] & ~ST_SKIN);
+}
+
+extern "C" reann_status reann_get_counters(const reann_ctx *c, reann_counters *out) {
+    if (!c || !out) return REANN_ERR_ARG;
+    *out = c->counters;
+    return REANN_OK;
+}
+
+extern "C" const char *reann_last_error(const reann_ctx *c) {
+    return c ? c->last_error.c_str() : g_create_error.c_str();
+}
+
+extern "C" reann_status reann_get_neighbors(reann_ctx *c, int64_t *row, int32_t *col, int64_t cap,
+                                            reann_stream stream) {
+    if (!c || !row || (!col && cap > 0)) return REANN_ERR_ARG;
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "no neighbour list");
+    if (cap < c->nnz) return fail(c, REANN_ERR_CAPACITY, "col is shorter than the list (" + std::to_string(c->nnz) + ")");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n;
+    std::vector<int> hrow(n + 1), hcol(c->nnz > 0 ? c->nnz : 1), hperm(n > 0 ? n : 1);
+    CK(cudaMemcpyAsync(hrow.data(), c->d_row, sizeof(int) * (n + 1), cudaMemcpyDeviceToHost, s));
+    if (c->nnz > 0) CK(cudaMemcpyAsync(hcol.data(), c->d_col, sizeof(int) * c->nnz, cudaMemcpyDeviceToHost, s));
+    if (n > 0) CK(cudaMemcpyAsync(hperm.data(), c->d_perm, sizeof(int) * n, cudaMemcpyDeviceToHost, s));
+    CK(sync_stream(c, s));
+    std::vector<int64_t> orow(n + 1, 0);
+    for (int64_t i = 0; i < n; ++i) orow[hperm[i] + 1] = hrow[i + 1] - hrow[i];
+    for (int64_t a = 0; a < n; ++a) orow[a + 1] += orow[a];
+    std::vector<int32_t> ocol(c->nnz > 0 ? c->nnz : 1);
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t a = hperm[i], o = orow[a];
+        for (int q = hrow[i]; q < hrow[i + 1]; ++q) ocol[o++] = hperm[hcol[q]];
+        std::sort(ocol.begin() + orow[a], ocol.begin() + o);
+    }
+    CK(cudaMemcpy(row, orow.data(), sizeof(int64_t) * (n + 1), cudaMemcpyDefault));
+    if (c->nnz > 0) CK(cudaMemcpy(col, ocol.data(), sizeof(int32_t) * c->nnz, cudaMemcpyDefault));
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_get_features(reann_ctx *c, int32_t t, float *rho, float *coef, reann_stream stream) {
+    if (!c) return REANN_ERR_ARG;
+    if (t < 0 || t >= c->T) return fail(c, REANN_ERR_ARG, "layer out of range");
+    if (!c->have_eval) return fail(c, REANN_ERR_STATE, "no evaluation yet");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n, nD = n * c->D;
+    if (n == 0) return REANN_OK;
+    if (rho) {
+        CK(launch_to_caller_rows(c, c->d_rho + t * nD, c->D, c->d_diag, s));
+        CK(cudaMemcpyAsync(rho, c->d_diag, sizeof(float) * nD, cudaMemcpyDefault, s));
+        CK(sync_stream(c, s));
+    }
+    if (coef) {
+        if (t == 0) {
+            std::vector<int> types(n);
+            CK(cudaMemcpy(types.data(), c->d_types_caller, sizeof(int) * n, cudaMemcpyDeviceToHost));
+            std::vector<float> h((size_t)nD);
+            for (int64_t a = 0; a < n; ++a)
+                std::memcpy(&h[a * c->D], &c->h_C0[(size_t)types[a] * c->D], sizeof(float) * c->D);
+            CK(cudaMemcpy(coef, h.data(), sizeof(float) * nD, cudaMemcpyDefault));
+        } else {
+            CK(launch_to_caller_rows(c, c->d_coef + t * nD, c->D, c->d_diag, s));
+            CK(cudaMemcpyAsync(coef, c->d_diag, sizeof(float) * nD, cudaMemcpyDefault, s));
+            CK(sync_stream(c, s));
+        }
+    }
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_profile(reann_ctx *c, int32_t enable) {
+    if (!c) return REANN_ERR_ARG;
+    DeviceGuard guard(c->device);
+    c->prof = enable != 0;
+    if (c->prof) {
+        for (auto &r : c->prof_pending) {
+            c->prof_pool.push_back(r.a);
+            c->prof_pool.push_back(r.b);
+        }
+        c->prof_pending.clear();
+        for (int g = 0; g < REANN_K_COUNT; ++g) {
+            c->prof_ms[g] = 0.0;
+            c->prof_n[g] = 0;
+        }
+    }
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_profile_read(const reann_ctx *c, int32_t group, double *ms, int64_t *launches) {
+    if (!c || group < 0 || group >= REANN_K_COUNT) return REANN_ERR_ARG;
+    if (ms) *ms = c->prof_ms[group];
+    if (launches) *launches = c->prof_n[group];
+    return REANN_OK;
+}

@@ -1,0 +1,165 @@
+// Internal declarations shared by the translation units of libreann.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/reann.h"
+
+namespace reann {
+
+constexpr int NT = 10;          // Cartesian tuples for L = 2
+constexpr int MAX_ELEMENTS = 8;
+constexpr int MAX_T = 8;
+
+// device status bits (or-ed into ctx->d_status)
+enum : int {
+    ST_NONFINITE = 1,
+    ST_CAPACITY = 2,
+    ST_SKIN = 4,
+    ST_BADTYPE = 8,
+    ST_TIMEOUT = 16,
+};
+
+// geometry and model constants passed by value to the edge kernels
+struct EdgeParams {
+    double box[3];
+    double inv_box[3];
+    float r_cut, r_cut2;
+    float pi_over_rc;
+    float alpha;
+    float mu_step;      // mu_n = n * mu_step
+};
+
+// offsets (in floats) of one atomic network inside the device weight blob
+struct NetOffsets {
+    int64_t shift, scale, W1, b1, W2, b2, W3, b3;
+    int n_out;
+};
+
+struct Ctx;
+
+// --- host orchestration helpers (defined across the .cu files) -------------
+cudaError_t scan_exclusive(const int *in, int *out, int64_t n, int64_t *d_total, void *tmp, cudaStream_t s);
+size_t scan_tmp_bytes(int64_t n);
+
+}  // namespace reann
+
+// The context.  All device pointers are owned by the context.
+struct reann_ctx {
+    reann_config cfg;
+    int device = 0;
+    int sm_count = 0;
+    int NP = 0, D = 0, NA = 0, T = 0, ne = 0, H1 = 0, H2 = 0;
+
+    // weights
+    float *d_w = nullptr;
+    int64_t n_w = 0;
+    std::vector<reann::NetOffsets> coef_nets;  // [(T-1) * ne]
+    std::vector<reann::NetOffsets> energy_nets;  // [ne]
+
+    // atoms
+    int64_t n = 0;          // atoms the workspaces are sized for
+    int64_t n_alloc = 0;
+    bool have_list = false;
+    bool have_eval = false;
+    double box[3] = {0, 0, 0};
+    int m[3] = {0, 0, 0};   // cells per axis
+    int ncell = 0;
+    int nbins = 0;          // ne * ncell
+    int64_t nbins_alloc = 0;
+    std::vector<int> elem_start;  // [ne + 1], host copy of the element segments
+    int *h_seg = nullptr;         // pinned [MAX_ELEMENTS + 1]
+    std::vector<float> h_C0;      // element coefficient table c^0
+
+    // neighbour search
+    int *d_bin_count = nullptr, *d_bin_start = nullptr, *d_bin_fill = nullptr;
+    int *d_key = nullptr;          // caller order
+    int *d_perm = nullptr;         // internal -> caller
+    int *d_perm_tmp = nullptr;
+    int *d_inv = nullptr;          // caller -> internal
+    int *d_types_caller = nullptr; // caller order
+    float4 *d_pos = nullptr;       // internal order: x, y, z, type bits
+    float4 *d_pos_build = nullptr; // positions at the last build
+    int *d_row = nullptr;          // [n + 1]
+    int *d_cnt = nullptr;          // [n]
+    int *d_col = nullptr;          // [cap]
+    int *d_act_cnt = nullptr;      // [n]
+    int *d_act_col = nullptr;      // [cap]
+    int64_t nnz = 0, cap = 0, max_row = 0;
+    void *d_scan_tmp = nullptr;
+    size_t scan_tmp_size = 0;
+    int64_t *d_i64 = nullptr;      // small scratch of int64 scalars
+    int64_t *h_i64 = nullptr;      // pinned mirror
+
+    // per-layer activations
+    float *d_A = nullptr;      // [T][n][NA]
+    float *d_rho = nullptr;    // [T][n][D]
+    float *d_coef = nullptr;   // [T][n][D]  (layer 0 unused: c^0 comes from C0)
+    float *d_G = nullptr;      // [n][NA]  dE/dA^t
+    float *d_dc = nullptr;     // [n][D]   dE/dc^t
+    float *d_Ei = nullptr;     // [n]
+    float *d_F = nullptr;      // [n][3] internal order
+    double *d_Epart = nullptr; // block partial sums of E
+    double *d_E = nullptr;     // [4] energies (pot, kin, ...)
+    int n_part = 0;
+
+    // MLP tile table: per tile (element, first row, rows)
+    int4 *d_tiles = nullptr;
+    int n_tiles = 0, n_tiles_alloc = 0;
+
+    // staging for host arrays and caller-order scratch
+    float *d_stage_f = nullptr;    // [n][3] floats
+    int *d_stage_i = nullptr;      // [n]
+    double *d_stage_x = nullptr;   // [n][3]
+    double *d_stage_v = nullptr;   // [n][3]
+    float *d_stage_e = nullptr;    // [n]
+    float *d_diag = nullptr;       // [n][max(D, NA)] diagnostics scratch
+    // MD state in internal order
+    double *d_x = nullptr, *d_v = nullptr;  // [n][3]
+    // state returned by the last MD call (caller order), for continuation checks
+    double *d_last_x = nullptr, *d_last_v = nullptr;
+    bool md_valid = false;
+    double md_dt = 0.0;
+    double md_mass[reann::MAX_ELEMENTS] = {};
+
+    // status
+    int *d_status = nullptr;
+    int *h_status = nullptr;   // pinned
+    double *h_E = nullptr;     // pinned
+
+    reann_counters counters{};
+    std::string last_error;
+
+    // per-launch CUDA-event timing (reann_profile)
+    bool prof = false;
+    struct ProfRec {
+        int group;
+        cudaEvent_t a, b;
+    };
+    std::vector<ProfRec> prof_pending;
+    std::vector<cudaEvent_t> prof_pool;
+    double prof_ms[REANN_K_COUNT] = {};
+    int64_t prof_n[REANN_K_COUNT] = {};
+};
+
+namespace reann {
+// Brackets one kernel launch: counts it and, when profiling, records an event
+// pair on the launching stream.
+struct LaunchScope {
+    reann_ctx *c;
+    int group;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    LaunchScope(reann_ctx *c_, int g, cudaStream_t s_, int kernels = 1);
+    ~LaunchScope();
+};
+void prof_harvest(reann_ctx *c);  // after a synchronisation of the stream
+}  // namespace reann
+#define REANN_CAT2(a, b) a##b
+#define REANN_CAT(a, b) REANN_CAT2(a, b)
+#define REANN_TIMED(...) ::reann::LaunchScope REANN_CAT(_reann_scope_, __LINE__)(__VA_ARGS__)

@@ -1,0 +1,48 @@
+// Launch wrappers shared between translation units.
+#pragma once
+
+#include "common.cuh"
+
+namespace reann {
+
+struct BinParams {
+    double box[3];
+    int m[3];
+    int ncell;
+    int ne;
+    double thr;  // (r_cut + skin)^2
+};
+
+BinParams make_bin_params(const reann_ctx *c);
+EdgeParams make_edge_params(const reann_ctx *c);
+
+// neighbour search (nbr.cu)
+cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s);
+cudaError_t launch_fill(reann_ctx *c, cudaStream_t s);
+cudaError_t launch_skin_check(reann_ctx *c, int *flag, cudaStream_t s);
+
+// edge kernels (edge.cu)
+cudaError_t launch_active(reann_ctx *c, cudaStream_t s);
+cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s);
+cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s);
+
+// atomic networks (mlp.cu)
+cudaError_t launch_mlp_coef_fwd(reann_ctx *c, int t, cudaStream_t s);   // rho^t -> c^{t+1}
+cudaError_t launch_mlp_energy(reann_ctx *c, cudaStream_t s);            // rho^{T-1} -> E_i, G^{T-1}
+cudaError_t launch_mlp_coef_bwd(reann_ctx *c, int t, cudaStream_t s);   // (rho^{t-1}, dE/dc^t) -> G^{t-1}
+
+// reductions, gathers and the integrator (md.cu)
+cudaError_t launch_pos_from_caller(reann_ctx *c, const float *d_pos_caller, cudaStream_t s);
+cudaError_t launch_energy_sum(reann_ctx *c, cudaStream_t s);            // -> d_E[0], status on non-finite
+cudaError_t launch_scatter_outputs(reann_ctx *c, float *d_forces, float *d_atom_energy, cudaStream_t s);
+cudaError_t launch_md_gather(reann_ctx *c, const double *d_x_caller, const double *d_v_caller, cudaStream_t s);
+cudaError_t launch_md_scatter(reann_ctx *c, double *d_x_caller, double *d_v_caller, float *d_pos_caller,
+                              cudaStream_t s);
+cudaError_t launch_md_kick_drift(reann_ctx *c, double dt, const double *inv_mass, int *flag, cudaStream_t s);
+cudaError_t launch_md_kick(reann_ctx *c, double dt, const double *inv_mass, cudaStream_t s);
+cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cudaStream_t s);
+cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s);
+cudaError_t launch_wrap_state(reann_ctx *c, double *d_x_caller, float *d_pos_caller, cudaStream_t s);
+cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s);
+
+}  // namespace reann

@@ -1,0 +1,304 @@
+// Reductions, order changes between the caller's atom order and the internal
+// (element, cell) order, and the velocity-Verlet integrator.
+//
+// The integrator is the plain velocity-Verlet update that drives the NVE runs
+// of "Efficient Parallelization of Message Passing Neural Network Potentials
+// for Large-Scale Molecular Dynamics" (section "Strong Scaling", NVE energy
+// conservation): v += F/m dt/2; x += v dt; F(x); v += F/m dt/2.  State x, v is
+// fp64; the force evaluation reads the fp32 rounding of x.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace reann {
+
+constexpr double ACC_UNIT = 1.0 / 103.6426965;   // eV/(A amu) -> A/fs^2
+constexpr double KE_UNIT = 103.6426965;          // amu A^2/fs^2 -> eV
+constexpr int RED_THREADS = 256;
+
+static inline unsigned blocks(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
+
+__global__ void k_pos_from_caller(int64_t n, const float *__restrict__ pos, const int *__restrict__ perm,
+                                  const int *__restrict__ types, float4 *__restrict__ pos4, int *__restrict__ status) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    int64_t a = perm[s];
+    float x = pos[3 * a], y = pos[3 * a + 1], z = pos[3 * a + 2];
+    if (!isfinite(x) || !isfinite(y) || !isfinite(z)) atomicOr(status, ST_NONFINITE);
+    pos4[s] = make_float4(x, y, z, __int_as_float(types[a]));
+}
+
+cudaError_t launch_pos_from_caller(reann_ctx *c, const float *d_pos_caller, cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0)
+        k_pos_from_caller<<<blocks(c->n, 256), 256, 0, s>>>(c->n, d_pos_caller, c->d_perm, c->d_types_caller,
+                                                            c->d_pos, c->d_status);
+    return cudaGetLastError();
+}
+
+// Deterministic fp64 sum: fixed per-block tree, then one block over the partials.
+__device__ __forceinline__ double block_sum(double v) {
+    __shared__ double sh[RED_THREADS];
+    sh[threadIdx.x] = v;
+    __syncthreads();
+    for (int w = RED_THREADS / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+        __syncthreads();
+    }
+    double r = sh[0];
+    __syncthreads();
+    return r;
+}
+
+__global__ void k_energy_partial(int64_t n, const float *__restrict__ Ei, const float *__restrict__ F,
+                                 double *__restrict__ part, int *__restrict__ status) {
+    int64_t i = (int64_t)blockIdx.x * RED_THREADS + threadIdx.x;
+    double v = 0.0;
+    bool bad = false;
+    if (i < n) {
+        float e = Ei[i];
+        v = (double)e;
+        bad = !isfinite(e) || !isfinite(F[3 * i]) || !isfinite(F[3 * i + 1]) || !isfinite(F[3 * i + 2]);
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+    double s = block_sum(v);
+    if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+
+__global__ void k_sum_partials(int np, const double *__restrict__ part, double *__restrict__ out) {
+    double v = 0.0;
+    for (int k = threadIdx.x; k < np; k += RED_THREADS) v += part[k];
+    double s = block_sum(v);
+    if (threadIdx.x == 0) *out = s;
+}
+
+cudaError_t launch_energy_sum(reann_ctx *c, cudaStream_t s) {
+    int np = (int)blocks(c->n, RED_THREADS);
+    REANN_TIMED(c, REANN_K_ENERGY_SUM, s, 2);
+    if (c->n > 0) k_energy_partial<<<np, RED_THREADS, 0, s>>>(c->n, c->d_Ei, c->d_F, c->d_Epart, c->d_status);
+    k_sum_partials<<<1, RED_THREADS, 0, s>>>(c->n > 0 ? np : 0, c->d_Epart, c->d_E);
+    return cudaGetLastError();
+}
+
+__global__ void k_scatter_outputs(int64_t n, const int *__restrict__ perm, const float *__restrict__ F,
+                                  const float *__restrict__ Ei, float *__restrict__ Fo, float *__restrict__ Eo) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    int64_t a = perm[s];
+    if (Fo) {
+        Fo[3 * a] = F[3 * s];
+        Fo[3 * a + 1] = F[3 * s + 1];
+        Fo[3 * a + 2] = F[3 * s + 2];
+    }
+    if (Eo) Eo[a] = Ei[s];
+}
+
+cudaError_t launch_scatter_outputs(reann_ctx *c, float *d_forces, float *d_atom_energy, cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0 && (d_forces || d_atom_energy))
+        k_scatter_outputs<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, c->d_F, c->d_Ei, d_forces,
+                                                            d_atom_energy);
+    return cudaGetLastError();
+}
+
+// internal rows of `width` floats -> caller order
+__global__ void k_rows_to_caller(int64_t n, int width, const int *__restrict__ perm, const float *__restrict__ in,
+                                 float *__restrict__ out) {
+    int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n * width) return;
+    int64_t s = k / width, f = k % width;
+    out[(int64_t)perm[s] * width + f] = in[k];
+}
+
+cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0) k_rows_to_caller<<<blocks(c->n * width, 256), 256, 0, s>>>(c->n, width, c->d_perm, d_internal, d_caller);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// MD state
+
+__global__ void k_md_gather(int64_t n, const int *__restrict__ perm, const double *__restrict__ xc,
+                            const double *__restrict__ vc, double *__restrict__ x, double *__restrict__ v) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    int64_t a = perm[s];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        x[3 * s + k] = xc[3 * a + k];
+        v[3 * s + k] = vc[3 * a + k];
+    }
+}
+
+cudaError_t launch_md_gather(reann_ctx *c, const double *d_x_caller, const double *d_v_caller, cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0) k_md_gather<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, d_x_caller, d_v_caller, c->d_x, c->d_v);
+    return cudaGetLastError();
+}
+
+__global__ void k_md_scatter(int64_t n, const int *__restrict__ perm, const double *__restrict__ x,
+                             const double *__restrict__ v, double *__restrict__ xc, double *__restrict__ vc,
+                             float *__restrict__ pc) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    int64_t a = perm[s];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        double xv = x[3 * s + k];
+        if (xc) xc[3 * a + k] = xv;
+        if (vc) vc[3 * a + k] = v[3 * s + k];
+        if (pc) pc[3 * a + k] = (float)xv;
+    }
+}
+
+cudaError_t launch_md_scatter(reann_ctx *c, double *d_x_caller, double *d_v_caller, float *d_pos_caller,
+                              cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0)
+        k_md_scatter<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, c->d_x, c->d_v, d_x_caller, d_v_caller,
+                                                       d_pos_caller);
+    return cudaGetLastError();
+}
+
+// flag = 1 when the caller-order state (x, v) differs bitwise from the state
+// the previous MD call returned
+__global__ void k_md_compare(int64_t m, const unsigned long long *__restrict__ x, const unsigned long long *__restrict__ v,
+                             const unsigned long long *__restrict__ lx, const unsigned long long *__restrict__ lv,
+                             int *__restrict__ flag) {
+    int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    bool diff = k < m && (x[k] != lx[k] || v[k] != lv[k]);
+    if (__any_sync(0xffffffffu, diff) && (threadIdx.x & 31) == 0) atomicOr(flag, 1);
+}
+
+cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s) {
+    int64_t m = 3 * c->n;
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (m > 0)
+        k_md_compare<<<blocks(m, 256), 256, 0, s>>>(m, (const unsigned long long *)x, (const unsigned long long *)v,
+                                                    (const unsigned long long *)c->d_last_x,
+                                                    (const unsigned long long *)c->d_last_v, flag);
+    return cudaGetLastError();
+}
+
+// caller-order fp64 positions wrapped into [0, L) in place, plus their fp32 copy
+__global__ void k_wrap_state(int64_t n, double bx, double by, double bz, double *__restrict__ x,
+                             float *__restrict__ p) {
+    int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= 3 * n) return;
+    double L = (k % 3 == 0) ? bx : ((k % 3 == 1) ? by : bz);
+    double v = x[k];
+    v -= L * floor(v / L);
+    if (v >= L) v -= L;
+    x[k] = v;
+    p[k] = (float)v;
+}
+
+cudaError_t launch_wrap_state(reann_ctx *c, double *d_x_caller, float *d_pos_caller, cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_OTHER, s, 1);
+    if (c->n > 0)
+        k_wrap_state<<<blocks(3 * c->n, 256), 256, 0, s>>>(c->n, c->box[0], c->box[1], c->box[2], d_x_caller,
+                                                           d_pos_caller);
+    return cudaGetLastError();
+}
+
+struct MdParams {
+    double inv_mass[MAX_ELEMENTS];
+    double half_dt_acc;   // dt/2 * ACC_UNIT
+    double dt;
+    double box[3];
+    double half_skin2;
+};
+
+// v += F/m dt/2; x += v dt; wrap into [0, L); fp32 copy; flag a rebuild when
+// the fp32 position moved more than skin/2 from the build position.
+__global__ void k_md_kick_drift(int64_t n, double *__restrict__ x, double *__restrict__ v, const float *__restrict__ F,
+                                float4 *__restrict__ pos4, const float4 *__restrict__ pos_build, MdParams M,
+                                int *__restrict__ flag) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    bool moved = false;
+    if (s < n) {
+        float4 p = pos4[s];
+        int e = __float_as_int(p.w);
+        double k = M.half_dt_acc * M.inv_mass[e];
+        float q[3];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            double vv = v[3 * s + a] + k * (double)F[3 * s + a];
+            double xx = x[3 * s + a] + M.dt * vv;
+            xx -= M.box[a] * floor(xx / M.box[a]);
+            if (xx >= M.box[a]) xx -= M.box[a];
+            v[3 * s + a] = vv;
+            x[3 * s + a] = xx;
+            q[a] = (float)xx;
+        }
+        pos4[s] = make_float4(q[0], q[1], q[2], p.w);
+        float4 b = pos_build[s];
+        double d[3] = {(double)q[0] - (double)b.x, (double)q[1] - (double)b.y, (double)q[2] - (double)b.z};
+#pragma unroll
+        for (int a = 0; a < 3; ++a) d[a] -= M.box[a] * rint(d[a] / M.box[a]);
+        double r2 = d[0] * d[0] + d[1] * d[1] + d[2] * d[2];
+        moved = !(r2 <= M.half_skin2);
+    }
+    if (__any_sync(0xffffffffu, moved) && (threadIdx.x & 31) == 0) atomicOr(flag, 1);
+}
+
+static MdParams md_params(const reann_ctx *c, double dt, const double *inv_mass) {
+    MdParams M;
+    for (int e = 0; e < MAX_ELEMENTS; ++e) M.inv_mass[e] = e < c->ne ? inv_mass[e] : 0.0;
+    M.half_dt_acc = 0.5 * dt * ACC_UNIT;
+    M.dt = dt;
+    for (int a = 0; a < 3; ++a) M.box[a] = c->box[a];
+    double h = 0.5 * c->cfg.skin;
+    M.half_skin2 = h * h;
+    return M;
+}
+
+cudaError_t launch_md_kick_drift(reann_ctx *c, double dt, const double *inv_mass, int *flag, cudaStream_t s) {
+    MdParams M = md_params(c, dt, inv_mass);
+    REANN_TIMED(c, REANN_K_INTEGRATE, s, 1);
+    if (c->n > 0)
+        k_md_kick_drift<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_x, c->d_v, c->d_F, c->d_pos, c->d_pos_build, M,
+                                                          flag);
+    return cudaGetLastError();
+}
+
+__global__ void k_md_kick(int64_t n, double *__restrict__ v, const float *__restrict__ F,
+                          const float4 *__restrict__ pos4, MdParams M) {
+    int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    int e = __float_as_int(pos4[s].w);
+    double k = M.half_dt_acc * M.inv_mass[e];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) v[3 * s + a] += k * (double)F[3 * s + a];
+}
+
+cudaError_t launch_md_kick(reann_ctx *c, double dt, const double *inv_mass, cudaStream_t s) {
+    MdParams M = md_params(c, dt, inv_mass);
+    REANN_TIMED(c, REANN_K_INTEGRATE, s, 1);
+    if (c->n > 0) k_md_kick<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_v, c->d_F, c->d_pos, M);
+    return cudaGetLastError();
+}
+
+__global__ void k_kinetic_partial(int64_t n, const double *__restrict__ v, const float4 *__restrict__ pos4,
+                                  MdParams M, double *__restrict__ part) {
+    int64_t s = (int64_t)blockIdx.x * RED_THREADS + threadIdx.x;
+    double k = 0.0;
+    if (s < n) {
+        int e = __float_as_int(pos4[s].w);
+        double m = M.inv_mass[e];   // holds the mass here
+        k = 0.5 * m * (v[3 * s] * v[3 * s] + v[3 * s + 1] * v[3 * s + 1] + v[3 * s + 2] * v[3 * s + 2]) * KE_UNIT;
+    }
+    double t = block_sum(k);
+    if (threadIdx.x == 0) part[blockIdx.x] = t;
+}
+
+cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cudaStream_t s) {
+    MdParams M = md_params(c, 0.0, mass);
+    int np = (int)blocks(c->n, RED_THREADS);
+    REANN_TIMED(c, REANN_K_OTHER, s, 2);
+    if (c->n > 0) k_kinetic_partial<<<np, RED_THREADS, 0, s>>>(c->n, c->d_v, c->d_pos, M, c->d_Epart);
+    k_sum_partials<<<1, RED_THREADS, 0, s>>>(c->n > 0 ? np : 0, c->d_Epart, d_out);
+    return cudaGetLastError();
+}
+
+}  // namespace reann

@@ -26,8 +26,10 @@ Readings of unstated recipe details:
     temperature with 3N-3 degrees of freedom;
   * weights: Xavier-uniform matrices, U(-0.1, 0.1) biases, U(-1, 1) initial
     element coefficients c^0, and a per-feature input standardisation
-    (shift mu, scale s) in front of every atomic network.  The shift and
-    scale are measured once on each workload's own structure and stored in
+    (shift mu, scale s) in front of every atomic network; the energy
+    network's output layer is multiplied by an energy scale that gives
+    forces of RMS 1 eV/A.  Shift, scale and energy scale are measured once
+    on each workload's own structure and stored in
     molecular_dynamics_b200/data/norm_<workload>.json.
 
 Positions are returned as float32 values wrapped into [0, L): both the GPU
@@ -248,14 +250,27 @@ def raw_c0(p: Preset) -> np.ndarray:
     return np.random.default_rng([seeds(p)[1], 999]).uniform(-1.0, 1.0, size=(p.n_elements, p.D))
 
 
-def load_norm(p: Preset):
-    """Standardisation (shift, scale) per layer t, element and feature, or None."""
+def _load_data(p: Preset):
     path = os.path.join(_DATA, f"norm_{p.key}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f)
+        return json.load(f)
+
+
+def load_norm(p: Preset):
+    """Standardisation (shift, scale) per layer t, element and feature, or None."""
+    d = _load_data(p)
+    if d is None:
+        return None
     return np.asarray(d["shift"], np.float64), np.asarray(d["scale"], np.float64)
+
+
+def load_energy_scale(p: Preset) -> float:
+    d = _load_data(p)
+    if d is None or "energy_scale" not in d:
+        raise FileNotFoundError(f"no energy scale for workload {p.key}")
+    return float(d["energy_scale"])
 
 
 def blob_layout(p: Preset, T: int):
@@ -286,13 +301,19 @@ def blob_layout(p: Preset, T: int):
     return lay
 
 
-def weight_blob(p: Preset, T: Optional[int] = None, norm=None, use_stored_norm: bool = True) -> np.ndarray:
-    """The float32 weight blob read by both the GPU library and the oracle."""
+def weight_blob(p: Preset, T: Optional[int] = None, norm=None, use_stored_norm: bool = True,
+                energy_scale: Optional[float] = None) -> np.ndarray:
+    """The float32 weight blob read by both the GPU library and the oracle.
+
+    energy_scale multiplies the energy network's output layer (W3, b3); by
+    default the stored per-workload value is used."""
     T = p.T if T is None else T
     if norm is None and use_stored_norm:
         norm = load_norm(p)
         if norm is None:
             raise FileNotFoundError(f"no standardisation data for workload {p.key}")
+    if energy_scale is None:
+        energy_scale = load_energy_scale(p) if use_stored_norm else 1.0
     lay = blob_layout(p, T)
     blob = np.zeros(lay["total"], dtype=np.float32)
 
@@ -304,6 +325,9 @@ def weight_blob(p: Preset, T: Optional[int] = None, norm=None, use_stored_norm: 
 
     def fill(net, layer, t_in, e):
         raw = raw_network(p, layer, e)
+        if layer == ENERGY_LAYER:
+            raw["W3"] = raw["W3"] * energy_scale
+            raw["b3"] = raw["b3"] * energy_scale
         if norm is not None and t_in < norm[0].shape[0]:
             put(net["shift"], norm[0][t_in, e])
             put(net["scale"], norm[1][t_in, e])

@@ -11,6 +11,12 @@ with shift = mean(rho^t_f) and scale = std(rho^t_f) + 1e-3 mean|rho^t_f|
 feature f on the workload's own seeded structure.  Layer t's statistics are
 measured with the networks of layers < t already standardised.
 
+The same script fixes the energy scale: the energy network's output layer
+(W3, b3) is multiplied by lambda = 1 / rms(F), with F the oracle forces of
+the unscaled model on the same structure, so that the synthetic potential
+has forces of physical size (RMS 1 eV/A) rather than the tens of eV/A that
+random weights on standardised densities give.
+
 Only the oracle and the seeded input generators run here; the output file
 molecular_dynamics_b200/data/norm_<workload>.json is read by
 molecular_dynamics_b200.synth.weight_blob.
@@ -63,14 +69,21 @@ def measure(p, verbose=True):
             sat.append(float((np.abs(z) > 3).mean()))
         if verbose:
             print(f"  {p.key} layer {t}: {time.time() - t0:.1f}s, saturated fraction {sat[-1]:.3f}", flush=True)
-    return shift, scale, sat
+    # energy scale from the unscaled model at the workload's own depth T
+    blob = synth.weight_blob(p, T=p.T, norm=(shift, scale), use_stored_norm=False, energy_scale=1.0)
+    model = oracle.Model.from_preset(p, blob, T=p.T)
+    res = oracle.energy_forces(model, pos, types, box, pairs)
+    lam = float(np.float32(1.0 / np.sqrt(np.mean(res.forces ** 2))))
+    if verbose:
+        print(f"  {p.key} energy scale {lam:.6g} ({time.time() - t0:.1f}s)", flush=True)
+    return shift, scale, sat, lam
 
 
 def main(keys):
     os.makedirs(OUT, exist_ok=True)
     for k in keys:
         p = presets.get(k)
-        shift, scale, sat = measure(p)
+        shift, scale, sat, lam = measure(p)
         out = {
             "workload": k,
             "recipe": "shift = mean(rho^t_f), scale = std(rho^t_f) + 1e-3 mean|rho^t_f| + 1e-6, per layer t, "
@@ -78,6 +91,8 @@ def main(keys):
             "shift": shift.tolist(),
             "scale": scale.tolist(),
             "saturated_fraction": sat,
+            "energy_scale": lam,
+            "energy_scale_recipe": "energy network output layer multiplied by 1/rms(F) of the unscaled model",
         }
         with open(os.path.join(OUT, f"norm_{k}.json"), "w") as f:
             json.dump(out, f)

@@ -1,0 +1,71 @@
+"""The five workloads at full size, in the launch configuration the benchmark
+times, checked against the oracle on outputs it can compute one by one:
+
+  * pair-list rows of sampled atoms against brute force over all N atoms
+    (bit-exact);
+  * forces and atomic energies of sampled atoms against the oracle run on the
+    cluster of every atom within 2 T r_c (+ margin) of the sample -- exactly
+    the atoms a force depends on through T message-passing layers;
+  * properties that hold at any size: zero net force, and the total energy
+    equal to the sum of the atomic energies.
+Small workloads (up to 3,000 atoms) are compared in full.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_helpers import (F_TOL, assert_atom_energies_close, assert_energy_close, assert_forces_close, cluster_around,
+                         gpu_eval, oracle_eval)
+from molecular_dynamics_b200 import presets, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", params=list(presets.ORDER))
+def full(request):
+    p = presets.get(request.param)
+    pos, types, box = synth.make_structure(p)
+    ctx, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=0)
+    return p, pos, types, box, ctx, E, F, Ei
+
+
+def test_sampled_rows_bit_exact(full):
+    p, pos, types, box, ctx, E, F, Ei = full
+    row, col = ctx.reann_get_neighbors()
+    rng = np.random.default_rng(p.index)
+    cen = np.sort(rng.choice(len(pos), size=min(64, len(pos)), replace=False))
+    orow, ocol = oracle.pairs_brute(pos, box, p.r_cut, p.skin, centres=cen)
+    for k, a in enumerate(cen):
+        assert np.array_equal(col[row[a]:row[a + 1]], ocol[orow[k]:orow[k + 1]]), a
+    cnt = ctx.reann_get_counters()
+    assert cnt.nnz == row[-1]
+
+
+def test_net_force_and_energy_sum(full):
+    p, pos, types, box, ctx, E, F, Ei = full
+    n = len(pos)
+    # fp32 force errors of ~1e-5 eV/A add up like a random walk
+    assert np.abs(F.sum(0)).max() <= 1e-4 * np.sqrt(n) + 1e-3
+    assert abs(Ei.sum() - E) <= 1e-6 * n + 1e-4 * abs(E)
+
+
+def test_sampled_forces_and_energies(full):
+    p, pos, types, box, ctx, E, F, Ei = full
+    n = len(pos)
+    w = synth.weight_blob(p)
+    if n <= 3000:
+        ref = oracle_eval(p, pos, types, box, weights=w)
+        assert_energy_close(E, ref.energy, n)
+        assert_atom_energies_close(Ei, ref.atom_energy)
+        assert_forces_close(F, ref.forces)
+        return
+    radius = 2 * p.T * p.r_cut + 0.5
+    assert radius < box[0] / 2
+    rng = np.random.default_rng(100 + p.index)
+    samples = rng.choice(n, size=4, replace=False)
+    for k in samples:
+        cpos, ctypes_, cbox, sel = cluster_around(pos, types, box, k, radius)
+        ref = oracle_eval(p, cpos, ctypes_, cbox, weights=w)
+        assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[0], (k, F[k], ref.forces[0])
+        rel = abs(Ei[k] - ref.atom_energy[0]) / max(abs(ref.atom_energy[0]), 1e-2)
+        assert rel <= 1e-4, (k, Ei[k], ref.atom_energy[0])

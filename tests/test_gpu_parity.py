@@ -1,0 +1,165 @@
+"""GPU path vs the fp64 oracle on the same seeded inputs, through the C ABI.
+
+Sizes span several 32-row network tiles and 128-atom thread blocks with
+ragged tails; one system has fewer than three cells per axis (the cell
+stencil must not double count wrapped cells).  Pair lists must be
+bit-identical as sets; energies and forces must meet the tolerances in
+gpu_helpers.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_helpers import (assert_atom_energies_close, assert_energy_close, assert_forces_close, gpu_eval, oracle_eval,
+                         torch_cuda)
+from helpers import small
+from molecular_dynamics_b200 import presets, reann, synth
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "ag256": lambda: small("ag256"),                                           # 2 cells per axis
+    "ag500": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.scaled("ag1m", ncell=5)),
+    "water300": lambda: small("water"),
+    "water3k": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.get("water3k")),
+    "hea256": lambda: small("hea"),
+    "hea1372": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.scaled("hea108k", ncell=7)),
+    "chon976": lambda: small("chon"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_pair_list_bit_exact(case):
+    p, pos, types, box = CASES[case]()
+    ctx, _, _, _ = gpu_eval(p, pos, types, box)
+    row, col = ctx.reann_get_neighbors()
+    orow, ocol = oracle.pairs_brute(pos, box, p.r_cut, p.skin)
+    assert np.array_equal(row, orow)
+    assert np.array_equal(col, ocol)
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_energy_forces_match_oracle(case):
+    p, pos, types, box = CASES[case]()
+    _, E, F, Ei = gpu_eval(p, pos, types, box)
+    ref = oracle_eval(p, pos, types, box)
+    assert_energy_close(E, ref.energy, len(pos))
+    assert_atom_energies_close(Ei, ref.atom_energy)
+    assert_forces_close(F, ref.forces)
+    assert abs(Ei.sum() - E) <= 1e-4 * max(1.0, abs(E))
+
+
+@pytest.mark.parametrize("case", ["ag500", "water300", "hea1372", "chon976"])
+def test_every_layer_matches_oracle(case):
+    p, pos, types, box = CASES[case]()
+    ctx, _, _, _ = gpu_eval(p, pos, types, box)
+    ref = oracle_eval(p, pos, types, box, intermediates=True)
+    for t in range(p.T):
+        rho, coef = ctx.reann_get_features(t)
+        scale_r = np.abs(ref.rho[t]).max(axis=0) + 1e-6
+        assert (np.abs(rho - ref.rho[t]) / scale_r).max() <= 2e-5, t
+        scale_c = np.abs(ref.coef[t]).max(axis=0) + 1e-6
+        assert (np.abs(coef - ref.coef[t]) / scale_c).max() <= 2e-5, t
+
+
+@pytest.mark.parametrize("T", [1, 2, 4])
+def test_depths_other_than_the_preset(T):
+    p, pos, types, box = small("chon")
+    w = synth.weight_blob(p, T=T)
+    _, E, F, Ei = gpu_eval(p, pos, types, box, T=T, weights=w)
+    ref = oracle_eval(p, pos, types, box, T=T, weights=w)
+    assert_energy_close(E, ref.energy, len(pos))
+    assert_forces_close(F, ref.forces)
+
+
+def test_repeated_evaluation_is_bit_identical():
+    p, pos, types, box = small("hea")
+    ctx, E1, F1, Ei1 = gpu_eval(p, pos, types, box)
+    torch = torch_cuda()
+    pos_d = torch.from_numpy(pos).cuda()
+    F2 = torch.empty_like(pos_d)
+    E2 = ctx.reann_energy_forces(pos_d, F2)
+    assert E1 == E2
+    assert np.array_equal(F1, F2.cpu().numpy().astype(np.float64))
+
+
+def test_host_and_device_arrays_give_identical_results():
+    p, pos, types, box = small("water")
+    ctx, E1, F1, Ei1 = gpu_eval(p, pos, types, box)
+    F2 = np.zeros_like(pos)
+    Ei2 = np.zeros(len(pos), np.float32)
+    ctx2 = reann.Context(reann.ModelSpec.from_preset(p, mlp_precision=0), synth.weight_blob(p))
+    ctx2.reann_build_neighbors(pos, types, box)
+    E2 = ctx2.reann_energy_forces(pos, F2, Ei2)
+    assert E1 == E2
+    assert np.array_equal(F1, F2.astype(np.float64))
+    assert np.array_equal(Ei1, Ei2.astype(np.float64))
+
+
+def test_permuted_input_gives_permuted_output():
+    p, pos, types, box = small("chon")
+    _, E1, F1, _ = gpu_eval(p, pos, types, box)
+    perm = np.random.default_rng(11).permutation(len(pos))
+    _, E2, F2, _ = gpu_eval(p, pos[perm], types[perm], box)
+    # the internal order is (element, cell, caller index): summation order may differ
+    assert abs(E1 - E2) <= 1e-6 * max(1.0, abs(E1))
+    assert np.abs(F2 - F1[perm]).max() <= 1e-4
+
+
+def test_images_outside_the_box_are_accepted():
+    p, pos, types, box = small("hea")
+    shift = np.array([1, -2, 3], np.float32) * box.astype(np.float32)
+    _, E1, F1, _ = gpu_eval(p, pos, types, box)
+    _, E2, F2, _ = gpu_eval(p, pos + shift, types, box)
+    ref = oracle_eval(p, pos + shift, types, box)
+    assert_energy_close(E2, ref.energy, len(pos))
+    assert_forces_close(F2, ref.forces)
+
+
+def test_isolated_atom_and_pair():
+    p = presets.get("water3k")
+    box = np.array([30.0, 30.0, 30.0])
+    for pos, types in ((np.array([[1.0, 2.0, 3.0]], np.float32), np.array([1], np.int32)),
+                       (np.array([[5.0, 5.0, 5.0], [6.1, 5.3, 4.2]], np.float32), np.array([1, 0], np.int32))):
+        _, E, F, Ei = gpu_eval(p, pos, types, box)
+        ref = oracle_eval(p, pos, types, box)
+        assert_energy_close(E, ref.energy, len(pos))
+        assert_forces_close(F, ref.forces)
+
+
+def test_empty_system():
+    p = presets.get("ag256")
+    ctx, E, F, Ei = gpu_eval(p, np.zeros((0, 3), np.float32), np.zeros(0, np.int32), np.array([20.0, 20.0, 20.0]))
+    assert E == 0.0 and F.shape == (0, 3)
+
+
+def test_error_statuses():
+    torch = torch_cuda()
+    p, pos, types, box = small("ag256")
+    spec = reann.ModelSpec.from_preset(p, mlp_precision=0)
+    ctx = reann.Context(spec, synth.weight_blob(p))
+    with pytest.raises(reann.ReannError) as e:
+        ctx.reann_energy_forces(pos)
+    assert e.value.status == 6                                        # no list yet
+    with pytest.raises(reann.ReannError) as e:
+        ctx.reann_build_neighbors(pos, types, np.array([13.0, 20.0, 20.0]))
+    assert e.value.status == 2                                        # box < 2 (r_c + skin)
+    bad = types.copy()
+    bad[3] = 5
+    with pytest.raises(reann.ReannError) as e:
+        ctx.reann_build_neighbors(pos, bad, box)
+    assert e.value.status == 1                                        # type out of range
+    nan = pos.copy()
+    nan[7, 1] = np.nan
+    with pytest.raises(reann.ReannError) as e:
+        ctx.reann_build_neighbors(nan, types, box)
+    assert e.value.status == 4                                        # non-finite
+    ctx.reann_build_neighbors(pos, types, box)
+    moved = pos.copy()
+    moved[0] += np.float32(0.6)                                       # > skin / 2
+    with pytest.raises(reann.ReannError) as e:
+        ctx.reann_energy_forces(moved)
+    assert e.value.status == 5
+    ctx.reann_energy_forces(pos)                                      # context still usable
+    with pytest.raises(reann.ReannError):
+        ctx.reann_get_features(p.T)                                   # layer out of range
