@@ -175,7 +175,7 @@ def main():
     v0 = synth.maxwell_boltzmann(p, types)
     n = len(pos)
     dt_fs = 1.0   # the metric's step (the water workload's own 0.5 fs is reported beside it)
-    spec = reann.ModelSpec.from_preset(p, mlp_precision=0)
+    spec = reann.ModelSpec.from_preset(p)   # the workload's own network precision (bf16 for ag1m)
     ctx = reann.Context(spec, synth.weight_blob(p), device=local)
     stream = torch.cuda.current_stream()
     x = torch.from_numpy(pos.astype(np.float64)).cuda()
@@ -276,10 +276,11 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32 (networks bf16, fp32 accumulate)" if p.mlp_precision else "f32",
+        "data": "synthetic",
         "config": {"workload": f"{p.key}: {p.description}", "atoms": n, "T": p.T, "r_cut": p.r_cut,
                    "n_radial": p.n_radial, "l_max": p.l_max, "hidden": list(p.hidden), "dt_fs": dt_fs,
-                   "networks": "fp32 CUDA-core", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "networks": "bf16 tcgen05, fp32 accumulate" if p.mlp_precision else "fp32 CUDA-core", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"working set > L2 ({n * (p.T * (10 * p.n_radial + 6 * p.n_radial) * 4) / 1e9:.1f} GB of "
                          f"per-layer activations vs 126 MB L2); no flush needed"},
         "ns_per_day": (args.steps / (t_ms * 1e-3)) * dt_fs * 86400 / 1e6,

@@ -208,22 +208,35 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
     CK(launch_fill(c, s));
     c->nnz = nnz;
     c->max_row = c->h_i64[2];
-    // tile table of the atomic networks: element segments cut into 32-row tiles
-    std::vector<int4> tiles;
-    for (int e = 0; e < c->ne; ++e)
-        for (int r = c->h_seg[e]; r < c->h_seg[e + 1]; r += 32)
-            tiles.push_back(make_int4(e, r, std::min(32, c->h_seg[e + 1] - r), 0));
-    bool same = (int)tiles.size() == c->n_tiles && c->elem_start.size() == (size_t)c->ne + 1 &&
+    // tile tables of the atomic networks: element segments cut into 32-row
+    // (CUDA cores) and 128-row (tensor cores) tiles; segments only change when
+    // the atoms' element counts do
+    bool same = c->elem_start.size() == (size_t)c->ne + 1 &&
                 std::equal(c->elem_start.begin(), c->elem_start.end(), c->h_seg);
     if (!same) {
+        std::vector<int4> tiles, tiles128;
+        for (int e = 0; e < c->ne; ++e) {
+            for (int r = c->h_seg[e]; r < c->h_seg[e + 1]; r += 32)
+                tiles.push_back(make_int4(e, r, std::min(32, c->h_seg[e + 1] - r), 0));
+            for (int r = c->h_seg[e]; r < c->h_seg[e + 1]; r += 128)
+                tiles128.push_back(make_int4(e, r, std::min(128, c->h_seg[e + 1] - r), 0));
+        }
         if ((int)tiles.size() > c->n_tiles_alloc) {
             CK(dalloc(&c->d_tiles, tiles.size()));
             c->n_tiles_alloc = (int)tiles.size();
         }
+        if ((int)tiles128.size() > c->n_tiles128_alloc) {
+            CK(dalloc(&c->d_tiles128, tiles128.size()));
+            c->n_tiles128_alloc = (int)tiles128.size();
+        }
         if (!tiles.empty())
             CK(cudaMemcpyAsync(c->d_tiles, tiles.data(), sizeof(int4) * tiles.size(), cudaMemcpyHostToDevice, s));
+        if (!tiles128.empty())
+            CK(cudaMemcpyAsync(c->d_tiles128, tiles128.data(), sizeof(int4) * tiles128.size(),
+                               cudaMemcpyHostToDevice, s));
         CK(sync_stream(c, s));
         c->n_tiles = (int)tiles.size();
+        c->n_tiles128 = (int)tiles128.size();
         c->elem_start.assign(c->h_seg, c->h_seg + c->ne + 1);
     }
     c->have_list = true;
@@ -233,15 +246,16 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
 
 // One energy+force evaluation on the internal positions d_pos.
 reann_status run_ef(reann_ctx *c, cudaStream_t s) {
+    const bool tc = c->cfg.mlp_precision == 1;
     CK(launch_active(c, s));
     for (int t = 0; t < c->T; ++t) {
         CK(launch_density_fwd(c, t, s));
-        if (t + 1 < c->T) CK(launch_mlp_coef_fwd(c, t, s));
+        if (t + 1 < c->T) CK(tc ? launch_mlp_tc_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s));
     }
-    CK(launch_mlp_energy(c, s));
+    CK(tc ? launch_mlp_tc_energy(c, s) : launch_mlp_energy(c, s));
     for (int t = c->T - 1; t >= 0; --t) {
         CK(launch_edge_bwd(c, t, t != c->T - 1, s));
-        if (t >= 1) CK(launch_mlp_coef_bwd(c, t, s));
+        if (t >= 1) CK(tc ? launch_mlp_tc_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s));
     }
     CK(launch_energy_sum(c, s));
     c->counters.evaluations++;
@@ -313,8 +327,8 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
         !(cfg->r_cut > 0) || !(cfg->skin >= 0) || !(cfg->alpha > 0) || !std::isfinite(cfg->r_cut) ||
         !std::isfinite(cfg->skin) || cfg->mlp_precision < 0 || cfg->mlp_precision > 1)
         return fail(nullptr, REANN_ERR_ARG, "invalid configuration");
-    if (cfg->mlp_precision == 1)
-        return fail(nullptr, REANN_ERR_UNSUPPORTED, "bf16 tensor-core networks are not built yet");
+    if (cfg->mlp_precision == 1 && (cfg->hidden[0] != 128 || cfg->hidden[1] != 128))
+        return fail(nullptr, REANN_ERR_UNSUPPORTED, "bf16 tensor-core networks need hidden widths [128, 128]");
     if (cfg->l_max != 2 || (cfg->n_radial != 8 && cfg->n_radial != 10) ||
         (cfg->hidden[0] != 64 && cfg->hidden[0] != 128) || (cfg->hidden[1] != 64 && cfg->hidden[1] != 128))
         return fail(nullptr, REANN_ERR_UNSUPPORTED, "supported: l_max 2, n_radial 8 or 10, hidden widths 64 or 128");
@@ -378,7 +392,7 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     DeviceGuard guard(c->device);
     free_atoms(c);
     dfree(c->d_w); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
-    dfree(c->d_act_col); dfree(c->d_tiles); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
+    dfree(c->d_act_col); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
     if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
     if (c->h_status) cudaFreeHost(c->h_status);
     if (c->h_i64) cudaFreeHost(c->h_i64);
@@ -544,7 +558,9 @@ extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs
         CK(cudaMemcpyAsync(v, c->d_last_v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, s));
     }
     CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_i64 + 3, c->d_i64 + 3, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
     CK(sync_stream(c, s));
+    c->counters.active_pairs = c->h_i64[3];
     c->md_valid = (c->h_status[0] & ~ST_SKIN) == 0;
     c->md_dt = dt_fs;
     std::copy(mass, mass + c->ne, c->md_mass);

@@ -108,9 +108,12 @@ struct reann_ctx {
     double *d_E = nullptr;     // [4] energies (pot, kin, ...)
     int n_part = 0;
 
-    // MLP tile table: per tile (element, first row, rows)
+    // MLP tile tables: per tile (element, first row, rows); 32-row tiles for
+    // the CUDA-core networks, 128-row tiles for the tensor-core networks
     int4 *d_tiles = nullptr;
     int n_tiles = 0, n_tiles_alloc = 0;
+    int4 *d_tiles128 = nullptr;
+    int n_tiles128 = 0, n_tiles128_alloc = 0;
 
     // staging for host arrays and caller-order scratch
     float *d_stage_f = nullptr;    // [n][3] floats

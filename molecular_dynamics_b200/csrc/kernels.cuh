@@ -31,6 +31,12 @@ cudaError_t launch_mlp_coef_fwd(reann_ctx *c, int t, cudaStream_t s);   // rho^t
 cudaError_t launch_mlp_energy(reann_ctx *c, cudaStream_t s);            // rho^{T-1} -> E_i, G^{T-1}
 cudaError_t launch_mlp_coef_bwd(reann_ctx *c, int t, cudaStream_t s);   // (rho^{t-1}, dE/dc^t) -> G^{t-1}
 
+// atomic networks on tcgen05 tensor cores, bf16 operands (mlp_tc.cu)
+bool tc_supported(const reann_ctx *c);
+cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
+cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s);
+cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
+
 // reductions, gathers and the integrator (md.cu)
 cudaError_t launch_pos_from_caller(reann_ctx *c, const float *d_pos_caller, cudaStream_t s);
 cudaError_t launch_energy_sum(reann_ctx *c, cudaStream_t s);            // -> d_E[0], status on non-finite

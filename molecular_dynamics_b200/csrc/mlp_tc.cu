@@ -1,0 +1,494 @@
+// Per-element atomic networks on the 5th-generation tensor cores (tcgen05),
+// bf16 operands with fp32 accumulation in tensor memory.
+//
+// Same networks as mlp.cu ("Efficient Parallelization of Message Passing
+// Neural Network Potentials for Large-Scale Molecular Dynamics", section "REANN
+// Architecture", Eq. 2 and the atomic energy; section "Parallelization
+// Algorithm", Eqs. 3 and 5 for the vector-Jacobian products):
+//   y = W3 tanh(W2 tanh(W1 ((x - shift) / scale) + b1) + b2) + b3.
+// A tile is 128 atoms of one element.  Each layer is one 128 x N x K GEMM
+// (tcgen05.mma, M = 128, K = 16 per instruction) whose accumulator sits in
+// TMEM; TMEM lane i holds atom i, so the epilogue (bias, tanh, tanh', the
+// energy dot product, dE/dA) is one thread per atom with no cross-thread
+// reduction.  The epilogue writes the next layer's bf16 operand straight into
+// shared memory in the canonical K-major layout, and one thread issues the
+// next MMA.
+//
+// Block: 128 threads (4 warps, warp w reads TMEM lanes 32w..32w+31), one
+// block per SM (shared memory > half an SM), persistent over the tiles.  All
+// waits on the MMA-completion barrier are bounded: a wait that gives up sets
+// ST_TIMEOUT, the block frees its tensor memory and returns.
+//
+// Shared-memory operand layout (K-major, no swizzle): an R x K bf16 tile keeps
+// element (r, k) at byte (k/8) R 16 + (r/8) 128 + (r%8) 16 + (k%8) 2, i.e.
+// 8-row x 16-byte core matrices, 128 B between 8-row groups (SBO) and R*16 B
+// between 16-byte K chunks (LBO).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace reann {
+namespace {
+
+constexpr int TM = 128;            // atoms per tile (MMA M)
+constexpr int TC_THREADS = 128;
+constexpr int KPAD = 32;           // feature dimension padded to a multiple of 16
+constexpr int TMEM_COLS = 512;
+
+enum { TC_FWD = 0, TC_ENERGY = 1, TC_BWD = 2 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t kmaj(int r, int k, int R) {
+    return (uint32_t)((k >> 3) * (R * 16) + (r >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2);
+}
+
+// shared-memory matrix descriptor: start, LBO, SBO (bytes), version 1, no swizzle
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128
+__host__ __device__ constexpr uint32_t idesc_bf16(int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// D[128 x N] (+)= A[128 x K] B[N x K]^T, both operands canonical K-major tiles
+template <int N, int K>
+__device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+    constexpr uint32_t idesc = idesc_bf16(N);
+#pragma unroll
+    for (int s = 0; s < K / 16; ++s) {
+        uint64_t a = sdesc(a_smem + (uint32_t)(2 * s * TM * 16), TM * 16, 128);
+        uint64_t b = sdesc(b_smem + (uint32_t)(2 * s * N * 16), N * 16, 128);
+        mma_bf16(d_tmem, a, b, idesc, s > 0 ? 1u : 0u);
+    }
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_smem_to_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// bounded wait for the barrier phase with the given parity
+__device__ __forceinline__ bool bar_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t a = smem_u32(bar);
+    for (int it = 0; it < (1 << 20); ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+// 32 consecutive fp32 TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// 8 bf16 values (columns c..c+7 of row r) -> one 16-byte chunk of a K-major tile
+__device__ __forceinline__ void st_chunk(unsigned char *tile, int R, int r, int c, const float *v) {
+    uint4 w = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    *reinterpret_cast<uint4 *>(tile + kmaj(r, c, R)) = w;
+}
+
+__device__ __forceinline__ void ld_chunk(const unsigned char *tile, int R, int r, int c, float *v) {
+    uint4 w = *reinterpret_cast<const uint4 *>(tile + kmaj(r, c, R));
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float2 f = __bfloat1622float2(h[k]);
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+    }
+}
+
+// one bf16 element of a K-major tile (weight preparation)
+__device__ __forceinline__ void st_elem(unsigned char *tile, int R, int r, int k, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(tile + kmaj(r, k, R)) = __float2bfloat16_rn(x);
+}
+
+struct TcNets {
+    NetOffsets net[MAX_ELEMENTS];
+};
+
+template <int NP, int H1, int H2, int MODE>
+struct TcLayout {
+    static constexpr int D = 3 * NP;
+    static constexpr int NA = NP * NT;
+    // bf16 operand tiles (bytes)
+    static constexpr int W1 = 0;                                        // [H1][KPAD]  B of layer 1
+    static constexpr int W2 = W1 + H1 * KPAD * 2;                       // [H2][H1]    B of layer 2
+    static constexpr int W3 = W2 + H2 * H1 * 2;                         // [KPAD][H2]  B of layer 3 (FWD)
+    static constexpr int W2T = W3 + (MODE == TC_FWD ? KPAD * H2 * 2 : 0);   // [H1][H2]  B of dE/da1
+    static constexpr int W3T = W2T + (MODE != TC_FWD ? H1 * H2 * 2 : 0);    // [H2][KPAD] B of dE/da2 (BWD)
+    static constexpr int W1T = W3T + (MODE == TC_BWD ? H2 * KPAD * 2 : 0);  // [KPAD][H1] B of dE/dx
+    static constexpr int X = W1T + (MODE != TC_FWD ? KPAD * H1 * 2 : 0);    // [TM][KPAD] standardised input
+    static constexpr int DY = X + TM * KPAD * 2;                        // [TM][KPAD] upstream gradient (BWD)
+    static constexpr int A1 = DY + (MODE == TC_BWD ? TM * KPAD * 2 : 0);    // [TM][H1]
+    static constexpr int A2 = A1 + TM * H1 * 2;                         // [TM][H2] (FWD: a2; else g2, then g1)
+    static constexpr int F32 = A2 + TM * (H1 > H2 ? H1 : H2) * 2;       // fp32 vectors
+    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2;         // b1, b2, b3, shift, scale, inv_scale, w3
+    static constexpr int BAR = F32 + nf32 * 4;
+    static constexpr int bytes = BAR + 16 + 16;
+    // TMEM columns
+    static constexpr int C_Z1 = 0, C_Z2 = 128, C_P2 = 256, C_OUT = 384;
+};
+
+template <int NP, int H1, int H2, int MODE>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_mlp_tc(const int4 *__restrict__ tiles, int n_tiles, const float *__restrict__ w, TcNets nets,
+             const float *__restrict__ X, float *__restrict__ Y, const float *__restrict__ dY, float *__restrict__ Ei,
+             const float *__restrict__ A, float *__restrict__ Gout, int *__restrict__ status) {
+    using L = TcLayout<NP, H1, H2, MODE>;
+    constexpr int D = L::D, NA = L::NA;
+    constexpr int DOUT = MODE == TC_ENERGY ? 1 : D;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    float *f32 = reinterpret_cast<float *>(sm + L::F32);
+    float *sb1 = f32, *sb2 = sb1 + H1, *sb3 = sb2 + H2, *sshift = sb3 + KPAD, *sscale = sshift + KPAD,
+          *sinv = sscale + KPAD, *sw3 = sinv + KPAD;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid;                       // this thread's atom within the tile (TMEM lane)
+    const uint32_t base = smem_u32(sm);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t phase = 0;
+    bool failed = false;
+    int cur = -1;
+
+    // one MMA group issued by thread 0, completion awaited by all threads
+    auto wait_mma = [&]() -> bool {
+        bool ok = bar_wait(bar, phase);
+        phase ^= 1u;
+        fence_after();
+        return !__syncthreads_or(!ok);
+    };
+
+    for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
+        const int4 tile = tiles[ti];
+        const int e = tile.x, r0 = tile.y, rows = tile.z;
+        if (e != cur) {
+            // element weights -> bf16 operand tiles and fp32 vectors
+            const NetOffsets &o = nets.net[e];
+            for (int k = tid; k < H1 * KPAD; k += TC_THREADS) {
+                int n = k / KPAD, f = k % KPAD;
+                st_elem(sm + L::W1, H1, n, f, f < D ? w[o.W1 + (int64_t)n * D + f] : 0.f);
+            }
+            for (int k = tid; k < H2 * H1; k += TC_THREADS) {
+                int n = k / H1, h = k % H1;
+                float v = w[o.W2 + k];
+                st_elem(sm + L::W2, H2, n, h, v);
+                if (MODE != TC_FWD) st_elem(sm + L::W2T, H1, h, n, v);
+            }
+            if (MODE == TC_FWD) {
+                for (int k = tid; k < KPAD * H2; k += TC_THREADS) {
+                    int n = k / H2, h = k % H2;
+                    st_elem(sm + L::W3, KPAD, n, h, n < DOUT ? w[o.W3 + (int64_t)n * H2 + h] : 0.f);
+                }
+            }
+            if (MODE == TC_BWD) {
+                for (int k = tid; k < H2 * KPAD; k += TC_THREADS) {
+                    int h = k / KPAD, j = k % KPAD;
+                    st_elem(sm + L::W3T, H2, h, j, j < DOUT ? w[o.W3 + (int64_t)j * H2 + h] : 0.f);
+                }
+            }
+            if (MODE != TC_FWD) {
+                for (int k = tid; k < KPAD * H1; k += TC_THREADS) {
+                    int f = k / H1, h = k % H1;
+                    st_elem(sm + L::W1T, KPAD, f, h, f < D ? w[o.W1 + (int64_t)h * D + f] : 0.f);
+                }
+            }
+            for (int k = tid; k < H1; k += TC_THREADS) sb1[k] = w[o.b1 + k];
+            for (int k = tid; k < H2; k += TC_THREADS) {
+                sb2[k] = w[o.b2 + k];
+                if (MODE == TC_ENERGY) sw3[k] = w[o.W3 + k];
+            }
+            for (int k = tid; k < KPAD; k += TC_THREADS) {
+                sb3[k] = k < DOUT ? w[o.b3 + k] : 0.f;
+                sshift[k] = k < D ? w[o.shift + k] : 0.f;
+                sscale[k] = k < D ? w[o.scale + k] : 1.f;
+                sinv[k] = k < D ? 1.0f / w[o.scale + k] : 0.f;
+            }
+            cur = e;
+        }
+        __syncthreads();
+        // input tile: standardised rho (and the upstream gradient) as bf16
+        {
+            const bool live = row < rows;
+            const int64_t gi = (int64_t)(r0 + row);
+#pragma unroll
+            for (int c = 0; c < KPAD; c += 8) {
+                float v[8], g[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    int f = c + u;
+                    float x = (live && f < D) ? X[gi * D + f] : 0.f;
+                    v[u] = f < D ? (x - sshift[f]) / sscale[f] : 0.f;
+                    if (!live) v[u] = 0.f;
+                    if (MODE == TC_BWD) g[u] = (live && f < D) ? dY[gi * D + f] : 0.f;
+                }
+                st_chunk(sm + L::X, TM, row, c, v);
+                if (MODE == TC_BWD) st_chunk(sm + L::DY, TM, row, c, g);
+            }
+        }
+        fence_smem_to_async();
+        __syncthreads();
+
+        // layer 1 (and, for the backward network, dE/da2 = dY W3)
+        if (tid == 0) {
+            fence_after();
+            gemm<H1, KPAD>(tmem + L::C_Z1, base + L::X, base + L::W1);
+            if (MODE == TC_BWD) gemm<H2, KPAD>(tmem + L::C_P2, base + L::DY, base + L::W3T);
+            mma_commit(bar);
+        }
+        if (!wait_mma()) { failed = true; break; }
+        // a1 = tanh(z1 + b1) -> A1
+#pragma unroll 1
+        for (int c = 0; c < H1; c += 32) {
+            float v[32];
+            tmem_ld32(lane_base + L::C_Z1 + c, v);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb1[c + u]);
+#pragma unroll
+            for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A1, TM, row, c + u, &v[u]);
+        }
+        fence_smem_to_async();
+        fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            fence_after();
+            gemm<H2, H1>(tmem + L::C_Z2, base + L::A1, base + L::W2);
+            mma_commit(bar);
+        }
+        if (!wait_mma()) { failed = true; break; }
+
+        if (MODE == TC_FWD) {
+            // a2 = tanh(z2 + b2) -> A2, then y = a2 W3^T + b3
+#pragma unroll 1
+            for (int c = 0; c < H2; c += 32) {
+                float v[32];
+                tmem_ld32(lane_base + L::C_Z2 + c, v);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb2[c + u]);
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A2, TM, row, c + u, &v[u]);
+            }
+            fence_smem_to_async();
+            fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after();
+                gemm<KPAD, H2>(tmem + L::C_OUT, base + L::A2, base + L::W3);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            float v[32];
+            tmem_ld32(lane_base + L::C_OUT, v);
+            if (row < rows) {
+                float *yo = Y + (int64_t)(r0 + row) * D;
+#pragma unroll
+                for (int f = 0; f < D; ++f) yo[f] = v[f] + sb3[f];
+            }
+        } else {
+            // g2 = dE/dz2: energy network dE_i/da2 = w3; backward network dY W3 (TMEM)
+            float e_row = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < H2; c += 32) {
+                float z[32], p[32];
+                tmem_ld32(lane_base + L::C_Z2 + c, z);
+                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P2 + c, p);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    float a = tanh_fast(z[u] + sb2[c + u]);
+                    float up = MODE == TC_ENERGY ? sw3[c + u] : p[u];
+                    if (MODE == TC_ENERGY) e_row = fmaf(sw3[c + u], a, e_row);
+                    z[u] = up * (1.f - a * a);
+                }
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A2, TM, row, c + u, &z[u]);
+            }
+            if (MODE == TC_ENERGY && row < rows) Ei[r0 + row] = e_row + sb3[0];
+            fence_smem_to_async();
+            fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after();
+                gemm<H1, H2>(tmem + L::C_Z1, base + L::A2, base + L::W2T);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            // g1 = (g2 W2) (1 - a1^2) -> over the g2 tile (its MMA has completed)
+#pragma unroll 1
+            for (int c = 0; c < H1; c += 32) {
+                float v[32];
+                tmem_ld32(lane_base + L::C_Z1 + c, v);
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) {
+                    float a[8];
+                    ld_chunk(sm + L::A1, TM, row, c + u, a);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[u + q] *= 1.f - a[q] * a[q];
+                    st_chunk(sm + L::A2, TM, row, c + u, &v[u]);
+                }
+            }
+            fence_smem_to_async();
+            fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after();
+                gemm<KPAD, H1>(tmem + L::C_OUT, base + L::A2, base + L::W1T);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            // dE/drho = (g1 W1) / scale; G = dE/dA = 2 w_tau A dE/drho
+            float gx[32];
+            tmem_ld32(lane_base + L::C_OUT, gx);
+            if (row < rows) {
+#pragma unroll
+                for (int f = 0; f < D; ++f) gx[f] *= sinv[f];
+                const int64_t gi = (int64_t)(r0 + row) * NA;
+                const float4 *a4 = reinterpret_cast<const float4 *>(A + gi);
+                float4 *g4 = reinterpret_cast<float4 *>(Gout + gi);
+#pragma unroll
+                for (int q = 0; q < NA / 4; ++q) {
+                    float4 a = a4[q];
+                    float av[4] = {a.x, a.y, a.z, a.w}, gv[4];
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const int k = 4 * q + s, nn = k / NT, u = k % NT;
+                        const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
+                        const float wt = u >= 7 ? 4.f : 2.f;
+                        gv[s] = wt * av[s] * gx[l * NP + nn];
+                    }
+                    g4[q] = make_float4(gv[0], gv[1], gv[2], gv[3]);
+                }
+            }
+        }
+        fence_before();
+        __syncthreads();
+    }
+
+    if (failed && tid == 0) atomicOr(status, ST_TIMEOUT);
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+}
+
+template <int NP, int H1, int H2, int MODE>
+cudaError_t run_tc(reann_ctx *c, const TcNets &nets, const float *X, float *Y, const float *dY, float *Ei,
+                   const float *A, float *G, cudaStream_t s) {
+    using L = TcLayout<NP, H1, H2, MODE>;
+    static_assert(L::bytes > 116 * 1024 && L::bytes <= 227 * 1024, "one block per SM keeps TMEM allocation safe");
+    static bool configured[64] = {};
+    auto kern = k_mlp_tc<NP, H1, H2, MODE>;
+    if (c->device < 0 || c->device >= 64) return cudaErrorInvalidDevice;
+    if (!configured[c->device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::bytes);
+        if (e) return e;
+        configured[c->device] = true;
+    }
+    if (c->n_tiles128 == 0) return cudaSuccess;
+    int grid = c->sm_count < c->n_tiles128 ? c->sm_count : c->n_tiles128;
+    REANN_TIMED(c, MODE == TC_FWD ? REANN_K_MLP_FWD : (MODE == TC_ENERGY ? REANN_K_MLP_ENERGY : REANN_K_MLP_BWD), s);
+    kern<<<grid, TC_THREADS, L::bytes, s>>>(c->d_tiles128, c->n_tiles128, c->d_w, nets, X, Y, dY, Ei, A, G,
+                                            c->d_status);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t dispatch_tc(reann_ctx *c, const TcNets &nets, const float *X, float *Y, const float *dY, float *Ei,
+                        const float *A, float *G, cudaStream_t s) {
+    if (c->NP == 8 && c->H1 == 128 && c->H2 == 128) return run_tc<8, 128, 128, MODE>(c, nets, X, Y, dY, Ei, A, G, s);
+    if (c->NP == 10 && c->H1 == 128 && c->H2 == 128) return run_tc<10, 128, 128, MODE>(c, nets, X, Y, dY, Ei, A, G, s);
+    return cudaErrorInvalidValue;
+}
+
+TcNets tc_nets(const std::vector<NetOffsets> &v, int first, int ne) {
+    TcNets m;
+    for (int e = 0; e < ne; ++e) m.net[e] = v[first + e];
+    return m;
+}
+
+}  // namespace
+
+bool tc_supported(const reann_ctx *c) { return (c->NP == 8 || c->NP == 10) && c->H1 == 128 && c->H2 == 128; }
+
+cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
+    const int64_t nD = c->n * c->D;
+    return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD, c->d_coef + (t + 1) * nD,
+                               nullptr, nullptr, nullptr, nullptr, s);
+}
+
+cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s) {
+    const int64_t nD = c->n * c->D, nA = c->n * c->NA;
+    const int t = c->T - 1;
+    return dispatch_tc<TC_ENERGY>(c, tc_nets(c->energy_nets, 0, c->ne), c->d_rho + t * nD, nullptr, nullptr, c->d_Ei,
+                                  c->d_A + t * nA, c->d_G, s);
+}
+
+cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s) {
+    const int64_t nD = c->n * c->D, nA = c->n * c->NA;
+    return dispatch_tc<TC_BWD>(c, tc_nets(c->coef_nets, (t - 1) * c->ne, c->ne), c->d_rho + (t - 1) * nD, nullptr,
+                               c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
+}
+
+}  // namespace reann

@@ -26,7 +26,8 @@ Readings of unstated recipe details:
     temperature with 3N-3 degrees of freedom;
   * weights: Xavier-uniform matrices, U(-0.1, 0.1) biases, U(-1, 1) initial
     element coefficients c^0, and a per-feature input standardisation
-    (shift mu, scale s) in front of every atomic network; the energy
+    (shift = mean, scale = std + 0.05 mean|.|, so that mean/scale <= 20) in
+    front of every atomic network; the energy
     network's output layer is multiplied by an energy scale that gives
     forces of RMS 1 eV/A.  Shift, scale and energy scale are measured once
     on each workload's own structure and stored in

@@ -6,10 +6,16 @@ Part of the weight recipe, not of the model: the paper's trained weights are
 not available, and random Xavier weights applied to raw embedded densities
 (values up to ~1e3 with a spread of a few percent) would saturate tanh and
 leave the forces near zero.  So each network sees (rho - shift) / scale,
-with shift = mean(rho^t_f) and scale = std(rho^t_f) + 1e-3 mean|rho^t_f|
+with shift = mean(rho^t_f) and scale = std(rho^t_f) + 0.05 mean|rho^t_f|
 + 1e-6, measured per layer t, per element of the centre atom and per
 feature f on the workload's own seeded structure.  Layer t's statistics are
 measured with the networks of layers < t already standardised.
+
+The 0.05 mean|rho| floor bounds the conditioning mean|rho| / scale by 20.
+A thermal crystal has density spreads of about 1 % of the mean, far below
+the spread of the varied structures a real model is fitted on; scaling by
+that spread alone made the synthetic model amplify any rounding of rho up
+to a thousandfold.
 
 The same script fixes the energy scale: the energy network's output layer
 (W3, b3) is multiplied by lambda = 1 / rms(F), with F the oracle forces of
@@ -33,6 +39,7 @@ import numpy as np
 import oracle
 from molecular_dynamics_b200 import presets, synth
 
+FLOOR = 0.05
 OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "molecular_dynamics_b200", "data")
 
 
@@ -59,7 +66,7 @@ def measure(p, verbose=True):
             sel = types == e
             r = rho[sel]
             mu = r.mean(0)
-            sd = r.std(0) + 1e-3 * np.abs(r).mean(0) + 1e-6
+            sd = r.std(0) + FLOOR * np.abs(r).mean(0) + 1e-6
             shift[t, e] = np.float32(mu)
             scale[t, e] = np.float32(sd)
             # diagnostic: fraction of first-layer pre-activations beyond |3|
@@ -86,7 +93,7 @@ def main(keys):
         shift, scale, sat, lam = measure(p)
         out = {
             "workload": k,
-            "recipe": "shift = mean(rho^t_f), scale = std(rho^t_f) + 1e-3 mean|rho^t_f| + 1e-6, per layer t, "
+            "recipe": "shift = mean(rho^t_f), scale = std(rho^t_f) + 0.05 mean|rho^t_f| + 1e-6, per layer t, "
                       "element of the centre atom and feature f, on the workload's seeded structure",
             "shift": shift.tolist(),
             "scale": scale.tolist(),

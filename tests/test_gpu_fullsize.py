@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_helpers import (F_TOL, assert_atom_energies_close, assert_energy_close, assert_forces_close, cluster_around,
+from gpu_helpers import (E_TOL, F_TOL, assert_atom_energies_close, assert_energy_close, assert_forces_close, cluster_around,
                          gpu_eval, oracle_eval)
 from molecular_dynamics_b200 import presets, synth
 
@@ -25,7 +25,8 @@ pytestmark = pytest.mark.gpu
 def full(request):
     p = presets.get(request.param)
     pos, types, box = synth.make_structure(p)
-    ctx, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=0)
+    # the launch configuration the benchmark times: the workload's own network precision
+    ctx, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=p.mlp_precision)
     return p, pos, types, box, ctx, E, F, Ei
 
 
@@ -53,11 +54,12 @@ def test_sampled_forces_and_energies(full):
     p, pos, types, box, ctx, E, F, Ei = full
     n = len(pos)
     w = synth.weight_blob(p)
+    prec = p.mlp_precision
     if n <= 3000:
         ref = oracle_eval(p, pos, types, box, weights=w)
-        assert_energy_close(E, ref.energy, n)
-        assert_atom_energies_close(Ei, ref.atom_energy)
-        assert_forces_close(F, ref.forces)
+        assert_energy_close(E, ref.energy, n, prec)
+        assert_atom_energies_close(Ei, ref.atom_energy, prec)
+        assert_forces_close(F, ref.forces, prec)
         return
     radius = 2 * p.T * p.r_cut + 0.5
     assert radius < box[0] / 2
@@ -66,6 +68,6 @@ def test_sampled_forces_and_energies(full):
     for k in samples:
         cpos, ctypes_, cbox, sel = cluster_around(pos, types, box, k, radius)
         ref = oracle_eval(p, cpos, ctypes_, cbox, weights=w)
-        assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[0], (k, F[k], ref.forces[0])
+        assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[prec], (k, F[k], ref.forces[0])
         rel = abs(Ei[k] - ref.atom_energy[0]) / max(abs(ref.atom_energy[0]), 1e-2)
-        assert rel <= 1e-4, (k, Ei[k], ref.atom_energy[0])
+        assert rel <= 10 * E_TOL[prec], (k, Ei[k], ref.atom_energy[0])

@@ -62,14 +62,42 @@ def test_every_layer_matches_oracle(case):
         assert (np.abs(coef - ref.coef[t]) / scale_c).max() <= 2e-5, t
 
 
-@pytest.mark.parametrize("T", [1, 2, 4])
-def test_depths_other_than_the_preset(T):
-    p, pos, types, box = small("chon")
+@pytest.mark.parametrize("key,T", [("chon", 1), ("chon", 2), ("ag", 1), ("ag", 4), ("ag", 6)])
+def test_depths_other_than_the_preset(key, T):
+    # the Ag model's standardisation covers layers up to 6 (its T sweep)
+    p, pos, types, box = small(key)
     w = synth.weight_blob(p, T=T)
     _, E, F, Ei = gpu_eval(p, pos, types, box, T=T, weights=w)
     ref = oracle_eval(p, pos, types, box, T=T, weights=w)
     assert_energy_close(E, ref.energy, len(pos))
     assert_forces_close(F, ref.forces)
+
+
+BF16_CASES = {
+    "ag500": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.scaled("ag1m", ncell=5)),
+    "ag2048": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.scaled("ag1m", ncell=8)),
+    # five elements with N_phi = 10 and [128,128] networks: ragged 128-row tiles per element
+    "hea1372_h128": lambda: (lambda p: (p, *synth.make_structure(p)))(
+        presets.scaled("hea108k", ncell=7).with_(hidden=(128, 128))),
+}
+
+
+@pytest.mark.parametrize("case", sorted(BF16_CASES))
+def test_bf16_tensor_core_networks_match_oracle(case):
+    p, pos, types, box = BF16_CASES[case]()
+    w = synth.weight_blob(p)
+    _, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=1, weights=w)
+    ref = oracle_eval(p, pos, types, box, weights=w)
+    assert_energy_close(E, ref.energy, len(pos), prec=1)
+    assert_atom_energies_close(Ei, ref.atom_energy, prec=1)
+    assert_forces_close(F, ref.forces, prec=1)
+
+
+def test_bf16_networks_are_deterministic():
+    p, pos, types, box = BF16_CASES["ag500"]()
+    _, E1, F1, _ = gpu_eval(p, pos, types, box, mlp_precision=1)
+    _, E2, F2, _ = gpu_eval(p, pos, types, box, mlp_precision=1)
+    assert E1 == E2 and np.array_equal(F1, F2)
 
 
 def test_repeated_evaluation_is_bit_identical():

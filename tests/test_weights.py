@@ -1,0 +1,47 @@
+"""The stored weight-recipe data: standardisation conditioning, energy scale,
+and determinism of the seeded draws."""
+import numpy as np
+import pytest
+
+from molecular_dynamics_b200 import presets, synth
+
+
+@pytest.mark.parametrize("key", presets.ORDER)
+def test_standardisation_is_well_conditioned(key):
+    p = presets.get(key)
+    shift, scale = synth.load_norm(p)
+    assert shift.shape == (p.stats_depth, p.n_elements, p.D)
+    assert np.all(scale > 0)
+    # the recipe's floor bounds mean / scale by 20 (1 / 0.05)
+    assert np.all(np.abs(shift) / scale <= 20.0 + 1e-3)
+
+
+@pytest.mark.parametrize("key", presets.ORDER)
+def test_energy_scale_present_and_positive(key):
+    lam = synth.load_energy_scale(presets.get(key))
+    assert 0 < lam < 10
+
+
+def test_weight_blob_is_deterministic_and_sized():
+    p = presets.get("hea108k")
+    a, b = synth.weight_blob(p), synth.weight_blob(p)
+    assert a.dtype == np.float32 and np.array_equal(a, b)
+    assert len(a) == synth.blob_layout(p, p.T)["total"]
+
+
+def test_energy_scale_multiplies_only_the_energy_output_layer():
+    p = presets.get("water3k")
+    a = synth.weight_blob(p, energy_scale=1.0)
+    b = synth.weight_blob(p, energy_scale=2.0)
+    lay = synth.blob_layout(p, p.T)
+    diff = np.nonzero(a != b)[0]
+    allowed = set()
+    for net in lay["energy"]:
+        for k in ("W3", "b3"):
+            o, shape = net[k]
+            allowed.update(range(o, o + int(np.prod(shape))))
+    assert set(diff.tolist()) <= allowed
+    for net in lay["energy"]:
+        o, shape = net["W3"]
+        m = int(np.prod(shape))
+        assert np.allclose(b[o:o + m], 2 * a[o:o + m])
