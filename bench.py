@@ -152,6 +152,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=16)
+    ap.add_argument("--ncell", type=int, default=0,
+                    help="FCC workloads: cells per axis (smaller lattices for profiling captures)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -171,6 +173,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
 
     p = presets.get(args.workload)
+    if args.ncell:
+        p = presets.scaled(args.workload, ncell=args.ncell)
     pos, types, box = synth.make_structure(p)
     v0 = synth.maxwell_boltzmann(p, types)
     n = len(pos)

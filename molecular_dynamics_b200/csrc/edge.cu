@@ -16,7 +16,8 @@
 //   dE/dc_k[n,l] = (-1)^l sum_j phi_n(r) sum_{|tau|=l} G_j[n,tau] Y_tau(d),
 // where d = x_j - x_k and G = dE/dA.  Both directed edges k->j and j->k are
 // folded into the row of k because the list is symmetric; the parity (-1)^l
-// comes from Y_tau(-d) = (-1)^l Y_tau(d).
+// comes from Y_tau(-d) = (-1)^l Y_tau(d).  The per-atom active-pair counts
+// of the last evaluation choose the lanes per centre of the backward pass.
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
@@ -176,109 +177,134 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
 }
 
 // ---------------------------------------------------------------------------
-// backward: one thread per centre atom k; G_k and c_k in registers, the
-// neighbour's G_j and c_j gathered per edge.
-template <int NP, bool HAS_DC>
+// backward: a group of W lanes per centre atom k.  G_k and c_k sit in shared
+// memory (read as broadcasts); lane g of the group takes the centre's active
+// neighbours g, g + W, ...; the per-lane force and dE/dc_k partials are summed
+// by a fixed shuffle tree, so the result is deterministic.
+template <int NP, bool HAS_DC, int W>
 __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                   const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
                                                   float *__restrict__ dc, bool accumulate, EdgeParams P) {
-    constexpr int D = 3 * NP, NA = NP * NT;
+    constexpr int D = 3 * NP, NA = NP * NT, GROUPS = 128 / W;
     __shared__ float sC0[MAX_ELEMENTS * D];
+    __shared__ float sG[GROUPS][NA];
+    __shared__ float sc[GROUPS][D];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
+    const int grp = threadIdx.x / W, gl = threadIdx.x % W;
+    const int i = blockIdx.x * GROUPS + grp;
+    const bool live = i < n;
+    float4 pi = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live) {
+        pi = pos[i];
+        for (int k = gl; k < NA; k += W) sG[grp][k] = G[(int64_t)i * NA + k];
+    }
     __syncthreads();
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-
-    float4 pi = pos[i];
-    float Gk[NA], ck[D];
-    {
-        const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)i * NA);
-#pragma unroll
-        for (int k = 0; k < NA / 4; ++k) {
-            float4 v = g4[k];
-            Gk[4 * k] = v.x; Gk[4 * k + 1] = v.y; Gk[4 * k + 2] = v.z; Gk[4 * k + 3] = v.w;
+    if (live) {
+        if (coef) {
+            for (int k = gl; k < D; k += W) sc[grp][k] = coef[(int64_t)i * D + k];
+        } else {
+            const int ti = __float_as_int(pi.w);
+            for (int k = gl; k < D; k += W) sc[grp][k] = sC0[ti * D + k];
         }
     }
-    load_coef<D>(ck, coef, sC0, i, __float_as_int(pi.w));
+    __syncthreads();
+    const float *Gk = sG[grp];
+    const float *ck = sc[grp];
+
     float fx = 0.f, fy = 0.f, fz = 0.f;
     float dck[HAS_DC ? D : 1];
 #pragma unroll
     for (int k = 0; k < (HAS_DC ? D : 1); ++k) dck[k] = 0.f;
 
-    int q0 = row[i], cnt = act_cnt[i];
-    for (int q = q0; q < q0 + cnt; ++q) {
-        int j = act_col[q];
-        float4 pj = pos[j];
-        float3 d = displacement(pi, pj, P);
-        float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
-        float inv_r = 1.0f / r;
+    const int q0 = live ? row[i] : 0, cnt = live ? act_cnt[i] : 0;
+    for (int q = q0 + gl; q < q0 + cnt; q += W) {
+        const int j = act_col[q];
+        const float4 pj = pos[j];
+        const float3 d = displacement(pi, pj, P);
+        const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
+        const float inv_r = 1.0f / r;
         float sn, cs;
         sincospif(r * (1.0f / P.r_cut), &sn, &cs);
-        float fc = 0.5f * (cs + 1.0f);
-        float dfc = -0.5f * P.pi_over_rc * sn;
-        float cj[D];
-        load_coef<D>(cj, coef, sC0, j, __float_as_int(pj.w));
+        const float fc = 0.5f * (cs + 1.0f);
+        const float dfc = -0.5f * P.pi_over_rc * sn;
+        const float *cjp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
         const float xx = d.x * d.x, yy = d.y * d.y, zz = d.z * d.z;
         const float xy = d.x * d.y, xz = d.x * d.z, yz = d.y * d.z;
         const float *Gj = G + (int64_t)j * NA;
 #pragma unroll
         for (int nn = 0; nn < NP; ++nn) {
-            float t = r - (float)nn * P.mu_step;
-            float g = expf(-P.alpha * t * t);
-            float phi = g * fc;
-            float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
+            const float t = r - (float)nn * P.mu_step;
+            const float g = expf(-P.alpha * t * t);
+            const float phi = g * fc;
+            const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
             float gj[NT];
 #pragma unroll
             for (int u = 0; u < NT / 2; ++u) {
-                float2 v = __ldg(reinterpret_cast<const float2 *>(Gj + nn * NT) + u);
-                gj[2 * u] = v.x; gj[2 * u + 1] = v.y;
+                const float2 v = __ldg(reinterpret_cast<const float2 *>(Gj + nn * NT) + u);
+                gj[2 * u] = v.x;
+                gj[2 * u + 1] = v.y;
             }
             const float *gk = &Gk[nn * NT];
-            float c0j = cj[nn], c1j = cj[NP + nn], c2j = cj[2 * NP + nn];
-            float c0k = ck[nn], c1k = ck[NP + nn], c2k = ck[2 * NP + nn];
-            // l = 0 (parity +)
-            float H0 = gk[0] * c0j + gj[0] * c0k;
-            // l = 1 (parity -)
-            float Hx = gk[1] * c1j - gj[1] * c1k;
-            float Hy = gk[2] * c1j - gj[2] * c1k;
-            float Hz = gk[3] * c1j - gj[3] * c1k;
-            // l = 2 (parity +)
-            float Hxx = gk[4] * c2j + gj[4] * c2k;
-            float Hyy = gk[5] * c2j + gj[5] * c2k;
-            float Hzz = gk[6] * c2j + gj[6] * c2k;
-            float Hxy = gk[7] * c2j + gj[7] * c2k;
-            float Hxz = gk[8] * c2j + gj[8] * c2k;
-            float Hyz = gk[9] * c2j + gj[9] * c2k;
-            float Pv = H0 + Hx * d.x + Hy * d.y + Hz * d.z + Hxx * xx + Hyy * yy + Hzz * zz + Hxy * xy + Hxz * xz +
-                       Hyz * yz;
-            float Qx = Hx + 2.f * Hxx * d.x + Hxy * d.y + Hxz * d.z;
-            float Qy = Hy + 2.f * Hyy * d.y + Hxy * d.x + Hyz * d.z;
-            float Qz = Hz + 2.f * Hzz * d.z + Hxz * d.x + Hyz * d.y;
-            float s = dphi * Pv * inv_r;
+            const float c0j = cjp[nn], c1j = cjp[NP + nn], c2j = cjp[2 * NP + nn];
+            const float c0k = ck[nn], c1k = ck[NP + nn], c2k = ck[2 * NP + nn];
+            // l = 0 (parity +), l = 1 (parity -), l = 2 (parity +)
+            const float H0 = gk[0] * c0j + gj[0] * c0k;
+            const float Hx = gk[1] * c1j - gj[1] * c1k;
+            const float Hy = gk[2] * c1j - gj[2] * c1k;
+            const float Hz = gk[3] * c1j - gj[3] * c1k;
+            const float Hxx = gk[4] * c2j + gj[4] * c2k;
+            const float Hyy = gk[5] * c2j + gj[5] * c2k;
+            const float Hzz = gk[6] * c2j + gj[6] * c2k;
+            const float Hxy = gk[7] * c2j + gj[7] * c2k;
+            const float Hxz = gk[8] * c2j + gj[8] * c2k;
+            const float Hyz = gk[9] * c2j + gj[9] * c2k;
+            const float Pv = H0 + Hx * d.x + Hy * d.y + Hz * d.z + Hxx * xx + Hyy * yy + Hzz * zz + Hxy * xy +
+                             Hxz * xz + Hyz * yz;
+            const float Qx = Hx + 2.f * Hxx * d.x + Hxy * d.y + Hxz * d.z;
+            const float Qy = Hy + 2.f * Hyy * d.y + Hxy * d.x + Hyz * d.z;
+            const float Qz = Hz + 2.f * Hzz * d.z + Hxz * d.x + Hyz * d.y;
+            const float s = dphi * Pv * inv_r;
             fx += s * d.x + phi * Qx;
             fy += s * d.y + phi * Qy;
             fz += s * d.z + phi * Qz;
             if (HAS_DC) {
-                float S0 = gj[0];
-                float S1 = gj[1] * d.x + gj[2] * d.y + gj[3] * d.z;
-                float S2 = gj[4] * xx + gj[5] * yy + gj[6] * zz + gj[7] * xy + gj[8] * xz + gj[9] * yz;
+                const float S0 = gj[0];
+                const float S1 = gj[1] * d.x + gj[2] * d.y + gj[3] * d.z;
+                const float S2 = gj[4] * xx + gj[5] * yy + gj[6] * zz + gj[7] * xy + gj[8] * xz + gj[9] * yz;
                 dck[nn] += phi * S0;
                 dck[NP + nn] -= phi * S1;
                 dck[2 * NP + nn] += phi * S2;
             }
         }
     }
-    float *Fo = F + 3 * (int64_t)i;
-    if (accumulate) {
-        fx += Fo[0]; fy += Fo[1]; fz += Fo[2];
-    }
-    Fo[0] = fx; Fo[1] = fy; Fo[2] = fz;
-    if (HAS_DC) {
-        float *o = dc + (int64_t)i * D;
+    // sum over the group's lanes (groups are aligned W-lane segments of a warp)
 #pragma unroll
-        for (int k = 0; k < D / 2; ++k) reinterpret_cast<float2 *>(o)[k] = make_float2(dck[2 * k], dck[2 * k + 1]);
+    for (int o = W / 2; o > 0; o >>= 1) {
+        fx += __shfl_xor_sync(0xffffffffu, fx, o);
+        fy += __shfl_xor_sync(0xffffffffu, fy, o);
+        fz += __shfl_xor_sync(0xffffffffu, fz, o);
+        if (HAS_DC) {
+#pragma unroll
+            for (int k = 0; k < D; ++k) dck[k] += __shfl_xor_sync(0xffffffffu, dck[k], o);
+        }
+    }
+    if (live && gl == 0) {
+        float *Fo = F + 3 * (int64_t)i;
+        if (accumulate) {
+            fx += Fo[0];
+            fy += Fo[1];
+            fz += Fo[2];
+        }
+        Fo[0] = fx;
+        Fo[1] = fy;
+        Fo[2] = fz;
+        if (HAS_DC) {
+            float *o = dc + (int64_t)i * D;
+#pragma unroll
+            for (int k = 0; k < D / 2; ++k) reinterpret_cast<float2 *>(o)[k] = make_float2(dck[2 * k], dck[2 * k + 1]);
+        }
     }
 }
 
@@ -304,24 +330,45 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// lanes per centre: about a third of the mean active degree, 4..16
+static int group_width(const reann_ctx *c) {
+    double deg = c->n > 0 ? (double)c->counters.active_pairs / (double)c->n : 0.0;
+    if (deg <= 0.0) deg = c->n > 0 ? 0.6 * (double)c->nnz / (double)c->n : 0.0;
+    return deg >= 36.0 ? 16 : (deg >= 18.0 ? 8 : 4);
+}
+
+template <int NP, bool DC, int W>
+static void edge_bwd_launch(reann_ctx *c, const float *coef, bool accumulate, const EdgeParams &P, cudaStream_t s) {
+    constexpr int GROUPS = 128 / W;
+    unsigned g = (unsigned)((c->n + GROUPS - 1) / GROUPS);
+    k_edge_bwd<NP, DC, W><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w,
+                                            c->ne, c->d_G, c->d_F, c->d_dc, accumulate, P);
+}
+
+template <int NP, bool DC>
+static void edge_bwd_width(reann_ctx *c, const float *coef, bool accumulate, const EdgeParams &P, cudaStream_t s) {
+    switch (group_width(c)) {
+        case 16: edge_bwd_launch<NP, DC, 16>(c, coef, accumulate, P, s); break;
+        case 8: edge_bwd_launch<NP, DC, 8>(c, coef, accumulate, P, s); break;
+        default: edge_bwd_launch<NP, DC, 4>(c, coef, accumulate, P, s); break;
+    }
+}
+
 cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s) {
     if (c->n == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
-    unsigned g = (unsigned)((c->n + 127) / 128);
-    bool has_dc = t >= 1;
+    const bool has_dc = t >= 1;
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
-#define REANN_EDGE_BWD(NPV, DC)                                                                                   \
-    k_edge_bwd<NPV, DC><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w, \
-                                          c->ne, c->d_G, c->d_F, c->d_dc, accumulate, P)
     if (c->NP == 8) {
-        if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
+        if (has_dc) edge_bwd_width<8, true>(c, coef, accumulate, P, s);
+        else edge_bwd_width<8, false>(c, coef, accumulate, P, s);
     } else if (c->NP == 10) {
-        if (has_dc) REANN_EDGE_BWD(10, true); else REANN_EDGE_BWD(10, false);
+        if (has_dc) edge_bwd_width<10, true>(c, coef, accumulate, P, s);
+        else edge_bwd_width<10, false>(c, coef, accumulate, P, s);
     } else {
         return cudaErrorInvalidValue;
     }
-#undef REANN_EDGE_BWD
     return cudaGetLastError();
 }
 

@@ -1,5 +1,8 @@
 // Per-element atomic networks on the 5th-generation tensor cores (tcgen05),
-// bf16 operands with fp32 accumulation in tensor memory.
+// bf16 operands with fp32 accumulation in tensor memory.  Weights are bf16
+// values; activations and gradients enter each GEMM as a pair of bf16 terms
+// (hi = bf16(v), lo = bf16(v - hi)), two MMA passes into one accumulator, so
+// an operand keeps 16 significant bits.
 //
 // Same networks as mlp.cu ("Efficient Parallelization of Message Passing
 // Neural Network Potentials for Large-Scale Molecular Dynamics", section "REANN
@@ -64,15 +67,27 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 
-// D[128 x N] (+)= A[128 x K] B[N x K]^T, both operands canonical K-major tiles
-template <int N, int K>
-__device__ __forceinline__ void gemm(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-    constexpr uint32_t idesc = idesc_bf16(N);
+// D[128 x N] (+)= (A_hi + A_lo)[128 x K] B^T over two passes (split bf16
+// activations, exact bf16 weights).  B is either a canonical K-major N x K tile
+// (BT = false) or, BT = true, the MN-major view of a stored K-major tile with
+// R_B = K rows and N columns: the same bytes, read transposed.  For that view
+// the 16-byte chunks run along N (stride R_B*16 between chunk groups, the SBO)
+// and 8-row groups run along K (stride 128, the LBO).
+template <int N, int K, bool BT, int RB>
+__device__ __forceinline__ void gemm2(uint32_t d_tmem, uint32_t a_hi, uint32_t a_lo, uint32_t b_smem) {
+    constexpr uint32_t idesc = idesc_bf16(N) | (BT ? (1u << 16) : 0u);
+    uint32_t acc = 0;
 #pragma unroll
-    for (int s = 0; s < K / 16; ++s) {
-        uint64_t a = sdesc(a_smem + (uint32_t)(2 * s * TM * 16), TM * 16, 128);
-        uint64_t b = sdesc(b_smem + (uint32_t)(2 * s * N * 16), N * 16, 128);
-        mma_bf16(d_tmem, a, b, idesc, s > 0 ? 1u : 0u);
+    for (int pass = 0; pass < 2; ++pass) {
+        const uint32_t a_smem = pass == 0 ? a_hi : a_lo;
+#pragma unroll
+        for (int s = 0; s < K / 16; ++s) {
+            uint64_t a = sdesc(a_smem + (uint32_t)(2 * s * TM * 16), TM * 16, 128);
+            uint64_t b = BT ? sdesc(b_smem + (uint32_t)(256 * s), 128, RB * 16)
+                            : sdesc(b_smem + (uint32_t)(2 * s * N * 16), N * 16, 128);
+            mma_bf16(d_tmem, a, b, idesc, acc);
+            acc = 1;
+        }
     }
 }
 
@@ -134,15 +149,16 @@ __device__ __forceinline__ void st_chunk(unsigned char *tile, int R, int r, int 
     *reinterpret_cast<uint4 *>(tile + kmaj(r, c, R)) = w;
 }
 
-__device__ __forceinline__ void ld_chunk(const unsigned char *tile, int R, int r, int c, float *v) {
-    uint4 w = *reinterpret_cast<const uint4 *>(tile + kmaj(r, c, R));
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w);
+// 8 values as a bf16 pair: hi = bf16(v), lo = bf16(v - hi) (16 significant bits)
+__device__ __forceinline__ void st_chunk2(unsigned char *hi, unsigned char *lo, int R, int r, int c, const float *v) {
+    float h[8], l[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        float2 f = __bfloat1622float2(h[k]);
-        v[2 * k] = f.x;
-        v[2 * k + 1] = f.y;
+    for (int u = 0; u < 8; ++u) {
+        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
+        l[u] = v[u] - h[u];
     }
+    st_chunk(hi, R, r, c, h);
+    st_chunk(lo, R, r, c, l);
 }
 
 // one bf16 element of a K-major tile (weight preparation)
@@ -158,23 +174,22 @@ template <int NP, int H1, int H2, int MODE>
 struct TcLayout {
     static constexpr int D = 3 * NP;
     static constexpr int NA = NP * NT;
-    // bf16 operand tiles (bytes)
-    static constexpr int W1 = 0;                                        // [H1][KPAD]  B of layer 1
-    static constexpr int W2 = W1 + H1 * KPAD * 2;                       // [H2][H1]    B of layer 2
-    static constexpr int W3 = W2 + H2 * H1 * 2;                         // [KPAD][H2]  B of layer 3 (FWD)
-    static constexpr int W2T = W3 + (MODE == TC_FWD ? KPAD * H2 * 2 : 0);   // [H1][H2]  B of dE/da1
-    static constexpr int W3T = W2T + (MODE != TC_FWD ? H1 * H2 * 2 : 0);    // [H2][KPAD] B of dE/da2 (BWD)
-    static constexpr int W1T = W3T + (MODE == TC_BWD ? H2 * KPAD * 2 : 0);  // [KPAD][H1] B of dE/dx
-    static constexpr int X = W1T + (MODE != TC_FWD ? KPAD * H1 * 2 : 0);    // [TM][KPAD] standardised input
-    static constexpr int DY = X + TM * KPAD * 2;                        // [TM][KPAD] upstream gradient (BWD)
-    static constexpr int A1 = DY + (MODE == TC_BWD ? TM * KPAD * 2 : 0);    // [TM][H1]
-    static constexpr int A2 = A1 + TM * H1 * 2;                         // [TM][H2] (FWD: a2; else g2, then g1)
-    static constexpr int F32 = A2 + TM * (H1 > H2 ? H1 : H2) * 2;       // fp32 vectors
-    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2;         // b1, b2, b3, shift, scale, inv_scale, w3
+    // bf16 weight tiles, K-major, one copy each (the backward products read
+    // them through the MN-major view)
+    static constexpr int W1 = 0;                                 // [H1][KPAD]
+    static constexpr int W2 = W1 + H1 * KPAD * 2;                // [H2][H1]
+    static constexpr int W3 = W2 + H2 * H1 * 2;                  // [KPAD][H2] (rows >= n_out are zero)
+    // split activation tiles (hi, lo)
+    static constexpr int X = W3 + KPAD * H2 * 2;                 // [TM][KPAD] x 2
+    static constexpr int DY = X + 2 * TM * KPAD * 2;             // [TM][KPAD] x 2 (BWD)
+    static constexpr int A1 = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][H1] x 2
+    static constexpr int A2 = A1 + 2 * TM * H1 * 2;              // [TM][H2] x 2
+    static constexpr int F32 = A2 + 2 * TM * H2 * 2;
+    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2;  // b1, b2, b3, shift, scale, 1/scale, w3
     static constexpr int BAR = F32 + nf32 * 4;
     static constexpr int bytes = BAR + 16 + 16;
     // TMEM columns
-    static constexpr int C_Z1 = 0, C_Z2 = 128, C_P2 = 256, C_OUT = 384;
+    static constexpr int C_Z1 = 0, C_Z2 = 128, C_P = 256, C_OUT = 384;
 };
 
 template <int NP, int H1, int H2, int MODE>
@@ -191,10 +206,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           *sinv = sscale + KPAD, *sw3 = sinv + KPAD;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
+    unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KPAD * 2;
+    unsigned char *dy_hi = sm + L::DY, *dy_lo = dy_hi + TM * KPAD * 2;
+    unsigned char *a1_hi = sm + L::A1, *a1_lo = a1_hi + TM * H1 * 2;
+    unsigned char *a2_hi = sm + L::A2, *a2_lo = a2_hi + TM * H2 * 2;
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid;                       // this thread's atom within the tile (TMEM lane)
     const uint32_t base = smem_u32(sm);
+    auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -214,47 +234,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool failed = false;
     int cur = -1;
 
-    // one MMA group issued by thread 0, completion awaited by all threads
+    // completion of the MMA group thread 0 committed, awaited by all threads
     auto wait_mma = [&]() -> bool {
         bool ok = bar_wait(bar, phase);
         phase ^= 1u;
         fence_after();
         return !__syncthreads_or(!ok);
     };
+    // operand stores (generic proxy) and TMEM reads done -> next MMA may start
+    auto handoff = [&]() {
+        fence_smem_to_async();
+        fence_before();
+        __syncthreads();
+    };
 
     for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
         const int4 tile = tiles[ti];
         const int e = tile.x, r0 = tile.y, rows = tile.z;
         if (e != cur) {
-            // element weights -> bf16 operand tiles and fp32 vectors
+            // element weights -> bf16 tiles and fp32 vectors
             const NetOffsets &o = nets.net[e];
             for (int k = tid; k < H1 * KPAD; k += TC_THREADS) {
                 int n = k / KPAD, f = k % KPAD;
                 st_elem(sm + L::W1, H1, n, f, f < D ? w[o.W1 + (int64_t)n * D + f] : 0.f);
             }
-            for (int k = tid; k < H2 * H1; k += TC_THREADS) {
-                int n = k / H1, h = k % H1;
-                float v = w[o.W2 + k];
-                st_elem(sm + L::W2, H2, n, h, v);
-                if (MODE != TC_FWD) st_elem(sm + L::W2T, H1, h, n, v);
-            }
-            if (MODE == TC_FWD) {
-                for (int k = tid; k < KPAD * H2; k += TC_THREADS) {
-                    int n = k / H2, h = k % H2;
-                    st_elem(sm + L::W3, KPAD, n, h, n < DOUT ? w[o.W3 + (int64_t)n * H2 + h] : 0.f);
-                }
-            }
-            if (MODE == TC_BWD) {
-                for (int k = tid; k < H2 * KPAD; k += TC_THREADS) {
-                    int h = k / KPAD, j = k % KPAD;
-                    st_elem(sm + L::W3T, H2, h, j, j < DOUT ? w[o.W3 + (int64_t)j * H2 + h] : 0.f);
-                }
-            }
-            if (MODE != TC_FWD) {
-                for (int k = tid; k < KPAD * H1; k += TC_THREADS) {
-                    int f = k / H1, h = k % H1;
-                    st_elem(sm + L::W1T, KPAD, f, h, f < D ? w[o.W1 + (int64_t)h * D + f] : 0.f);
-                }
+            for (int k = tid; k < H2 * H1; k += TC_THREADS) st_elem(sm + L::W2, H2, k / H1, k % H1, w[o.W2 + k]);
+            for (int k = tid; k < KPAD * H2; k += TC_THREADS) {
+                int n = k / H2, h = k % H2;
+                st_elem(sm + L::W3, KPAD, n, h, n < DOUT ? w[o.W3 + (int64_t)n * H2 + h] : 0.f);
             }
             for (int k = tid; k < H1; k += TC_THREADS) sb1[k] = w[o.b1 + k];
             for (int k = tid; k < H2; k += TC_THREADS) {
@@ -270,7 +277,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             cur = e;
         }
         __syncthreads();
-        // input tile: standardised rho (and the upstream gradient) as bf16
+        // input tile: standardised rho (and the upstream gradient), split bf16
         {
             const bool live = row < rows;
             const int64_t gi = (int64_t)(r0 + row);
@@ -279,28 +286,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 float v[8], g[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    int f = c + u;
-                    float x = (live && f < D) ? X[gi * D + f] : 0.f;
-                    v[u] = f < D ? (x - sshift[f]) / sscale[f] : 0.f;
-                    if (!live) v[u] = 0.f;
-                    if (MODE == TC_BWD) g[u] = (live && f < D) ? dY[gi * D + f] : 0.f;
+                    const int f = c + u;
+                    const bool ok = live && f < D;
+                    v[u] = ok ? (X[gi * D + f] - sshift[f]) / sscale[f] : 0.f;
+                    g[u] = (MODE == TC_BWD && ok) ? dY[gi * D + f] : 0.f;
                 }
-                st_chunk(sm + L::X, TM, row, c, v);
-                if (MODE == TC_BWD) st_chunk(sm + L::DY, TM, row, c, g);
+                st_chunk2(x_hi, x_lo, TM, row, c, v);
+                if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, c, g);
             }
         }
-        fence_smem_to_async();
-        __syncthreads();
+        handoff();
 
-        // layer 1 (and, for the backward network, dE/da2 = dY W3)
+        // layer 1 (and, for the coefficient backward, dE/da2 = dY W3 via the MN-major view of W3)
         if (tid == 0) {
             fence_after();
-            gemm<H1, KPAD>(tmem + L::C_Z1, base + L::X, base + L::W1);
-            if (MODE == TC_BWD) gemm<H2, KPAD>(tmem + L::C_P2, base + L::DY, base + L::W3T);
+            gemm2<H1, KPAD, false, 0>(tmem + L::C_Z1, sa(x_hi), sa(x_lo), base + L::W1);
+            if (MODE == TC_BWD) gemm2<H2, KPAD, true, KPAD>(tmem + L::C_P, sa(dy_hi), sa(dy_lo), base + L::W3);
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
-        // a1 = tanh(z1 + b1) -> A1
+        // a1 = tanh(z1 + b1)
 #pragma unroll 1
         for (int c = 0; c < H1; c += 32) {
             float v[32];
@@ -308,20 +313,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb1[c + u]);
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A1, TM, row, c + u, &v[u]);
+            for (int u = 0; u < 32; u += 8) st_chunk2(a1_hi, a1_lo, TM, row, c + u, &v[u]);
         }
-        fence_smem_to_async();
-        fence_before();
-        __syncthreads();
+        handoff();
         if (tid == 0) {
             fence_after();
-            gemm<H2, H1>(tmem + L::C_Z2, base + L::A1, base + L::W2);
+            gemm2<H2, H1, false, 0>(tmem + L::C_Z2, sa(a1_hi), sa(a1_lo), base + L::W2);
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
 
         if (MODE == TC_FWD) {
-            // a2 = tanh(z2 + b2) -> A2, then y = a2 W3^T + b3
+            // a2 = tanh(z2 + b2), then y = a2 W3^T + b3
 #pragma unroll 1
             for (int c = 0; c < H2; c += 32) {
                 float v[32];
@@ -329,14 +332,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb2[c + u]);
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A2, TM, row, c + u, &v[u]);
+                for (int u = 0; u < 32; u += 8) st_chunk2(a2_hi, a2_lo, TM, row, c + u, &v[u]);
             }
-            fence_smem_to_async();
-            fence_before();
-            __syncthreads();
+            handoff();
             if (tid == 0) {
                 fence_after();
-                gemm<KPAD, H2>(tmem + L::C_OUT, base + L::A2, base + L::W3);
+                gemm2<KPAD, H2, false, 0>(tmem + L::C_OUT, sa(a2_hi), sa(a2_lo), base + L::W3);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
@@ -348,53 +349,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int f = 0; f < D; ++f) yo[f] = v[f] + sb3[f];
             }
         } else {
-            // g2 = dE/dz2: energy network dE_i/da2 = w3; backward network dY W3 (TMEM)
+            // g2 = dE/dz2 = (energy: w3, backward: dY W3) * (1 - a2^2); energy E_i = w3 . a2 + b3
             float e_row = 0.f;
 #pragma unroll 1
             for (int c = 0; c < H2; c += 32) {
-                float z[32], p[32];
+                float z[32], up[32];
                 tmem_ld32(lane_base + L::C_Z2 + c, z);
-                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P2 + c, p);
+                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P + c, up);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                    float a = tanh_fast(z[u] + sb2[c + u]);
-                    float up = MODE == TC_ENERGY ? sw3[c + u] : p[u];
+                    const float a = tanh_fast(z[u] + sb2[c + u]);
+                    const float g = MODE == TC_ENERGY ? sw3[c + u] : up[u];
                     if (MODE == TC_ENERGY) e_row = fmaf(sw3[c + u], a, e_row);
-                    z[u] = up * (1.f - a * a);
+                    z[u] = g * (1.f - a * a);
                 }
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) st_chunk(sm + L::A2, TM, row, c + u, &z[u]);
+                for (int u = 0; u < 32; u += 8) st_chunk2(a2_hi, a2_lo, TM, row, c + u, &z[u]);
             }
             if (MODE == TC_ENERGY && row < rows) Ei[r0 + row] = e_row + sb3[0];
-            fence_smem_to_async();
-            fence_before();
-            __syncthreads();
+            handoff();
+            // p1 = g2 W2 (MN-major view of W2), into the columns dY W3 used
             if (tid == 0) {
                 fence_after();
-                gemm<H1, H2>(tmem + L::C_Z1, base + L::A2, base + L::W2T);
+                gemm2<H1, H2, true, H2>(tmem + L::C_P, sa(a2_hi), sa(a2_lo), base + L::W2);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            // g1 = (g2 W2) (1 - a1^2) -> over the g2 tile (its MMA has completed)
+            // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation still in TMEM
 #pragma unroll 1
             for (int c = 0; c < H1; c += 32) {
-                float v[32];
-                tmem_ld32(lane_base + L::C_Z1 + c, v);
+                float p[32], z[32];
+                tmem_ld32(lane_base + L::C_P + c, p);
+                tmem_ld32(lane_base + L::C_Z1 + c, z);
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) {
-                    float a[8];
-                    ld_chunk(sm + L::A1, TM, row, c + u, a);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) v[u + q] *= 1.f - a[q] * a[q];
-                    st_chunk(sm + L::A2, TM, row, c + u, &v[u]);
+                for (int u = 0; u < 32; ++u) {
+                    const float a = tanh_fast(z[u] + sb1[c + u]);
+                    p[u] *= 1.f - a * a;
                 }
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk2(a1_hi, a1_lo, TM, row, c + u, &p[u]);
             }
-            fence_smem_to_async();
-            fence_before();
-            __syncthreads();
+            handoff();
+            // dE/dx = g1 W1 (MN-major view of W1)
             if (tid == 0) {
                 fence_after();
-                gemm<KPAD, H1>(tmem + L::C_OUT, base + L::A2, base + L::W1T);
+                gemm2<KPAD, H1, true, H1>(tmem + L::C_OUT, sa(a1_hi), sa(a1_lo), base + L::W1);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
@@ -409,8 +408,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 float4 *g4 = reinterpret_cast<float4 *>(Gout + gi);
 #pragma unroll
                 for (int q = 0; q < NA / 4; ++q) {
-                    float4 a = a4[q];
-                    float av[4] = {a.x, a.y, a.z, a.w}, gv[4];
+                    const float4 a = a4[q];
+                    const float av[4] = {a.x, a.y, a.z, a.w};
+                    float gv[4];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
                         const int k = 4 * q + s, nn = k / NT, u = k % NT;

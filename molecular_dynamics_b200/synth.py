@@ -24,13 +24,15 @@ Readings of unstated recipe details:
   * Maxwell-Boltzmann velocities: Gaussian per component with variance
     kT/m, centre-of-mass velocity removed, rescaled to exactly the target
     temperature with 3N-3 degrees of freedom;
+  * workloads with bf16 networks store their matrices as bf16 values;
   * weights: Xavier-uniform matrices, U(-0.1, 0.1) biases, U(-1, 1) initial
     element coefficients c^0, and a per-feature input standardisation
     (shift = mean, scale = std + 0.05 mean|.|, so that mean/scale <= 20) in
     front of every atomic network; the energy
     network's output layer is multiplied by an energy scale that gives
     forces of RMS 1 eV/A.  Shift, scale and energy scale are measured once
-    on each workload's own structure and stored in
+    on each workload's own structure (FCC lattices: with five times the
+    thermal displacement, a training-set-like spread) and stored in
     molecular_dynamics_b200/data/norm_<workload>.json.
 
 Positions are returned as float32 values wrapped into [0, L): both the GPU
@@ -228,6 +230,13 @@ _KIND = {"W1": 1, "b1": 2, "W2": 3, "b2": 4, "W3": 5, "b3": 6}
 ENERGY_LAYER = 100
 
 
+def to_bf16_values(a) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), returned as float32."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
 def _xavier(rng, fan_out, fan_in):
     b = np.sqrt(6.0 / (fan_in + fan_out))
     return rng.uniform(-b, b, size=(fan_out, fan_in))
@@ -329,6 +338,11 @@ def weight_blob(p: Preset, T: Optional[int] = None, norm=None, use_stored_norm: 
         if layer == ENERGY_LAYER:
             raw["W3"] = raw["W3"] * energy_scale
             raw["b3"] = raw["b3"] * energy_scale
+        if p.mlp_precision == 1:
+            # bf16 networks: the matrices are stored as bf16 values, as bf16
+            # inference stores them (biases and standardisation stay fp32)
+            for k in ("W1", "W2", "W3"):
+                raw[k] = to_bf16_values(raw[k])
         if norm is not None and t_in < norm[0].shape[0]:
             put(net["shift"], norm[0][t_in, e])
             put(net["scale"], norm[1][t_in, e])
