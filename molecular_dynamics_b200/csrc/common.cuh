@@ -41,6 +41,21 @@ struct NetOffsets {
     int n_out;
 };
 
+// Lane decomposition of the edge kernels: a slot of LPE = N_phi / 2 lanes
+// works on one edge, lane `sub` of the slot owning radial indices 2 sub and
+// 2 sub + 1.  dE/dA rows (G) are stored lane-interleaved so that a slot's
+// loads of one neighbour's row are contiguous: the 20 values of lane `sub`
+// (index m*10 + tau for its radial index 2 sub + m) sit at
+//   p = (idx / 4) * 4 LPE + 4 sub + idx % 4.
+__host__ __device__ constexpr int g_slot_index(int n, int tau, int NP) {
+    return ((((n % 2) * NT + tau) / 4) * 4 * (NP / 2)) + 4 * (n / 2) + (((n % 2) * NT + tau) % 4);
+}
+// inverse: the (radial index, tuple) stored at position p
+__host__ __device__ constexpr int g_slot_source(int p, int NP) {
+    return (2 * ((p % (4 * (NP / 2))) / 4) + ((p / (4 * (NP / 2))) * 4 + p % 4) / NT) * NT +
+           ((p / (4 * (NP / 2))) * 4 + p % 4) % NT;
+}
+
 struct Ctx;
 
 // --- host orchestration helpers (defined across the .cu files) -------------

@@ -16,8 +16,7 @@
 //   dE/dc_k[n,l] = (-1)^l sum_j phi_n(r) sum_{|tau|=l} G_j[n,tau] Y_tau(d),
 // where d = x_j - x_k and G = dE/dA.  Both directed edges k->j and j->k are
 // folded into the row of k because the list is symmetric; the parity (-1)^l
-// comes from Y_tau(-d) = (-1)^l Y_tau(d).  The per-atom active-pair counts
-// of the last evaluation choose the lanes per centre of the backward pass.
+// comes from Y_tau(-d) = (-1)^l Y_tau(d).
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
@@ -90,207 +89,245 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// loads of one atom's D coefficients (layer 0: the element table in shared
-// memory; later layers: the message vector written by the coefficient network)
+// Lane decomposition shared by both edge passes: one warp per centre atom,
+// EPW = 32 / LPE edge slots of LPE = N_phi / 2 lanes; lane `sub` of a slot
+// owns radial indices 2 sub and 2 sub + 1.  A slot's lanes read one
+// neighbour's coefficients and dE/dA row as contiguous runs, and each lane
+// keeps only its own radial indices' accumulators.
+template <int NP>
+struct Lanes {
+    static constexpr int LPE = NP / 2;
+    static constexpr int EPW = 32 / LPE;
+    static constexpr int USED = EPW * LPE;
+};
 
-template <int D>
-__device__ __forceinline__ void load_coef(float (&c)[D], const float *__restrict__ coef, const float *sC0, int j,
-                                          int type_j) {
-    if (coef) {
-        const float *p = coef + (int64_t)j * D;
-        if (D % 4 == 0) {
-#pragma unroll
-            for (int k = 0; k < D / 4; ++k) {
-                float4 v = __ldg(reinterpret_cast<const float4 *>(p) + k);
-                c[4 * k] = v.x; c[4 * k + 1] = v.y; c[4 * k + 2] = v.z; c[4 * k + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < D / 2; ++k) {
-                float2 v = __ldg(reinterpret_cast<const float2 *>(p) + k);
-                c[2 * k] = v.x; c[2 * k + 1] = v.y;
-            }
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < D; ++k) c[k] = sC0[type_j * D + k];
-    }
-}
-
-// ---------------------------------------------------------------------------
-// forward: one thread per centre atom, A^t accumulated in registers over the
-// centre's active neighbours in row order (deterministic), then rho^t.
+// forward: A^t for the lane's two radial indices accumulated in fp64 (the
+// odd-l components are small residuals of cancelling neighbour sums), products
+// c phi formed exactly in fp64, monomials from the fp64 displacement; slots
+// summed in a fixed order through shared memory; rho^t in fp64, stored fp32.
 template <int NP>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
                                                      EdgeParams P) {
-    constexpr int D = 3 * NP, NA = NP * NT;
-    __shared__ float sC0[MAX_ELEMENTS * D];
+    using Ln = Lanes<NP>;
+    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE, EPW = Ln::EPW;
+    __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
+    __shared__ double sred[4][EPW][LPE][2 * NT];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
     __syncthreads();
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 4 + warp;
+    const int slot = lane / LPE, sub = lane % LPE;
+    const bool active_lane = lane < Ln::USED && i < n;
+    const int n0 = 2 * sub;
 
-    float acc[NA];
+    double acc[2][NT];
 #pragma unroll
-    for (int k = 0; k < NA; ++k) acc[k] = 0.f;
-    float4 pi = pos[i];
-    int q0 = row[i], cnt = act_cnt[i];
-    for (int q = q0; q < q0 + cnt; ++q) {
-        int j = act_col[q];
-        float4 pj = pos[j];
-        float3 d = displacement(pi, pj, P);
-        float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
-        float fc = 0.5f * (cospif(r * (1.0f / P.r_cut) ) + 1.0f);
-        float c[D];
-        load_coef<D>(c, coef, sC0, j, __float_as_int(pj.w));
-        const float Y[NT] = {1.f, d.x, d.y, d.z, d.x * d.x, d.y * d.y, d.z * d.z, d.x * d.y, d.x * d.z, d.y * d.z};
+    for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int nn = 0; nn < NP; ++nn) {
-            float t = r - (float)nn * P.mu_step;
-            float phi = expf(-P.alpha * t * t) * fc;
-            float a0 = c[nn] * phi, a1 = c[NP + nn] * phi, a2 = c[2 * NP + nn] * phi;
-            acc[nn * NT + 0] += a0;
+        for (int u = 0; u < NT; ++u) acc[m][u] = 0.0;
+    if (active_lane) {
+        const float4 pi = pos[i];
+        const int q0 = row[i], cnt = act_cnt[i];
+        for (int q = q0 + slot; q < q0 + cnt; q += EPW) {
+            const int j = act_col[q];
+            const float4 pj = pos[j];
+            double dx = (double)pj.x - (double)pi.x, dy = (double)pj.y - (double)pi.y,
+                   dz = (double)pj.z - (double)pi.z;
+            dx -= P.box[0] * rint(dx * P.inv_box[0]);
+            dy -= P.box[1] * rint(dy * P.inv_box[1]);
+            dz -= P.box[2] * rint(dz * P.inv_box[2]);
+            const float r = (float)sqrt(dx * dx + dy * dy + dz * dz);
+            const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
+            const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
+            float c[3][2];
 #pragma unroll
-            for (int u = 1; u < 4; ++u) acc[nn * NT + u] += a1 * Y[u];
+            for (int l = 0; l < 3; ++l) {
+                const float2 v = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
+                c[l][0] = v.x;
+                c[l][1] = v.y;
+            }
+            const double Y[NT] = {1.0, dx, dy, dz, dx * dx, dy * dy, dz * dz, dx * dy, dx * dz, dy * dz};
 #pragma unroll
-            for (int u = 4; u < NT; ++u) acc[nn * NT + u] += a2 * Y[u];
+            for (int m = 0; m < 2; ++m) {
+                const float t = r - (float)(n0 + m) * P.mu_step;
+                const double phi = (double)(expf(-P.alpha * t * t) * fc);
+                const double a0 = (double)c[0][m] * phi, a1 = (double)c[1][m] * phi, a2 = (double)c[2][m] * phi;
+                acc[m][0] += a0;
+#pragma unroll
+                for (int u = 1; u < 4; ++u) acc[m][u] = fma(a1, Y[u], acc[m][u]);
+#pragma unroll
+                for (int u = 4; u < NT; ++u) acc[m][u] = fma(a2, Y[u], acc[m][u]);
+            }
         }
     }
-    float *Ao = A_out + (int64_t)i * NA;
+    if (lane < Ln::USED) {
 #pragma unroll
-    for (int k = 0; k < NA / 4; ++k)
-        reinterpret_cast<float4 *>(Ao)[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
-    float rho[D];
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int nn = 0; nn < NP; ++nn) {
-        const float *a = &acc[nn * NT];
-        rho[nn] = a[0] * a[0];
-        rho[NP + nn] = a[1] * a[1] + a[2] * a[2] + a[3] * a[3];
-        rho[2 * NP + nn] = a[4] * a[4] + a[5] * a[5] + a[6] * a[6] + 2.f * (a[7] * a[7] + a[8] * a[8] + a[9] * a[9]);
+            for (int u = 0; u < NT; ++u) sred[warp][slot][sub][m * NT + u] = acc[m][u];
     }
-    float *ro = rho_out + (int64_t)i * D;
+    __syncwarp();
+    if (i < n && lane < LPE) {
+        // lane == sub here: sum the slots in order, then this lane's two radial indices
+        double a[2][NT];
 #pragma unroll
-    for (int k = 0; k < D / 2; ++k) reinterpret_cast<float2 *>(ro)[k] = make_float2(rho[2 * k], rho[2 * k + 1]);
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int u = 0; u < NT; ++u) {
+                double v = 0.0;
+#pragma unroll
+                for (int s2 = 0; s2 < EPW; ++s2) v += sred[warp][s2][lane][m * NT + u];
+                a[m][u] = v;
+            }
+        float *Ao = A_out + (int64_t)i * NA;
+        float *ro = rho_out + (int64_t)i * D;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int nn = n0 + m;
+#pragma unroll
+            for (int u = 0; u < NT; u += 2)
+                *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2((float)a[m][u], (float)a[m][u + 1]);
+            const double *v = a[m];
+            ro[nn] = (float)(v[0] * v[0]);
+            ro[NP + nn] = (float)(v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+            ro[2 * NP + nn] = (float)(v[4] * v[4] + v[5] * v[5] + v[6] * v[6] +
+                                      2.0 * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]));
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
-// backward: a group of W lanes per centre atom k.  G_k and c_k sit in shared
-// memory (read as broadcasts); lane g of the group takes the centre's active
-// neighbours g, g + W, ...; the per-lane force and dE/dc_k partials are summed
-// by a fixed shuffle tree, so the result is deterministic.
-template <int NP, bool HAS_DC, int W>
+// backward: one warp per centre atom k, the same slots and lanes as the
+// forward.  Lane `sub` keeps G_k and c_k of its two radial indices in
+// registers and reads the neighbour's 20 interleaved dE/dA values as five
+// contiguous float4 per slot.  Force partials are summed over the warp by a
+// shuffle tree, dE/dc_k partials over the slots in order through shared memory.
+template <int NP, bool HAS_DC>
 __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                   const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
                                                   float *__restrict__ dc, bool accumulate, EdgeParams P) {
-    constexpr int D = 3 * NP, NA = NP * NT, GROUPS = 128 / W;
-    __shared__ float sC0[MAX_ELEMENTS * D];
-    __shared__ float sG[GROUPS][NA];
-    __shared__ float sc[GROUPS][D];
+    using Ln = Lanes<NP>;
+    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE, EPW = Ln::EPW;
+    __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
+    __shared__ float sred[4][EPW][LPE][6];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
-    const int grp = threadIdx.x / W, gl = threadIdx.x % W;
-    const int i = blockIdx.x * GROUPS + grp;
-    const bool live = i < n;
-    float4 pi = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (live) {
-        pi = pos[i];
-        for (int k = gl; k < NA; k += W) sG[grp][k] = G[(int64_t)i * NA + k];
-    }
     __syncthreads();
-    if (live) {
-        if (coef) {
-            for (int k = gl; k < D; k += W) sc[grp][k] = coef[(int64_t)i * D + k];
-        } else {
-            const int ti = __float_as_int(pi.w);
-            for (int k = gl; k < D; k += W) sc[grp][k] = sC0[ti * D + k];
-        }
-    }
-    __syncthreads();
-    const float *Gk = sG[grp];
-    const float *ck = sc[grp];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 4 + warp;
+    const int slot = lane / LPE, sub = lane % LPE;
+    const bool active_lane = lane < Ln::USED && i < n;
+    const int n0 = 2 * sub;
 
     float fx = 0.f, fy = 0.f, fz = 0.f;
-    float dck[HAS_DC ? D : 1];
+    float dck[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+    if (active_lane) {
+        const float4 pi = pos[i];
+        float gk[2 * NT], ck[3][2];
+        {
+            const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)i * NA);
 #pragma unroll
-    for (int k = 0; k < (HAS_DC ? D : 1); ++k) dck[k] = 0.f;
-
-    const int q0 = live ? row[i] : 0, cnt = live ? act_cnt[i] : 0;
-    for (int q = q0 + gl; q < q0 + cnt; q += W) {
-        const int j = act_col[q];
-        const float4 pj = pos[j];
-        const float3 d = displacement(pi, pj, P);
-        const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
-        const float inv_r = 1.0f / r;
-        float sn, cs;
-        sincospif(r * (1.0f / P.r_cut), &sn, &cs);
-        const float fc = 0.5f * (cs + 1.0f);
-        const float dfc = -0.5f * P.pi_over_rc * sn;
-        const float *cjp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
-        const float xx = d.x * d.x, yy = d.y * d.y, zz = d.z * d.z;
-        const float xy = d.x * d.y, xz = d.x * d.z, yz = d.y * d.z;
-        const float *Gj = G + (int64_t)j * NA;
-#pragma unroll
-        for (int nn = 0; nn < NP; ++nn) {
-            const float t = r - (float)nn * P.mu_step;
-            const float g = expf(-P.alpha * t * t);
-            const float phi = g * fc;
-            const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
-            float gj[NT];
-#pragma unroll
-            for (int u = 0; u < NT / 2; ++u) {
-                const float2 v = __ldg(reinterpret_cast<const float2 *>(Gj + nn * NT) + u);
-                gj[2 * u] = v.x;
-                gj[2 * u + 1] = v.y;
+            for (int q = 0; q < 5; ++q) {
+                const float4 v = g4[q * LPE + sub];
+                gk[4 * q] = v.x; gk[4 * q + 1] = v.y; gk[4 * q + 2] = v.z; gk[4 * q + 3] = v.w;
             }
-            const float *gk = &Gk[nn * NT];
-            const float c0j = cjp[nn], c1j = cjp[NP + nn], c2j = cjp[2 * NP + nn];
-            const float c0k = ck[nn], c1k = ck[NP + nn], c2k = ck[2 * NP + nn];
-            // l = 0 (parity +), l = 1 (parity -), l = 2 (parity +)
-            const float H0 = gk[0] * c0j + gj[0] * c0k;
-            const float Hx = gk[1] * c1j - gj[1] * c1k;
-            const float Hy = gk[2] * c1j - gj[2] * c1k;
-            const float Hz = gk[3] * c1j - gj[3] * c1k;
-            const float Hxx = gk[4] * c2j + gj[4] * c2k;
-            const float Hyy = gk[5] * c2j + gj[5] * c2k;
-            const float Hzz = gk[6] * c2j + gj[6] * c2k;
-            const float Hxy = gk[7] * c2j + gj[7] * c2k;
-            const float Hxz = gk[8] * c2j + gj[8] * c2k;
-            const float Hyz = gk[9] * c2j + gj[9] * c2k;
-            const float Pv = H0 + Hx * d.x + Hy * d.y + Hz * d.z + Hxx * xx + Hyy * yy + Hzz * zz + Hxy * xy +
-                             Hxz * xz + Hyz * yz;
-            const float Qx = Hx + 2.f * Hxx * d.x + Hxy * d.y + Hxz * d.z;
-            const float Qy = Hy + 2.f * Hyy * d.y + Hxy * d.x + Hyz * d.z;
-            const float Qz = Hz + 2.f * Hzz * d.z + Hxz * d.x + Hyz * d.y;
-            const float s = dphi * Pv * inv_r;
-            fx += s * d.x + phi * Qx;
-            fy += s * d.y + phi * Qy;
-            fz += s * d.z + phi * Qz;
-            if (HAS_DC) {
-                const float S0 = gj[0];
-                const float S1 = gj[1] * d.x + gj[2] * d.y + gj[3] * d.z;
-                const float S2 = gj[4] * xx + gj[5] * yy + gj[6] * zz + gj[7] * xy + gj[8] * xz + gj[9] * yz;
-                dck[nn] += phi * S0;
-                dck[NP + nn] -= phi * S1;
-                dck[2 * NP + nn] += phi * S2;
+            const float *cp = coef ? coef + (int64_t)i * D : sC0 + __float_as_int(pi.w) * D;
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                const float2 v = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+                ck[l][0] = v.x;
+                ck[l][1] = v.y;
+            }
+        }
+        const int q0 = row[i], cnt = act_cnt[i];
+        for (int q = q0 + slot; q < q0 + cnt; q += EPW) {
+            const int j = act_col[q];
+            const float4 pj = pos[j];
+            const float3 d = displacement(pi, pj, P);
+            const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
+            const float inv_r = 1.0f / r;
+            float sn, cs;
+            sincospif(r * (1.0f / P.r_cut), &sn, &cs);
+            const float fc = 0.5f * (cs + 1.0f);
+            const float dfc = -0.5f * P.pi_over_rc * sn;
+            float gj[2 * NT], cj[3][2];
+            {
+                const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)j * NA);
+#pragma unroll
+                for (int q2 = 0; q2 < 5; ++q2) {
+                    const float4 v = __ldg(g4 + q2 * LPE + sub);
+                    gj[4 * q2] = v.x; gj[4 * q2 + 1] = v.y; gj[4 * q2 + 2] = v.z; gj[4 * q2 + 3] = v.w;
+                }
+                const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                    const float2 v = coef ? __ldg(reinterpret_cast<const float2 *>(cp + l * NP + n0))
+                                          : *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+                    cj[l][0] = v.x;
+                    cj[l][1] = v.y;
+                }
+            }
+            const float xx = d.x * d.x, yy = d.y * d.y, zz = d.z * d.z;
+            const float xy = d.x * d.y, xz = d.x * d.z, yz = d.y * d.z;
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const float t = r - (float)(n0 + m) * P.mu_step;
+                const float g = expf(-P.alpha * t * t);
+                const float phi = g * fc;
+                const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
+                const float *a = &gk[m * NT];
+                const float *b = &gj[m * NT];
+                const float c0j = cj[0][m], c1j = cj[1][m], c2j = cj[2][m];
+                const float c0k = ck[0][m], c1k = ck[1][m], c2k = ck[2][m];
+                // l = 0 (parity +), l = 1 (parity -), l = 2 (parity +)
+                const float H0 = a[0] * c0j + b[0] * c0k;
+                const float Hx = a[1] * c1j - b[1] * c1k;
+                const float Hy = a[2] * c1j - b[2] * c1k;
+                const float Hz = a[3] * c1j - b[3] * c1k;
+                const float Hxx = a[4] * c2j + b[4] * c2k;
+                const float Hyy = a[5] * c2j + b[5] * c2k;
+                const float Hzz = a[6] * c2j + b[6] * c2k;
+                const float Hxy = a[7] * c2j + b[7] * c2k;
+                const float Hxz = a[8] * c2j + b[8] * c2k;
+                const float Hyz = a[9] * c2j + b[9] * c2k;
+                const float Pv = H0 + Hx * d.x + Hy * d.y + Hz * d.z + Hxx * xx + Hyy * yy + Hzz * zz + Hxy * xy +
+                                 Hxz * xz + Hyz * yz;
+                const float Qx = Hx + 2.f * Hxx * d.x + Hxy * d.y + Hxz * d.z;
+                const float Qy = Hy + 2.f * Hyy * d.y + Hxy * d.x + Hyz * d.z;
+                const float Qz = Hz + 2.f * Hzz * d.z + Hxz * d.x + Hyz * d.y;
+                const float s = dphi * Pv * inv_r;
+                fx += s * d.x + phi * Qx;
+                fy += s * d.y + phi * Qy;
+                fz += s * d.z + phi * Qz;
+                if (HAS_DC) {
+                    const float S1 = b[1] * d.x + b[2] * d.y + b[3] * d.z;
+                    const float S2 = b[4] * xx + b[5] * yy + b[6] * zz + b[7] * xy + b[8] * xz + b[9] * yz;
+                    dck[m][0] += phi * b[0];
+                    dck[m][1] -= phi * S1;
+                    dck[m][2] += phi * S2;
+                }
             }
         }
     }
-    // sum over the group's lanes (groups are aligned W-lane segments of a warp)
 #pragma unroll
-    for (int o = W / 2; o > 0; o >>= 1) {
+    for (int o = 16; o > 0; o >>= 1) {
         fx += __shfl_xor_sync(0xffffffffu, fx, o);
         fy += __shfl_xor_sync(0xffffffffu, fy, o);
         fz += __shfl_xor_sync(0xffffffffu, fz, o);
-        if (HAS_DC) {
-#pragma unroll
-            for (int k = 0; k < D; ++k) dck[k] += __shfl_xor_sync(0xffffffffu, dck[k], o);
-        }
     }
-    if (live && gl == 0) {
+    if (HAS_DC && lane < Ln::USED) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int l = 0; l < 3; ++l) sred[warp][slot][sub][m * 3 + l] = dck[m][l];
+    }
+    __syncwarp();
+    if (i >= n) return;
+    if (lane == 0) {
         float *Fo = F + 3 * (int64_t)i;
         if (accumulate) {
             fx += Fo[0];
@@ -300,10 +337,18 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restric
         Fo[0] = fx;
         Fo[1] = fy;
         Fo[2] = fz;
-        if (HAS_DC) {
-            float *o = dc + (int64_t)i * D;
+    }
+    if (HAS_DC && lane < LPE) {
+        float *o = dc + (int64_t)i * D;
 #pragma unroll
-            for (int k = 0; k < D / 2; ++k) reinterpret_cast<float2 *>(o)[k] = make_float2(dck[2 * k], dck[2 * k + 1]);
+        for (int l = 0; l < 3; ++l) {
+            float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < EPW; ++s2) {
+                v0 += sred[warp][s2][lane][l];
+                v1 += sred[warp][s2][lane][3 + l];
+            }
+            *reinterpret_cast<float2 *>(o + l * NP + n0) = make_float2(v0, v1);
         }
     }
 }
@@ -317,7 +362,7 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
     float *rho = c->d_rho + (int64_t)t * c->n * c->D;
-    unsigned g = (unsigned)((c->n + 127) / 128);
+    const unsigned g = (unsigned)((c->n + 3) / 4);   // one warp per centre, 4 per block
     REANN_TIMED(c, REANN_K_DENSITY, s);
     if (c->NP == 8)
         k_density_fwd<8><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w,
@@ -330,45 +375,24 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// lanes per centre: about a third of the mean active degree, 4..16
-static int group_width(const reann_ctx *c) {
-    double deg = c->n > 0 ? (double)c->counters.active_pairs / (double)c->n : 0.0;
-    if (deg <= 0.0) deg = c->n > 0 ? 0.6 * (double)c->nnz / (double)c->n : 0.0;
-    return deg >= 36.0 ? 16 : (deg >= 18.0 ? 8 : 4);
-}
-
-template <int NP, bool DC, int W>
-static void edge_bwd_launch(reann_ctx *c, const float *coef, bool accumulate, const EdgeParams &P, cudaStream_t s) {
-    constexpr int GROUPS = 128 / W;
-    unsigned g = (unsigned)((c->n + GROUPS - 1) / GROUPS);
-    k_edge_bwd<NP, DC, W><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w,
-                                            c->ne, c->d_G, c->d_F, c->d_dc, accumulate, P);
-}
-
-template <int NP, bool DC>
-static void edge_bwd_width(reann_ctx *c, const float *coef, bool accumulate, const EdgeParams &P, cudaStream_t s) {
-    switch (group_width(c)) {
-        case 16: edge_bwd_launch<NP, DC, 16>(c, coef, accumulate, P, s); break;
-        case 8: edge_bwd_launch<NP, DC, 8>(c, coef, accumulate, P, s); break;
-        default: edge_bwd_launch<NP, DC, 4>(c, coef, accumulate, P, s); break;
-    }
-}
-
 cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s) {
     if (c->n == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
+    const unsigned g = (unsigned)((c->n + 3) / 4);
     const bool has_dc = t >= 1;
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
+#define REANN_EDGE_BWD(NPV, DC)                                                                                   \
+    k_edge_bwd<NPV, DC><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w, \
+                                          c->ne, c->d_G, c->d_F, c->d_dc, accumulate, P)
     if (c->NP == 8) {
-        if (has_dc) edge_bwd_width<8, true>(c, coef, accumulate, P, s);
-        else edge_bwd_width<8, false>(c, coef, accumulate, P, s);
+        if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
     } else if (c->NP == 10) {
-        if (has_dc) edge_bwd_width<10, true>(c, coef, accumulate, P, s);
-        else edge_bwd_width<10, false>(c, coef, accumulate, P, s);
+        if (has_dc) REANN_EDGE_BWD(10, true); else REANN_EDGE_BWD(10, false);
     } else {
         return cudaErrorInvalidValue;
     }
+#undef REANN_EDGE_BWD
     return cudaGetLastError();
 }
 

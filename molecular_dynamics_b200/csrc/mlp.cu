@@ -12,7 +12,8 @@
 // rows uses one network.  A persistent block keeps its element's weights in
 // shared memory across tiles.  The backward kernels finish with
 //   G[i][n,tau] = dE/dA^t_{i,n,tau} = 2 w_tau A^t_{i,n,tau} dE/drho^t_{i,(n,l)},
-// the derivative of the squared sum of Eq. 1, so the edge pass can read G.
+// the derivative of the squared sum of Eq. 1, so the edge pass can read G
+// (stored in the edge kernels' lane-interleaved order, see g_slot_index).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -168,13 +169,15 @@ __global__ void __launch_bounds__(MLP_THREADS) k_mlp(const int4 *__restrict__ ti
                 sX[r * LDX + c] = v / sscale[c];
             });
             __syncthreads();
+            // G rows are stored in the edge kernels' lane-interleaved order
             for (int k = tid; k < rows * NA; k += MLP_THREADS) {
-                int r = k / NA, q = k % NA;
-                int nn = q / NT, u = q % NT;
-                int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
-                float wt = u >= 7 ? 4.f : 2.f;  // 2 * l!/(lx! ly! lz!)
-                int64_t gi = (int64_t)(r0 + r) * NA + q;
-                Gout[gi] = wt * A[gi] * sX[r * LDX + l * NP + nn];
+                const int r = k / NA, q = k % NA;
+                const int src = g_slot_source(q, NP);
+                const int nn = src / NT, u = src % NT;
+                const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
+                const float wt = u >= 7 ? 4.f : 2.f;  // 2 * l!/(lx! ly! lz!)
+                const int64_t rb = (int64_t)(r0 + r) * NA;
+                Gout[rb + q] = wt * A[rb + src] * sX[r * LDX + l * NP + nn];
             }
         }
         __syncthreads();

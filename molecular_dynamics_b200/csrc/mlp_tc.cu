@@ -406,17 +406,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int64_t gi = (int64_t)(r0 + row) * NA;
                 const float4 *a4 = reinterpret_cast<const float4 *>(A + gi);
                 float4 *g4 = reinterpret_cast<float4 *>(Gout + gi);
+                float av[NA];
 #pragma unroll
                 for (int q = 0; q < NA / 4; ++q) {
                     const float4 a = a4[q];
-                    const float av[4] = {a.x, a.y, a.z, a.w};
+                    av[4 * q] = a.x; av[4 * q + 1] = a.y; av[4 * q + 2] = a.z; av[4 * q + 3] = a.w;
+                }
+                // G rows in the edge kernels' lane-interleaved order
+#pragma unroll
+                for (int q = 0; q < NA / 4; ++q) {
                     float gv[4];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        const int k = 4 * q + s, nn = k / NT, u = k % NT;
+                        const int src = g_slot_source(4 * q + s, NP), nn = src / NT, u = src % NT;
                         const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
                         const float wt = u >= 7 ? 4.f : 2.f;
-                        gv[s] = wt * av[s] * gx[l * NP + nn];
+                        gv[s] = wt * av[src] * gx[l * NP + nn];
                     }
                     g4[q] = make_float4(gv[0], gv[1], gv[2], gv[3]);
                 }

@@ -78,7 +78,7 @@ BF16_CASES = {
     "ag2048": lambda: (lambda p: (p, *synth.make_structure(p)))(presets.scaled("ag1m", ncell=8)),
     # five elements with N_phi = 10 and [128,128] networks: ragged 128-row tiles per element
     "hea1372_h128": lambda: (lambda p: (p, *synth.make_structure(p)))(
-        presets.scaled("hea108k", ncell=7).with_(hidden=(128, 128))),
+        presets.scaled("hea108k", ncell=7).with_(hidden=(128, 128), mlp_precision=1)),
 }
 
 
