@@ -29,6 +29,7 @@ enum : int {
 struct EdgeParams {
     double box[3];
     double inv_box[3];
+    float L_hi[3], L_lo[3], inv_L[3];   // box edge as an fp32 pair L_hi + L_lo, and 1/L
     float r_cut, r_cut2;
     float pi_over_rc;
     float alpha;

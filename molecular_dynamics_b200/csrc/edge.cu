@@ -30,6 +30,9 @@ EdgeParams make_edge_params(const reann_ctx *c) {
     for (int a = 0; a < 3; ++a) {
         P.box[a] = c->box[a];
         P.inv_box[a] = 1.0 / c->box[a];
+        P.L_hi[a] = (float)c->box[a];
+        P.L_lo[a] = (float)(c->box[a] - (double)P.L_hi[a]);
+        P.inv_L[a] = (float)(1.0 / c->box[a]);
     }
     P.r_cut = (float)c->cfg.r_cut;
     P.r_cut2 = (float)(c->cfg.r_cut * c->cfg.r_cut);
@@ -39,16 +42,24 @@ EdgeParams make_edge_params(const reann_ctx *c) {
     return P;
 }
 
-// Minimum-image displacement x_j - x_i: difference and image shift in fp64
-// (so that boundary-crossing pairs keep full precision), rounded to fp32.
+// Minimum-image displacement x_j - x_i in fp32 without losing the fp32
+// precision of the result: TwoSum gives s + t = x_j - x_i exactly; the image
+// shift k L is removed from s exactly (for k != 0, s and k L_hi are within a
+// factor of two, so the difference is exact) and the small terms t - k L_lo
+// added last.  The result is the correctly rounded displacement up to the
+// L_lo rounding (~1e-13 A).
+__device__ __forceinline__ float min_image(float xi, float xj, float L_hi, float L_lo, float inv_L) {
+    const float s = xj - xi;
+    const float bb = s - xj;
+    const float t = (xj - (s - bb)) + (-xi - bb);
+    const float k = rintf(s * inv_L);
+    return (s - k * L_hi) + (t - k * L_lo);
+}
+
 __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeParams &P) {
-    double dx = (double)pj.x - (double)pi.x;
-    double dy = (double)pj.y - (double)pi.y;
-    double dz = (double)pj.z - (double)pi.z;
-    dx -= P.box[0] * rint(dx * P.inv_box[0]);
-    dy -= P.box[1] * rint(dy * P.inv_box[1]);
-    dz -= P.box[2] * rint(dz * P.inv_box[2]);
-    return make_float3((float)dx, (float)dy, (float)dz);
+    return make_float3(min_image(pi.x, pj.x, P.L_hi[0], P.L_lo[0], P.inv_L[0]),
+                       min_image(pi.y, pj.y, P.L_hi[1], P.L_lo[1], P.inv_L[1]),
+                       min_image(pi.z, pj.z, P.L_hi[2], P.L_lo[2], P.inv_L[2]));
 }
 
 // ---------------------------------------------------------------------------
@@ -101,10 +112,9 @@ struct Lanes {
     static constexpr int USED = EPW * LPE;
 };
 
-// forward: A^t for the lane's two radial indices accumulated in fp64 (the
-// odd-l components are small residuals of cancelling neighbour sums), products
-// c phi formed exactly in fp64, monomials from the fp64 displacement; slots
-// summed in a fixed order through shared memory; rho^t in fp64, stored fp32.
+// forward: A^t for the lane's two radial indices accumulated over the slot's
+// edges in row order, then the slots summed in a fixed order through shared
+// memory; rho^t from the summed A^t.
 template <int NP>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
@@ -114,7 +124,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE, EPW = Ln::EPW;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
-    __shared__ double sred[4][EPW][LPE][2 * NT];
+    __shared__ float sred[4][EPW][LPE][2 * NT + 1];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,23 +133,19 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
     const bool active_lane = lane < Ln::USED && i < n;
     const int n0 = 2 * sub;
 
-    double acc[2][NT];
+    float acc[2][NT];
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int u = 0; u < NT; ++u) acc[m][u] = 0.0;
+        for (int u = 0; u < NT; ++u) acc[m][u] = 0.f;
     if (active_lane) {
         const float4 pi = pos[i];
         const int q0 = row[i], cnt = act_cnt[i];
         for (int q = q0 + slot; q < q0 + cnt; q += EPW) {
             const int j = act_col[q];
             const float4 pj = pos[j];
-            double dx = (double)pj.x - (double)pi.x, dy = (double)pj.y - (double)pi.y,
-                   dz = (double)pj.z - (double)pi.z;
-            dx -= P.box[0] * rint(dx * P.inv_box[0]);
-            dy -= P.box[1] * rint(dy * P.inv_box[1]);
-            dz -= P.box[2] * rint(dz * P.inv_box[2]);
-            const float r = (float)sqrt(dx * dx + dy * dy + dz * dz);
+            const float3 d = displacement(pi, pj, P);
+            const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
             const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
             const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
             float c[3][2];
@@ -149,17 +155,17 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
                 c[l][0] = v.x;
                 c[l][1] = v.y;
             }
-            const double Y[NT] = {1.0, dx, dy, dz, dx * dx, dy * dy, dz * dz, dx * dy, dx * dz, dy * dz};
+            const float Y[NT] = {1.f, d.x, d.y, d.z, d.x * d.x, d.y * d.y, d.z * d.z, d.x * d.y, d.x * d.z, d.y * d.z};
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const float t = r - (float)(n0 + m) * P.mu_step;
-                const double phi = (double)(expf(-P.alpha * t * t) * fc);
-                const double a0 = (double)c[0][m] * phi, a1 = (double)c[1][m] * phi, a2 = (double)c[2][m] * phi;
+                const float phi = expf(-P.alpha * t * t) * fc;
+                const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
                 acc[m][0] += a0;
 #pragma unroll
-                for (int u = 1; u < 4; ++u) acc[m][u] = fma(a1, Y[u], acc[m][u]);
+                for (int u = 1; u < 4; ++u) acc[m][u] = fmaf(a1, Y[u], acc[m][u]);
 #pragma unroll
-                for (int u = 4; u < NT; ++u) acc[m][u] = fma(a2, Y[u], acc[m][u]);
+                for (int u = 4; u < NT; ++u) acc[m][u] = fmaf(a2, Y[u], acc[m][u]);
             }
         }
     }
@@ -172,12 +178,12 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
     __syncwarp();
     if (i < n && lane < LPE) {
         // lane == sub here: sum the slots in order, then this lane's two radial indices
-        double a[2][NT];
+        float a[2][NT];
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
             for (int u = 0; u < NT; ++u) {
-                double v = 0.0;
+                float v = 0.f;
 #pragma unroll
                 for (int s2 = 0; s2 < EPW; ++s2) v += sred[warp][s2][lane][m * NT + u];
                 a[m][u] = v;
@@ -188,13 +194,11 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
         for (int m = 0; m < 2; ++m) {
             const int nn = n0 + m;
 #pragma unroll
-            for (int u = 0; u < NT; u += 2)
-                *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2((float)a[m][u], (float)a[m][u + 1]);
-            const double *v = a[m];
-            ro[nn] = (float)(v[0] * v[0]);
-            ro[NP + nn] = (float)(v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
-            ro[2 * NP + nn] = (float)(v[4] * v[4] + v[5] * v[5] + v[6] * v[6] +
-                                      2.0 * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]));
+            for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(a[m][u], a[m][u + 1]);
+            const float *v = a[m];
+            ro[nn] = v[0] * v[0];
+            ro[NP + nn] = v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+            ro[2 * NP + nn] = v[4] * v[4] + v[5] * v[5] + v[6] * v[6] + 2.f * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]);
         }
     }
 }
