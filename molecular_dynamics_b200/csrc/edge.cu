@@ -64,11 +64,13 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 
 // ---------------------------------------------------------------------------
 // active pairs: the entries of each row closer than r_cut, compacted to the
-// front of the row's slot (same offsets as the full list).
+// front of the row's slot (same offsets as the full list), each with its
+// displacement and distance (dx, dy, dz, r), which every edge pass of the
+// evaluation then reads instead of recomputing.
 __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
-                                                int *__restrict__ act_col, EdgeParams P,
-                                                unsigned long long *__restrict__ total) {
+                                                int *__restrict__ act_col, float4 *__restrict__ act_geo,
+                                                EdgeParams P, unsigned long long *__restrict__ total) {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     int k = 0;
     if (i < n) {
@@ -78,7 +80,11 @@ __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict_
             int j = col[q];
             float3 d = displacement(pi, pos[j], P);
             float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
-            if (r2 < P.r_cut2) act_col[q0 + k++] = j;
+            if (r2 < P.r_cut2) {
+                act_col[q0 + k] = j;
+                act_geo[q0 + k] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+                ++k;
+            }
         }
         act_cnt[i] = k;
     }
@@ -95,42 +101,43 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
     k_active<<<(unsigned)((c->n + 127) / 128), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_col, c->d_act_cnt,
-                                                            c->d_act_col, P, (unsigned long long *)(c->d_i64 + 3));
+                                                            c->d_act_col, c->d_act_geo, P,
+                                                            (unsigned long long *)(c->d_i64 + 3));
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Lane decomposition shared by both edge passes: one warp per centre atom,
-// EPW = 32 / LPE edge slots of LPE = N_phi / 2 lanes; lane `sub` of a slot
-// owns radial indices 2 sub and 2 sub + 1.  A slot's lanes read one
+// Lane decomposition shared by both edge passes: a slot of LPE = N_phi / 2
+// lanes owns one centre atom and walks its active neighbours in row order;
+// lane `sub` owns radial indices 2 sub and 2 sub + 1.  A warp holds
+// CPW = 32 / LPE slots (8 centres for N_phi = 8).  The slot's lanes read one
 // neighbour's coefficients and dE/dA row as contiguous runs, and each lane
-// keeps only its own radial indices' accumulators.
+// keeps only its own radial indices' accumulators, so the forward needs no
+// cross-lane reduction and the backward only a sum of the force over the slot.
 template <int NP>
 struct Lanes {
     static constexpr int LPE = NP / 2;
-    static constexpr int EPW = 32 / LPE;
-    static constexpr int USED = EPW * LPE;
+    static constexpr int CPW = 32 / LPE;        // centres per warp
+    static constexpr int USED = CPW * LPE;
+    static constexpr int CPB = 4 * CPW;         // centres per 128-thread block
 };
 
-// forward: A^t for the lane's two radial indices accumulated over the slot's
-// edges in row order, then the slots summed in a fixed order through shared
-// memory; rho^t from the summed A^t.
 template <int NP>
-__global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
+__global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
+                                                     const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
                                                      EdgeParams P) {
     using Ln = Lanes<NP>;
-    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE, EPW = Ln::EPW;
+    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
-    __shared__ float sred[4][EPW][LPE][2 * NT + 1];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i = blockIdx.x * 4 + warp;
     const int slot = lane / LPE, sub = lane % LPE;
-    const bool active_lane = lane < Ln::USED && i < n;
+    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    if (lane >= Ln::USED || i >= n) return;
     const int n0 = 2 * sub;
 
     float acc[2][NT];
@@ -138,99 +145,73 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const float4 *__rest
     for (int m = 0; m < 2; ++m)
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = 0.f;
-    if (active_lane) {
-        const float4 pi = pos[i];
-        const int q0 = row[i], cnt = act_cnt[i];
-        for (int q = q0 + slot; q < q0 + cnt; q += EPW) {
-            const int j = act_col[q];
-            const float4 pj = pos[j];
-            const float3 d = displacement(pi, pj, P);
-            const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
-            const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
-            const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
-            float c[3][2];
+    const int q0 = row[i], q1 = q0 + act_cnt[i];
+    for (int q = q0; q < q1; ++q) {
+        const int j = act_col[q];
+        const float4 g = act_geo[q];     // dx, dy, dz, r
+        const float r = g.w;
+        const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
+        const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
+        float c[3][2];
 #pragma unroll
-            for (int l = 0; l < 3; ++l) {
-                const float2 v = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
-                c[l][0] = v.x;
-                c[l][1] = v.y;
-            }
-            const float Y[NT] = {1.f, d.x, d.y, d.z, d.x * d.x, d.y * d.y, d.z * d.z, d.x * d.y, d.x * d.z, d.y * d.z};
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const float t = r - (float)(n0 + m) * P.mu_step;
-                const float phi = expf(-P.alpha * t * t) * fc;
-                const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
-                acc[m][0] += a0;
-#pragma unroll
-                for (int u = 1; u < 4; ++u) acc[m][u] = fmaf(a1, Y[u], acc[m][u]);
-#pragma unroll
-                for (int u = 4; u < NT; ++u) acc[m][u] = fmaf(a2, Y[u], acc[m][u]);
-            }
+        for (int l = 0; l < 3; ++l) {
+            const float2 v = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
+            c[l][0] = v.x;
+            c[l][1] = v.y;
         }
-    }
-    if (lane < Ln::USED) {
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int u = 0; u < NT; ++u) sred[warp][slot][sub][m * NT + u] = acc[m][u];
-    }
-    __syncwarp();
-    if (i < n && lane < LPE) {
-        // lane == sub here: sum the slots in order, then this lane's two radial indices
-        float a[2][NT];
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int u = 0; u < NT; ++u) {
-                float v = 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < EPW; ++s2) v += sred[warp][s2][lane][m * NT + u];
-                a[m][u] = v;
-            }
-        float *Ao = A_out + (int64_t)i * NA;
-        float *ro = rho_out + (int64_t)i * D;
+        const float Y[NT] = {1.f, g.x, g.y, g.z, g.x * g.x, g.y * g.y, g.z * g.z, g.x * g.y, g.x * g.z, g.y * g.z};
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            const int nn = n0 + m;
+            const float t = r - (float)(n0 + m) * P.mu_step;
+            const float phi = expf(-P.alpha * t * t) * fc;
+            const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
+            acc[m][0] += a0;
 #pragma unroll
-            for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(a[m][u], a[m][u + 1]);
-            const float *v = a[m];
-            ro[nn] = v[0] * v[0];
-            ro[NP + nn] = v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
-            ro[2 * NP + nn] = v[4] * v[4] + v[5] * v[5] + v[6] * v[6] + 2.f * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]);
+            for (int u = 1; u < 4; ++u) acc[m][u] = fmaf(a1, Y[u], acc[m][u]);
+#pragma unroll
+            for (int u = 4; u < NT; ++u) acc[m][u] = fmaf(a2, Y[u], acc[m][u]);
         }
+    }
+    float *Ao = A_out + (int64_t)i * NA;
+    float *ro = rho_out + (int64_t)i * D;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const int nn = n0 + m;
+        const float *v = acc[m];
+#pragma unroll
+        for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(v[u], v[u + 1]);
+        ro[nn] = v[0] * v[0];
+        ro[NP + nn] = v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+        ro[2 * NP + nn] = v[4] * v[4] + v[5] * v[5] + v[6] * v[6] + 2.f * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]);
     }
 }
 
-// ---------------------------------------------------------------------------
-// backward: one warp per centre atom k, the same slots and lanes as the
-// forward.  Lane `sub` keeps G_k and c_k of its two radial indices in
-// registers and reads the neighbour's 20 interleaved dE/dA values as five
-// contiguous float4 per slot.  Force partials are summed over the warp by a
-// shuffle tree, dE/dc_k partials over the slots in order through shared memory.
+// backward: same slots and lanes.  Lane `sub` keeps G_k and c_k of its two
+// radial indices in registers and reads the neighbour's 20 interleaved dE/dA
+// values as five float4 (the slot's four lanes read 64 contiguous bytes per
+// load).  dE/dc_k of the lane's radial indices needs no reduction; the force
+// is summed over the slot's lanes in a fixed order.
 template <int NP, bool HAS_DC>
-__global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
+__global__ void __launch_bounds__(128) k_edge_bwd(int n, const int *__restrict__ row,
                                                   const int *__restrict__ act_cnt, const int *__restrict__ act_col,
+                                                  const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
                                                   float *__restrict__ dc, bool accumulate, EdgeParams P) {
     using Ln = Lanes<NP>;
-    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE, EPW = Ln::EPW;
+    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
-    __shared__ float sred[4][EPW][LPE][6];
     for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i = blockIdx.x * 4 + warp;
     const int slot = lane / LPE, sub = lane % LPE;
-    const bool active_lane = lane < Ln::USED && i < n;
+    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const bool live = lane < Ln::USED && i < n;
     const int n0 = 2 * sub;
 
     float fx = 0.f, fy = 0.f, fz = 0.f;
     float dck[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
-    if (active_lane) {
-        const float4 pi = pos[i];
+    if (live) {
         float gk[2 * NT], ck[3][2];
         {
             const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)i * NA);
@@ -239,7 +220,7 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restric
                 const float4 v = g4[q * LPE + sub];
                 gk[4 * q] = v.x; gk[4 * q + 1] = v.y; gk[4 * q + 2] = v.z; gk[4 * q + 3] = v.w;
             }
-            const float *cp = coef ? coef + (int64_t)i * D : sC0 + __float_as_int(pi.w) * D;
+            const float *cp = coef ? coef + (int64_t)i * D : sC0 + __float_as_int(pos[i].w) * D;
 #pragma unroll
             for (int l = 0; l < 3; ++l) {
                 const float2 v = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
@@ -247,12 +228,12 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restric
                 ck[l][1] = v.y;
             }
         }
-        const int q0 = row[i], cnt = act_cnt[i];
-        for (int q = q0 + slot; q < q0 + cnt; q += EPW) {
+        const int q0 = row[i], q1 = q0 + act_cnt[i];
+        for (int q = q0; q < q1; ++q) {
             const int j = act_col[q];
-            const float4 pj = pos[j];
-            const float3 d = displacement(pi, pj, P);
-            const float r = sqrtf(d.x * d.x + d.y * d.y + d.z * d.z);
+            const float4 geo = act_geo[q];
+            const float3 d = make_float3(geo.x, geo.y, geo.z);
+            const float r = geo.w;
             const float inv_r = 1.0f / r;
             float sn, cs;
             sincospif(r * (1.0f / P.r_cut), &sn, &cs);
@@ -266,11 +247,10 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restric
                     const float4 v = __ldg(g4 + q2 * LPE + sub);
                     gj[4 * q2] = v.x; gj[4 * q2 + 1] = v.y; gj[4 * q2 + 2] = v.z; gj[4 * q2 + 3] = v.w;
                 }
-                const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pj.w) * D;
+                const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
 #pragma unroll
                 for (int l = 0; l < 3; ++l) {
-                    const float2 v = coef ? __ldg(reinterpret_cast<const float2 *>(cp + l * NP + n0))
-                                          : *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+                    const float2 v = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
                     cj[l][0] = v.x;
                     cj[l][1] = v.y;
                 }
@@ -317,43 +297,32 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const float4 *__restric
             }
         }
     }
+    // force: sum over the slot's lanes (sub 0 .. LPE-1) in a fixed order
+    const int base = (lane / LPE) * LPE;
+    float sx = 0.f, sy = 0.f, sz = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        fx += __shfl_xor_sync(0xffffffffu, fx, o);
-        fy += __shfl_xor_sync(0xffffffffu, fy, o);
-        fz += __shfl_xor_sync(0xffffffffu, fz, o);
+    for (int s2 = 0; s2 < LPE; ++s2) {
+        const int src = base + s2 < 32 ? base + s2 : lane;
+        sx += __shfl_sync(0xffffffffu, fx, src);
+        sy += __shfl_sync(0xffffffffu, fy, src);
+        sz += __shfl_sync(0xffffffffu, fz, src);
     }
-    if (HAS_DC && lane < Ln::USED) {
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int l = 0; l < 3; ++l) sred[warp][slot][sub][m * 3 + l] = dck[m][l];
-    }
-    __syncwarp();
-    if (i >= n) return;
-    if (lane == 0) {
+    if (!live) return;
+    if (sub == 0) {
         float *Fo = F + 3 * (int64_t)i;
         if (accumulate) {
-            fx += Fo[0];
-            fy += Fo[1];
-            fz += Fo[2];
+            sx += Fo[0];
+            sy += Fo[1];
+            sz += Fo[2];
         }
-        Fo[0] = fx;
-        Fo[1] = fy;
-        Fo[2] = fz;
+        Fo[0] = sx;
+        Fo[1] = sy;
+        Fo[2] = sz;
     }
-    if (HAS_DC && lane < LPE) {
+    if (HAS_DC) {
         float *o = dc + (int64_t)i * D;
 #pragma unroll
-        for (int l = 0; l < 3; ++l) {
-            float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < EPW; ++s2) {
-                v0 += sred[warp][s2][lane][l];
-                v1 += sred[warp][s2][lane][3 + l];
-            }
-            *reinterpret_cast<float2 *>(o + l * NP + n0) = make_float2(v0, v1);
-        }
+        for (int l = 0; l < 3; ++l) *reinterpret_cast<float2 *>(o + l * NP + n0) = make_float2(dck[0][l], dck[1][l]);
     }
 }
 
@@ -366,14 +335,13 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
     float *rho = c->d_rho + (int64_t)t * c->n * c->D;
-    const unsigned g = (unsigned)((c->n + 3) / 4);   // one warp per centre, 4 per block
     REANN_TIMED(c, REANN_K_DENSITY, s);
     if (c->NP == 8)
-        k_density_fwd<8><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w,
-                                           c->ne, A, rho, P);
+        k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
     else if (c->NP == 10)
-        k_density_fwd<10><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w,
-                                            c->ne, A, rho, P);
+        k_density_fwd<10><<<(unsigned)((c->n + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
@@ -383,12 +351,12 @@ cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s
     if (c->n == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
-    const unsigned g = (unsigned)((c->n + 3) / 4);
     const bool has_dc = t >= 1;
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
-#define REANN_EDGE_BWD(NPV, DC)                                                                                   \
-    k_edge_bwd<NPV, DC><<<g, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_act_cnt, c->d_act_col, coef, c->d_w, \
-                                          c->ne, c->d_G, c->d_F, c->d_dc, accumulate, P)
+#define REANN_EDGE_BWD(NPV, DC)                                                                                  \
+    k_edge_bwd<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
+        (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, c->d_G, c->d_F, \
+        c->d_dc, accumulate, P)
     if (c->NP == 8) {
         if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
     } else if (c->NP == 10) {
