@@ -71,27 +71,38 @@ __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict_
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
                                                 EdgeParams P, unsigned long long *__restrict__ total) {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    // one warp per row: lanes test consecutive entries, a ballot compacts the
+    // active ones in row order and the writes stay contiguous
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (i >= n) return;
+    const float4 pi = pos[i];
+    const int q0 = row[i], q1 = row[i + 1];
     int k = 0;
-    if (i < n) {
-        float4 pi = pos[i];
-        int q0 = row[i], q1 = row[i + 1];
-        for (int q = q0; q < q1; ++q) {
-            int j = col[q];
-            float3 d = displacement(pi, pos[j], P);
-            float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
-            if (r2 < P.r_cut2) {
-                act_col[q0 + k] = j;
-                act_geo[q0 + k] = make_float4(d.x, d.y, d.z, sqrtf(r2));
-                ++k;
-            }
+    for (int base = q0; base < q1; base += 32) {
+        const int q = base + lane;
+        bool act = false;
+        int j = 0;
+        float3 d = make_float3(0.f, 0.f, 0.f);
+        float r2 = 0.f;
+        if (q < q1) {
+            j = col[q];
+            d = displacement(pi, pos[j], P);
+            r2 = d.x * d.x + d.y * d.y + d.z * d.z;
+            act = r2 < P.r_cut2;
         }
-        act_cnt[i] = k;
+        const unsigned mask = __ballot_sync(0xffffffffu, act);
+        if (act) {
+            const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
+            act_col[o] = j;
+            act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+        }
+        k += __popc(mask);
     }
-    unsigned long long v = (unsigned long long)k;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((threadIdx.x & 31) == 0 && v) atomicAdd(total, v);
+    if (lane == 0) {
+        act_cnt[i] = k;
+        atomicAdd(total, (unsigned long long)k);
+    }
 }
 
 cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
@@ -100,7 +111,7 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(c->d_i64 + 3, 0, sizeof(int64_t), s);
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
-    k_active<<<(unsigned)((c->n + 127) / 128), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_col, c->d_act_cnt,
+    k_active<<<(unsigned)((c->n + 3) / 4), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_col, c->d_act_cnt,
                                                             c->d_act_col, c->d_act_geo, P,
                                                             (unsigned long long *)(c->d_i64 + 3));
     return cudaGetLastError();

@@ -2,9 +2,9 @@
 oracle on the same inputs, and compare with the stated tolerances.
 
 Tolerances (fp32 path): total energy |E_gpu - E_ref| / N <= 1e-5 max(|E_ref| / N,
-1e-2 eV); per-atom energies |dE_i| <= 1e-5 max(|E_i|, 1e-2 eV) in the worst atom
-is reported and bounded by 1e-4; forces max-abs <= 1e-4 eV/A.  BF16-network
-path: forces max-abs <= 5e-3 eV/A, energy per atom 1e-3 relative.
+1e-2 eV); the worst atom's |dE_i| <= 1e-4 of the RMS per-atom energy; forces
+max-abs <= 1e-4 eV/A.  BF16-network path: forces max-abs <= 5e-3 eV/A, the
+same energy tolerances (the split-bf16 networks keep 16 significant bits).
 """
 from __future__ import annotations
 
@@ -14,7 +14,7 @@ import oracle
 from molecular_dynamics_b200 import reann, synth
 
 F_TOL = {0: 1e-4, 1: 5e-3}
-E_TOL = {0: 1e-5, 1: 1e-3}
+E_TOL = {0: 1e-5, 1: 1e-5}
 
 
 def torch_cuda():
@@ -56,8 +56,12 @@ def assert_forces_close(F_gpu, F_ref, prec=0):
 
 
 def assert_atom_energies_close(Ei_gpu, Ei_ref, prec=0):
-    rel = np.abs(Ei_gpu - Ei_ref) / np.maximum(np.abs(Ei_ref), 1e-2)
-    assert rel.max() <= 10 * E_TOL[prec], rel.max()
+    # worst atom against the system's per-atom energy scale (RMS of E_i): the
+    # per-atom figure is reported beside the total-energy tolerance, and an
+    # atom whose own E_i happens to be near zero is not a scale
+    scale = max(float(np.sqrt(np.mean(Ei_ref ** 2))), 1e-2)
+    err = np.abs(Ei_gpu - Ei_ref).max() / scale
+    assert err <= 10 * E_TOL[prec], err
 
 
 def cluster_around(pos, types, box, k, radius):

@@ -69,5 +69,6 @@ def test_sampled_forces_and_energies(full):
         cpos, ctypes_, cbox, sel = cluster_around(pos, types, box, k, radius)
         ref = oracle_eval(p, cpos, ctypes_, cbox, weights=w)
         assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[prec], (k, F[k], ref.forces[0])
-        rel = abs(Ei[k] - ref.atom_energy[0]) / max(abs(ref.atom_energy[0]), 1e-2)
+        # against the system's per-atom energy scale, as in gpu_helpers
+        rel = abs(Ei[k] - ref.atom_energy[0]) / max(float(np.sqrt(np.mean(Ei ** 2))), 1e-2)
         assert rel <= 10 * E_TOL[prec], (k, Ei[k], ref.atom_energy[0])
