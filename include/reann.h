@@ -236,6 +236,39 @@ reann_status reann_profile(reann_ctx *ctx, int32_t enable);
  */
 reann_status reann_profile_read(const reann_ctx *ctx, int32_t group, double *ms, int64_t *launches);
 
+/*
+ * Allocation-free pair list (the paper has no counterpart: this serves
+ * callers, not the method).  Some callers cannot allocate device memory:
+ * programs that own the whole device through their own pool or a fixed
+ * memory budget (an MD engine's force plug-in, for example, receives its
+ * buffers and may not grow the footprint), and latency-critical loops that
+ * avoid cudaMalloc/cudaFree because those can synchronise the whole device.
+ * This call needs no context and allocates nothing: the caller passes inputs
+ * and outputs, and the scratch
+ * (cell bins, sorted cell lists, row counts) lives in one fixed file-scope
+ * device array of about 2.5 MB that every GPU loading the library holds until
+ * the process exits.
+ *
+ * Computes the list reann_build_neighbors builds, in the caller's order: row
+ * [n+1] (device int32) receives the offsets, col [cap] (device int32) every j
+ * with (i, j), i != j, within r_cut + skin under the same fp64 no-FMA test,
+ * rows sorted by j.  pos: device float32 [n][3] (A); box: host double[3];
+ * nnz: host, receives the list length.  At most 131,072 atoms: larger n is
+ * rejected with REANN_ERR_CAPACITY before any GPU work; if the list outgrows
+ * cap, REANN_ERR_CAPACITY is returned with *nnz set, row filled and col not
+ * written.  Other errors: REANN_ERR_ARG, REANN_ERR_BOX, REANN_ERR_NONFINITE,
+ * REANN_ERR_CUDA; reann_last_error(NULL) gives the message.
+ *
+ * All calls share the scratch array and it keeps the last call's contents;
+ * each call clears what must start at zero.  Calls whose GPU work overlaps
+ * (two streams, or two host threads on one device) race on the array:
+ * serialise them.  The first call on a device looks up the array's device
+ * address with that device current (cudaGetSymbolAddress); make that first
+ * call before any stream capture.  Synchronises the stream twice.
+ */
+reann_status reann_pair_list_noalloc(int64_t n, const float *pos, const double box[3], double r_cut, double skin,
+                                     int32_t *row, int32_t *col, int64_t cap, int64_t *nnz, reann_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

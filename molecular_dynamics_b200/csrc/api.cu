@@ -276,6 +276,8 @@ void fill_counters(reann_ctx *c) {
 
 namespace reann {
 
+void set_context_free_error(const std::string &msg) { g_create_error = msg; }
+
 LaunchScope::LaunchScope(reann_ctx *c_, int g, cudaStream_t s_, int kernels) : c(c_), group(g), s(s_) {
     c->counters.kernel_launches += kernels;
     if (!c->prof) return;

@@ -61,6 +61,8 @@ struct Ctx;
 
 // --- host orchestration helpers (defined across the .cu files) -------------
 cudaError_t scan_exclusive(const int *in, int *out, int64_t n, int64_t *d_total, void *tmp, cudaStream_t s);
+// message returned by reann_last_error(NULL) on this host thread
+void set_context_free_error(const std::string &msg);
 size_t scan_tmp_bytes(int64_t n);
 
 }  // namespace reann

@@ -24,7 +24,7 @@ STATUS = {
 
 EXPORTS = ("reann_create", "reann_destroy", "reann_build_neighbors", "reann_energy_forces", "reann_md_step",
            "reann_get_counters", "reann_last_error", "reann_get_neighbors", "reann_get_features", "reann_profile",
-           "reann_profile_read")
+           "reann_profile_read", "reann_pair_list_noalloc")
 
 KERNEL_GROUPS = ("active", "density", "mlp_fwd", "mlp_energy", "edge_bwd", "mlp_bwd", "energy_sum", "integrate",
                  "neighbors", "other")
@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH):
     lib.reann_get_neighbors.argtypes = [P, P, P, I64, P]
     lib.reann_get_features.argtypes = [P, I32, P, P, P]
     lib.reann_profile.argtypes = [P, I32]
+    lib.reann_pair_list_noalloc.argtypes = [I64, P, C.POINTER(D), D, D, P, P, I64, C.POINTER(I64), P]
     lib.reann_profile_read.argtypes = [P, I32, C.POINTER(D), C.POINTER(I64)]
     for name in EXPORTS:
         if name != "reann_last_error":
@@ -110,6 +111,20 @@ def _stream(stream) -> Optional[int]:
     except ImportError:
         pass
     return None
+
+
+def reann_pair_list_noalloc(pos, box, r_cut: float, skin: float, row, col, stream=None) -> int:
+    """Allocation-free pair list into caller buffers (device tensors): row
+    int32 [n+1], col int32 [cap].  Returns the list length."""
+    lib = load()
+    n = int(pos.shape[0])
+    b = (C.c_double * 3)(*[float(x) for x in box])
+    nnz = C.c_int64(0)
+    st = lib.reann_pair_list_noalloc(n, _ptr(pos), b, float(r_cut), float(skin), _ptr(row), _ptr(col),
+                                     int(col.shape[0]), C.byref(nnz), _stream(stream))
+    if st:
+        raise ReannError(st, lib.reann_last_error(None).decode())
+    return nnz.value
 
 
 @dataclass
