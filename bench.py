@@ -47,6 +47,12 @@ FLOP_DENSITY_PER_PAIR = {8: 240, 10: 298}
 FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without dE/dc, layers >= 1)
 
 
+# DRAM read + write of one k_edge_bwd launch from the ncu capture summarised in
+# profiles/k_edge_bwd_ag256k.md (256,000 atoms), scaled to the atom count of the
+# run; None when the kernel has changed since that capture
+EDGE_BWD_TRAFFIC_PER_ATOM = (446.367488e6 + 26.646272e6) / 256000
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -272,7 +278,8 @@ def main():
         achieved = flop_per_launch / (ms_dom / n_dom * 1e-3) / 1e12
         roof = {"kernel": {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}[dominant], "bound": "alu",
                 "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                "traffic": None,
+                "traffic": (EDGE_BWD_TRAFFIC_PER_ATOM * n if dominant == "edge_bwd" else None),
+                "traffic_note": "bytes per launch: DRAM read+write of a 256,000-atom capture scaled by the atom count",
                 "peak_note": f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {pk.get('sm_max_mhz', 1965.0):.0f} MHz "
                              f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz",
                 "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
