@@ -18,6 +18,10 @@
 // folded into the row of k because the list is symmetric; the parity (-1)^l
 // comes from Y_tau(-d) = (-1)^l Y_tau(d).
 //
+// Transcendentals use the SFU intrinsics (__expf, __sincosf, __fdividef):
+// their arguments are bounded (cosine argument in [0, pi), exponent <= 0) and
+// the parity tests hold the results to the stated tolerances.
+//
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
 #include "common.cuh"
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         const int j = act_col[q];
         const float4 g = act_geo[q];     // dx, dy, dz, r
         const float r = g.w;
-        const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
+        const float fc = 0.5f * (__cosf(r * P.pi_over_rc) + 1.0f);   // argument in [0, pi)
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
         float c[3][2];
 #pragma unroll
@@ -174,7 +178,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
             const float t = r - (float)(n0 + m) * P.mu_step;
-            const float phi = expf(-P.alpha * t * t) * fc;
+            const float phi = __expf(-P.alpha * t * t) * fc;
             const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
             acc[m][0] += a0;
 #pragma unroll
@@ -245,9 +249,9 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const int *__restrict__
             const float4 geo = act_geo[q];
             const float3 d = make_float3(geo.x, geo.y, geo.z);
             const float r = geo.w;
-            const float inv_r = 1.0f / r;
+            const float inv_r = __fdividef(1.0f, r);
             float sn, cs;
-            sincospif(r * (1.0f / P.r_cut), &sn, &cs);
+            __sincosf(r * P.pi_over_rc, &sn, &cs);   // argument in [0, pi)
             const float fc = 0.5f * (cs + 1.0f);
             const float dfc = -0.5f * P.pi_over_rc * sn;
             float gj[2 * NT], cj[3][2];
@@ -271,7 +275,7 @@ __global__ void __launch_bounds__(128) k_edge_bwd(int n, const int *__restrict__
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const float t = r - (float)(n0 + m) * P.mu_step;
-                const float g = expf(-P.alpha * t * t);
+                const float g = __expf(-P.alpha * t * t);
                 const float phi = g * fc;
                 const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
                 const float *a = &gk[m * NT];

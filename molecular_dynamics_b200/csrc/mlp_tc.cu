@@ -17,8 +17,10 @@
 // shared memory in the canonical K-major layout, and one thread issues the
 // next MMA.
 //
-// Block: 128 threads (4 warps, warp w reads TMEM lanes 32w..32w+31), one
-// block per SM (shared memory > half an SM), persistent over the tiles.  All
+// Block: 256 threads; warp w reads TMEM lanes 32 (w % 4) .. + 31 and works on
+// half w / 4 of each accumulator's columns, so a tile row (atom) is shared by
+// two threads.  One block per SM (shared memory > half an SM), persistent
+// over the tiles.  All
 // waits on the MMA-completion barrier are bounded: a wait that gives up sets
 // ST_TIMEOUT, the block frees its tensor memory and returns.
 //
@@ -35,7 +37,7 @@ namespace reann {
 namespace {
 
 constexpr int TM = 128;            // atoms per tile (MMA M)
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 256;    // two warp groups: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
 constexpr int KPAD = 32;           // feature dimension padded to a multiple of 16
 constexpr int TMEM_COLS = 512;
 
@@ -185,7 +187,7 @@ struct TcLayout {
     static constexpr int A1 = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][H1] x 2
     static constexpr int A2 = A1 + 2 * TM * H1 * 2;              // [TM][H2] x 2
     static constexpr int F32 = A2 + 2 * TM * H2 * 2;
-    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2;  // b1, b2, b3, shift, scale, 1/scale, w3
+    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2 + 2 * TM;  // b1, b2, b3, shift, scale, 1/scale, w3, e_part
     static constexpr int BAR = F32 + nf32 * 4;
     static constexpr int bytes = BAR + 16 + 16;
     // TMEM columns
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     extern __shared__ __align__(1024) unsigned char sm[];
     float *f32 = reinterpret_cast<float *>(sm + L::F32);
     float *sb1 = f32, *sb2 = sb1 + H1, *sb3 = sb2 + H2, *sshift = sb3 + KPAD, *sscale = sshift + KPAD,
-          *sinv = sscale + KPAD, *sw3 = sinv + KPAD;
+          *sinv = sscale + KPAD, *sw3 = sinv + KPAD, *se = sw3 + H2;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
     unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KPAD * 2;
@@ -212,7 +214,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     unsigned char *a2_hi = sm + L::A2, *a2_lo = a2_hi + TM * H2 * 2;
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int row = tid;                       // this thread's atom within the tile (TMEM lane)
+    const int row = tid & (TM - 1);            // this thread's atom within the tile (TMEM lane)
+    const int half = tid / TM;                 // which half of each accumulator's columns
     const uint32_t base = smem_u32(sm);
     auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
 
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __syncthreads();
     fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t phase = 0;
     bool failed = false;
     int cur = -1;
@@ -282,7 +285,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const bool live = row < rows;
             const int64_t gi = (int64_t)(r0 + row);
 #pragma unroll
-            for (int c = 0; c < KPAD; c += 8) {
+            for (int c = half * (KPAD / 2); c < (half + 1) * (KPAD / 2); c += 8) {
                 float v[8], g[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!wait_mma()) { failed = true; break; }
         // a1 = tanh(z1 + b1)
 #pragma unroll 1
-        for (int c = 0; c < H1; c += 32) {
+        for (int c = half * (H1 / 2); c < (half + 1) * (H1 / 2); c += 32) {
             float v[32];
             tmem_ld32(lane_base + L::C_Z1 + c, v);
 #pragma unroll
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (MODE == TC_FWD) {
             // a2 = tanh(z2 + b2), then y = a2 W3^T + b3
 #pragma unroll 1
-            for (int c = 0; c < H2; c += 32) {
+            for (int c = half * (H2 / 2); c < (half + 1) * (H2 / 2); c += 32) {
                 float v[32];
                 tmem_ld32(lane_base + L::C_Z2 + c, v);
 #pragma unroll
@@ -346,13 +349,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (row < rows) {
                 float *yo = Y + (int64_t)(r0 + row) * D;
 #pragma unroll
-                for (int f = 0; f < D; ++f) yo[f] = v[f] + sb3[f];
+                for (int f = 0; f < D; ++f)
+                    if ((f < (D + 1) / 2) == (half == 0)) yo[f] = v[f] + sb3[f];
             }
         } else {
             // g2 = dE/dz2 = (energy: w3, backward: dY W3) * (1 - a2^2); energy E_i = w3 . a2 + b3
             float e_row = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < H2; c += 32) {
+            for (int c = half * (H2 / 2); c < (half + 1) * (H2 / 2); c += 32) {
                 float z[32], up[32];
                 tmem_ld32(lane_base + L::C_Z2 + c, z);
                 if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P + c, up);
@@ -366,8 +370,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 32; u += 8) st_chunk2(a2_hi, a2_lo, TM, row, c + u, &z[u]);
             }
-            if (MODE == TC_ENERGY && row < rows) Ei[r0 + row] = e_row + sb3[0];
+            if (MODE == TC_ENERGY) se[half * TM + row] = e_row;
             handoff();
+            if (MODE == TC_ENERGY && half == 0 && row < rows) Ei[r0 + row] = se[row] + se[TM + row] + sb3[0];
             // p1 = g2 W2 (MN-major view of W2), into the columns dY W3 used
             if (tid == 0) {
                 fence_after();
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (!wait_mma()) { failed = true; break; }
             // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation still in TMEM
 #pragma unroll 1
-            for (int c = 0; c < H1; c += 32) {
+            for (int c = half * (H1 / 2); c < (half + 1) * (H1 / 2); c += 32) {
                 float p[32], z[32];
                 tmem_ld32(lane_base + L::C_P + c, p);
                 tmem_ld32(lane_base + L::C_Z1 + c, z);
@@ -412,9 +417,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     const float4 a = a4[q];
                     av[4 * q] = a.x; av[4 * q + 1] = a.y; av[4 * q + 2] = a.z; av[4 * q + 3] = a.w;
                 }
-                // G rows in the edge kernels' lane-interleaved order
+                // G rows in the edge kernels' lane-interleaved order; each half writes half of the row
+                constexpr int QS = (NA / 4 + 1) / 2;
 #pragma unroll
                 for (int q = 0; q < NA / 4; ++q) {
+                    if ((q < QS) != (half == 0)) continue;
                     float gv[4];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
