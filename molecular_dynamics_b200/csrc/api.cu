@@ -170,6 +170,7 @@ reann_status ensure_capacity(reann_ctx *c, int64_t nnz) {
     CK(dalloc(&c->d_col, (size_t)cap));
     CK(dalloc(&c->d_act_col, (size_t)cap));
     CK(dalloc(&c->d_act_geo, (size_t)cap));
+    CK(dalloc(&c->d_act_fc, (size_t)cap));
     c->cap = cap;
     return REANN_OK;
 }
@@ -395,7 +396,7 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     DeviceGuard guard(c->device);
     free_atoms(c);
     dfree(c->d_w); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
-    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
+    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_act_fc); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
     if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
     if (c->h_status) cudaFreeHost(c->h_status);
     if (c->h_i64) cudaFreeHost(c->h_i64);

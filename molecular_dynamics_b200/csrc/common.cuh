@@ -109,6 +109,7 @@ struct reann_ctx {
     int *d_act_cnt = nullptr;      // [n]
     int *d_act_col = nullptr;      // [cap]
     float4 *d_act_geo = nullptr;   // [cap] displacement and distance of each active entry
+    float *d_act_fc = nullptr;     // [cap] cutoff function of each active entry
     int64_t nnz = 0, cap = 0, max_row = 0;
     void *d_scan_tmp = nullptr;
     size_t scan_tmp_size = 0;

@@ -18,9 +18,11 @@
 // folded into the row of k because the list is symmetric; the parity (-1)^l
 // comes from Y_tau(-d) = (-1)^l Y_tau(d).
 //
-// Transcendentals use the SFU intrinsics (__expf, __sincosf, __fdividef):
-// their arguments are bounded (cosine argument in [0, pi), exponent <= 0) and
-// the parity tests hold the results to the stated tolerances.
+// The backward pass uses the SFU intrinsics (__expf, __sincosf, __fdividef):
+// their arguments are bounded (sine/cosine argument in [0, pi), exponent <= 0)
+// and only forces depend on them.  The forward pass keeps the accurate
+// expf/cospif: the densities feed standardised network inputs, where the
+// intrinsics' ~1e-7 errors showed up as 1e-5-level per-atom energy errors.
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
@@ -69,12 +71,13 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 // ---------------------------------------------------------------------------
 // active pairs: the entries of each row closer than r_cut, compacted to the
 // front of the row's slot (same offsets as the full list), each with its
-// displacement and distance (dx, dy, dz, r), which every edge pass of the
-// evaluation then reads instead of recomputing.
+// displacement and distance (dx, dy, dz, r) and cutoff function f_c(r), which
+// every edge pass of the evaluation then reads instead of recomputing.
 __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
-                                                EdgeParams P, unsigned long long *__restrict__ total) {
+                                                float *__restrict__ act_fc, EdgeParams P,
+                                                unsigned long long *__restrict__ total) {
     // one warp per row: lanes test consecutive entries, a ballot compacts the
     // active ones in row order and the writes stay contiguous
     const int lane = threadIdx.x & 31;
@@ -98,8 +101,10 @@ __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict_
         const unsigned mask = __ballot_sync(0xffffffffu, act);
         if (act) {
             const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
+            const float r = sqrtf(r2);
             act_col[o] = j;
-            act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+            act_geo[o] = make_float4(d.x, d.y, d.z, r);
+            act_fc[o] = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
         }
         k += __popc(mask);
     }
@@ -116,7 +121,7 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
     k_active<<<(unsigned)((c->n + 3) / 4), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_col, c->d_act_cnt,
-                                                            c->d_act_col, c->d_act_geo, P,
+                                                            c->d_act_col, c->d_act_geo, c->d_act_fc, P,
                                                             (unsigned long long *)(c->d_i64 + 3));
     return cudaGetLastError();
 }
@@ -140,7 +145,8 @@ struct Lanes {
 template <int NP>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
-                                                     const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
+                                                     const float4 *__restrict__ act_geo,
+                                                     const float *__restrict__ act_fc, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
                                                      EdgeParams P) {
@@ -165,7 +171,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         const int j = act_col[q];
         const float4 g = act_geo[q];     // dx, dy, dz, r
         const float r = g.w;
-        const float fc = 0.5f * (__cosf(r * P.pi_over_rc) + 1.0f);   // argument in [0, pi)
+        const float fc = act_fc[q];
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
         float c[3][2];
 #pragma unroll
@@ -178,7 +184,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
             const float t = r - (float)(n0 + m) * P.mu_step;
-            const float phi = __expf(-P.alpha * t * t) * fc;
+            const float phi = expf(-P.alpha * t * t) * fc;
             const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
             acc[m][0] += a0;
 #pragma unroll
@@ -207,7 +213,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 // load).  dE/dc_k of the lane's radial indices needs no reduction; the force
 // is summed over the slot's lanes in a fixed order.
 template <int NP, bool HAS_DC>
-__global__ void __launch_bounds__(128) k_edge_bwd(int n, const int *__restrict__ row,
+__global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restrict__ row,
                                                   const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                   const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
@@ -353,10 +359,12 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     REANN_TIMED(c, REANN_K_DENSITY, s);
     if (c->NP == 8)
         k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_act_fc, c->d_pos, coef, c->d_w, c->ne,
+            A, rho, P);
     else if (c->NP == 10)
         k_density_fwd<10><<<(unsigned)((c->n + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_act_fc, c->d_pos, coef, c->d_w, c->ne,
+            A, rho, P);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
