@@ -148,6 +148,58 @@ def run_reference(args, rank, world):
     return 0
 
 
+def dd_sweep(args):
+    """Monolithic vs domain-decomposed E+F for T = 1..6 on the workload: time,
+    ghost bytes per layer and per evaluation, and bit-identity of the results.
+    One JSON line per T."""
+    import torch
+    from molecular_dynamics_b200 import reann
+
+    p = presets.get(args.workload)
+    if args.ncell:
+        p = presets.scaled(args.workload, ncell=args.ncell)
+    pos, types, box = synth.make_structure(p)
+    n = len(pos)
+    pos_d = torch.from_numpy(pos).cuda()
+    types_d = torch.from_numpy(types).cuda()
+    grid = tuple(int(x) for x in args.dd_grid.split("x"))
+    stream = torch.cuda.current_stream()
+
+    def timed(ctx, F):
+        for _ in range(2):
+            ctx.reann_energy_forces(pos_d, F)
+        times = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            E = ctx.reann_energy_forces(pos_d, F)
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return E, statistics.median(times)
+
+    for T in range(1, max(p.stats_depth, p.T) + 1):
+        w = synth.weight_blob(p, T=T)
+        out = {}
+        for name, g in (("mono", (0, 0, 0)), ("dd", grid)):
+            ctx = reann.Context(reann.ModelSpec.from_preset(p, T=T, dd_grid=g), w)
+            ctx.reann_build_neighbors(pos_d, types_d, box)
+            F = torch.empty_like(pos_d)
+            E, ms = timed(ctx, F)
+            out[name] = (E, ms, F.clone(), ctx.reann_get_counters())
+            ctx.close()
+        c = out["dd"][3]
+        print(json.dumps({
+            "mode": "dd_sweep", "workload": p.key, "atoms": n, "T": T, "dd_grid": list(grid),
+            "ef_ms_monolithic": out["mono"][1], "ef_ms_dd": out["dd"][1],
+            "ghost_slots": c.ghost_slots, "ghost_bytes_per_layer_fwd": c.ghost_bytes_fwd,
+            "ghost_bytes_per_layer_bwd": c.ghost_bytes_bwd,
+            "ghost_bytes_per_evaluation": (T - 1) * c.ghost_bytes_fwd + T * c.ghost_bytes_bwd + 16 * c.ghost_slots,
+            "bit_identical": bool(out["mono"][0] == out["dd"][0] and torch.equal(out["mono"][2], out["dd"][2])),
+        }), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -158,6 +210,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=16)
+    ap.add_argument("--dd-sweep", action="store_true",
+                    help="monolithic vs domain-decomposed E+F for T = 1..6 (one JSON line per T)")
+    ap.add_argument("--dd-grid", default="8x8x8")
     ap.add_argument("--ncell", type=int, default=0,
                     help="FCC workloads: cells per axis (smaller lattices for profiling captures)")
     args = ap.parse_args()
@@ -167,6 +222,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.dd_sweep:
+        return dd_sweep(args)
 
     import torch
     from molecular_dynamics_b200 import reann

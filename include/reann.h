@@ -80,6 +80,7 @@ typedef struct {
     double alpha;          /* A^-2 */
     int32_t mlp_precision; /* 0 = fp32 networks; 1 = bf16 tensor-core GEMMs, fp32 accumulate */
     int32_t dd_grid[3];    /* {0,0,0} = monolithic; else subdomains per axis (checking mode) */
+    int32_t dd_stale_ghosts; /* checking mode only: 1 = skip the per-layer ghost refresh (negative control) */
 } reann_config;
 
 /*
@@ -129,7 +130,8 @@ typedef enum {
     REANN_K_INTEGRATE = 7,   /* velocity-Verlet kicks and drift */
     REANN_K_NEIGHBORS = 8,   /* binning + neighbour list build (all kernels of one build) */
     REANN_K_OTHER = 9,       /* gathers, scatters, checks */
-    REANN_K_COUNT = 10
+    REANN_K_GHOST = 10,      /* domain-decomposed mode: ghost planning and per-layer ghost refresh */
+    REANN_K_COUNT = 11
 } reann_kernel_group;
 
 /*

@@ -103,8 +103,9 @@ void free_atoms(reann_ctx *c) {
     dfree(c->d_A); dfree(c->d_rho); dfree(c->d_coef); dfree(c->d_G); dfree(c->d_dc); dfree(c->d_Ei);
     dfree(c->d_F); dfree(c->d_Epart); dfree(c->d_stage_f); dfree(c->d_stage_i); dfree(c->d_stage_x);
     dfree(c->d_stage_v); dfree(c->d_stage_e); dfree(c->d_x); dfree(c->d_v); dfree(c->d_diag);
-    dfree(c->d_last_x); dfree(c->d_last_v);
+    dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub);
     c->md_valid = false;
+    c->slots_alloc = 0;
     c->n_alloc = 0;
 }
 
@@ -140,7 +141,26 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_diag, N * (size_t)std::max(c->D, c->NA)));
     CK(dalloc(&c->d_last_x, 3 * N));
     CK(dalloc(&c->d_last_v, 3 * N));
+    if (c->dd) CK(dalloc(&c->d_dd_sub, N));
+    c->slots_alloc = n;
     c->n_alloc = n;
+    return REANN_OK;
+}
+
+// slot-sized arrays (positions, coefficients, dE/dA) for n_slots >= n slots;
+// the first n positions are kept
+reann_status ensure_slots(reann_ctx *c, int64_t n_slots, cudaStream_t s) {
+    c->n_slots = n_slots;
+    if (n_slots <= c->slots_alloc) return REANN_OK;
+    float4 *pos = nullptr;
+    CK(cudaMalloc(&pos, sizeof(float4) * (size_t)n_slots));
+    if (c->n > 0) CK(cudaMemcpyAsync(pos, c->d_pos, sizeof(float4) * (size_t)c->n, cudaMemcpyDeviceToDevice, s));
+    CK(cudaStreamSynchronize(s));
+    dfree(c->d_pos);
+    c->d_pos = pos;
+    CK(dalloc(&c->d_coef, (size_t)c->T * n_slots * c->D));
+    CK(dalloc(&c->d_G, (size_t)n_slots * c->NA));
+    c->slots_alloc = n_slots;
     return REANN_OK;
 }
 
@@ -170,7 +190,6 @@ reann_status ensure_capacity(reann_ctx *c, int64_t nnz) {
     CK(dalloc(&c->d_col, (size_t)cap));
     CK(dalloc(&c->d_act_col, (size_t)cap));
     CK(dalloc(&c->d_act_geo, (size_t)cap));
-    CK(dalloc(&c->d_act_fc, (size_t)cap));
     c->cap = cap;
     return REANN_OK;
 }
@@ -241,6 +260,27 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
         c->n_tiles128 = (int)tiles128.size();
         c->elem_start.assign(c->h_seg, c->h_seg + c->ne + 1);
     }
+    c->n_slots = c->n;
+    if (c->dd) {
+        int64_t ng = 0;
+        CK(dd_plan(c, s, &ng));
+        if (ng > INT32_MAX - c->n) return fail(c, REANN_ERR_CAPACITY, "too many ghost slots");
+        if (ng > c->dd_owner_alloc) {
+            CK(dalloc(&c->d_dd_owner, (size_t)ng));
+            c->dd_owner_alloc = ng;
+        }
+        if (c->cap > c->col_dd_alloc) {
+            CK(dalloc(&c->d_col_dd, (size_t)c->cap));
+            c->col_dd_alloc = c->cap;
+        }
+        reann_status st2 = ensure_slots(c, c->n + ng, s);
+        if (st2) return st2;
+        c->dd_ghosts = ng;
+        CK(dd_finish(c, s));
+        c->counters.ghost_slots = ng;
+        c->counters.ghost_bytes_fwd = ng * c->D * (int64_t)sizeof(float);
+        c->counters.ghost_bytes_bwd = ng * c->NA * (int64_t)sizeof(float);
+    }
     c->have_list = true;
     c->counters.builds++;
     return REANN_OK;
@@ -249,15 +289,30 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
 // One energy+force evaluation on the internal positions d_pos.
 reann_status run_ef(reann_ctx *c, cudaStream_t s) {
     const bool tc = c->cfg.mlp_precision == 1;
+    const int64_t cstride = c->n_slots * c->D;
+    // domain-decomposed mode: ghost positions follow their owners
+    if (c->dd) CK(dd_gather_rows(c, reinterpret_cast<float *>(c->d_pos), 4, s));
     CK(launch_active(c, s));
     for (int t = 0; t < c->T; ++t) {
         CK(launch_density_fwd(c, t, s));
-        if (t + 1 < c->T) CK(tc ? launch_mlp_tc_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s));
+        if (t + 1 < c->T) {
+            CK(tc ? launch_mlp_tc_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s));
+            // the per-layer message sync: ghost c^{t+1} from the owners (or, as
+            // a negative control, the ghosts keep c^0)
+            if (c->dd) {
+                float *coef = c->d_coef + (t + 1) * cstride;
+                CK(c->cfg.dd_stale_ghosts ? dd_stale_coef(c, coef, s) : dd_gather_rows(c, coef, c->D, s));
+            }
+        }
     }
     CK(tc ? launch_mlp_tc_energy(c, s) : launch_mlp_energy(c, s));
+    if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
     for (int t = c->T - 1; t >= 0; --t) {
         CK(launch_edge_bwd(c, t, t != c->T - 1, s));
-        if (t >= 1) CK(tc ? launch_mlp_tc_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s));
+        if (t >= 1) {
+            CK(tc ? launch_mlp_tc_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s));
+            if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
+        }
     }
     CK(launch_energy_sum(c, s));
     c->counters.evaluations++;
@@ -336,8 +391,13 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     if (cfg->l_max != 2 || (cfg->n_radial != 8 && cfg->n_radial != 10) ||
         (cfg->hidden[0] != 64 && cfg->hidden[0] != 128) || (cfg->hidden[1] != 64 && cfg->hidden[1] != 128))
         return fail(nullptr, REANN_ERR_UNSUPPORTED, "supported: l_max 2, n_radial 8 or 10, hidden widths 64 or 128");
-    for (int a = 0; a < 3; ++a)
-        if (cfg->dd_grid[a] != 0) return fail(nullptr, REANN_ERR_UNSUPPORTED, "domain-decomposed mode is not built");
+    {
+        const bool any = cfg->dd_grid[0] || cfg->dd_grid[1] || cfg->dd_grid[2];
+        for (int a = 0; a < 3; ++a)
+            if (any && (cfg->dd_grid[a] < 1 || cfg->dd_grid[a] > 64))
+                return fail(nullptr, REANN_ERR_ARG, "dd_grid: all zero, or 1..64 subdomains per axis");
+        if (cfg->dd_stale_ghosts < 0 || cfg->dd_stale_ghosts > 1) return fail(nullptr, REANN_ERR_ARG, "dd_stale_ghosts");
+    }
     reann_ctx *c = new reann_ctx();
     c->cfg = *cfg;
     c->device = device;
@@ -348,6 +408,7 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     c->ne = cfg->n_elements;
     c->H1 = cfg->hidden[0];
     c->H2 = cfg->hidden[1];
+    c->dd = cfg->dd_grid[0] > 0;
     int64_t expect = (int64_t)c->ne * c->D + (int64_t)(c->T - 1) * c->ne * net_size(c, c->D) + (int64_t)c->ne * net_size(c, 1);
     if ((int64_t)nbytes != expect * (int64_t)sizeof(float)) {
         delete c;
@@ -396,7 +457,8 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     DeviceGuard guard(c->device);
     free_atoms(c);
     dfree(c->d_w); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
-    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_act_fc); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
+    dfree(c->d_dd_bits); dfree(c->d_dd_prefix); dfree(c->d_dd_cnt); dfree(c->d_dd_owner); dfree(c->d_col_dd);
+    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
     if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
     if (c->h_status) cudaFreeHost(c->h_status);
     if (c->h_i64) cudaFreeHost(c->h_i64);
@@ -639,7 +701,7 @@ extern "C" reann_status reann_get_features(reann_ctx *c, int32_t t, float *rho, 
                 std::memcpy(&h[a * c->D], &c->h_C0[(size_t)types[a] * c->D], sizeof(float) * c->D);
             CK(cudaMemcpy(coef, h.data(), sizeof(float) * nD, cudaMemcpyDefault));
         } else {
-            CK(launch_to_caller_rows(c, c->d_coef + t * nD, c->D, c->d_diag, s));
+            CK(launch_to_caller_rows(c, c->d_coef + t * c->n_slots * c->D, c->D, c->d_diag, s));
             CK(cudaMemcpyAsync(coef, c->d_diag, sizeof(float) * nD, cudaMemcpyDefault, s));
             CK(sync_stream(c, s));
         }

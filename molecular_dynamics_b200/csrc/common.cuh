@@ -101,7 +101,7 @@ struct reann_ctx {
     int *d_perm_tmp = nullptr;
     int *d_inv = nullptr;          // caller -> internal
     int *d_types_caller = nullptr; // caller order
-    float4 *d_pos = nullptr;       // internal order: x, y, z, type bits
+    float4 *d_pos = nullptr;       // [n_slots] internal order: x, y, z, type bits
     float4 *d_pos_build = nullptr; // positions at the last build
     int *d_row = nullptr;          // [n + 1]
     int *d_cnt = nullptr;          // [n]
@@ -109,18 +109,30 @@ struct reann_ctx {
     int *d_act_cnt = nullptr;      // [n]
     int *d_act_col = nullptr;      // [cap]
     float4 *d_act_geo = nullptr;   // [cap] displacement and distance of each active entry
-    float *d_act_fc = nullptr;     // [cap] cutoff function of each active entry
     int64_t nnz = 0, cap = 0, max_row = 0;
     void *d_scan_tmp = nullptr;
     size_t scan_tmp_size = 0;
     int64_t *d_i64 = nullptr;      // small scratch of int64 scalars
     int64_t *h_i64 = nullptr;      // pinned mirror
 
+    // domain-decomposed checking mode: slots [0, n) local atoms, [n, n_slots) ghosts
+    bool dd = false;
+    int64_t n_slots = 0, slots_alloc = 0;
+    int64_t dd_ghosts = 0;
+    int *d_dd_sub = nullptr;       // [n] subdomain of each internal atom
+    unsigned *d_dd_bits = nullptr; // [P][ceil(n/32)] ghost membership
+    int *d_dd_prefix = nullptr, *d_dd_cnt = nullptr;
+    int64_t dd_words_alloc = 0;
+    int *d_dd_owner = nullptr;     // [n_ghost] internal index of each ghost's owner
+    int64_t dd_owner_alloc = 0;
+    int *d_col_dd = nullptr;       // [cap] list columns as slots
+    int64_t col_dd_alloc = 0;
+
     // per-layer activations
     float *d_A = nullptr;      // [T][n][NA]
     float *d_rho = nullptr;    // [T][n][D]
-    float *d_coef = nullptr;   // [T][n][D]  (layer 0 unused: c^0 comes from C0)
-    float *d_G = nullptr;      // [n][NA]  dE/dA^t
+    float *d_coef = nullptr;   // [T][n_slots][D]  (layer 0 unused: c^0 comes from C0)
+    float *d_G = nullptr;      // [n_slots][NA]  dE/dA^t
     float *d_dc = nullptr;     // [n][D]   dE/dc^t
     float *d_Ei = nullptr;     // [n]
     float *d_F = nullptr;      // [n][3] internal order

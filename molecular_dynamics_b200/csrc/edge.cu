@@ -71,13 +71,12 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 // ---------------------------------------------------------------------------
 // active pairs: the entries of each row closer than r_cut, compacted to the
 // front of the row's slot (same offsets as the full list), each with its
-// displacement and distance (dx, dy, dz, r) and cutoff function f_c(r), which
-// every edge pass of the evaluation then reads instead of recomputing.
+// displacement and distance (dx, dy, dz, r), which every edge pass of the
+// evaluation then reads instead of recomputing.
 __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
-                                                float *__restrict__ act_fc, EdgeParams P,
-                                                unsigned long long *__restrict__ total) {
+                                                EdgeParams P, unsigned long long *__restrict__ total) {
     // one warp per row: lanes test consecutive entries, a ballot compacts the
     // active ones in row order and the writes stay contiguous
     const int lane = threadIdx.x & 31;
@@ -101,10 +100,8 @@ __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict_
         const unsigned mask = __ballot_sync(0xffffffffu, act);
         if (act) {
             const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
-            const float r = sqrtf(r2);
             act_col[o] = j;
-            act_geo[o] = make_float4(d.x, d.y, d.z, r);
-            act_fc[o] = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
+            act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
         }
         k += __popc(mask);
     }
@@ -120,8 +117,9 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(c->d_i64 + 3, 0, sizeof(int64_t), s);
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
-    k_active<<<(unsigned)((c->n + 3) / 4), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, c->d_col, c->d_act_cnt,
-                                                            c->d_act_col, c->d_act_geo, c->d_act_fc, P,
+    k_active<<<(unsigned)((c->n + 3) / 4), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row,
+                                                        c->dd ? c->d_col_dd : c->d_col, c->d_act_cnt,
+                                                            c->d_act_col, c->d_act_geo, P,
                                                             (unsigned long long *)(c->d_i64 + 3));
     return cudaGetLastError();
 }
@@ -145,8 +143,7 @@ struct Lanes {
 template <int NP>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
-                                                     const float4 *__restrict__ act_geo,
-                                                     const float *__restrict__ act_fc, const float4 *__restrict__ pos,
+                                                     const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
                                                      EdgeParams P) {
@@ -171,7 +168,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         const int j = act_col[q];
         const float4 g = act_geo[q];     // dx, dy, dz, r
         const float r = g.w;
-        const float fc = act_fc[q];
+        const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
         float c[3][2];
 #pragma unroll
@@ -353,18 +350,16 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
 cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     if (c->n == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
-    const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
+    const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
     float *rho = c->d_rho + (int64_t)t * c->n * c->D;
     REANN_TIMED(c, REANN_K_DENSITY, s);
     if (c->NP == 8)
         k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_act_fc, c->d_pos, coef, c->d_w, c->ne,
-            A, rho, P);
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
     else if (c->NP == 10)
         k_density_fwd<10><<<(unsigned)((c->n + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_act_fc, c->d_pos, coef, c->d_w, c->ne,
-            A, rho, P);
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
@@ -373,7 +368,7 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
 cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s) {
     if (c->n == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
-    const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n * c->D;
+    const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     const bool has_dc = t >= 1;
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
 #define REANN_EDGE_BWD(NPV, DC)                                                                                  \

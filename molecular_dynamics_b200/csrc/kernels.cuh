@@ -31,6 +31,12 @@ cudaError_t launch_mlp_coef_fwd(reann_ctx *c, int t, cudaStream_t s);   // rho^t
 cudaError_t launch_mlp_energy(reann_ctx *c, cudaStream_t s);            // rho^{T-1} -> E_i, G^{T-1}
 cudaError_t launch_mlp_coef_bwd(reann_ctx *c, int t, cudaStream_t s);   // (rho^{t-1}, dE/dc^t) -> G^{t-1}
 
+// domain-decomposed checking mode (dd.cu)
+cudaError_t dd_plan(reann_ctx *c, cudaStream_t s, int64_t *n_ghost);
+cudaError_t dd_finish(reann_ctx *c, cudaStream_t s);
+cudaError_t dd_gather_rows(reann_ctx *c, float *base, int width, cudaStream_t s);
+cudaError_t dd_stale_coef(reann_ctx *c, float *coef, cudaStream_t s);
+
 // atomic networks on tcgen05 tensor cores, bf16 operands (mlp_tc.cu)
 bool tc_supported(const reann_ctx *c);
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s);

@@ -236,7 +236,7 @@ static MlpNets nets_of(const std::vector<NetOffsets> &v, int first, int ne) {
 cudaError_t launch_mlp_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nD = c->n * c->D;
     return dispatch<MODE_FWD>(c, nets_of(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD,
-                              c->d_coef + (t + 1) * nD, nullptr, nullptr, nullptr, nullptr, s);
+                              c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_mlp_energy(reann_ctx *c, cudaStream_t s) {

@@ -486,8 +486,8 @@ bool tc_supported(const reann_ctx *c) { return (c->NP == 8 || c->NP == 10) && c-
 
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nD = c->n * c->D;
-    return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD, c->d_coef + (t + 1) * nD,
-                               nullptr, nullptr, nullptr, nullptr, s);
+    return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD,
+                               c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s) {

@@ -27,7 +27,7 @@ EXPORTS = ("reann_create", "reann_destroy", "reann_build_neighbors", "reann_ener
            "reann_profile_read", "reann_pair_list_noalloc")
 
 KERNEL_GROUPS = ("active", "density", "mlp_fwd", "mlp_energy", "edge_bwd", "mlp_bwd", "energy_sum", "integrate",
-                 "neighbors", "other")
+                 "neighbors", "other", "ghost")
 
 
 class ReannError(RuntimeError):
@@ -39,7 +39,7 @@ class ReannError(RuntimeError):
 class Config(C.Structure):
     _fields_ = [("n_elements", C.c_int32), ("T", C.c_int32), ("n_radial", C.c_int32), ("l_max", C.c_int32),
                 ("hidden", C.c_int32 * 2), ("r_cut", C.c_double), ("skin", C.c_double), ("alpha", C.c_double),
-                ("mlp_precision", C.c_int32), ("dd_grid", C.c_int32 * 3)]
+                ("mlp_precision", C.c_int32), ("dd_grid", C.c_int32 * 3), ("dd_stale_ghosts", C.c_int32)]
 
 
 class MdStats(C.Structure):
@@ -139,11 +139,14 @@ class ModelSpec:
     alpha: float
     mlp_precision: int = 0
     dd_grid: Sequence[int] = (0, 0, 0)
+    dd_stale_ghosts: int = 0
 
     @classmethod
-    def from_preset(cls, p, T: Optional[int] = None, mlp_precision: Optional[int] = None, dd_grid=(0, 0, 0)):
+    def from_preset(cls, p, T: Optional[int] = None, mlp_precision: Optional[int] = None, dd_grid=(0, 0, 0),
+                    dd_stale_ghosts: int = 0):
         return cls(p.n_elements, p.T if T is None else T, p.n_radial, p.l_max, tuple(p.hidden), p.r_cut, p.skin,
-                   p.alpha, p.mlp_precision if mlp_precision is None else mlp_precision, tuple(dd_grid))
+                   p.alpha, p.mlp_precision if mlp_precision is None else mlp_precision, tuple(dd_grid),
+                   dd_stale_ghosts)
 
     def config(self) -> Config:
         c = Config()
@@ -153,6 +156,7 @@ class ModelSpec:
         c.mlp_precision = self.mlp_precision
         for k in range(3):
             c.dd_grid[k] = self.dd_grid[k]
+        c.dd_stale_ghosts = self.dd_stale_ghosts
         return c
 
 
