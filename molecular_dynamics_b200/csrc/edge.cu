@@ -85,25 +85,31 @@ __global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict_
     const float4 pi = pos[i];
     const int q0 = row[i], q1 = row[i + 1];
     int k = 0;
-    for (int base = q0; base < q1; base += 32) {
-        const int q = base + lane;
-        bool act = false;
-        int j = 0;
-        float3 d = make_float3(0.f, 0.f, 0.f);
-        float r2 = 0.f;
-        if (q < q1) {
-            j = col[q];
-            d = displacement(pi, pos[j], P);
-            r2 = d.x * d.x + d.y * d.y + d.z * d.z;
-            act = r2 < P.r_cut2;
+    constexpr int B = 4;   // entries per lane whose loads are issued together
+    for (int base = q0; base < q1; base += 32 * B) {
+        int j[B];
+        float4 pj[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int q = base + 32 * b + lane;
+            j[b] = q < q1 ? col[q] : -1;
         }
-        const unsigned mask = __ballot_sync(0xffffffffu, act);
-        if (act) {
-            const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
-            act_col[o] = j;
-            act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+#pragma unroll
+        for (int b = 0; b < B; ++b) pj[b] = j[b] >= 0 ? pos[j[b]] : pi;
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            if (base + 32 * b >= q1) break;
+            const float3 d = displacement(pi, pj[b], P);
+            const float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
+            const bool act = j[b] >= 0 && r2 < P.r_cut2;
+            const unsigned mask = __ballot_sync(0xffffffffu, act);
+            if (act) {
+                const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
+                act_col[o] = j[b];
+                act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+            }
+            k += __popc(mask);
         }
-        k += __popc(mask);
     }
     if (lane == 0) {
         act_cnt[i] = k;
@@ -164,9 +170,16 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = 0.f;
     const int q0 = row[i], q1 = q0 + act_cnt[i];
+    int j_next = q0 < q1 ? act_col[q0] : 0;
+    float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int q = q0; q < q1; ++q) {
-        const int j = act_col[q];
-        const float4 g = act_geo[q];     // dx, dy, dz, r
+        // the next edge's index and geometry are in flight while this one computes
+        const int j = j_next;
+        const float4 g = g_next;         // dx, dy, dz, r
+        if (q + 1 < q1) {
+            j_next = act_col[q + 1];
+            g_next = act_geo[q + 1];
+        }
         const float r = g.w;
         const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
@@ -247,9 +260,16 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             }
         }
         const int q0 = row[i], q1 = q0 + act_cnt[i];
+        int j_next = q0 < q1 ? act_col[q0] : 0;
+        float4 geo_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; ++q) {
-            const int j = act_col[q];
-            const float4 geo = act_geo[q];
+            // the next edge's index and geometry are in flight while this one computes
+            const int j = j_next;
+            const float4 geo = geo_next;
+            if (q + 1 < q1) {
+                j_next = act_col[q + 1];
+                geo_next = act_geo[q + 1];
+            }
             const float3 d = make_float3(geo.x, geo.y, geo.z);
             const float r = geo.w;
             const float inv_r = __fdividef(1.0f, r);

@@ -251,6 +251,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncthreads();
     };
 
+    // raw inputs of this thread's row and column half for the next tile, loaded
+    // while the current tile computes
+    constexpr int HC = KPAD / 2;
+    float xr[HC], dr[HC];
+    auto prefetch = [&](int t2) {
+        int4 tl = t2 < n_tiles ? tiles[t2] : make_int4(0, 0, 0, 0);
+        const bool live = row < tl.z;
+        const int64_t gi = (int64_t)(tl.y + row);
+#pragma unroll
+        for (int u = 0; u < HC; ++u) {
+            const int f = half * HC + u;
+            const bool ok = live && f < D;
+            xr[u] = ok ? X[gi * D + f] : 0.f;
+            dr[u] = (MODE == TC_BWD && ok) ? dY[gi * D + f] : 0.f;
+        }
+    };
+    prefetch(blockIdx.x);
+
     for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
         const int4 tile = tiles[ti];
         const int e = tile.x, r0 = tile.y, rows = tile.z;
@@ -283,21 +301,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // input tile: standardised rho (and the upstream gradient), split bf16
         {
             const bool live = row < rows;
-            const int64_t gi = (int64_t)(r0 + row);
 #pragma unroll
-            for (int c = half * (KPAD / 2); c < (half + 1) * (KPAD / 2); c += 8) {
+            for (int c8 = 0; c8 < HC; c8 += 8) {
+                const int c = half * HC + c8;
                 float v[8], g[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int f = c + u;
                     const bool ok = live && f < D;
-                    v[u] = ok ? (X[gi * D + f] - sshift[f]) / sscale[f] : 0.f;
-                    g[u] = (MODE == TC_BWD && ok) ? dY[gi * D + f] : 0.f;
+                    v[u] = ok ? (xr[c8 + u] - sshift[f]) / sscale[f] : 0.f;
+                    g[u] = dr[c8 + u];
                 }
                 st_chunk2(x_hi, x_lo, TM, row, c, v);
                 if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, c, g);
             }
         }
+        prefetch(ti + gridDim.x);
         handoff();
 
         // layer 1 (and, for the coefficient backward, dE/da2 = dY W3 via the MN-major view of W3)
