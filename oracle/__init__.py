@@ -50,20 +50,53 @@ class Cfg(C.Structure):
 _lib = None
 
 
+def _bind(cdll):
+    _bind_signatures(cdll)
+    return cdll
+
+
 def lib():
     global _lib
     if _lib is None:
-        _lib = C.CDLL(build())
-        P = C.c_void_p
-        _lib.oracle_pairs_brute.argtypes = [C.c_int64, P, P, C.c_double, C.c_double, C.c_int64, P, C.c_int64, P, P, P]
-        _lib.oracle_pairs_cells.argtypes = [C.c_int64, P, P, C.c_double, C.c_double, C.c_int64, P, P, P]
-        _lib.oracle_energy_forces.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, P, P, P, P, P, P]
-        _lib.oracle_rho_pairwise.argtypes = [P, C.c_int64, P, P, P, P, P, P]
-        _lib.oracle_md_verlet.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, C.c_double, C.c_int32, P, P]
-        _lib.oracle_weight_count.argtypes = [P]
-        _lib.oracle_weight_count.restype = C.c_int64
-        _lib.oracle_num_threads.restype = C.c_int
+        _lib = _bind(C.CDLL(build()))
     return _lib
+
+
+class use_library:
+    """Temporarily route every oracle call through another build of the C
+    source (the planted-mistake tests compile deliberately broken copies)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = _bind(C.CDLL(self.path))
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+
+
+def compile_source(src: str, out: str) -> str:
+    """Compile an oracle C source with the oracle's own flags."""
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-std=c99", "-D_DEFAULT_SOURCE",
+                           "-shared", "-fPIC", "-o", out, src, "-lm"])
+    return out
+
+
+def _bind_signatures(cdll):
+    P = C.c_void_p
+    cdll.oracle_pairs_brute.argtypes = [C.c_int64, P, P, C.c_double, C.c_double, C.c_int64, P, C.c_int64, P, P, P]
+    cdll.oracle_pairs_cells.argtypes = [C.c_int64, P, P, C.c_double, C.c_double, C.c_int64, P, P, P]
+    cdll.oracle_energy_forces.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, P, P, P, P, P, P]
+    cdll.oracle_rho_pairwise.argtypes = [P, C.c_int64, P, P, P, P, P, P]
+    cdll.oracle_md_verlet.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, C.c_double, C.c_int32, P, P]
+    cdll.oracle_weight_count.argtypes = [P]
+    cdll.oracle_weight_count.restype = C.c_int64
+    cdll.oracle_num_threads.restype = C.c_int
 
 
 def num_threads() -> int:

@@ -1,0 +1,62 @@
+"""The oracle's pins have teeth: plausible mistakes planted into a copy of
+the oracle's C source (a dropped term, a wrong sign, a transposed operand, a
+wrong index or layer) must each make at least one pin fail.
+
+Each case patches one expression of oracle/reann_oracle.c, compiles the copy,
+routes the oracle through it and runs an existing pin test expecting an
+AssertionError.  The real oracle is restored afterwards.  Everything here is
+CPU only.
+"""
+import os
+
+import pytest
+
+import oracle
+import test_oracle_density as dens
+import test_oracle_forces as forc
+import test_oracle_pairs as pairs
+
+MUTANTS = [
+    ("multinomial weight dropped",
+     "return factorial(t[0] + t[1] + t[2]) / (factorial(t[0]) * factorial(t[1]) * factorial(t[2]));",
+     "return 1.0;",
+     lambda: dens.test_density_matches_multinomial_formula_every_layer("ag256")),
+    ("force on the centre with the wrong sign",
+     "gx[i * 3 + a] -= V[a];", "gx[i * 3 + a] += V[a];",
+     lambda: forc.test_zero_net_force("ag256")),
+    ("second hidden layer transposed",
+     "(double)v->W2[(int64_t)h * H1 + k] * a1[k]", "(double)v->W2[(int64_t)k * H1 + h] * a1[k]",
+     lambda: dens.test_t1_energy_is_the_local_eann_network_on_closed_form_density()),
+    ("feature index (n, l) swapped",
+     "coef[j * D + tuple_l(tau) * NP + nn]", "coef[j * D + nn * 3 + tuple_l(tau)]",
+     lambda: dens.test_dimer_closed_form(2.9)),
+    ("cutoff derivative dropped",
+     "double dfc = -0.5 * (pi / c->r_cut) * sin(pi * r / c->r_cut);", "double dfc = 0.0;",
+     lambda: forc.test_forces_match_central_differences("ag256", 10)),
+    ("minimum image dropped",
+     "v = v - box[a] * rint(v / box[a]);", "v = v;",
+     lambda: pairs.test_fcc_shell_counts(4.09, 6.0, 78, 54)),
+    ("energy read from the wrong layer",
+     "&rho[((T - 1) * n + i) * D], a1, a2, &Ei[i]", "&rho[((T > 1 ? T - 2 : 0) * n + i) * D], a1, a2, &Ei[i]",
+     lambda: forc.test_receptive_field_is_T_hops(2)),
+    ("tanh derivative wrong",
+     "g2[k] = s * (1.0 - a2[k] * a2[k]);", "g2[k] = s * (1.0 - a2[k]);",
+     lambda: forc.test_forces_match_central_differences("water", 10)),
+    ("input standardisation dropped in the backward",
+     "gx[f] = s / (double)v->scale[f];", "gx[f] = s;",
+     lambda: forc.test_forces_match_central_differences("hea", 10)),
+]
+
+
+@pytest.mark.parametrize("name,old,new,pin", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new, pin, tmp_path):
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation site not found once: {old}"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.compile_source(str(path), str(tmp_path / "libmutant.so"))
+    with oracle.use_library(lib):
+        with pytest.raises(AssertionError):
+            pin()
+    # the real oracle still passes the same pin
+    pin()
