@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from molecular_dynamics_b200 import presets, synth  # noqa: E402
+from molecular_dynamics_b200.ranks import RankGroup, RankInfo, cuda_event_clock, timed_region  # noqa: E402
 
 METRIC = "atom-steps/s (MD step = E+F, T=3)"
 UNIT = "atom-steps/s"
@@ -51,6 +52,7 @@ FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without d
 # profiles/k_edge_bwd_ag256k.md (256,000 atoms), scaled to the atom count of the
 # run; None when the kernel has changed since that capture
 EDGE_BWD_TRAFFIC_PER_ATOM = (446.367488e6 + 26.646272e6) / 256000
+EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom capture scaled by the atom count"
 
 
 def peaks():
@@ -200,16 +202,47 @@ def dd_sweep(args):
     return 0
 
 
+def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk):
+    """Roofline entry of the dominant kernel group: algorithmic FP32 operations
+    per launch (per-pair counts x active pairs) over its mean CUDA-event launch
+    time, against the FP32 FMA peak of the SM count at clocks.max.sm."""
+    shares = {k: v_[0] for k, v_ in prof.items()}
+    dominant = max(shares, key=shares.get)
+    if dominant == "edge_bwd":
+        flop_per_launch = active_pairs * (FLOP_EDGE_BWD_PER_PAIR[NP][0] + (T - 1) * FLOP_EDGE_BWD_PER_PAIR[NP][1]) / T
+    elif dominant == "density":
+        flop_per_launch = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
+    else:
+        return None
+    ms_dom, n_dom = prof[dominant]
+    if not n_dom:
+        return None
+    smax = pk.get("sm_max_mhz", 1965.0)
+    clock_mhz = clk.get("sm_mhz") or smax
+    peak_tf = sm_count * 128 * 2 * smax * 1e6 / 1e12
+    achieved = flop_per_launch / (ms_dom / n_dom * 1e-3) / 1e12
+    traffic = None
+    if dominant == "edge_bwd" and EDGE_BWD_TRAFFIC_PER_ATOM is not None:
+        traffic = EDGE_BWD_TRAFFIC_PER_ATOM * n_atoms
+    return {"kernel": {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}[dominant], "bound": "alu",
+            "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+            "traffic": traffic,
+            "traffic_note": EDGE_BWD_TRAFFIC_NOTE,
+            "peak_note": f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {smax:.0f} MHz "
+                         f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz",
+            "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--workload", default="ag1m", choices=presets.ORDER)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-steps", type=int, default=16)
+    ap.add_argument("--cpu-steps", type=int, default=64)
     ap.add_argument("--dd-sweep", action="store_true",
                     help="monolithic vs domain-decomposed E+F for T = 1..6 (one JSON line per T)")
     ap.add_argument("--dd-grid", default="8x8x8")
@@ -217,23 +250,17 @@ def main():
                     help="FCC workloads: cells per axis (smaller lattices for profiling captures)")
     args = ap.parse_args()
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    info = RankInfo.from_env()
     if args.impl == "reference":
-        return run_reference(args, rank, world)
+        return run_reference(args, info.rank, info.world)
     if args.dd_sweep:
         return dd_sweep(args)
 
     import torch
     from molecular_dynamics_b200 import reann
 
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(info.local)
+    group = RankGroup.init(info, "nccl")
 
     p = presets.get(args.workload)
     if args.ncell:
@@ -243,47 +270,32 @@ def main():
     n = len(pos)
     dt_fs = 1.0   # the metric's step (the water workload's own 0.5 fs is reported beside it)
     spec = reann.ModelSpec.from_preset(p)   # the workload's own network precision (bf16 for ag1m)
-    ctx = reann.Context(spec, synth.weight_blob(p), device=local)
+    ctx = reann.Context(spec, synth.weight_blob(p), device=info.local)
     stream = torch.cuda.current_stream()
+    clock = cuda_event_clock(stream)
     x = torch.from_numpy(pos.astype(np.float64)).cuda()
     v = torch.from_numpy(v0.copy()).cuda()
     ctx.reann_build_neighbors(torch.from_numpy(pos).cuda(), torch.from_numpy(types).cuda(), box)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(val):
-        if dist is None:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # warm-up (the first call also evaluates the entry forces)
     ctx.reann_md_step(args.warmup, dt_fs, x, v, p.masses)
     torch.cuda.synchronize()
 
     # ---- device-resident timed region: K steps in one call (a continuation)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(info.local)
     launches0 = ctx.reann_get_counters().kernel_launches
     ctx.reann_profile(True)
-    barrier()
-    torch.cuda.synchronize()
     clocks.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    st = ctx.reann_md_step(args.steps, dt_fs, x, v, p.masses)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    run = timed_region(group, lambda: ctx.reann_md_step(args.steps, dt_fs, x, v, p.masses), clock,
+                       n * args.steps)
     clk = clocks.stop()
-    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    st = run.result
+    t_ms = run.ms
+    value = run.throughput
     prof = ctx.reann_profile_read()
     ctx.reann_profile(False)
     cnt = ctx.reann_get_counters()
     launches = cnt.kernel_launches - launches0
-    value = world * n * args.steps / (t_ms * 1e-3)
 
     # ---- end to end: one public call per step with pinned host state
     e2e = None
@@ -293,53 +305,27 @@ def main():
         xh.copy_(x.cpu())
         vh.copy_(v.cpu())
         ctx.reann_md_step(1, dt_fs, xh.numpy(), vh.numpy(), p.masses)      # warm the host path
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            ctx.reann_md_step(1, dt_fs, xh.numpy(), vh.numpy(), p.masses)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        te = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": world * n * args.steps / (te * 1e-3), "unit": UNIT,
+
+        def host_steps():
+            for _ in range(args.steps):
+                ctx.reann_md_step(1, dt_fs, xh.numpy(), vh.numpy(), p.masses)
+
+        run_e = timed_region(group, host_steps, clock, n * args.steps)
+        e2e = {"value": run_e.throughput, "unit": UNIT,
                "h2d_bytes_per_step": 2 * 3 * 8 * n, "d2h_bytes_per_step": 2 * 3 * 8 * n,
                "note": "reann_md_step(1) per step with pinned host x, v: x and v copied in and out every step"}
 
-    if rank != 0:
-        if dist is not None:
-            dist.destroy_process_group()
+    if info.rank != 0:
+        group.close()
         return 0
+    world = info.world
 
     # ---- roofline of the dominant kernel group (FP32-ALU bound edge passes)
     pk, pk_kind = peaks()
-    sm_count = torch.cuda.get_device_properties(local).multi_processor_count
+    sm_count = torch.cuda.get_device_properties(info.local).multi_processor_count
     shares = {k: v_[0] for k, v_ in prof.items()}
     total = sum(shares.values()) or 1.0
-    dominant = max(shares, key=shares.get)
-    active_pairs = cnt.active_pairs
-    NP = p.n_radial
-    T = p.T
-    if dominant == "edge_bwd":
-        flop_per_launch = active_pairs * (FLOP_EDGE_BWD_PER_PAIR[NP][0] + (T - 1) * FLOP_EDGE_BWD_PER_PAIR[NP][1]) / T
-    elif dominant == "density":
-        flop_per_launch = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
-    else:
-        flop_per_launch = None
-    ms_dom, n_dom = prof[dominant]
-    roof = None
-    if flop_per_launch is not None and n_dom:
-        clock_mhz = clk["sm_mhz"] or pk.get("sm_max_mhz", 1965.0)
-        peak_tf = sm_count * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        achieved = flop_per_launch / (ms_dom / n_dom * 1e-3) / 1e12
-        roof = {"kernel": {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}[dominant], "bound": "alu",
-                "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                "traffic": (EDGE_BWD_TRAFFIC_PER_ATOM * n if dominant == "edge_bwd" else None),
-                "traffic_note": "bytes per launch: DRAM read+write of a 256,000-atom capture scaled by the atom count",
-                "peak_note": f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {pk.get('sm_max_mhz', 1965.0):.0f} MHz "
-                             f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz",
-                "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
+    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -365,8 +351,7 @@ def main():
         cb, _ = cpu_sample(args.cpu_steps)
         line["cpu_baseline"] = cb
     print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    group.close()
     return 0
 
 

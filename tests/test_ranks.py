@@ -1,0 +1,107 @@
+"""Replica ranks on the CPU: world-size-2 gloo process groups.
+
+The benchmark runs one independent system per GPU; its only collectives
+bracket the timed region.  These tests run the same host logic with gloo:
+the reported time is the slowest rank's, the units are summed over ranks,
+every rank takes the same collective steps, and the reference arm does its
+work on rank 0 alone.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+import time
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+from molecular_dynamics_b200.ranks import RankGroup, RankInfo, Timed, host_clock, timed_region  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, sleeps, units, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    info = RankInfo.from_env()
+    group = RankGroup.init(info, "gloo", timeout_s=60)
+    try:
+        res = timed_region(group, lambda: time.sleep(sleeps[rank]) or rank, host_clock, units[rank])
+        # a second region, as the benchmark's end-to-end leg does, on every rank
+        res2 = timed_region(group, lambda: rank * 10, host_clock, units[rank])
+        out.put((rank, res.ms, res.units, res.result, res2.units, res2.result))
+    finally:
+        group.close()
+
+
+def _run(world, sleeps, units):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, sleeps, units, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    rows = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return sorted(rows)
+
+
+def test_two_ranks_max_time_and_summed_units():
+    rows = _run(2, sleeps=[0.05, 0.4], units=[1000.0, 3000.0])
+    ms = [r[1] for r in rows]
+    # both ranks report the same (slowest) time, at least rank 1's own sleep
+    assert ms[0] == ms[1]
+    assert ms[0] >= 400.0
+    for rank, _, u, result, u2, result2 in rows:
+        assert u == 4000.0 and u2 == 4000.0
+        assert result == rank and result2 == 10 * rank
+
+
+def test_single_process_group_is_identity():
+    g = RankGroup()
+    res = timed_region(g, lambda: 7, lambda run: (12.5, run()), 100.0)
+    assert res.ms == 12.5 and res.units == 100.0 and res.result == 7
+    assert res.throughput == pytest.approx(100.0 / 12.5e-3)
+
+
+def test_throughput_is_whole_job():
+    # replicas: value = units of all ranks / the slowest rank's time
+    t = Timed(ms=250.0, units=4 * 1_048_576 * 20, result=None)
+    assert t.throughput == pytest.approx(4 * 1_048_576 * 20 / 0.25)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    t0 = time.perf_counter()
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "0", "--gpus", "2"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+    assert time.perf_counter() - t0 < 60
+
+
+def test_roofline_arithmetic():
+    import bench
+    # 10 launches of 3 ms each of the edge backward; T = 3, N_phi = 8
+    prof = {"edge_bwd": (30.0, 10), "density": (9.0, 9), "active": (1.0, 3)}
+    pairs = 1_000_000
+    roof = bench.roofline(prof, pairs, 8, 3, 50_000, 148, {"sm_max_mhz": 2000.0}, "measured", {"sm_mhz": 1900.0})
+    flop = pairs * (bench.FLOP_EDGE_BWD_PER_PAIR[8][0] + 2 * bench.FLOP_EDGE_BWD_PER_PAIR[8][1]) / 3
+    assert roof["kernel"] == "k_edge_bwd" and roof["bound"] == "alu"
+    assert roof["flop_per_launch"] == pytest.approx(flop)
+    assert roof["achieved"] == pytest.approx(flop / 3e-3 / 1e12)
+    assert roof["peak"] == pytest.approx(148 * 128 * 2 * 2000e6 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    # a dominant group with no algorithmic count has no entry
+    assert bench.roofline({"mlp_bwd": (5.0, 1)}, pairs, 8, 3, 1, 148, {}, "fallback", {}) is None
+    json.dumps(roof)
