@@ -12,17 +12,27 @@
 // A tile is 128 atoms of one element.  Each layer is one 128 x N x K GEMM
 // (tcgen05.mma, M = 128, K = 16 per instruction) whose accumulator sits in
 // TMEM; TMEM lane i holds atom i, so the epilogue (bias, tanh, tanh', the
-// energy dot product, dE/dA) is one thread per atom with no cross-thread
-// reduction.  The epilogue writes the next layer's bf16 operand straight into
-// shared memory in the canonical K-major layout, and one thread issues the
-// next MMA.
+// energy dot product) is per atom with no cross-lane reduction.  The epilogue
+// writes the next layer's bf16 operand straight into shared memory in the
+// canonical K-major layout (one activation buffer, reused by every layer once
+// the product that read it has completed), and one thread issues the next MMA.
 //
-// Block: 256 threads; warp w reads TMEM lanes 32 (w % 4) .. + 31 and works on
-// half w / 4 of each accumulator's columns, so a tile row (atom) is shared by
-// two threads.  One block per SM (shared memory > half an SM), persistent
-// over the tiles.  All
-// waits on the MMA-completion barrier are bounded: a wait that gives up sets
-// ST_TIMEOUT, the block frees its tensor memory and returns.
+// Block: 512 threads, one per SM (shared memory > half an SM), persistent over
+// the tiles.  Warp w reads TMEM lanes 32 (w % 4) .. + 31; warp group w / 4
+// takes one 32-column chunk of every 128-wide accumulator, so a tile row is
+// shared by four threads.  The epilogue is bound by the tanh unit: bf16
+// rounding of the split operands is done with integer instructions so that
+// the special-function pipe only evaluates tanh.
+//
+// Global traffic is contiguous: the next tile's raw inputs are prefetched in
+// element order while the current tile computes and transposed to rows through
+// the idle activation buffer; forward outputs leave through the idle input
+// buffer; for the energy network and the coefficient backward the tile's A rows
+// arrive by one bulk copy (cp.async.bulk, completion on an mbarrier) issued at
+// the start of the tile, and dE/dA = 2 w_tau A dE/drho is written one warp per
+// row in the edge kernels' lane-interleaved order.  All waits (MMA completion,
+// bulk copy) are bounded: a wait that gives up sets ST_TIMEOUT, the block waits
+// once more for a copy still in flight, frees its tensor memory and returns.
 //
 // Shared-memory operand layout (K-major, no swizzle): an R x K bf16 tile keeps
 // element (r, k) at byte (k/8) R 16 + (r/8) 128 + (r%8) 16 + (k%8) 2, i.e.
@@ -37,11 +47,14 @@ namespace reann {
 namespace {
 
 constexpr int TM = 128;            // atoms per tile (MMA M)
-constexpr int TC_THREADS = 256;    // two warp groups: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
+constexpr int TC_THREADS = 512;    // four warp groups: warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) ..
 constexpr int KPAD = 32;           // feature dimension padded to a multiple of 16
 constexpr int TMEM_COLS = 512;
 
 enum { TC_FWD = 0, TC_ENERGY = 1, TC_BWD = 2 };
+
+template <int NP>
+__host__ __device__ constexpr int NA_BYTES() { return NP * NT * 4; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -140,27 +153,24 @@ __device__ __forceinline__ float tanh_fast(float x) {
     return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// 8 bf16 values (columns c..c+7 of row r) -> one 16-byte chunk of a K-major tile
-__device__ __forceinline__ void st_chunk(unsigned char *tile, int R, int r, int c, const float *v) {
-    uint4 w = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-    *reinterpret_cast<uint4 *>(tile + kmaj(r, c, R)) = w;
-}
-
-// 8 values as a bf16 pair: hi = bf16(v), lo = bf16(v - hi) (16 significant bits)
+// 8 values (columns c..c+7 of row r) as a bf16 pair, hi = bf16(v) and
+// lo = bf16(v - hi) (16 significant bits), into one 16-byte chunk of each
+// K-major tile.  Rounding to bf16 is done on the bit pattern (add half a bf16
+// ulp, keep the upper 16 bits: round to nearest, ties away from zero), which
+// runs on the integer pipe; v - hi is exact in fp32.
 __device__ __forceinline__ void st_chunk2(unsigned char *hi, unsigned char *lo, int R, int r, int c, const float *v) {
-    float h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        h[u] = __bfloat162float(__float2bfloat16_rn(v[u]));
-        l[u] = v[u] - h[u];
+    for (int u = 0; u < 8; u += 2) {
+        const uint32_t a = __float_as_uint(v[u]) + 0x8000u, b = __float_as_uint(v[u + 1]) + 0x8000u;
+        const float la = v[u] - __uint_as_float(a & 0xFFFF0000u);
+        const float lb = v[u + 1] - __uint_as_float(b & 0xFFFF0000u);
+        h[u / 2] = __byte_perm(a, b, 0x7632);
+        l[u / 2] = __byte_perm(__float_as_uint(la) + 0x8000u, __float_as_uint(lb) + 0x8000u, 0x7632);
     }
-    st_chunk(hi, R, r, c, h);
-    st_chunk(lo, R, r, c, l);
+    const uint32_t off = kmaj(r, c, R);
+    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // one bf16 element of a K-major tile (weight preparation)
@@ -172,24 +182,48 @@ struct TcNets {
     NetOffsets net[MAX_ELEMENTS];
 };
 
+// 8 consecutive fp32 TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+// bulk (non-tensor) copy global -> this CTA's shared memory, completing on an
+// mbarrier; both addresses 16-byte aligned, size a multiple of 16
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 template <int NP, int H1, int H2, int MODE>
 struct TcLayout {
     static constexpr int D = 3 * NP;
     static constexpr int NA = NP * NT;
+    static constexpr bool STAGE = MODE != TC_FWD;   // A tile through shared memory
     // bf16 weight tiles, K-major, one copy each (the backward products read
     // them through the MN-major view)
     static constexpr int W1 = 0;                                 // [H1][KPAD]
     static constexpr int W2 = W1 + H1 * KPAD * 2;                // [H2][H1]
     static constexpr int W3 = W2 + H2 * H1 * 2;                  // [KPAD][H2] (rows >= n_out are zero)
-    // split activation tiles (hi, lo)
+    // split operand tiles (hi, lo)
     static constexpr int X = W3 + KPAD * H2 * 2;                 // [TM][KPAD] x 2
     static constexpr int DY = X + 2 * TM * KPAD * 2;             // [TM][KPAD] x 2 (BWD)
-    static constexpr int A1 = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][H1] x 2
-    static constexpr int A2 = A1 + 2 * TM * H1 * 2;              // [TM][H2] x 2
-    static constexpr int F32 = A2 + 2 * TM * H2 * 2;
-    static constexpr int nf32 = H1 + H2 + KPAD + 3 * KPAD + H2 + 2 * TM;  // b1, b2, b3, shift, scale, 1/scale, w3, e_part
+    static constexpr int ACT = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][128] x 2, every layer
+    // fp32 staging: the tile's A rows ([TM][NA]) and dE/drho ([TM][KPAD + 1])
+    static constexpr int STG = ACT + 2 * TM * 128 * 2;
+    static constexpr int GX = STG + (STAGE ? TM * NA * 4 : 0);
+    static constexpr int GXS = KPAD + 1;                          // padded row stride (no bank conflicts)
+    static constexpr int F32 = GX + (STAGE ? TM * GXS * 4 : 0);
+    static constexpr int nf32 = H1 + H2 + KPAD + 2 * KPAD + H2 + 4 * TM;  // b1, b2, b3, shift, 1/scale, w3, e parts
     static constexpr int BAR = F32 + nf32 * 4;
-    static constexpr int bytes = BAR + 16 + 16;
+    static constexpr int bytes = BAR + 32;
     // TMEM columns
     static constexpr int C_Z1 = 0, C_Z2 = 128, C_P = 256, C_OUT = 384;
 };
@@ -199,23 +233,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     k_mlp_tc(const int4 *__restrict__ tiles, int n_tiles, const float *__restrict__ w, TcNets nets,
              const float *__restrict__ X, float *__restrict__ Y, const float *__restrict__ dY, float *__restrict__ Ei,
              const float *__restrict__ A, float *__restrict__ Gout, int *__restrict__ status) {
+    static_assert(H1 == 4 * 32 && H2 == 4 * 32, "one 32-column chunk per warp group and layer");
     using L = TcLayout<NP, H1, H2, MODE>;
     constexpr int D = L::D, NA = L::NA;
     constexpr int DOUT = MODE == TC_ENERGY ? 1 : D;
     extern __shared__ __align__(1024) unsigned char sm[];
     float *f32 = reinterpret_cast<float *>(sm + L::F32);
-    float *sb1 = f32, *sb2 = sb1 + H1, *sb3 = sb2 + H2, *sshift = sb3 + KPAD, *sscale = sshift + KPAD,
-          *sinv = sscale + KPAD, *sw3 = sinv + KPAD, *se = sw3 + H2;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    float *sb1 = f32, *sb2 = sb1 + H1, *sb3 = sb2 + H2, *sshift = sb3 + KPAD, *sinv = sshift + KPAD,
+          *sw3 = sinv + KPAD, *se = sw3 + H2;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);   // [0] MMA completion, [1] A tile landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
     unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KPAD * 2;
     unsigned char *dy_hi = sm + L::DY, *dy_lo = dy_hi + TM * KPAD * 2;
-    unsigned char *a1_hi = sm + L::A1, *a1_lo = a1_hi + TM * H1 * 2;
-    unsigned char *a2_hi = sm + L::A2, *a2_lo = a2_hi + TM * H2 * 2;
+    unsigned char *act_hi = sm + L::ACT, *act_lo = act_hi + TM * 128 * 2;
+    float *stg = reinterpret_cast<float *>(sm + L::STG);
+    float *gxs = reinterpret_cast<float *>(sm + L::GX);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & (TM - 1);            // this thread's atom within the tile (TMEM lane)
-    const int half = tid / TM;                 // which half of each accumulator's columns
+    const int qc = tid / TM;                   // warp group: columns 32 qc .. 32 qc + 31 of each accumulator
+    const int c = 32 * qc;
     const uint32_t base = smem_u32(sm);
     auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
 
@@ -226,6 +263,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar + 1)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     fence_before();
@@ -233,8 +271,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    uint32_t phase = 0;
-    bool failed = false;
+    uint32_t phase = 0, phase_ld = 0;
+    bool failed = false, load_pending = false;
     int cur = -1;
 
     // completion of the MMA group thread 0 committed, awaited by all threads
@@ -251,26 +289,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncthreads();
     };
 
-    // raw inputs of this thread's row and column half for the next tile, loaded
-    // while the current tile computes
-    constexpr int HC = KPAD / 2;
-    float xr[HC], dr[HC];
+    // raw inputs of the next tile, loaded while the current tile computes:
+    // the tile's rows are contiguous in X (and dY), so thread tid takes
+    // elements tid, tid + 512, ... of that run (coalesced).  The tile
+    // descriptor is read one tile further ahead, so the addresses are known
+    // when the loads issue.
+    constexpr int NXR = (TM * D + TC_THREADS - 1) / TC_THREADS;
+    float xr[NXR], dr[NXR];
+    int4 tl = make_int4(0, 0, 0, 0);                                   // tile whose inputs are in xr
+    int4 tl2 = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);   // the one after
     auto prefetch = [&](int t2) {
-        int4 tl = t2 < n_tiles ? tiles[t2] : make_int4(0, 0, 0, 0);
-        const bool live = row < tl.z;
-        const int64_t gi = (int64_t)(tl.y + row);
+        tl = tl2;
+        const int64_t g0 = (int64_t)tl.y * D;
+        const int cnt = tl.z * D;
 #pragma unroll
-        for (int u = 0; u < HC; ++u) {
-            const int f = half * HC + u;
-            const bool ok = live && f < D;
-            xr[u] = ok ? X[gi * D + f] : 0.f;
-            dr[u] = (MODE == TC_BWD && ok) ? dY[gi * D + f] : 0.f;
+        for (int u = 0; u < NXR; ++u) {
+            const int k = tid + u * TC_THREADS;
+            xr[u] = k < cnt ? X[g0 + k] : 0.f;
+            dr[u] = (MODE == TC_BWD && k < cnt) ? dY[g0 + k] : 0.f;
         }
+        const int t3 = t2 + gridDim.x;
+        tl2 = t3 < n_tiles ? tiles[t3] : make_int4(0, 0, 0, 0);
     };
+    // dE/dA positions of this lane (element pk = lane + 32 j of a row, in the
+    // edge kernels' lane-interleaved order), packed: source A index (bits 0-7),
+    // dE/drho index (bits 8-15), mixed second-order tuple (bit 16: 2 w_tau = 4)
+    constexpr int NJ = (NA + 31) / 32;
+    int posj[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int pk = (tid & 31) + 32 * j;
+        const int src = g_slot_source(pk < NA ? pk : 0, NP), nn = src / NT, u = src - nn * NT;
+        const int gi = (u == 0 ? 0 : (u < 4 ? 1 : 2)) * NP + nn;
+        posj[j] = src | (gi << 8) | ((u >= 7 ? 1 : 0) << 16);
+    }
     prefetch(blockIdx.x);
 
     for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
-        const int4 tile = tiles[ti];
+        const int4 tile = tl;
         const int e = tile.x, r0 = tile.y, rows = tile.z;
         if (e != cur) {
             // element weights -> bf16 tiles and fp32 vectors
@@ -292,29 +348,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int k = tid; k < KPAD; k += TC_THREADS) {
                 sb3[k] = k < DOUT ? w[o.b3 + k] : 0.f;
                 sshift[k] = k < D ? w[o.shift + k] : 0.f;
-                sscale[k] = k < D ? w[o.scale + k] : 1.f;
                 sinv[k] = k < D ? 1.0f / w[o.scale + k] : 0.f;
             }
             cur = e;
         }
+        // the tile's A rows (energy and backward) stream into the staging buffer
+        // while the networks run (the previous tile finished reading it before
+        // the barrier that ended it)
+        if (L::STAGE && tid == 0) {
+            bulk_load(stg, A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4), bar + 1);
+            load_pending = true;
+        }
         __syncthreads();
-        // input tile: standardised rho (and the upstream gradient), split bf16
+        // input tile: raw values -> padded fp32 rows in the (idle) activation
+        // buffer, then standardised rho (and the upstream gradient) split bf16
         {
-            const bool live = row < rows;
+            constexpr int RS = D + 1;   // odd row stride: conflict-free row reads
+            float *xs = reinterpret_cast<float *>(act_hi), *ds = xs + TM * RS;
 #pragma unroll
-            for (int c8 = 0; c8 < HC; c8 += 8) {
-                const int c = half * HC + c8;
-                float v[8], g[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int f = c + u;
-                    const bool ok = live && f < D;
-                    v[u] = ok ? (xr[c8 + u] - sshift[f]) / sscale[f] : 0.f;
-                    g[u] = dr[c8 + u];
+            for (int u = 0; u < NXR; ++u) {
+                const int k = tid + u * TC_THREADS;
+                if (k < rows * D) {
+                    const int rk = k / D, f = k - rk * D;
+                    xs[rk * RS + f] = xr[u];
+                    if (MODE == TC_BWD) ds[rk * RS + f] = dr[u];
                 }
-                st_chunk2(x_hi, x_lo, TM, row, c, v);
-                if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, c, g);
             }
+            __syncthreads();
+            const bool live = row < rows;
+            float v[8], g[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int f = 8 * qc + u;
+                const bool ok = live && f < D;
+                v[u] = ok ? (xs[row * RS + f] - sshift[f]) * sinv[f] : 0.f;
+                g[u] = (MODE == TC_BWD && ok) ? ds[row * RS + f] : 0.f;
+            }
+            st_chunk2(x_hi, x_lo, TM, row, 8 * qc, v);
+            if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, 8 * qc, g);
         }
         prefetch(ti + gridDim.x);
         handoff();
@@ -328,57 +399,62 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!wait_mma()) { failed = true; break; }
         // a1 = tanh(z1 + b1)
-#pragma unroll 1
-        for (int c = half * (H1 / 2); c < (half + 1) * (H1 / 2); c += 32) {
+        {
             float v[32];
             tmem_ld32(lane_base + L::C_Z1 + c, v);
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb1[c + u]);
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) st_chunk2(a1_hi, a1_lo, TM, row, c + u, &v[u]);
+            for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
         }
         handoff();
         if (tid == 0) {
             fence_after();
-            gemm2<H2, H1, false, 0>(tmem + L::C_Z2, sa(a1_hi), sa(a1_lo), base + L::W2);
+            gemm2<H2, H1, false, 0>(tmem + L::C_Z2, sa(act_hi), sa(act_lo), base + L::W2);
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
 
         if (MODE == TC_FWD) {
-            // a2 = tanh(z2 + b2), then y = a2 W3^T + b3
-#pragma unroll 1
-            for (int c = half * (H2 / 2); c < (half + 1) * (H2 / 2); c += 32) {
+            // a2 = tanh(z2 + b2) (the layer-2 product has consumed a1), then y = a2 W3^T + b3
+            {
                 float v[32];
                 tmem_ld32(lane_base + L::C_Z2 + c, v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb2[c + u]);
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) st_chunk2(a2_hi, a2_lo, TM, row, c + u, &v[u]);
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
             }
             handoff();
             if (tid == 0) {
                 fence_after();
-                gemm2<KPAD, H2, false, 0>(tmem + L::C_OUT, sa(a2_hi), sa(a2_lo), base + L::W3);
+                gemm2<KPAD, H2, false, 0>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W3);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            float v[32];
-            tmem_ld32(lane_base + L::C_OUT, v);
-            if (row < rows) {
-                float *yo = Y + (int64_t)(r0 + row) * D;
+            // y rows through the (idle) input tile buffer, then contiguous stores
+            {
+                constexpr int RS = D + 1;
+                float *ys = reinterpret_cast<float *>(x_hi);
+                float v[8];
+                tmem_ld8(lane_base + L::C_OUT + 8 * qc, v);
 #pragma unroll
-                for (int f = 0; f < D; ++f)
-                    if ((f < (D + 1) / 2) == (half == 0)) yo[f] = v[f] + sb3[f];
+                for (int u = 0; u < 8; ++u)
+                    if (8 * qc + u < D) ys[row * RS + 8 * qc + u] = v[u] + sb3[8 * qc + u];
+                __syncthreads();
+                float *yo = Y + (int64_t)r0 * D;
+                for (int k = tid; k < rows * D; k += TC_THREADS) {
+                    const int rk = k / D;
+                    yo[k] = ys[rk * RS + (k - rk * D)];
+                }
             }
         } else {
             // g2 = dE/dz2 = (energy: w3, backward: dY W3) * (1 - a2^2); energy E_i = w3 . a2 + b3
-            float e_row = 0.f;
-#pragma unroll 1
-            for (int c = half * (H2 / 2); c < (half + 1) * (H2 / 2); c += 32) {
+            {
                 float z[32], up[32];
                 tmem_ld32(lane_base + L::C_Z2 + c, z);
                 if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P + c, up);
+                float e_row = 0.f;
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                     const float a = tanh_fast(z[u] + sb2[c + u]);
@@ -387,21 +463,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     z[u] = g * (1.f - a * a);
                 }
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) st_chunk2(a2_hi, a2_lo, TM, row, c + u, &z[u]);
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &z[u]);
+                if (MODE == TC_ENERGY) se[qc * TM + row] = e_row;
             }
-            if (MODE == TC_ENERGY) se[half * TM + row] = e_row;
             handoff();
-            if (MODE == TC_ENERGY && half == 0 && row < rows) Ei[r0 + row] = se[row] + se[TM + row] + sb3[0];
+            if (MODE == TC_ENERGY && qc == 0 && row < rows)
+                Ei[r0 + row] = ((se[row] + se[TM + row]) + (se[2 * TM + row] + se[3 * TM + row])) + sb3[0];
             // p1 = g2 W2 (MN-major view of W2), into the columns dY W3 used
             if (tid == 0) {
                 fence_after();
-                gemm2<H1, H2, true, H2>(tmem + L::C_P, sa(a2_hi), sa(a2_lo), base + L::W2);
+                gemm2<H1, H2, true, H2>(tmem + L::C_P, sa(act_hi), sa(act_lo), base + L::W2);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
             // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation still in TMEM
-#pragma unroll 1
-            for (int c = half * (H1 / 2); c < (half + 1) * (H1 / 2); c += 32) {
+            {
                 float p[32], z[32];
                 tmem_ld32(lane_base + L::C_P + c, p);
                 tmem_ld32(lane_base + L::C_Z1 + c, z);
@@ -411,45 +487,38 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     p[u] *= 1.f - a * a;
                 }
 #pragma unroll
-                for (int u = 0; u < 32; u += 8) st_chunk2(a1_hi, a1_lo, TM, row, c + u, &p[u]);
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &p[u]);
             }
             handoff();
             // dE/dx = g1 W1 (MN-major view of W1)
             if (tid == 0) {
                 fence_after();
-                gemm2<KPAD, H1, true, H1>(tmem + L::C_OUT, sa(a1_hi), sa(a1_lo), base + L::W1);
+                gemm2<KPAD, H1, true, H1>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W1);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            // dE/drho = (g1 W1) / scale; G = dE/dA = 2 w_tau A dE/drho
-            float gx[32];
-            tmem_ld32(lane_base + L::C_OUT, gx);
-            if (row < rows) {
+            // dE/drho = (g1 W1) / scale, shared by the row's four threads
+            {
+                float v[8];
+                tmem_ld8(lane_base + L::C_OUT + 8 * qc, v);
 #pragma unroll
-                for (int f = 0; f < D; ++f) gx[f] *= sinv[f];
-                const int64_t gi = (int64_t)(r0 + row) * NA;
-                const float4 *a4 = reinterpret_cast<const float4 *>(A + gi);
-                float4 *g4 = reinterpret_cast<float4 *>(Gout + gi);
-                float av[NA];
+                for (int u = 0; u < 8; ++u) gxs[row * L::GXS + 8 * qc + u] = v[u] * sinv[8 * qc + u];
+            }
+            const bool landed = bar_wait(bar + 1, phase_ld);
+            if (__syncthreads_or(!landed)) { failed = true; break; }
+            phase_ld ^= 1u;
+            if (tid == 0) load_pending = false;
+            // G = dE/dA = 2 w_tau A dE/drho, warp per row, lanes along the row in
+            // the edge kernels' lane-interleaved order (contiguous stores)
+            float *go = Gout + (int64_t)r0 * NA;
+            for (int rk = warp; rk < rows; rk += TC_THREADS / 32) {
+                const float *ar = stg + rk * NA, *gr = gxs + rk * L::GXS;
+                float *orow = go + (int64_t)rk * NA;
 #pragma unroll
-                for (int q = 0; q < NA / 4; ++q) {
-                    const float4 a = a4[q];
-                    av[4 * q] = a.x; av[4 * q + 1] = a.y; av[4 * q + 2] = a.z; av[4 * q + 3] = a.w;
-                }
-                // G rows in the edge kernels' lane-interleaved order; each half writes half of the row
-                constexpr int QS = (NA / 4 + 1) / 2;
-#pragma unroll
-                for (int q = 0; q < NA / 4; ++q) {
-                    if ((q < QS) != (half == 0)) continue;
-                    float gv[4];
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const int src = g_slot_source(4 * q + s, NP), nn = src / NT, u = src % NT;
-                        const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
-                        const float wt = u >= 7 ? 4.f : 2.f;
-                        gv[s] = wt * av[src] * gx[l * NP + nn];
-                    }
-                    g4[q] = make_float4(gv[0], gv[1], gv[2], gv[3]);
+                for (int j = 0; j < NJ; ++j) {
+                    const int pk = (tid & 31) + 32 * j;
+                    const int c = posj[j];
+                    if (pk < NA) orow[pk] = ((c >> 16) ? 4.f : 2.f) * ar[c & 255] * gr[(c >> 8) & 255];
                 }
             }
         }
@@ -457,7 +526,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncthreads();
     }
 
-    if (failed && tid == 0) atomicOr(status, ST_TIMEOUT);
+    if (tid == 0) {
+        if (failed) atomicOr(status, ST_TIMEOUT);
+        // a tile load that never completed: wait for it once more, with the same bound
+        if (load_pending) bar_wait(bar + 1, phase_ld);
+    }
     fence_before();
     __syncthreads();
     fence_after();
@@ -469,6 +542,8 @@ cudaError_t run_tc(reann_ctx *c, const TcNets &nets, const float *X, float *Y, c
                    const float *A, float *G, cudaStream_t s) {
     using L = TcLayout<NP, H1, H2, MODE>;
     static_assert(L::bytes > 116 * 1024 && L::bytes <= 227 * 1024, "one block per SM keeps TMEM allocation safe");
+    static_assert(L::STG % 16 == 0 && L::GX % 16 == 0 && L::BAR % 16 == 0, "bulk copies need 16-byte alignment");
+    static_assert((NA_BYTES<NP>() % 16) == 0, "A rows must be whole 16-byte units for the bulk copy");
     static bool configured[64] = {};
     auto kern = k_mlp_tc<NP, H1, H2, MODE>;
     if (c->device < 0 || c->device >= 64) return cudaErrorInvalidDevice;
