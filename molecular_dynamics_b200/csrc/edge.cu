@@ -26,6 +26,8 @@
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -73,48 +75,49 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 // front of the row's slot (same offsets as the full list), each with its
 // displacement and distance (dx, dy, dz, r), which every edge pass of the
 // evaluation then reads instead of recomputing.
-__global__ void __launch_bounds__(128) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
+__global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
                                                 EdgeParams P, unsigned long long *__restrict__ total) {
     // one warp per row: lanes test consecutive entries, a ballot compacts the
-    // active ones in row order and the writes stay contiguous
+    // active ones in row order and the writes stay contiguous.  Warps stride
+    // over the rows and add their count of active pairs to the total once.
     const int lane = threadIdx.x & 31;
-    const int i = blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (i >= n) return;
-    const float4 pi = pos[i];
-    const int q0 = row[i], q1 = row[i + 1];
-    int k = 0;
-    constexpr int B = 4;   // entries per lane whose loads are issued together
-    for (int base = q0; base < q1; base += 32 * B) {
-        int j[B];
-        float4 pj[B];
+    unsigned long long tot = 0;
+    for (int i = blockIdx.x * 4 + (threadIdx.x >> 5); i < n; i += gridDim.x * 4) {
+        const float4 pi = pos[i];
+        const int q0 = row[i], q1 = row[i + 1];
+        int k = 0;
+        constexpr int B = 4;   // entries per lane whose loads are issued together
+        for (int base = q0; base < q1; base += 32 * B) {
+            int j[B];
+            float4 pj[B];
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-            const int q = base + 32 * b + lane;
-            j[b] = q < q1 ? col[q] : -1;
-        }
-#pragma unroll
-        for (int b = 0; b < B; ++b) pj[b] = j[b] >= 0 ? pos[j[b]] : pi;
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            if (base + 32 * b >= q1) break;
-            const float3 d = displacement(pi, pj[b], P);
-            const float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
-            const bool act = j[b] >= 0 && r2 < P.r_cut2;
-            const unsigned mask = __ballot_sync(0xffffffffu, act);
-            if (act) {
-                const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
-                act_col[o] = j[b];
-                act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+            for (int b = 0; b < B; ++b) {
+                const int q = base + 32 * b + lane;
+                j[b] = q < q1 ? col[q] : -1;
             }
-            k += __popc(mask);
+#pragma unroll
+            for (int b = 0; b < B; ++b) pj[b] = j[b] >= 0 ? pos[j[b]] : pi;
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+                if (base + 32 * b >= q1) break;
+                const float3 d = displacement(pi, pj[b], P);
+                const float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
+                const bool act = j[b] >= 0 && r2 < P.r_cut2;
+                const unsigned mask = __ballot_sync(0xffffffffu, act);
+                if (act) {
+                    const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
+                    act_col[o] = j[b];
+                    act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+                }
+                k += __popc(mask);
+            }
         }
+        if (lane == 0) act_cnt[i] = k;
+        tot += (unsigned long long)k;
     }
-    if (lane == 0) {
-        act_cnt[i] = k;
-        atomicAdd(total, (unsigned long long)k);
-    }
+    if (lane == 0 && tot) atomicAdd(total, tot);
 }
 
 cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
@@ -123,7 +126,9 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(c->d_i64 + 3, 0, sizeof(int64_t), s);
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
-    k_active<<<(unsigned)((c->n + 3) / 4), 128, 0, s>>>((int)c->n, c->d_pos, c->d_row,
+    // one resident wave (8 blocks of 128 threads per SM at <= 64 registers)
+    const unsigned grid = (unsigned)std::min<int64_t>((c->n + 3) / 4, (int64_t)c->sm_count * 8);
+    k_active<<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row,
                                                         c->dd ? c->d_col_dd : c->d_col, c->d_act_cnt,
                                                             c->d_act_col, c->d_act_geo, P,
                                                             (unsigned long long *)(c->d_i64 + 3));
