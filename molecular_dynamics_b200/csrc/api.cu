@@ -246,18 +246,36 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
             CK(dalloc(&c->d_tiles, tiles.size()));
             c->n_tiles_alloc = (int)tiles.size();
         }
-        if ((int)tiles128.size() > c->n_tiles128_alloc) {
-            CK(dalloc(&c->d_tiles128, tiles128.size()));
-            c->n_tiles128_alloc = (int)tiles128.size();
+        // block ranges of the tensor-core networks, stored after the 128-row
+        // tiles: each block takes a contiguous run of one element's tiles (its
+        // weights are loaded once), at most one block per SM
+        const int n128 = (int)tiles128.size();
+        std::vector<int4> table(tiles128);
+        if (n128) {
+            const int blocks = std::max(1, c->sm_count - c->ne);
+            const int per = (n128 + blocks - 1) / blocks;
+            for (int t = 0; t < n128;) {
+                int u = t;
+                while (u < n128 && tiles128[u].x == tiles128[t].x) ++u;
+                const int k = (u - t + per - 1) / per;
+                for (int b = 0; b < k; ++b)
+                    table.push_back(make_int4(t + (int)((int64_t)(u - t) * b / k),
+                                              t + (int)((int64_t)(u - t) * (b + 1) / k), tiles128[t].x, 0));
+                t = u;
+            }
+        }
+        if ((int)table.size() > c->n_tiles128_alloc) {
+            CK(dalloc(&c->d_tiles128, table.size()));
+            c->n_tiles128_alloc = (int)table.size();
         }
         if (!tiles.empty())
             CK(cudaMemcpyAsync(c->d_tiles, tiles.data(), sizeof(int4) * tiles.size(), cudaMemcpyHostToDevice, s));
-        if (!tiles128.empty())
-            CK(cudaMemcpyAsync(c->d_tiles128, tiles128.data(), sizeof(int4) * tiles128.size(),
-                               cudaMemcpyHostToDevice, s));
+        if (!table.empty())
+            CK(cudaMemcpyAsync(c->d_tiles128, table.data(), sizeof(int4) * table.size(), cudaMemcpyHostToDevice, s));
         CK(sync_stream(c, s));
         c->n_tiles = (int)tiles.size();
-        c->n_tiles128 = (int)tiles128.size();
+        c->n_tiles128 = n128;
+        c->n_tc_ranges = (int)table.size() - n128;
         c->elem_start.assign(c->h_seg, c->h_seg + c->ne + 1);
     }
     c->n_slots = c->n;

@@ -146,6 +146,7 @@ struct reann_ctx {
     int n_tiles = 0, n_tiles_alloc = 0;
     int4 *d_tiles128 = nullptr;
     int n_tiles128 = 0, n_tiles128_alloc = 0;
+    int n_tc_ranges = 0;   // tensor-core network blocks; their ranges follow the 128-row tiles
 
     // staging for host arrays and caller-order scratch
     float *d_stage_f = nullptr;    // [n][3] floats

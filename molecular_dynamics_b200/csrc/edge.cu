@@ -81,12 +81,22 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
                                                 EdgeParams P, unsigned long long *__restrict__ total) {
     // one warp per row: lanes test consecutive entries, a ballot compacts the
     // active ones in row order and the writes stay contiguous.  Warps stride
-    // over the rows and add their count of active pairs to the total once.
+    // over the rows (the next row's position and bounds are loaded while the
+    // current one is tested) and add their count of active pairs to the total once.
     const int lane = threadIdx.x & 31;
     unsigned long long tot = 0;
-    for (int i = blockIdx.x * 4 + (threadIdx.x >> 5); i < n; i += gridDim.x * 4) {
-        const float4 pi = pos[i];
-        const int q0 = row[i], q1 = row[i + 1];
+    int i = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int stride = gridDim.x * 4;
+    float4 pi_n = i < n ? pos[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    int q0_n = i < n ? row[i] : 0, q1_n = i < n ? row[i + 1] : 0;
+    for (; i < n; i += stride) {
+        const float4 pi = pi_n;
+        const int q0 = q0_n, q1 = q1_n;
+        if (i + stride < n) {
+            pi_n = pos[i + stride];
+            q0_n = row[i + stride];
+            q1_n = row[i + stride + 1];
+        }
         int k = 0;
         constexpr int B = 4;   // entries per lane whose loads are issued together
         for (int base = q0; base < q1; base += 32 * B) {

@@ -47,7 +47,8 @@ namespace reann {
 namespace {
 
 constexpr int TM = 128;            // atoms per tile (MMA M)
-constexpr int TC_THREADS = 512;    // four warp groups: warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) ..
+constexpr int TC_THREADS = 512;    // two independent groups of 256 threads
+constexpr int TC_GROUP = 256;
 constexpr int KPAD = 32;           // feature dimension padded to a multiple of 16
 constexpr int TMEM_COLS = 512;
 
@@ -193,124 +194,156 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
     for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// bulk (non-tensor) copy global -> this CTA's shared memory, completing on an
-// mbarrier; both addresses 16-byte aligned, size a multiple of 16
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
+// L2 prefetch of a contiguous global range (bulk, no shared-memory destination);
+// address 16-byte aligned, size a multiple of 16
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
+
+// named barrier of one thread group (ids 1 and 2; 0 is __syncthreads), and
+// the same barrier with an OR over the group's predicates
+__device__ __forceinline__ void group_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(TC_GROUP) : "memory");
+}
+__device__ __forceinline__ bool group_or(int g, bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, o;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred o, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, o;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(1 + g), "r"(TC_GROUP)
+        : "memory");
+    return r != 0;
+}
+
 template <int NP, int H1, int H2, int MODE>
 struct TcLayout {
     static constexpr int D = 3 * NP;
     static constexpr int NA = NP * NT;
-    static constexpr bool STAGE = MODE != TC_FWD;   // A tile through shared memory
-    // bf16 weight tiles, K-major, one copy each (the backward products read
-    // them through the MN-major view)
+    static constexpr int RS = D + 1;          // padded fp32 row stride of staged rows (odd: no bank conflicts)
+    static constexpr int GXS = KPAD + 1;      // padded row stride of dE/drho rows
+    // shared by both groups: bf16 weight tiles, K-major, one copy each (the
+    // backward products read them through the MN-major view), fp32 vectors
     static constexpr int W1 = 0;                                 // [H1][KPAD]
     static constexpr int W2 = W1 + H1 * KPAD * 2;                // [H2][H1]
     static constexpr int W3 = W2 + H2 * H1 * 2;                  // [KPAD][H2] (rows >= n_out are zero)
-    // split operand tiles (hi, lo)
-    static constexpr int X = W3 + KPAD * H2 * 2;                 // [TM][KPAD] x 2
-    static constexpr int DY = X + 2 * TM * KPAD * 2;             // [TM][KPAD] x 2 (BWD)
-    static constexpr int ACT = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][128] x 2, every layer
-    // fp32 staging: the tile's A rows ([TM][NA]) and dE/drho ([TM][KPAD + 1])
-    static constexpr int STG = ACT + 2 * TM * 128 * 2;
-    static constexpr int GX = STG + (STAGE ? TM * NA * 4 : 0);
-    static constexpr int GXS = KPAD + 1;                          // padded row stride (no bank conflicts)
-    static constexpr int F32 = GX + (STAGE ? TM * GXS * 4 : 0);
-    static constexpr int nf32 = H1 + H2 + KPAD + 2 * KPAD + H2 + 4 * TM;  // b1, b2, b3, shift, 1/scale, w3, e parts
-    static constexpr int BAR = F32 + nf32 * 4;
-    static constexpr int bytes = BAR + 32;
-    // TMEM columns
-    static constexpr int C_Z1 = 0, C_Z2 = 128, C_P = 256, C_OUT = 384;
+    static constexpr int F32 = W3 + KPAD * H2 * 2;
+    static constexpr int nf32 = H1 + H2 + KPAD + 2 * KPAD + H2;  // b1, b2, b3, shift, 1/scale, w3
+    static constexpr int GRP = (F32 + nf32 * 4 + 15) / 16 * 16;
+    // per group (offsets inside the group's region):
+    //   ACT  [TM][128] bf16 hi + lo: the operand of layers 2 and 3 (and of the
+    //        VJP products), reused by every layer once the product that read it
+    //        has completed; between products it also holds the raw input rows
+    //        (fp32 [TM][RS], x then dY), the dY operand (hi + lo at ACT_DY),
+    //        the output rows and the dE/drho rows
+    //   X    [TM][KPAD] bf16 hi + lo, kept for the whole tile (the backward
+    //        recomputes layer 1 from it)
+    static constexpr int ACT = 0;
+    static constexpr int ACT_DY = 48 * 1024;
+    static constexpr int X = ACT + 2 * TM * 128 * 2;
+    static constexpr int SE = X + 2 * TM * KPAD * 2;             // energy partials [2][TM] fp32
+    static constexpr int BAR = SE + 2 * TM * 4;                  // MMA-completion mbarrier
+    static constexpr int GROUP_BYTES = BAR + 16;
+    static constexpr int SLOT = GRP + 2 * GROUP_BYTES;           // TMEM base address
+    static constexpr int bytes = SLOT + 16;
+    static_assert(2 * TM * RS * 4 <= ACT_DY && ACT_DY + 2 * TM * KPAD * 2 <= X, "input staging fits the ACT buffer");
+    static_assert(TM * GXS * 4 <= X && TM * RS * 4 <= X, "output staging fits the ACT buffer");
+    static_assert(GRP % 16 == 0 && GROUP_BYTES % 16 == 0, "16-byte aligned operand tiles");
+    // TMEM columns of a group (its base is 256 g): two 128-column accumulators
+    static constexpr int C_A = 0, C_B = 128;
 };
 
+// Two independent groups of 256 threads (8 warps) per block, each working on
+// its own tiles of the block's tile range with its own TMEM columns, operand
+// buffers, MMA-completion barrier and named barrier, so that one group's
+// epilogue (tanh on the special-function pipe, shared-memory stores) overlaps
+// the other's tensor-core products.  Inside a group, warp w reads TMEM lanes
+// 32 (w % 4) .. + 31 and thread half h = (w / 4) % 2 takes columns 64 h .. 64 h + 63
+// of every 128-wide accumulator.
 template <int NP, int H1, int H2, int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    k_mlp_tc(const int4 *__restrict__ tiles, int n_tiles, const float *__restrict__ w, TcNets nets,
-             const float *__restrict__ X, float *__restrict__ Y, const float *__restrict__ dY, float *__restrict__ Ei,
-             const float *__restrict__ A, float *__restrict__ Gout, int *__restrict__ status) {
-    static_assert(H1 == 4 * 32 && H2 == 4 * 32, "one 32-column chunk per warp group and layer");
+    k_mlp_tc(const int4 *__restrict__ tiles, const int4 *__restrict__ ranges, const float *__restrict__ w,
+             TcNets nets, const float *__restrict__ X, float *__restrict__ Y, const float *__restrict__ dY,
+             float *__restrict__ Ei, const float *__restrict__ A, float *__restrict__ Gout, int *__restrict__ status) {
+    static_assert(H1 == 128 && H2 == 128, "two 32-column chunks per thread and layer");
     using L = TcLayout<NP, H1, H2, MODE>;
-    constexpr int D = L::D, NA = L::NA;
+    constexpr int D = L::D, NA = L::NA, RS = L::RS;
     constexpr int DOUT = MODE == TC_ENERGY ? 1 : D;
     extern __shared__ __align__(1024) unsigned char sm[];
     float *f32 = reinterpret_cast<float *>(sm + L::F32);
     float *sb1 = f32, *sb2 = sb1 + H1, *sb3 = sb2 + H2, *sshift = sb3 + KPAD, *sinv = sshift + KPAD,
-          *sw3 = sinv + KPAD, *se = sw3 + H2;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);   // [0] MMA completion, [1] A tile landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
-    unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KPAD * 2;
-    unsigned char *dy_hi = sm + L::DY, *dy_lo = dy_hi + TM * KPAD * 2;
-    unsigned char *act_hi = sm + L::ACT, *act_lo = act_hi + TM * 128 * 2;
-    float *stg = reinterpret_cast<float *>(sm + L::STG);
-    float *gxs = reinterpret_cast<float *>(sm + L::GX);
+          *sw3 = sinv + KPAD;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int row = tid & (TM - 1);            // this thread's atom within the tile (TMEM lane)
-    const int qc = tid / TM;                   // warp group: columns 32 qc .. 32 qc + 31 of each accumulator
-    const int c = 32 * qc;
+    const int g = tid / TC_GROUP, gt = tid - g * TC_GROUP, gw = gt >> 5;
+    const int row = gt & (TM - 1);             // this thread's atom within the tile (TMEM lane)
+    const int h = gt / TM;                     // column half
+    unsigned char *gs = sm + L::GRP + g * L::GROUP_BYTES;
+    unsigned char *act_hi = gs + L::ACT, *act_lo = act_hi + TM * 128 * 2;
+    unsigned char *dy_hi = gs + L::ACT_DY, *dy_lo = dy_hi + TM * KPAD * 2;
+    unsigned char *x_hi = gs + L::X, *x_lo = x_hi + TM * KPAD * 2;
+    float *stage = reinterpret_cast<float *>(gs + L::ACT);
+    float *se = reinterpret_cast<float *>(gs + L::SE);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(gs + L::BAR);
     const uint32_t base = smem_u32(sm);
     auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
 
+    const int4 rg = ranges[blockIdx.x];        // (first tile, end tile, element, -)
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    if (tid == 0) {
+    if (gt == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar + 1)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    {
+        // the block's element: weights -> bf16 tiles and fp32 vectors
+        const NetOffsets &o = nets.net[rg.z];
+        for (int k = tid; k < H1 * KPAD; k += TC_THREADS) {
+            int n = k / KPAD, f = k % KPAD;
+            st_elem(sm + L::W1, H1, n, f, f < D ? w[o.W1 + (int64_t)n * D + f] : 0.f);
+        }
+        for (int k = tid; k < H2 * H1; k += TC_THREADS) st_elem(sm + L::W2, H2, k / H1, k % H1, w[o.W2 + k]);
+        for (int k = tid; k < KPAD * H2; k += TC_THREADS) {
+            int n = k / H2, hh = k % H2;
+            st_elem(sm + L::W3, KPAD, n, hh, n < DOUT ? w[o.W3 + (int64_t)n * H2 + hh] : 0.f);
+        }
+        for (int k = tid; k < H1; k += TC_THREADS) sb1[k] = w[o.b1 + k];
+        for (int k = tid; k < H2; k += TC_THREADS) {
+            sb2[k] = w[o.b2 + k];
+            sw3[k] = MODE == TC_ENERGY ? w[o.W3 + k] : 0.f;
+        }
+        for (int k = tid; k < KPAD; k += TC_THREADS) {
+            sb3[k] = k < DOUT ? w[o.b3 + k] : 0.f;
+            sshift[k] = k < D ? w[o.shift + k] : 0.f;
+            sinv[k] = k < D ? 1.0f / w[o.scale + k] : 0.f;
+        }
     }
     fence_before();
     __syncthreads();
     fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot + (uint32_t)(256 * g);
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    uint32_t phase = 0, phase_ld = 0;
-    bool failed = false, load_pending = false;
-    int cur = -1;
+    uint32_t phase = 0;
+    bool failed = false;
 
-    // completion of the MMA group thread 0 committed, awaited by all threads
+    // completion of the MMA group the group's thread 0 committed, awaited by the group
     auto wait_mma = [&]() -> bool {
         bool ok = bar_wait(bar, phase);
         phase ^= 1u;
         fence_after();
-        return !__syncthreads_or(!ok);
+        return !group_or(g, !ok);
     };
     // operand stores (generic proxy) and TMEM reads done -> next MMA may start
     auto handoff = [&]() {
         fence_smem_to_async();
         fence_before();
-        __syncthreads();
+        group_sync(g);
     };
 
-    // raw inputs of the next tile, loaded while the current tile computes:
-    // the tile's rows are contiguous in X (and dY), so thread tid takes
-    // elements tid, tid + 512, ... of that run (coalesced).  The tile
-    // descriptor is read one tile further ahead, so the addresses are known
-    // when the loads issue.
-    constexpr int NXR = (TM * D + TC_THREADS - 1) / TC_THREADS;
-    float xr[NXR], dr[NXR];
-    int4 tl = make_int4(0, 0, 0, 0);                                   // tile whose inputs are in xr
-    int4 tl2 = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);   // the one after
-    auto prefetch = [&](int t2) {
-        tl = tl2;
-        const int64_t g0 = (int64_t)tl.y * D;
-        const int cnt = tl.z * D;
-#pragma unroll
-        for (int u = 0; u < NXR; ++u) {
-            const int k = tid + u * TC_THREADS;
-            xr[u] = k < cnt ? X[g0 + k] : 0.f;
-            dr[u] = (MODE == TC_BWD && k < cnt) ? dY[g0 + k] : 0.f;
-        }
-        const int t3 = t2 + gridDim.x;
-        tl2 = t3 < n_tiles ? tiles[t3] : make_int4(0, 0, 0, 0);
-    };
     // dE/dA positions of this lane (element pk = lane + 32 j of a row, in the
     // edge kernels' lane-interleaved order), packed: source A index (bits 0-7),
     // dE/drho index (bits 8-15), mixed second-order tuple (bit 16: 2 w_tau = 4)
@@ -323,164 +356,141 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int gi = (u == 0 ? 0 : (u < 4 ? 1 : 2)) * NP + nn;
         posj[j] = src | (gi << 8) | ((u >= 7 ? 1 : 0) << 16);
     }
-    prefetch(blockIdx.x);
 
-    for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
-        const int4 tile = tl;
-        const int e = tile.x, r0 = tile.y, rows = tile.z;
-        if (e != cur) {
-            // element weights -> bf16 tiles and fp32 vectors
-            const NetOffsets &o = nets.net[e];
-            for (int k = tid; k < H1 * KPAD; k += TC_THREADS) {
-                int n = k / KPAD, f = k % KPAD;
-                st_elem(sm + L::W1, H1, n, f, f < D ? w[o.W1 + (int64_t)n * D + f] : 0.f);
-            }
-            for (int k = tid; k < H2 * H1; k += TC_THREADS) st_elem(sm + L::W2, H2, k / H1, k % H1, w[o.W2 + k]);
-            for (int k = tid; k < KPAD * H2; k += TC_THREADS) {
-                int n = k / H2, h = k % H2;
-                st_elem(sm + L::W3, KPAD, n, h, n < DOUT ? w[o.W3 + (int64_t)n * H2 + h] : 0.f);
-            }
-            for (int k = tid; k < H1; k += TC_THREADS) sb1[k] = w[o.b1 + k];
-            for (int k = tid; k < H2; k += TC_THREADS) {
-                sb2[k] = w[o.b2 + k];
-                if (MODE == TC_ENERGY) sw3[k] = w[o.W3 + k];
-            }
-            for (int k = tid; k < KPAD; k += TC_THREADS) {
-                sb3[k] = k < DOUT ? w[o.b3 + k] : 0.f;
-                sshift[k] = k < D ? w[o.shift + k] : 0.f;
-                sinv[k] = k < D ? 1.0f / w[o.scale + k] : 0.f;
-            }
-            cur = e;
-        }
-        // the tile's A rows (energy and backward) stream into the staging buffer
-        // while the networks run (the previous tile finished reading it before
-        // the barrier that ended it)
-        if (L::STAGE && tid == 0) {
-            bulk_load(stg, A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4), bar + 1);
-            load_pending = true;
-        }
-        __syncthreads();
-        // input tile: raw values -> padded fp32 rows in the (idle) activation
-        // buffer, then standardised rho (and the upstream gradient) split bf16
+    for (int ti = rg.x + g; ti < rg.y && !failed; ti += 2) {
+        const int4 tile = tiles[ti];
+        const int r0 = tile.y, rows = tile.z;
+        // energy and backward: the tile's A rows are read at the end; start
+        // moving them into L2 now
+        if (MODE != TC_FWD && gt == 0) prefetch_l2(A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4));
+        // input tile: contiguous raw rows -> padded fp32 rows in ACT, then the
+        // standardised rho (and the upstream gradient) split bf16
         {
-            constexpr int RS = D + 1;   // odd row stride: conflict-free row reads
-            float *xs = reinterpret_cast<float *>(act_hi), *ds = xs + TM * RS;
-#pragma unroll
-            for (int u = 0; u < NXR; ++u) {
-                const int k = tid + u * TC_THREADS;
-                if (k < rows * D) {
-                    const int rk = k / D, f = k - rk * D;
-                    xs[rk * RS + f] = xr[u];
-                    if (MODE == TC_BWD) ds[rk * RS + f] = dr[u];
-                }
+            float *xs = stage, *ds = stage + TM * RS;
+            const float *xg = X + (int64_t)r0 * D;
+            const float *dg = MODE == TC_BWD ? dY + (int64_t)r0 * D : nullptr;
+            for (int k = gt; k < rows * D; k += TC_GROUP) {
+                const int rk = k / D, f = k - rk * D;
+                xs[rk * RS + f] = xg[k];
+                if (MODE == TC_BWD) ds[rk * RS + f] = dg[k];
             }
-            __syncthreads();
+            group_sync(g);
             const bool live = row < rows;
-            float v[8], g[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int f = 8 * qc + u;
-                const bool ok = live && f < D;
-                v[u] = ok ? (xs[row * RS + f] - sshift[f]) * sinv[f] : 0.f;
-                g[u] = (MODE == TC_BWD && ok) ? ds[row * RS + f] : 0.f;
+            for (int c8 = 0; c8 < 16; c8 += 8) {
+                float v[8], gv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int f = 16 * h + c8 + u;
+                    const bool ok = live && f < D;
+                    v[u] = ok ? (xs[row * RS + f] - sshift[f]) * sinv[f] : 0.f;
+                    gv[u] = (MODE == TC_BWD && ok) ? ds[row * RS + f] : 0.f;
+                }
+                st_chunk2(x_hi, x_lo, TM, row, 16 * h + c8, v);
+                if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, 16 * h + c8, gv);
             }
-            st_chunk2(x_hi, x_lo, TM, row, 8 * qc, v);
-            if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, 8 * qc, g);
         }
-        prefetch(ti + gridDim.x);
         handoff();
 
         // layer 1 (and, for the coefficient backward, dE/da2 = dY W3 via the MN-major view of W3)
-        if (tid == 0) {
+        if (gt == 0) {
             fence_after();
-            gemm2<H1, KPAD, false, 0>(tmem + L::C_Z1, sa(x_hi), sa(x_lo), base + L::W1);
-            if (MODE == TC_BWD) gemm2<H2, KPAD, true, KPAD>(tmem + L::C_P, sa(dy_hi), sa(dy_lo), base + L::W3);
+            gemm2<H1, KPAD, false, 0>(tmem + L::C_A, sa(x_hi), sa(x_lo), base + L::W1);
+            if (MODE == TC_BWD) gemm2<H2, KPAD, true, KPAD>(tmem + L::C_B, sa(dy_hi), sa(dy_lo), base + L::W3);
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
         // a1 = tanh(z1 + b1)
-        {
+#pragma unroll 1
+        for (int c = 64 * h; c < 64 * h + 64; c += 32) {
             float v[32];
-            tmem_ld32(lane_base + L::C_Z1 + c, v);
+            tmem_ld32(lane_base + L::C_A + c, v);
 #pragma unroll
             for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb1[c + u]);
 #pragma unroll
             for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
         }
         handoff();
-        if (tid == 0) {
+        // z2 = a1 W2^T: into B (forward, energy) or over z1 in A (backward, whose B holds dY W3)
+        constexpr int C_Z2 = MODE == TC_BWD ? L::C_A : L::C_B;
+        if (gt == 0) {
             fence_after();
-            gemm2<H2, H1, false, 0>(tmem + L::C_Z2, sa(act_hi), sa(act_lo), base + L::W2);
+            gemm2<H2, H1, false, 0>(tmem + C_Z2, sa(act_hi), sa(act_lo), base + L::W2);
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
 
         if (MODE == TC_FWD) {
-            // a2 = tanh(z2 + b2) (the layer-2 product has consumed a1), then y = a2 W3^T + b3
-            {
+            // a2 = tanh(z2 + b2), then y = a2 W3^T + b3 (into A)
+#pragma unroll 1
+            for (int c = 64 * h; c < 64 * h + 64; c += 32) {
                 float v[32];
-                tmem_ld32(lane_base + L::C_Z2 + c, v);
+                tmem_ld32(lane_base + C_Z2 + c, v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb2[c + u]);
 #pragma unroll
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
             }
             handoff();
-            if (tid == 0) {
+            if (gt == 0) {
                 fence_after();
-                gemm2<KPAD, H2, false, 0>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W3);
+                gemm2<KPAD, H2, false, 0>(tmem + L::C_A, sa(act_hi), sa(act_lo), base + L::W3);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            // y rows through the (idle) input tile buffer, then contiguous stores
-            {
-                constexpr int RS = D + 1;
-                float *ys = reinterpret_cast<float *>(x_hi);
-                float v[8];
-                tmem_ld8(lane_base + L::C_OUT + 8 * qc, v);
+            // y rows through ACT (the last product has consumed it), then contiguous stores
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (8 * qc + u < D) ys[row * RS + 8 * qc + u] = v[u] + sb3[8 * qc + u];
-                __syncthreads();
-                float *yo = Y + (int64_t)r0 * D;
-                for (int k = tid; k < rows * D; k += TC_THREADS) {
-                    const int rk = k / D;
-                    yo[k] = ys[rk * RS + (k - rk * D)];
+            for (int c8 = 0; c8 < 16; c8 += 8) {
+                float v[8];
+                tmem_ld8(lane_base + L::C_A + 16 * h + c8, v);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int f = 16 * h + c8 + u;
+                    if (f < D) stage[row * RS + f] = v[u] + sb3[f];
                 }
+            }
+            group_sync(g);
+            float *yo = Y + (int64_t)r0 * D;
+            for (int k = gt; k < rows * D; k += TC_GROUP) {
+                const int rk = k / D;
+                yo[k] = stage[rk * RS + (k - rk * D)];
             }
         } else {
             // g2 = dE/dz2 = (energy: w3, backward: dY W3) * (1 - a2^2); energy E_i = w3 . a2 + b3
-            {
+            float e_row = 0.f;
+#pragma unroll 1
+            for (int c = 64 * h; c < 64 * h + 64; c += 32) {
                 float z[32], up[32];
-                tmem_ld32(lane_base + L::C_Z2 + c, z);
-                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P + c, up);
-                float e_row = 0.f;
+                tmem_ld32(lane_base + C_Z2 + c, z);
+                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_B + c, up);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                     const float a = tanh_fast(z[u] + sb2[c + u]);
-                    const float g = MODE == TC_ENERGY ? sw3[c + u] : up[u];
+                    const float gg = MODE == TC_ENERGY ? sw3[c + u] : up[u];
                     if (MODE == TC_ENERGY) e_row = fmaf(sw3[c + u], a, e_row);
-                    z[u] = g * (1.f - a * a);
+                    z[u] = gg * (1.f - a * a);
                 }
 #pragma unroll
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &z[u]);
-                if (MODE == TC_ENERGY) se[qc * TM + row] = e_row;
             }
+            if (MODE == TC_ENERGY) se[h * TM + row] = e_row;
             handoff();
-            if (MODE == TC_ENERGY && qc == 0 && row < rows)
-                Ei[r0 + row] = ((se[row] + se[TM + row]) + (se[2 * TM + row] + se[3 * TM + row])) + sb3[0];
-            // p1 = g2 W2 (MN-major view of W2), into the columns dY W3 used
-            if (tid == 0) {
+            if (MODE == TC_ENERGY && h == 0 && row < rows) Ei[r0 + row] = (se[row] + se[TM + row]) + sb3[0];
+            // p1 = g2 W2 (MN-major view of W2) into B; the backward recomputes z1
+            // = x W1^T into A (its first copy was overwritten by z2)
+            if (gt == 0) {
                 fence_after();
-                gemm2<H1, H2, true, H2>(tmem + L::C_P, sa(act_hi), sa(act_lo), base + L::W2);
+                gemm2<H1, H2, true, H2>(tmem + L::C_B, sa(act_hi), sa(act_lo), base + L::W2);
+                if (MODE == TC_BWD) gemm2<H1, KPAD, false, 0>(tmem + L::C_A, sa(x_hi), sa(x_lo), base + L::W1);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation still in TMEM
-            {
+            // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation in TMEM
+#pragma unroll 1
+            for (int c = 64 * h; c < 64 * h + 64; c += 32) {
                 float p[32], z[32];
-                tmem_ld32(lane_base + L::C_P + c, p);
-                tmem_ld32(lane_base + L::C_Z1 + c, z);
+                tmem_ld32(lane_base + L::C_B + c, p);
+                tmem_ld32(lane_base + L::C_A + c, z);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                     const float a = tanh_fast(z[u] + sb1[c + u]);
@@ -490,51 +500,65 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &p[u]);
             }
             handoff();
-            // dE/dx = g1 W1 (MN-major view of W1)
-            if (tid == 0) {
+            // dE/dx = g1 W1 (MN-major view of W1), into A
+            if (gt == 0) {
                 fence_after();
-                gemm2<KPAD, H1, true, H1>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W1);
+                gemm2<KPAD, H1, true, H1>(tmem + L::C_A, sa(act_hi), sa(act_lo), base + L::W1);
                 mma_commit(bar);
             }
             if (!wait_mma()) { failed = true; break; }
-            // dE/drho = (g1 W1) / scale, shared by the row's four threads
-            {
+            // dE/drho = (g1 W1) / scale, rows through ACT (consumed by the last product)
+            float *gxs = stage;
+#pragma unroll
+            for (int c8 = 0; c8 < 16; c8 += 8) {
                 float v[8];
-                tmem_ld8(lane_base + L::C_OUT + 8 * qc, v);
+                tmem_ld8(lane_base + L::C_A + 16 * h + c8, v);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) gxs[row * L::GXS + 8 * qc + u] = v[u] * sinv[8 * qc + u];
+                for (int u = 0; u < 8; ++u) gxs[row * L::GXS + 16 * h + c8 + u] = v[u] * sinv[16 * h + c8 + u];
             }
-            const bool landed = bar_wait(bar + 1, phase_ld);
-            if (__syncthreads_or(!landed)) { failed = true; break; }
-            phase_ld ^= 1u;
-            if (tid == 0) load_pending = false;
-            // G = dE/dA = 2 w_tau A dE/drho, warp per row, lanes along the row in
-            // the edge kernels' lane-interleaved order (contiguous stores)
+            group_sync(g);
+            // G = dE/dA = 2 w_tau A dE/drho, warp per row, lanes along the row in the
+            // edge kernels' lane-interleaved order (contiguous stores); four rows'
+            // A values are loaded before any is used
+            const float *ag = A + (int64_t)r0 * NA;
             float *go = Gout + (int64_t)r0 * NA;
-            for (int rk = warp; rk < rows; rk += TC_THREADS / 32) {
-                const float *ar = stg + rk * NA, *gr = gxs + rk * L::GXS;
-                float *orow = go + (int64_t)rk * NA;
+            for (int rb = gw; rb < rows; rb += 4 * (TC_GROUP / 32)) {
+                float av[4][NJ];
 #pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    const int pk = (tid & 31) + 32 * j;
-                    const int c = posj[j];
-                    if (pk < NA) orow[pk] = ((c >> 16) ? 4.f : 2.f) * ar[c & 255] * gr[(c >> 8) & 255];
+                for (int q = 0; q < 4; ++q) {
+                    const int rk = rb + q * (TC_GROUP / 32);
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int pk = (tid & 31) + 32 * j;
+                        av[q][j] = (rk < rows && pk < NA) ? ag[(int64_t)rk * NA + (posj[j] & 255)] : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int rk = rb + q * (TC_GROUP / 32);
+                    if (rk >= rows) break;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int pk = (tid & 31) + 32 * j;
+                        const int c = posj[j];
+                        if (pk < NA)
+                            go[(int64_t)rk * NA + pk] =
+                                ((c >> 16) ? 4.f : 2.f) * av[q][j] * gxs[rk * L::GXS + ((c >> 8) & 255)];
+                    }
                 }
             }
         }
+        // the next tile's input staging overwrites ACT: all of this tile's reads are done
         fence_before();
-        __syncthreads();
+        group_sync(g);
     }
 
-    if (tid == 0) {
-        if (failed) atomicOr(status, ST_TIMEOUT);
-        // a tile load that never completed: wait for it once more, with the same bound
-        if (load_pending) bar_wait(bar + 1, phase_ld);
-    }
+    if (failed && gt == 0) atomicOr(status, ST_TIMEOUT);
     fence_before();
     __syncthreads();
     fence_after();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*tmem_slot),
+                                "r"(TMEM_COLS));
 }
 
 template <int NP, int H1, int H2, int MODE>
@@ -542,8 +566,7 @@ cudaError_t run_tc(reann_ctx *c, const TcNets &nets, const float *X, float *Y, c
                    const float *A, float *G, cudaStream_t s) {
     using L = TcLayout<NP, H1, H2, MODE>;
     static_assert(L::bytes > 116 * 1024 && L::bytes <= 227 * 1024, "one block per SM keeps TMEM allocation safe");
-    static_assert(L::STG % 16 == 0 && L::GX % 16 == 0 && L::BAR % 16 == 0, "bulk copies need 16-byte alignment");
-    static_assert((NA_BYTES<NP>() % 16) == 0, "A rows must be whole 16-byte units for the bulk copy");
+    static_assert((NA_BYTES<NP>() % 16) == 0, "A rows must be whole 16-byte units for the L2 prefetch");
     static bool configured[64] = {};
     auto kern = k_mlp_tc<NP, H1, H2, MODE>;
     if (c->device < 0 || c->device >= 64) return cudaErrorInvalidDevice;
@@ -552,11 +575,10 @@ cudaError_t run_tc(reann_ctx *c, const TcNets &nets, const float *X, float *Y, c
         if (e) return e;
         configured[c->device] = true;
     }
-    if (c->n_tiles128 == 0) return cudaSuccess;
-    int grid = c->sm_count < c->n_tiles128 ? c->sm_count : c->n_tiles128;
+    if (c->n_tc_ranges == 0) return cudaSuccess;
     REANN_TIMED(c, MODE == TC_FWD ? REANN_K_MLP_FWD : (MODE == TC_ENERGY ? REANN_K_MLP_ENERGY : REANN_K_MLP_BWD), s);
-    kern<<<grid, TC_THREADS, L::bytes, s>>>(c->d_tiles128, c->n_tiles128, c->d_w, nets, X, Y, dY, Ei, A, G,
-                                            c->d_status);
+    kern<<<c->n_tc_ranges, TC_THREADS, L::bytes, s>>>(c->d_tiles128, c->d_tiles128 + c->n_tiles128, c->d_w, nets, X,
+                                                      Y, dY, Ei, A, G, c->d_status);
     return cudaGetLastError();
 }
 
