@@ -1,6 +1,7 @@
 """Writes the per-feature input standardisation of every atomic network.
 
     python -m oracle.make_norm_stats [workload ...]
+    python -m oracle.make_norm_stats --sign-only [workload ...]
 
 Part of the weight recipe, not of the model: the paper's trained weights are
 not available, and random Xavier weights applied to raw embedded densities
@@ -23,10 +24,18 @@ molecular workloads (liquid water, C/H/O/N gas) are already varied and use
 their own structure.
 
 The same script fixes the energy scale: the energy network's output layer
-(W3, b3) is multiplied by lambda = 1 / rms(F), with F the oracle forces of
+(W3, b3) is multiplied by lambda = +-1 / rms(F), with F the oracle forces of
 the unscaled model on the same structure, so that the synthetic potential
 has forces of physical size (RMS 1 eV/A) rather than the tens of eV/A that
-random weights on standardised densities give.
+random weights on standardised densities give.  The sign matters for the
+FCC workloads: the perfect lattice is a stationary point of any such model
+(every atom is a centre of inversion), and a random output layer makes it a
+maximum or a minimum along the thermal displacements with equal odds; with
+a maximum the crystal heats up in an MD run and, after ~100 fs at 1 fs steps,
+throws atoms fast enough to break velocity Verlet.  A fitted potential has
+its crystal at a minimum, so the sign is chosen to make the workload's
+thermally displaced structure higher in energy than the perfect lattice.
+Molecular workloads keep the positive sign.
 
 Only the oracle and the seeded input generators run here; the output file
 molecular_dynamics_b200/data/norm_<workload>.json is read by
@@ -49,6 +58,8 @@ OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 
 
 STATS_SIGMA_FACTOR = 5.0
+ENERGY_SCALE_RECIPE = ("energy network output layer multiplied by +-1/rms(F) of the unscaled model; FCC workloads "
+                       "take the sign that puts the perfect lattice below the workload's thermal structure")
 
 
 def stats_structure(p):
@@ -96,9 +107,48 @@ def measure(p, verbose=True):
     model = oracle.Model.from_preset(p, blob, T=p.T)
     res = oracle.energy_forces(model, pos, types, box, pairs)
     lam = float(np.float32(1.0 / np.sqrt(np.mean(res.forces ** 2))))
+    lam *= energy_sign(p, shift, scale, lam, verbose)
     if verbose:
         print(f"  {p.key} energy scale {lam:.6g} ({time.time() - t0:.1f}s)", flush=True)
     return shift, scale, sat, lam
+
+
+def energy_sign(p, shift, scale, lam, verbose=True):
+    """+1 or -1 for the energy scale (see the module text): FCC workloads get
+    the sign that puts the perfect lattice below the workload's structure."""
+    if p.kind != "fcc":
+        return 1.0
+    blob = synth.weight_blob(p, T=p.T, norm=(shift, scale), use_stored_norm=False, energy_scale=abs(lam))
+    model = oracle.Model.from_preset(p, blob, T=p.T)
+    per_atom = []
+    for q in (p, p.with_(sigma=0.0)):
+        pos, types, box = synth.make_structure(q)
+        pairs = oracle.pairs_brute(pos, box, q.r_cut, q.skin) if len(pos) <= 20000 else \
+            oracle.pairs_cells(pos, box, q.r_cut, q.skin)
+        per_atom.append(oracle.energy_forces(model, pos, types, box, pairs, forces=False).energy / len(pos))
+    sign = 1.0 if per_atom[0] > per_atom[1] else -1.0
+    if verbose:
+        print(f"  {p.key} E/atom thermal {per_atom[0]:.6f}, perfect lattice {per_atom[1]:.6f} "
+              f"(positive scale) -> sign {sign:+.0f}", flush=True)
+    return sign
+
+
+def resign(keys):
+    """Recompute only the sign of the stored energy scales (the standardisation
+    and |lambda| do not depend on it)."""
+    for k in keys:
+        p = presets.get(k)
+        path = os.path.join(OUT, f"norm_{k}.json")
+        with open(path) as f:
+            d = json.load(f)
+        shift = np.asarray(d["shift"], np.float64)
+        scale = np.asarray(d["scale"], np.float64)
+        lam = abs(float(d["energy_scale"]))
+        d["energy_scale"] = lam * energy_sign(p, shift[:p.T], scale[:p.T], lam)
+        d["energy_scale_recipe"] = ENERGY_SCALE_RECIPE
+        with open(path, "w") as f:
+            json.dump(d, f)
+        print(f"wrote norm_{k}.json  energy scale {d['energy_scale']:.6g}")
 
 
 def main(keys):
@@ -115,7 +165,7 @@ def main(keys):
             "scale": scale.tolist(),
             "saturated_fraction": sat,
             "energy_scale": lam,
-            "energy_scale_recipe": "energy network output layer multiplied by 1/rms(F) of the unscaled model",
+            "energy_scale_recipe": ENERGY_SCALE_RECIPE,
         }
         with open(os.path.join(OUT, f"norm_{k}.json"), "w") as f:
             json.dump(out, f)
@@ -123,4 +173,8 @@ def main(keys):
 
 
 if __name__ == "__main__":
-    main(sys.argv[1:] or list(presets.ORDER))
+    args = sys.argv[1:]
+    if args and args[0] == "--sign-only":
+        resign(args[1:] or list(presets.ORDER))
+    else:
+        main(args or list(presets.ORDER))

@@ -17,9 +17,25 @@ def test_standardisation_is_well_conditioned(key):
 
 
 @pytest.mark.parametrize("key", presets.ORDER)
-def test_energy_scale_present_and_positive(key):
-    lam = synth.load_energy_scale(presets.get(key))
-    assert 0 < lam < 10
+def test_energy_scale_present_and_signed(key):
+    p = presets.get(key)
+    lam = synth.load_energy_scale(p)
+    assert 0 < abs(lam) < 10
+    if p.kind != "fcc":
+        assert lam > 0
+
+
+def test_crystal_lies_below_its_thermal_structure():
+    # the sign of the energy scale makes the perfect lattice the lower-energy
+    # structure, so an MD run of the crystal stays in its basin
+    import oracle
+    p = presets.get("ag256")
+    model = oracle.Model.from_preset(p, synth.weight_blob(p))
+    e = []
+    for q in (p, p.with_(sigma=0.0)):
+        pos, types, box = synth.make_structure(q)
+        e.append(oracle.energy_forces(model, pos, types, box, forces=False).energy / len(pos))
+    assert e[0] > e[1] + 1e-3
 
 
 def test_weight_blob_is_deterministic_and_sized():
