@@ -281,10 +281,10 @@ def main():
     ctx.reann_md_step(args.warmup, dt_fs, x, v, p.masses)
     torch.cuda.synchronize()
 
-    # ---- device-resident timed region: K steps in one call (a continuation)
+    # ---- device-resident timed region: K steps in one call (a continuation);
+    # each step's energy+forces and half kick replay as one CUDA graph
     clocks = ClockSampler(info.local)
     launches0 = ctx.reann_get_counters().kernel_launches
-    ctx.reann_profile(True)
     clocks.start()
     run = timed_region(group, lambda: ctx.reann_md_step(args.steps, dt_fs, x, v, p.masses), clock,
                        n * args.steps)
@@ -292,10 +292,16 @@ def main():
     st = run.result
     t_ms = run.ms
     value = run.throughput
+    launches = ctx.reann_get_counters().kernel_launches - launches0
+
+    # ---- kernel breakdown: a separate call with per-launch CUDA events (eager launches)
+    prof_steps = min(args.steps, 20)
+    ctx.reann_profile(True)
+    ctx.reann_md_step(prof_steps, dt_fs, x, v, p.masses)
+    torch.cuda.synchronize()
     prof = ctx.reann_profile_read()
     ctx.reann_profile(False)
     cnt = ctx.reann_get_counters()
-    launches = cnt.kernel_launches - launches0
 
     # ---- end to end: one public call per step with pinned host state
     e2e = None
@@ -334,14 +340,17 @@ def main():
         "data": "synthetic",
         "config": {"workload": f"{p.key}: {p.description}", "atoms": n, "T": p.T, "r_cut": p.r_cut,
                    "n_radial": p.n_radial, "l_max": p.l_max, "hidden": list(p.hidden), "dt_fs": dt_fs,
-                   "networks": "bf16 tcgen05, fp32 accumulate" if p.mlp_precision else "fp32 CUDA-core", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "networks": "bf16 tcgen05, fp32 accumulate" if p.mlp_precision else "fp32 CUDA-core",
+                   "launch": "energy+forces and half kick replayed as one CUDA graph per step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"working set > L2 ({n * (p.T * (10 * p.n_radial + 6 * p.n_radial) * 4) / 1e9:.1f} GB of "
                          f"per-layer activations vs 126 MB L2); no flush needed"},
         "ns_per_day": (args.steps / (t_ms * 1e-3)) * dt_fs * 86400 / 1e6,
         "rebuilds": st.rebuilds,
         "gpu_launches": launches,
         "clocks": clk,
-        "kernel_ms_per_step": {k: v_[0] / args.steps for k, v_ in prof.items() if v_[1]},
+        "kernel_ms_per_step": {k: v_[0] / prof_steps for k, v_ in prof.items() if v_[1]},
+        "kernel_profile_note": f"per-launch CUDA events over a separate {prof_steps}-step call with eager launches",
         "kernel_share": {k: v_ / total for k, v_ in shares.items() if v_},
         "roofline": roof,
     }

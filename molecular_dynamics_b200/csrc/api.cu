@@ -13,6 +13,7 @@
 //   E = sum_i E_i (deterministic fp64 tree)                      [md.cu]
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -213,6 +214,7 @@ reann_status check_status(reann_ctx *c, int st) {
 // Binning + CSR for the caller-order float positions/types already on the
 // device.  Reads nnz back (one synchronisation) and grows the list if needed.
 reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s) {
+    c->g_valid = false;   // list sizes and buffers may change: the step graph is recaptured
     CK(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
     CK(launch_build(c, d_pos_caller, d_types_caller, s));
     CK(cudaMemcpyAsync(c->h_i64, c->d_i64, sizeof(int64_t) * 3, cudaMemcpyDeviceToHost, s));
@@ -338,6 +340,60 @@ reann_status run_ef(reann_ctx *c, cudaStream_t s) {
     return REANN_OK;
 }
 
+// The part of an MD step after the skin check: energy+forces and the second
+// half kick.  Eager launches on `s` while profiling (per-launch events) or with
+// REANN_GRAPHS=0; otherwise one CUDA graph replay, captured on the library's
+// stream the first time a neighbour list (with this dt and these masses) is
+// used and ordered against `s` with events.
+reann_status ef_and_kick(reann_ctx *c, double dt_fs, const double *inv_mass, cudaStream_t s) {
+    reann_status st;
+    if (c->prof || c->g_disabled || c->n == 0) {
+        if ((st = run_ef(c, s))) return st;
+        CK(launch_md_kick(c, dt_fs, inv_mass, s));
+        return REANN_OK;
+    }
+    if (!c->g_stream) {
+        CK(cudaStreamCreateWithFlags(&c->g_stream, cudaStreamNonBlocking));
+        for (auto &ev : c->g_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    }
+    const bool same = c->g_valid && c->g_dt == dt_fs && std::equal(inv_mass, inv_mass + c->ne, c->g_inv_mass);
+    CK(cudaEventRecord(c->g_ev[0], s));
+    CK(cudaStreamWaitEvent(c->g_stream, c->g_ev[0], 0));
+    if (!same) {
+        if (c->g_exec) {
+            cudaGraphExecDestroy(c->g_exec);
+            c->g_exec = nullptr;
+        }
+        const int64_t k0 = c->counters.kernel_launches, e0 = c->counters.evaluations;
+        CK(cudaStreamBeginCapture(c->g_stream, cudaStreamCaptureModeThreadLocal));
+        st = run_ef(c, c->g_stream);
+        cudaError_t ek = st ? cudaSuccess : launch_md_kick(c, dt_fs, inv_mass, c->g_stream);
+        cudaGraph_t g = nullptr;
+        cudaError_t ee = cudaStreamEndCapture(c->g_stream, &g);
+        c->g_launches = c->counters.kernel_launches - k0;
+        c->counters.kernel_launches = k0;
+        c->counters.evaluations = e0;
+        if (st || ek || ee) {
+            if (g) cudaGraphDestroy(g);
+            if (st) return st;
+            CK(ek ? ek : ee);
+        }
+        cudaError_t ei = cudaGraphInstantiate(&c->g_exec, g, 0);
+        cudaGraphDestroy(g);
+        CK(ei);
+        c->g_valid = true;
+        c->g_dt = dt_fs;
+        std::copy(inv_mass, inv_mass + c->ne, c->g_inv_mass);
+    }
+    CK(cudaGraphLaunch(c->g_exec, c->g_stream));
+    CK(cudaEventRecord(c->g_ev[1], c->g_stream));
+    CK(cudaStreamWaitEvent(s, c->g_ev[1], 0));
+    c->counters.kernel_launches += c->g_launches;
+    c->counters.evaluations++;
+    c->have_eval = true;
+    return REANN_OK;
+}
+
 void fill_counters(reann_ctx *c) {
     c->counters.n_atoms = c->n;
     c->counters.nnz = c->nnz;
@@ -419,6 +475,10 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     reann_ctx *c = new reann_ctx();
     c->cfg = *cfg;
     c->device = device;
+    {
+        const char *gv = std::getenv("REANN_GRAPHS");
+        c->g_disabled = gv && std::strcmp(gv, "0") == 0;
+    }
     c->NP = cfg->n_radial;
     c->D = c->NP * (cfg->l_max + 1);
     c->NA = c->NP * NT;
@@ -487,6 +547,10 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
         cudaEventDestroy(r.b);
     }
     for (auto ev : c->prof_pool) cudaEventDestroy(ev);
+    if (c->g_exec) cudaGraphExecDestroy(c->g_exec);
+    for (auto ev : c->g_ev)
+        if (ev) cudaEventDestroy(ev);
+    if (c->g_stream) cudaStreamDestroy(c->g_stream);
     delete c;
     return REANN_OK;
 }
@@ -629,8 +693,7 @@ extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs
             CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
             ++rebuilds;
         }
-        if ((st = run_ef(c, s))) return st;
-        CK(launch_md_kick(c, dt_fs, inv_mass, s));
+        if ((st = ef_and_kick(c, dt_fs, inv_mass, s))) return st;
         ++done;
     }
     CK(launch_kinetic(c, mass, c->d_E + 1, s));

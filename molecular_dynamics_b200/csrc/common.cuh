@@ -162,6 +162,17 @@ struct reann_ctx {
     bool md_valid = false;
     double md_dt = 0.0;
     double md_mass[reann::MAX_ELEMENTS] = {};
+    // one MD step's energy+force evaluation and closing half kick as a CUDA
+    // graph, captured on a library stream once per neighbour list (and per
+    // dt / masses) and replayed for the following steps
+    cudaStream_t g_stream = nullptr;
+    cudaEvent_t g_ev[2] = {nullptr, nullptr};
+    cudaGraphExec_t g_exec = nullptr;
+    bool g_valid = false;
+    double g_dt = 0.0;
+    double g_inv_mass[reann::MAX_ELEMENTS] = {};
+    int64_t g_launches = 0;   // kernels one replay runs
+    bool g_disabled = false;  // REANN_GRAPHS=0 in the environment
 
     // status
     int *d_status = nullptr;
