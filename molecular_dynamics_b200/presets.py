@@ -54,6 +54,12 @@ class Preset:
     temperature: float = 300.0
     # largest T the standardisation statistics cover (T sweeps)
     t_stats: int = 0
+    # density features: 0 = sum_tau w A_{n,tau}^2 per (n, l) (Eq. 1);
+    # 1 = sum_tau w A_{n,tau} A_{m,tau} per (n <= m, l), N_phi (N_phi+1)(L+1)/2 features
+    density_form: int = 0
+    # FCC: cells per axis of the lattice the standardisation statistics are
+    # measured on (0 = the workload's own lattice)
+    stats_ncell: int = 0
 
     @property
     def n_elements(self) -> int:
@@ -61,7 +67,14 @@ class Preset:
 
     @property
     def D(self) -> int:
+        """orbital coefficients per atom, one per (n, l)"""
         return self.n_radial * (self.l_max + 1)
+
+    @property
+    def DR(self) -> int:
+        """density features per atom (the networks' input width)"""
+        pairs = self.n_radial * (self.n_radial + 1) // 2 if self.density_form == 1 else self.n_radial
+        return pairs * (self.l_max + 1)
 
     @property
     def masses(self) -> Tuple[float, ...]:
@@ -115,9 +128,23 @@ PRESETS = {
         description="40,000 C2H2 + 40,000 O2 + 2,000 N2 (244,000 atoms) in a 200 A cube, 2.0 A gap; E+F throughput",
         elements=("H", "C", "N", "O"), T=3, r_cut=5.0, n_radial=8, hidden=(64, 64),
         kind="chon", n_mol=(40000, 40000, 2000), box=200.0),
+    # pair-product density variant (D_rho = N_phi (N_phi+1)(L+1)/2 = 108 features)
+    "ag256p": Preset(
+        key="ag256p", index=6,
+        description="Ag FCC 4x4x4 cells (256 atoms), a=4.09 A, sigma=0.05 A, pair-product densities; single E+F",
+        elements=("Ag",), T=2, r_cut=6.0, n_radial=8, hidden=(64, 64),
+        kind="fcc", ncell=4, a=4.09, sigma=0.05, density_form=1),
+    "ag1mp": Preset(
+        key="ag1mp", index=7,
+        description="Ag FCC 64x64x64 cells (1,048,576 atoms), a=4.09 A, sigma=0.05 A, pair-product densities, "
+                    "fp32 networks; 200 velocity-Verlet steps of 1 fs",
+        elements=("Ag",), T=3, r_cut=6.0, n_radial=8, hidden=(128, 128),
+        kind="fcc", ncell=64, a=4.09, sigma=0.05, md_steps=200, dt_fs=1.0, density_form=1, stats_ncell=16),
 }
 
 ORDER = ("ag256", "water3k", "hea108k", "ag1m", "chon244k")
+VARIANTS = ("ag256p", "ag1mp")
+ALL = ORDER + VARIANTS
 
 
 def get(key: str) -> Preset:

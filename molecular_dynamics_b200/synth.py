@@ -246,11 +246,11 @@ def raw_network(p: Preset, layer: int, element: int) -> Dict[str, np.ndarray]:
     """Random draws of one atomic network; layer = t for the coefficient network
     M^t (rho^t -> c^{t+1}), or ENERGY_LAYER for the energy network."""
     seed = seeds(p)[1]
-    D, (H1, H2) = p.D, p.hidden
+    D, DR, (H1, H2) = p.D, p.DR, p.hidden
     n_out = 1 if layer == ENERGY_LAYER else D
     g = lambda k: np.random.default_rng([seed, layer, element, _KIND[k]])
     return {
-        "W1": _xavier(g("W1"), H1, D), "b1": g("b1").uniform(-0.1, 0.1, H1),
+        "W1": _xavier(g("W1"), H1, DR), "b1": g("b1").uniform(-0.1, 0.1, H1),
         "W2": _xavier(g("W2"), H2, H1), "b2": g("b2").uniform(-0.1, 0.1, H2),
         "W3": _xavier(g("W3"), n_out, H2), "b3": g("b3").uniform(-0.1, 0.1, n_out),
     }
@@ -288,10 +288,11 @@ def blob_layout(p: Preset, T: int):
 
     Layout: C0[n_el][D]; then for t = 0..T-2 and each element the coefficient
     network M^t; then for each element the energy network.  Each network is
-    shift[D], scale[D], W1[H1][D], b1[H1], W2[H2][H1], b2[H2], W3[n_out][H2],
-    b3[n_out] (matrices row-major, output index first).
+    shift[DR], scale[DR], W1[H1][DR], b1[H1], W2[H2][H1], b2[H2], W3[n_out][H2],
+    b3[n_out] (matrices row-major, output index first); DR is the density
+    feature count (D for the square form), n_out = D or 1.
     """
-    D, (H1, H2), ne = p.D, p.hidden, p.n_elements
+    D, DR, (H1, H2), ne = p.D, p.DR, p.hidden, p.n_elements
     off = 0
     lay = {"C0": (off, (ne, D))}
     off += ne * D
@@ -299,7 +300,7 @@ def blob_layout(p: Preset, T: int):
     def net(n_out):
         nonlocal off
         d = {}
-        for name, shape in (("shift", (D,)), ("scale", (D,)), ("W1", (H1, D)), ("b1", (H1,)),
+        for name, shape in (("shift", (DR,)), ("scale", (DR,)), ("W1", (H1, DR)), ("b1", (H1,)),
                             ("W2", (H2, H1)), ("b2", (H2,)), ("W3", (n_out, H2)), ("b3", (n_out,))):
             d[name] = (off, shape)
             off += int(np.prod(shape))
@@ -347,8 +348,8 @@ def weight_blob(p: Preset, T: Optional[int] = None, norm=None, use_stored_norm: 
             put(net["shift"], norm[0][t_in, e])
             put(net["scale"], norm[1][t_in, e])
         else:
-            put(net["shift"], np.zeros(p.D))
-            put(net["scale"], np.ones(p.D))
+            put(net["shift"], np.zeros(p.DR))
+            put(net["scale"], np.ones(p.DR))
         for k in ("W1", "b1", "W2", "b2", "W3", "b3"):
             put(net[k], raw[k])
 

@@ -44,7 +44,7 @@ def build(force: bool = False) -> str:
 class Cfg(C.Structure):
     _fields_ = [("n_elements", C.c_int32), ("T", C.c_int32), ("n_radial", C.c_int32), ("l_max", C.c_int32),
                 ("hidden1", C.c_int32), ("hidden2", C.c_int32), ("r_cut", C.c_double), ("skin", C.c_double),
-                ("alpha", C.c_double)]
+                ("alpha", C.c_double), ("density_form", C.c_int32)]
 
 
 _lib = None
@@ -123,15 +123,23 @@ class Model:
     skin: float
     alpha: float
     weights: np.ndarray
+    density_form: int = 0
 
     @classmethod
     def from_preset(cls, p, weights: np.ndarray, T: Optional[int] = None) -> "Model":
         return cls(p.n_elements, p.T if T is None else T, p.n_radial, p.l_max, tuple(p.hidden), p.r_cut, p.skin,
-                   p.alpha, np.ascontiguousarray(weights, dtype=np.float32))
+                   p.alpha, np.ascontiguousarray(weights, dtype=np.float32), getattr(p, "density_form", 0))
 
     @property
     def D(self) -> int:
+        """coefficients per atom: one per (n, l)"""
         return self.n_radial * (self.l_max + 1)
+
+    @property
+    def DR(self) -> int:
+        """density features per atom (network input width)"""
+        pairs = self.n_radial * (self.n_radial + 1) // 2 if self.density_form == 1 else self.n_radial
+        return pairs * (self.l_max + 1)
 
     @property
     def n_tuples(self) -> int:
@@ -139,7 +147,7 @@ class Model:
 
     def cfg(self) -> Cfg:
         return Cfg(self.n_elements, self.T, self.n_radial, self.l_max, self.hidden[0], self.hidden[1], self.r_cut,
-                   self.skin, self.alpha)
+                   self.skin, self.alpha, self.density_form)
 
 
 def _check(rc: int, what: str):
@@ -187,7 +195,7 @@ class Result:
     energy: float
     atom_energy: np.ndarray
     forces: Optional[np.ndarray]
-    rho: Optional[np.ndarray] = None      # [T, N, D]
+    rho: Optional[np.ndarray] = None      # [T, N, DR]
     coef: Optional[np.ndarray] = None     # [T, N, D]
     A: Optional[np.ndarray] = None        # [T, N, N_phi * n_tuples]
 
@@ -206,7 +214,7 @@ def energy_forces(model: Model, x, types, box, pairs=None, forces: bool = True, 
     F = np.zeros((n, 3)) if forces else None
     rho = coef = A = None
     if intermediates:
-        rho = np.zeros((model.T, n, model.D))
+        rho = np.zeros((model.T, n, model.DR))
         coef = np.zeros((model.T, n, model.D))
         A = np.zeros((model.T, n, model.n_radial * model.n_tuples))
     _check(lib().oracle_energy_forces(C.byref(cfg), _p(w), len(w), n, _p(x), _p(types), _p(box), _p(row),
@@ -223,7 +231,7 @@ def rho_pairwise(model: Model, x, box, coef, pairs=None) -> np.ndarray:
     if pairs is None:
         pairs = pairs_brute(x, box, model.r_cut, model.skin)
     row, col = np.ascontiguousarray(pairs[0], np.int64), np.ascontiguousarray(pairs[1], np.int32)
-    rho = np.zeros((n, model.D))
+    rho = np.zeros((n, model.DR))
     cfg = model.cfg()
     _check(lib().oracle_rho_pairwise(C.byref(cfg), n, _p(x), _p(box), _p(row),
                                      _p(col if len(col) else np.zeros(1, np.int32)), _p(coef), _p(rho)),

@@ -62,10 +62,18 @@ ENERGY_SCALE_RECIPE = ("energy network output layer multiplied by +-1/rms(F) of 
                        "take the sign that puts the perfect lattice below the workload's thermal structure")
 
 
+def stats_lattice(p):
+    """FCC workloads: the lattice the statistics and the energy scale are
+    measured on -- the workload's own, or a smaller one of the same recipe
+    (stats_ncell) where the per-feature statistics of the periodic crystal are
+    the same and the oracle is cheaper."""
+    return p.with_(ncell=p.stats_ncell) if p.kind == "fcc" and p.stats_ncell else p
+
+
 def stats_structure(p):
     """The structure the statistics are measured on (see the module text)."""
     if p.kind == "fcc":
-        return synth.make_structure(p.with_(sigma=STATS_SIGMA_FACTOR * p.sigma))
+        return synth.make_structure(stats_lattice(p).with_(sigma=STATS_SIGMA_FACTOR * p.sigma))
     return synth.make_structure(p)
 
 
@@ -78,7 +86,7 @@ def measure(p, verbose=True):
     else:
         pairs = oracle.pairs_cells(pos, box, p.r_cut, p.skin)
     depth = p.stats_depth
-    ne, D = p.n_elements, p.D
+    ne, D = p.n_elements, p.DR
     shift = np.zeros((depth, ne, D))
     scale = np.ones((depth, ne, D))
     sat = []
@@ -121,7 +129,8 @@ def energy_sign(p, shift, scale, lam, verbose=True):
     blob = synth.weight_blob(p, T=p.T, norm=(shift, scale), use_stored_norm=False, energy_scale=abs(lam))
     model = oracle.Model.from_preset(p, blob, T=p.T)
     per_atom = []
-    for q in (p, p.with_(sigma=0.0)):
+    base = stats_lattice(p)
+    for q in (base, base.with_(sigma=0.0)):
         pos, types, box = synth.make_structure(q)
         pairs = oracle.pairs_brute(pos, box, q.r_cut, q.skin) if len(pos) <= 20000 else \
             oracle.pairs_cells(pos, box, q.r_cut, q.skin)

@@ -25,6 +25,12 @@
  *   density    (Eq. 1) A^t_{i,n,tau} = sum_j c^t_{j,(n,l)} phi_n(r_ij) Y_tau(d_ij),
  *              rho^t_{i,(n,l)} = sum_{|tau| = l} l!/(lx! ly! lz!) (A^t_{i,n,tau})^2.
  *              Feature (n, l) sits at index l*N_phi + n; D = N_phi (L+1).
+ *   pair form  (density_form = 1; the dimension N_phi (N_phi+1)(L+1)/2 that
+ *              section "REANN Architecture" states for the density vector)
+ *              rho^t_{i,(n,m,l)} = sum_{|tau| = l} l!/tau! A_{i,n,tau} A_{i,m,tau}
+ *              for n <= m, at index l*P + pair(n, m), P = N_phi (N_phi+1)/2,
+ *              pair(n, m) = n N_phi - n (n-1)/2 + (m - n); the diagonal n = m
+ *              is the square form.  Messages c keep one value per (n, l).
  *   messages   c^0_j is the element row C0[Z_j]; for 1 <= t <= T-1,
  *              c^t_i = M^{t-1}_{Z_i}(rho^{t-1}_i)  (Eq. 2).
  *   energy     E_i = N_{Z_i}(rho^{T-1}_i), E = sum_i E_i (Eq. 3 input).
@@ -61,6 +67,7 @@ typedef struct {
     double r_cut;
     double skin;
     double alpha;
+    int32_t density_form; /* 0: squares per (n, l) (Eq. 1); 1: pair products per (n <= m, l) */
 } oracle_cfg;
 
 enum { ORACLE_OK = 0, ORACLE_ERR_ARG = 1, ORACLE_ERR_BOX = 2, ORACLE_ERR_CAPACITY = 3, ORACLE_ERR_MEM = 4 };
@@ -73,6 +80,15 @@ static const int TUPLE[ORACLE_MAX_TUPLES][3] = {
 };
 
 static int n_tuples(int L) { return (L + 1) * (L + 2) * (L + 3) / 6; }
+
+/* number of density features per atom (network input width) */
+static int n_feat(const oracle_cfg *c) {
+    int NP = c->n_radial;
+    return c->density_form == 1 ? NP * (NP + 1) / 2 * (c->l_max + 1) : NP * (c->l_max + 1);
+}
+
+/* index of the pair (n, m), n <= m, among the N_phi (N_phi+1)/2 pairs */
+static int pair_index(int NP, int n, int m) { return n * NP - n * (n - 1) / 2 + (m - n); }
 static int tuple_l(int tau) { return TUPLE[tau][0] + TUPLE[tau][1] + TUPLE[tau][2]; }
 
 static double factorial(int k) {
@@ -296,13 +312,13 @@ typedef struct {
 } weight_view;
 
 static int64_t net_size(const oracle_cfg *c, int n_out) {
-    int D = c->n_radial * (c->l_max + 1);
+    int D = n_feat(c);
     return 2 * D + (int64_t)c->hidden1 * D + c->hidden1 + (int64_t)c->hidden2 * c->hidden1 + c->hidden2 +
            (int64_t)n_out * c->hidden2 + n_out;
 }
 
 static const float *bind_net(const oracle_cfg *c, const float *p, int n_out, net_view *v) {
-    int D = c->n_radial * (c->l_max + 1);
+    int D = n_feat(c);
     v->n_out = n_out;
     v->shift = p; p += D;
     v->scale = p; p += D;
@@ -339,7 +355,8 @@ static void free_weights(weight_view *v) { free(v->coef); free(v->energy); }
 
 static int check_cfg(const oracle_cfg *c) {
     if (!c || c->n_elements < 1 || c->T < 1 || c->n_radial < 2 || c->l_max < 0 || c->l_max > ORACLE_MAX_L ||
-        c->hidden1 < 1 || c->hidden2 < 1 || !(c->r_cut > 0) || !(c->skin >= 0) || !(c->alpha > 0))
+        c->hidden1 < 1 || c->hidden2 < 1 || !(c->r_cut > 0) || !(c->skin >= 0) || !(c->alpha > 0) ||
+        c->density_form < 0 || c->density_form > 1 || n_feat(c) > 256)
         return ORACLE_ERR_ARG;
     return ORACLE_OK;
 }
@@ -349,8 +366,8 @@ static int check_cfg(const oracle_cfg *c) {
 
 /* hidden activations a1[H1], a2[H2] are returned for reuse by the VJP */
 static void net_forward(const oracle_cfg *c, const net_view *v, const double *x, double *a1, double *a2, double *y) {
-    int D = c->n_radial * (c->l_max + 1), H1 = c->hidden1, H2 = c->hidden2;
-    double xt[64];
+    int D = n_feat(c), H1 = c->hidden1, H2 = c->hidden2;
+    double xt[256];
     for (int f = 0; f < D; ++f) xt[f] = (x[f] - (double)v->shift[f]) / (double)v->scale[f];
     for (int h = 0; h < H1; ++h) {
         double z = v->b1[h];
@@ -372,7 +389,7 @@ static void net_forward(const oracle_cfg *c, const net_view *v, const double *x,
 /* gx = (dy/dx)^T gy, given the activations of net_forward at the same x */
 static void net_vjp(const oracle_cfg *c, const net_view *v, const double *a1, const double *a2, const double *gy,
                     double *gx) {
-    int D = c->n_radial * (c->l_max + 1), H1 = c->hidden1, H2 = c->hidden2;
+    int D = n_feat(c), H1 = c->hidden1, H2 = c->hidden2;
     double g2[512], g1[512];
     for (int k = 0; k < H2; ++k) {
         double s = 0.0;
@@ -430,12 +447,14 @@ static void angular(int ntau, const double d[3], double *Y, double (*dY)[3]) {
 /* Density of one layer (Eq. 1)                                             */
 
 /*
- * A[i][n*ntau + tau] and rho[i][l*N_phi + n] of layer t for every centre,
- * given the neighbour list and the coefficients c[j][l*N_phi + n] of layer t.
+ * A[i][n*ntau + tau] and rho[i][*] of layer t for every centre (n_feat
+ * features: l*N_phi + n, or l*P + pair(n, m) in the pair form), given the
+ * neighbour list and the coefficients c[j][l*N_phi + n] of layer t.
  */
 static void density_layer(const oracle_cfg *c, int64_t n, const double *x, const double *box, const int64_t *row,
                           const int32_t *col, const double *coef, double *A, double *rho) {
-    int D = c->n_radial * (c->l_max + 1), ntau = n_tuples(c->l_max), NP = c->n_radial;
+    int D = c->n_radial * (c->l_max + 1), ntau = n_tuples(c->l_max), NP = c->n_radial, DR = n_feat(c);
+    int P = NP * (NP + 1) / 2;
     #pragma omp parallel for schedule(dynamic, 64)
     for (int64_t i = 0; i < n; ++i) {
         double *Ai = &A[i * NP * ntau];
@@ -453,10 +472,19 @@ static void density_layer(const oracle_cfg *c, int64_t n, const double *x, const
                 for (int tau = 0; tau < ntau; ++tau)
                     Ai[nn * ntau + tau] += coef[j * D + tuple_l(tau) * NP + nn] * phi[nn] * Y[tau];
         }
-        for (int f = 0; f < D; ++f) rho[i * D + f] = 0.0;
-        for (int nn = 0; nn < NP; ++nn)
-            for (int tau = 0; tau < ntau; ++tau)
-                rho[i * D + tuple_l(tau) * NP + nn] += tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[nn * ntau + tau];
+        for (int f = 0; f < DR; ++f) rho[i * DR + f] = 0.0;
+        if (c->density_form == 1) {
+            for (int nn = 0; nn < NP; ++nn)
+                for (int mm = nn; mm < NP; ++mm)
+                    for (int tau = 0; tau < ntau; ++tau)
+                        rho[i * DR + tuple_l(tau) * P + pair_index(NP, nn, mm)] +=
+                            tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[mm * ntau + tau];
+        } else {
+            for (int nn = 0; nn < NP; ++nn)
+                for (int tau = 0; tau < ntau; ++tau)
+                    rho[i * DR + tuple_l(tau) * NP + nn] +=
+                        tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[nn * ntau + tau];
+        }
     }
 }
 
@@ -485,9 +513,10 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
     weight_view w;
     if (bind_weights(c, weights, &w)) return ORACLE_ERR_MEM;
 
-    int T = c->T, D = c->n_radial * (c->l_max + 1), NP = c->n_radial, ntau = n_tuples(c->l_max);
+    int T = c->T, D = c->n_radial * (c->l_max + 1), NP = c->n_radial, ntau = n_tuples(c->l_max), DR = n_feat(c);
+    int P = NP * (NP + 1) / 2;
     int64_t nA = (int64_t)NP * ntau;
-    double *rho = (double *)malloc(sizeof(double) * T * n * D + 1);
+    double *rho = (double *)malloc(sizeof(double) * T * n * DR + 1);
     double *coef = (double *)malloc(sizeof(double) * T * n * D + 1);
     double *A = (double *)malloc(sizeof(double) * T * n * nA + 1);
     double *Ei = (double *)malloc(sizeof(double) * n + 1);
@@ -497,12 +526,12 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
     for (int64_t i = 0; i < n; ++i)
         for (int f = 0; f < D; ++f) coef[i * D + f] = w.C0[types[i] * D + f];
     for (int t = 0; t < T; ++t) {
-        density_layer(c, n, x, box, row, col, &coef[t * n * D], &A[t * n * nA], &rho[t * n * D]);
+        density_layer(c, n, x, box, row, col, &coef[t * n * D], &A[t * n * nA], &rho[t * n * DR]);
         if (t + 1 < T) {
             #pragma omp parallel for schedule(static)
             for (int64_t i = 0; i < n; ++i) {
                 double a1[512], a2[512];
-                net_forward(c, &w.coef[t * c->n_elements + types[i]], &rho[(t * n + i) * D], a1, a2,
+                net_forward(c, &w.coef[t * c->n_elements + types[i]], &rho[(t * n + i) * DR], a1, a2,
                             &coef[((t + 1) * n + i) * D]);
             }
         }
@@ -510,7 +539,7 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
     #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         double a1[512], a2[512];
-        net_forward(c, &w.energy[types[i]], &rho[((T - 1) * n + i) * D], a1, a2, &Ei[i]);
+        net_forward(c, &w.energy[types[i]], &rho[((T - 1) * n + i) * DR], a1, a2, &Ei[i]);
     }
     double E = 0.0;
     for (int64_t i = 0; i < n; ++i) E += Ei[i];
@@ -520,7 +549,7 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
 
     if (forces) {
         int nth = oracle_num_threads();
-        double *g = (double *)malloc(sizeof(double) * n * D + 1);        /* dE/drho^t */
+        double *g = (double *)malloc(sizeof(double) * n * DR + 1);       /* dE/drho^t */
         double *gc = (double *)malloc(sizeof(double) * n * D + 1);       /* dE/dc^t */
         double *gx_t = (double *)calloc((size_t)nth * n * 3 + 1, sizeof(double));
         double *gc_t = (double *)calloc((size_t)nth * n * D + 1, sizeof(double));
@@ -531,8 +560,8 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
         for (int64_t i = 0; i < n; ++i) {
             double a1[512], a2[512], y, one = 1.0;
             const net_view *v = &w.energy[types[i]];
-            net_forward(c, v, &rho[((T - 1) * n + i) * D], a1, a2, &y);
-            net_vjp(c, v, a1, a2, &one, &g[i * D]);
+            net_forward(c, v, &rho[((T - 1) * n + i) * DR], a1, a2, &y);
+            net_vjp(c, v, a1, a2, &one, &g[i * DR]);
         }
         for (int t = T - 1; t >= 0; --t) {
             const double *ct = &coef[t * n * D];
@@ -540,6 +569,7 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
             memset(gc_t, 0, sizeof(double) * (size_t)nth * n * D);
             /* Eq. 4 for centre i and active neighbour j:
              *   dE/dA_{i,n,tau} = 2 w_tau A_{i,n,tau} dE/drho_{i,(n,l)}
+             *     (pair form: w_tau sum_m (1 + [m = n]) A_{i,m,tau} dE/drho_{i,(min, max of n m, l)})
              *   message term:  dE/dc_{j,(n,l)} += sum_tau dE/dA_{i,n,tau} phi_n Y_tau
              *   direct term:   dE/dd_ij = sum_{n,tau} dE/dA_{i,n,tau} c_{j,(n,l)} d(phi_n Y_tau)/dd
              *                  with dd_ij/dx_j = +1 and dd_ij/dx_i = -1 */
@@ -553,9 +583,20 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
                 double *gcl = &gc_t[(int64_t)th * n * D];
                 double GA[21 * ORACLE_MAX_TUPLES];
                 for (int nn = 0; nn < NP; ++nn)
-                    for (int tau = 0; tau < ntau; ++tau)
-                        GA[nn * ntau + tau] = 2.0 * tuple_weight(tau) * At[i * nA + nn * ntau + tau] *
-                                              g[i * D + tuple_l(tau) * NP + nn];
+                    for (int tau = 0; tau < ntau; ++tau) {
+                        if (c->density_form == 1) {
+                            double s = 0.0;
+                            for (int mm = 0; mm < NP; ++mm) {
+                                int a = nn < mm ? nn : mm, b = nn < mm ? mm : nn;
+                                s += (mm == nn ? 2.0 : 1.0) * At[i * nA + mm * ntau + tau] *
+                                     g[i * DR + tuple_l(tau) * P + pair_index(NP, a, b)];
+                            }
+                            GA[nn * ntau + tau] = tuple_weight(tau) * s;
+                        } else {
+                            GA[nn * ntau + tau] = 2.0 * tuple_weight(tau) * At[i * nA + nn * ntau + tau] *
+                                                  g[i * DR + tuple_l(tau) * NP + nn];
+                        }
+                    }
                 for (int64_t q = row[i]; q < row[i + 1]; ++q) {
                     int64_t j = col[q];
                     double d[3];
@@ -594,8 +635,8 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
                 for (int64_t i = 0; i < n; ++i) {
                     double a1[512], a2[512], y[64];
                     const net_view *v = &w.coef[(t - 1) * c->n_elements + types[i]];
-                    net_forward(c, v, &rho[((t - 1) * n + i) * D], a1, a2, y);
-                    net_vjp(c, v, a1, a2, &gc[i * D], &g[i * D]);
+                    net_forward(c, v, &rho[((t - 1) * n + i) * DR], a1, a2, y);
+                    net_vjp(c, v, a1, a2, &gc[i * D], &g[i * DR]);
                 }
             }
         }
@@ -607,7 +648,7 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
             }
         free(g); free(gc); free(gx_t); free(gc_t);
     }
-    if (rho_out) memcpy(rho_out, rho, sizeof(double) * T * n * D);
+    if (rho_out) memcpy(rho_out, rho, sizeof(double) * T * n * DR);
     if (coef_out) memcpy(coef_out, coef, sizeof(double) * T * n * D);
     if (A_out) memcpy(A_out, A, sizeof(double) * T * n * nA);
     free(rho); free(coef); free(A); free(Ei);
@@ -620,13 +661,14 @@ int oracle_energy_forces(const oracle_cfg *c, const float *weights, int64_t weig
  * multinomial theorem, sum_{|tau|=l} l!/tau! Y_tau(d_j) Y_tau(d_k) = (d_j . d_k)^l,
  * so rho_{i,(n,l)} = sum_{j,k} a_j a_k (d_ij . d_ik)^l with
  * a_j = c_{j,(n,l)} phi_n(r_ij), over the active neighbours j, k of i.
- * No Cartesian tuple appears.
+ * Pair form: rho_{i,(n,m,l)} = sum_{j,k} a_{j,n} b_{k,m} (d_ij . d_ik)^l with
+ * b_{k,m} = c_{k,(m,l)} phi_m(r_ik).  No Cartesian tuple appears.
  */
 int oracle_rho_pairwise(const oracle_cfg *c, int64_t n, const double *x, const double *box, const int64_t *row,
                         const int32_t *col, const double *coef, double *rho) {
     int rc = check_cfg(c);
     if (rc) return rc;
-    int D = c->n_radial * (c->l_max + 1), NP = c->n_radial;
+    int D = c->n_radial * (c->l_max + 1), NP = c->n_radial, DR = n_feat(c), P = NP * (NP + 1) / 2;
     #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t i = 0; i < n; ++i) {
         int64_t deg = row[i + 1] - row[i];
@@ -643,16 +685,18 @@ int oracle_rho_pairwise(const oracle_cfg *c, int64_t n, const double *x, const d
             for (int a = 0; a < 3; ++a) dv[3 * m + a] = d[a];
             nb[m++] = col[q];
         }
-        for (int f = 0; f < D; ++f) rho[i * D + f] = 0.0;
+        for (int f = 0; f < DR; ++f) rho[i * DR + f] = 0.0;
         for (int64_t p = 0; p < m; ++p)
             for (int64_t q = 0; q < m; ++q) {
                 double dot = dv[3 * p] * dv[3 * q] + dv[3 * p + 1] * dv[3 * q + 1] + dv[3 * p + 2] * dv[3 * q + 2];
                 for (int l = 0; l <= c->l_max; ++l)
-                    for (int nn = 0; nn < NP; ++nn) {
-                        int f = l * NP + nn;
-                        rho[i * D + f] += coef[nb[p] * D + f] * ph[p * NP + nn] * coef[nb[q] * D + f] *
-                                          ph[q * NP + nn] * ipow(dot, l);
-                    }
+                    for (int nn = 0; nn < NP; ++nn)
+                        for (int mm = nn; mm < (c->density_form == 1 ? NP : nn + 1); ++mm) {
+                            int fn = l * NP + nn, fm = l * NP + mm;
+                            int f = c->density_form == 1 ? l * P + pair_index(NP, nn, mm) : fn;
+                            rho[i * DR + f] += coef[nb[p] * D + fn] * ph[p * NP + nn] * coef[nb[q] * D + fm] *
+                                               ph[q * NP + mm] * ipow(dot, l);
+                        }
             }
         free(dv); free(ph); free(nb);
     }

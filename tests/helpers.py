@@ -19,6 +19,8 @@ def small(key: str):
         p = presets.scaled("chon244k", n_mol=(160, 160, 8), box=31.7)
     elif key == "ag":
         p = presets.scaled("ag1m", ncell=4)
+    elif key == "agp":
+        p = presets.get("ag256p")
     else:
         raise KeyError(key)
     pos, types, box = synth.make_structure(p)

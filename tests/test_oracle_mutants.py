@@ -14,6 +14,7 @@ import pytest
 import oracle
 import test_oracle_density as dens
 import test_oracle_forces as forc
+import test_oracle_pair_density as pairden
 import test_oracle_pairs as pairs
 
 MUTANTS = [
@@ -37,7 +38,7 @@ MUTANTS = [
      "v = v - box[a] * rint(v / box[a]);", "v = v;",
      lambda: pairs.test_fcc_shell_counts(4.09, 6.0, 78, 54)),
     ("energy read from the wrong layer",
-     "&rho[((T - 1) * n + i) * D], a1, a2, &Ei[i]", "&rho[((T > 1 ? T - 2 : 0) * n + i) * D], a1, a2, &Ei[i]",
+     "&rho[((T - 1) * n + i) * DR], a1, a2, &Ei[i]", "&rho[((T > 1 ? T - 2 : 0) * n + i) * DR], a1, a2, &Ei[i]",
      lambda: forc.test_receptive_field_is_T_hops(2)),
     ("tanh derivative wrong",
      "g2[k] = s * (1.0 - a2[k] * a2[k]);", "g2[k] = s * (1.0 - a2[k]);",
@@ -45,6 +46,13 @@ MUTANTS = [
     ("input standardisation dropped in the backward",
      "gx[f] = s / (double)v->scale[f];", "gx[f] = s;",
      lambda: forc.test_forces_match_central_differences("hea", 10)),
+    ("pair form: diagonal factor 2 dropped in the backward",
+     "s += (mm == nn ? 2.0 : 1.0) * At[i * nA + mm * ntau + tau] *", "s += 1.0 * At[i * nA + mm * ntau + tau] *",
+     lambda: pairden.test_pair_forces_match_central_differences()),
+    ("pair form: second factor taken from the same radial index",
+     "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[mm * ntau + tau];",
+     "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[nn * ntau + tau];",
+     lambda: pairden.test_pair_density_matches_pairwise_formula_every_layer()),
 ]
 
 
