@@ -81,6 +81,12 @@ typedef struct {
     int32_t mlp_precision; /* 0 = fp32 networks; 1 = bf16 tensor-core GEMMs, fp32 accumulate */
     int32_t dd_grid[3];    /* {0,0,0} = monolithic; else subdomains per axis (checking mode) */
     int32_t dd_stale_ghosts; /* checking mode only: 1 = skip the per-layer ghost refresh (negative control) */
+    int32_t density_form;    /* 0 = Eq. 1: rho_(n,l) = sum_tau w_tau A_{n,tau}^2, D_rho = N_phi (L+1) features;
+                                1 = pair products rho_(n,m,l) = sum_tau w_tau A_{n,tau} A_{m,tau} for n <= m,
+                                    D_rho = N_phi (N_phi+1)(L+1)/2 features (the density dimension stated in
+                                    section "REANN Architecture"); fp32 networks and N_phi = 8 only
+                                    (REANN_ERR_UNSUPPORTED otherwise).  The messages c keep one value per
+                                    (n, l) in both forms. */
 } reann_config;
 
 /*
@@ -89,8 +95,10 @@ typedef struct {
  *   for t = 0..T-2, for e = 0..n_elements-1: coefficient network M^t_e (rho^t -> c^{t+1}), n_out = D
  *   for e = 0..n_elements-1:                 energy network N_e (rho^{T-1} -> E_i), n_out = 1
  * and each network is
- *   shift[D], scale[D], W1[H1][D], b1[H1], W2[H2][H1], b2[H2], W3[n_out][H2], b3[n_out]
- * evaluating y = W3 tanh(W2 tanh(W1 ((x - shift) / scale) + b1) + b2) + b3.
+ *   shift[Dr], scale[Dr], W1[H1][Dr], b1[H1], W2[H2][H1], b2[H2], W3[n_out][H2], b3[n_out]
+ * evaluating y = W3 tanh(W2 tanh(W1 ((x - shift) / scale) + b1) + b2) + b3, with
+ * D = N_phi (L+1) coefficients per atom and Dr density features per atom
+ * (Dr = D, or N_phi (N_phi+1)(L+1)/2 for density_form = 1).
  */
 
 typedef struct {
@@ -217,8 +225,9 @@ reann_status reann_get_neighbors(reann_ctx *ctx, int64_t *row, int32_t *col, int
 
 /*
  * Diagnostics (parity tests).  After reann_energy_forces, copies layer t's
- * per-atom embedded density rho^t (float32 [n][D]) and coefficients c^t
- * (float32 [n][D]) in the caller's atom order.  Either pointer may be NULL.
+ * per-atom embedded density rho^t (float32 [n][Dr], Dr as in the weight blob)
+ * and coefficients c^t (float32 [n][D]) in the caller's atom order.  Either
+ * pointer may be NULL.
  * Synchronises the stream.  Errors: REANN_ERR_STATE, REANN_ERR_ARG.
  */
 reann_status reann_get_features(reann_ctx *ctx, int32_t t, float *rho, float *coef, reann_stream stream);

@@ -81,15 +81,16 @@ void dfree(T *&p) {
 }
 
 int64_t net_size(const reann_ctx *c, int n_out) {
-    return 2LL * c->D + (int64_t)c->H1 * c->D + c->H1 + (int64_t)c->H2 * c->H1 + c->H2 + (int64_t)n_out * c->H2 + n_out;
+    return 2LL * c->DR + (int64_t)c->H1 * c->DR + c->H1 + (int64_t)c->H2 * c->H1 + c->H2 + (int64_t)n_out * c->H2 +
+           n_out;
 }
 
 NetOffsets bind_net(const reann_ctx *c, int64_t &off, int n_out) {
     NetOffsets o;
     o.n_out = n_out;
-    o.shift = off; off += c->D;
-    o.scale = off; off += c->D;
-    o.W1 = off; off += (int64_t)c->H1 * c->D;
+    o.shift = off; off += c->DR;
+    o.scale = off; off += c->DR;
+    o.W1 = off; off += (int64_t)c->H1 * c->DR;
     o.b1 = off; off += c->H1;
     o.W2 = off; off += (int64_t)c->H2 * c->H1;
     o.b2 = off; off += c->H2;
@@ -125,7 +126,7 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_cnt, N));
     CK(dalloc(&c->d_act_cnt, N));
     CK(dalloc(&c->d_A, (size_t)c->T * N * c->NA));
-    CK(dalloc(&c->d_rho, (size_t)c->T * N * c->D));
+    CK(dalloc(&c->d_rho, (size_t)c->T * N * c->DR));
     CK(dalloc(&c->d_coef, (size_t)c->T * N * c->D));
     CK(dalloc(&c->d_G, N * c->NA));
     CK(dalloc(&c->d_dc, N * c->D));
@@ -139,7 +140,7 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_stage_e, N));
     CK(dalloc(&c->d_x, 3 * N));
     CK(dalloc(&c->d_v, 3 * N));
-    CK(dalloc(&c->d_diag, N * (size_t)std::max(c->D, c->NA)));
+    CK(dalloc(&c->d_diag, N * (size_t)std::max(c->DR, c->NA)));
     CK(dalloc(&c->d_last_x, 3 * N));
     CK(dalloc(&c->d_last_v, 3 * N));
     if (c->dd) CK(dalloc(&c->d_dd_sub, N));
@@ -472,6 +473,10 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
                 return fail(nullptr, REANN_ERR_ARG, "dd_grid: all zero, or 1..64 subdomains per axis");
         if (cfg->dd_stale_ghosts < 0 || cfg->dd_stale_ghosts > 1) return fail(nullptr, REANN_ERR_ARG, "dd_stale_ghosts");
     }
+    if (cfg->density_form < 0 || cfg->density_form > 1) return fail(nullptr, REANN_ERR_ARG, "density_form is 0 or 1");
+    if (cfg->density_form == 1 && (cfg->mlp_precision != 0 || cfg->n_radial != 8 || cfg->l_max != 2))
+        return fail(nullptr, REANN_ERR_UNSUPPORTED,
+                    "the pair-product density form is built for fp32 networks, N_phi = 8 and L = 2");
     reann_ctx *c = new reann_ctx();
     c->cfg = *cfg;
     c->device = device;
@@ -481,6 +486,7 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     }
     c->NP = cfg->n_radial;
     c->D = c->NP * (cfg->l_max + 1);
+    c->DR = cfg->density_form == 1 ? c->NP * (c->NP + 1) / 2 * (cfg->l_max + 1) : c->D;
     c->NA = c->NP * NT;
     c->T = cfg->T;
     c->ne = cfg->n_elements;
@@ -766,11 +772,11 @@ extern "C" reann_status reann_get_features(reann_ctx *c, int32_t t, float *rho, 
     if (!c->have_eval) return fail(c, REANN_ERR_STATE, "no evaluation yet");
     DeviceGuard guard(c->device);
     cudaStream_t s = (cudaStream_t)stream;
-    const int64_t n = c->n, nD = n * c->D;
+    const int64_t n = c->n, nD = n * c->D, nR = n * c->DR;
     if (n == 0) return REANN_OK;
     if (rho) {
-        CK(launch_to_caller_rows(c, c->d_rho + t * nD, c->D, c->d_diag, s));
-        CK(cudaMemcpyAsync(rho, c->d_diag, sizeof(float) * nD, cudaMemcpyDefault, s));
+        CK(launch_to_caller_rows(c, c->d_rho + t * nR, c->DR, c->d_diag, s));
+        CK(cudaMemcpyAsync(rho, c->d_diag, sizeof(float) * nR, cudaMemcpyDefault, s));
         CK(sync_stream(c, s));
     }
     if (coef) {

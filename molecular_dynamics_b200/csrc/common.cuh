@@ -73,6 +73,7 @@ struct reann_ctx {
     int device = 0;
     int sm_count = 0;
     int NP = 0, D = 0, NA = 0, T = 0, ne = 0, H1 = 0, H2 = 0;
+    int DR = 0;   // density features per atom (network input width): D, or N_phi (N_phi+1)(L+1)/2 in the pair form
 
     // weights
     float *d_w = nullptr;

@@ -219,13 +219,14 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         }
     }
     float *Ao = A_out + (int64_t)i * NA;
-    float *ro = rho_out + (int64_t)i * D;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
         const int nn = n0 + m;
         const float *v = acc[m];
 #pragma unroll
         for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(v[u], v[u + 1]);
+        if (!rho_out) continue;   // pair form: rho from A in k_rho_pair
+        float *ro = rho_out + (int64_t)i * D;
         ro[nn] = v[0] * v[0];
         ro[NP + nn] = v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
         ro[2 * NP + nn] = v[4] * v[4] + v[5] * v[5] + v[6] * v[6] + 2.f * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]);
@@ -380,6 +381,32 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
 }
 
 // ---------------------------------------------------------------------------
+// Pair-product densities (density_form = 1): rho_(n,m,l) = sum_{|tau|=l}
+// l!/tau! A_{n,tau} A_{m,tau} for n <= m, at index l P + pair(n, m) with
+// P = N_phi (N_phi+1)/2 and pair(n, m) = n N_phi - n (n-1)/2 + (m - n); the
+// density dimension N_phi (N_phi+1)(L+1)/2 of section "REANN Architecture".
+// One thread per (atom, pair); the atom's A row is read from L1.
+template <int NP>
+__global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict__ A, float *__restrict__ rho) {
+    constexpr int P = NP * (NP + 1) / 2, NA = NP * NT, DR = 3 * P;
+    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= (int64_t)n * P) return;
+    const int64_t i = k / P;
+    const int p = (int)(k - i * P);
+    int a = 0, first = 0;
+    while (first + (NP - a) <= p) {   // row a of the upper triangle holds pairs (a, a..NP-1)
+        first += NP - a;
+        ++a;
+    }
+    const int b = a + (p - first);
+    const float *x = A + i * NA + a * NT, *y = A + i * NA + b * NT;
+    float *ro = rho + i * DR;
+    ro[p] = x[0] * y[0];
+    ro[P + p] = x[1] * y[1] + x[2] * y[2] + x[3] * y[3];
+    ro[2 * P + p] = x[4] * y[4] + x[5] * y[5] + x[6] * y[6] + 2.f * (x[7] * y[7] + x[8] * y[8] + x[9] * y[9]);
+}
+
+// ---------------------------------------------------------------------------
 // host wrappers
 
 cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
@@ -387,8 +414,19 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
-    float *rho = c->d_rho + (int64_t)t * c->n * c->D;
-    REANN_TIMED(c, REANN_K_DENSITY, s);
+    const bool pair = c->cfg.density_form == 1;
+    float *rho = pair ? nullptr : c->d_rho + (int64_t)t * c->n * c->D;
+    REANN_TIMED(c, REANN_K_DENSITY, s, pair ? 2 : 1);
+    if (pair) {
+        if (c->NP != 8) return cudaErrorInvalidValue;
+        const int64_t threads = c->n * (8 * 9 / 2);
+        k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, nullptr,
+            P);
+        k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>((int)c->n, A,
+                                                                        c->d_rho + (int64_t)t * c->n * c->DR);
+        return cudaGetLastError();
+    }
     if (c->NP == 8)
         k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
             (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);

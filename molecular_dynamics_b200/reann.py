@@ -39,7 +39,8 @@ class ReannError(RuntimeError):
 class Config(C.Structure):
     _fields_ = [("n_elements", C.c_int32), ("T", C.c_int32), ("n_radial", C.c_int32), ("l_max", C.c_int32),
                 ("hidden", C.c_int32 * 2), ("r_cut", C.c_double), ("skin", C.c_double), ("alpha", C.c_double),
-                ("mlp_precision", C.c_int32), ("dd_grid", C.c_int32 * 3), ("dd_stale_ghosts", C.c_int32)]
+                ("mlp_precision", C.c_int32), ("dd_grid", C.c_int32 * 3), ("dd_stale_ghosts", C.c_int32),
+                ("density_form", C.c_int32)]
 
 
 class MdStats(C.Structure):
@@ -140,13 +141,20 @@ class ModelSpec:
     mlp_precision: int = 0
     dd_grid: Sequence[int] = (0, 0, 0)
     dd_stale_ghosts: int = 0
+    density_form: int = 0
 
     @classmethod
     def from_preset(cls, p, T: Optional[int] = None, mlp_precision: Optional[int] = None, dd_grid=(0, 0, 0),
                     dd_stale_ghosts: int = 0):
         return cls(p.n_elements, p.T if T is None else T, p.n_radial, p.l_max, tuple(p.hidden), p.r_cut, p.skin,
                    p.alpha, p.mlp_precision if mlp_precision is None else mlp_precision, tuple(dd_grid),
-                   dd_stale_ghosts)
+                   dd_stale_ghosts, getattr(p, "density_form", 0))
+
+    @property
+    def DR(self) -> int:
+        """density features per atom"""
+        pairs = self.n_radial * (self.n_radial + 1) // 2 if self.density_form == 1 else self.n_radial
+        return pairs * (self.l_max + 1)
 
     def config(self) -> Config:
         c = Config()
@@ -157,6 +165,7 @@ class ModelSpec:
         for k in range(3):
             c.dd_grid[k] = self.dd_grid[k]
         c.dd_stale_ghosts = self.dd_stale_ghosts
+        c.density_form = self.density_form
         return c
 
 
@@ -244,9 +253,9 @@ class Context:
         return out
 
     def reann_get_features(self, t: int, stream=None):
-        """(rho^t, c^t), float32 [n][D] each, caller order, numpy."""
+        """(rho^t [n][Dr], c^t [n][D]), float32, caller order, numpy."""
         D = self.spec.n_radial * (self.spec.l_max + 1)
-        rho = np.zeros((self.n, D), np.float32)
+        rho = np.zeros((self.n, self.spec.DR), np.float32)
         coef = np.zeros((self.n, D), np.float32)
         self._check(self.lib.reann_get_features(self.h, int(t), rho.ctypes.data, coef.ctypes.data, _stream(stream)))
         return rho, coef

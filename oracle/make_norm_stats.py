@@ -8,8 +8,9 @@ not available, and random Xavier weights applied to raw embedded densities
 (values up to ~1e3 with a spread of a few percent) would saturate tanh and
 leave the forces near zero.  So each network sees (rho - shift) / scale,
 with shift = mean(rho^t_f) and scale = std(rho^t_f) + 0.05 mean|rho^t_f|
-+ 1e-6, measured per layer t, per element of the centre atom and per
-feature f on the workload's own seeded structure.  Layer t's statistics are
++ 1e-6 (0.106 for the pair-product form, see floor()), measured per layer
+t, per element of the centre atom and per feature f on the workload's own
+seeded structure.  Layer t's statistics are
 measured with the networks of layers < t already standardised.
 
 The 0.05 mean|rho| floor bounds the conditioning mean|rho| / scale by 20.
@@ -54,6 +55,21 @@ import oracle
 from molecular_dynamics_b200 import presets, synth
 
 FLOOR = 0.05
+
+
+def floor(p):
+    """The floor of the standardisation scale, as a fraction of mean|rho|.
+
+    It bounds the conditioning mean|rho| / scale by 1 / floor, and with it how
+    far the fp32 rounding of a feature moves the standardised input.  In a
+    crystal that rounding is nearly the same in every atom, so its effect on
+    the first layer's pre-activation adds up coherently over the features: the
+    pair-product form (N_phi (N_phi+1)(L+1)/2 features instead of N_phi (L+1))
+    takes the floor times sqrt(features / N_phi (L+1)), which keeps that sum at
+    the square form's level (0.05 -> 0.106 for N_phi = 8)."""
+    return FLOOR * float(np.sqrt(p.DR / p.D))
+
+
 OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "molecular_dynamics_b200", "data")
 
 
@@ -100,7 +116,7 @@ def measure(p, verbose=True):
             sel = types == e
             r = rho[sel]
             mu = r.mean(0)
-            sd = r.std(0) + FLOOR * np.abs(r).mean(0) + 1e-6
+            sd = r.std(0) + floor(p) * np.abs(r).mean(0) + 1e-6
             shift[t, e] = np.float32(mu)
             scale[t, e] = np.float32(sd)
             # diagnostic: fraction of first-layer pre-activations beyond |3|
