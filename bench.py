@@ -202,16 +202,33 @@ def dd_sweep(args):
     return 0
 
 
-def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk):
-    """Roofline entry of the dominant kernel group: algorithmic FP32 operations
-    per launch (per-pair counts x active pairs) over its mean CUDA-event launch
-    time, against the FP32 FMA peak of the SM count at clocks.max.sm."""
+def network_flop_per_atom(group, d_in, d_out, hidden):
+    """Algorithmic flops of one network launch per atom: a forward pass is
+    2 (d_in H1 + H1 H2 + H2 d_out); the energy launch adds its VJP (same
+    count with d_out = 1), the coefficient backward recomputes the forward and
+    runs the VJP."""
+    h1, h2 = hidden
+    fwd = lambda o: 2 * (d_in * h1 + h1 * h2 + h2 * o)
+    return {"mlp_fwd": fwd(d_out), "mlp_energy": 2 * fwd(1), "mlp_bwd": 2 * fwd(d_out)}[group]
+
+
+def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None):
+    """Roofline entry of the dominant kernel group: algorithmic operations per
+    launch over its mean CUDA-event launch time.  Edge passes and fp32
+    networks: FP32 FMA peak of the SM count at clocks.max.sm; bf16 tensor-core
+    networks: the measured sustained bf16 peak.  `net` = (d_in, d_out, hidden,
+    mlp_precision) of the workload's networks."""
     shares = {k: v_[0] for k, v_ in prof.items()}
     dominant = max(shares, key=shares.get)
+    tensor = False
     if dominant == "edge_bwd":
         flop_per_launch = active_pairs * (FLOP_EDGE_BWD_PER_PAIR[NP][0] + (T - 1) * FLOP_EDGE_BWD_PER_PAIR[NP][1]) / T
     elif dominant == "density":
         flop_per_launch = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
+    elif dominant.startswith("mlp_") and net is not None:
+        d_in, d_out, hidden, prec = net
+        flop_per_launch = n_atoms * network_flop_per_atom(dominant, d_in, d_out, hidden)
+        tensor = prec == 1
     else:
         return None
     ms_dom, n_dom = prof[dominant]
@@ -219,18 +236,26 @@ def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk):
         return None
     smax = pk.get("sm_max_mhz", 1965.0)
     clock_mhz = clk.get("sm_mhz") or smax
-    peak_tf = sm_count * 128 * 2 * smax * 1e6 / 1e12
     achieved = flop_per_launch / (ms_dom / n_dom * 1e-3) / 1e12
     traffic = None
     if dominant == "edge_bwd" and EDGE_BWD_TRAFFIC_PER_ATOM is not None:
         traffic = EDGE_BWD_TRAFFIC_PER_ATOM * n_atoms
-    return {"kernel": {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}[dominant], "bound": "alu",
+    kernel = {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}.get(
+        dominant, ("k_mlp_tc" if tensor else "k_mlp") + {"mlp_fwd": " (coefficient networks)",
+                                                          "mlp_energy": " (energy network + VJP)",
+                                                          "mlp_bwd": " (coefficient-network VJP)"}.get(dominant, ""))
+    if tensor:
+        peak_tf = pk.get("bf16_tflops_sustained", 1400.0)
+        peak_note = f"bf16 dense, sustained ({pk_kind})"
+    else:
+        peak_tf = sm_count * 128 * 2 * smax * 1e6 / 1e12
+        peak_note = (f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {smax:.0f} MHz "
+                     f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz")
+    return {"kernel": kernel, "bound": "tensor" if tensor else "alu",
             "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
             "traffic": traffic,
-            "traffic_note": EDGE_BWD_TRAFFIC_NOTE,
-            "peak_note": f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {smax:.0f} MHz "
-                         f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz",
-            "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
+            "traffic_note": EDGE_BWD_TRAFFIC_NOTE if traffic is not None else "no DRAM capture of this kernel",
+            "peak_note": peak_note, "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
 
 
 def main():
@@ -331,7 +356,8 @@ def main():
     sm_count = torch.cuda.get_device_properties(info.local).multi_processor_count
     shares = {k: v_[0] for k, v_ in prof.items()}
     total = sum(shares.values()) or 1.0
-    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk)
+    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk,
+                    net=(p.DR, p.D, tuple(p.hidden), p.mlp_precision))
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -105,3 +105,13 @@ def test_roofline_arithmetic():
     # a dominant group with no algorithmic count has no entry
     assert bench.roofline({"mlp_bwd": (5.0, 1)}, pairs, 8, 3, 1, 148, {}, "fallback", {}) is None
     json.dumps(roof)
+    # dominant fp32 networks: 2 (108*128 + 128*128 + 128*24) flop per forward, doubled for the VJP launch
+    r2 = bench.roofline({"mlp_bwd": (8.0, 2), "edge_bwd": (1.0, 3)}, pairs, 8, 3, 1000, 148, {"sm_max_mhz": 2000.0},
+                        "measured", {}, net=(108, 24, (128, 128), 0))
+    assert r2["bound"] == "alu"
+    assert r2["flop_per_launch"] == 1000 * 2 * 2 * (108 * 128 + 128 * 128 + 128 * 24)
+    assert r2["achieved"] == pytest.approx(r2["flop_per_launch"] / 4e-3 / 1e12)
+    # bf16 tensor-core networks: against the sustained bf16 peak
+    r3 = bench.roofline({"mlp_fwd": (8.0, 2)}, pairs, 8, 3, 1000, 148, {"bf16_tflops_sustained": 1382.5}, "measured",
+                        {}, net=(24, 24, (128, 128), 1))
+    assert r3["bound"] == "tensor" and r3["peak"] == 1382.5
