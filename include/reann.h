@@ -84,9 +84,9 @@ typedef struct {
     int32_t density_form;    /* 0 = Eq. 1: rho_(n,l) = sum_tau w_tau A_{n,tau}^2, D_rho = N_phi (L+1) features;
                                 1 = pair products rho_(n,m,l) = sum_tau w_tau A_{n,tau} A_{m,tau} for n <= m,
                                     D_rho = N_phi (N_phi+1)(L+1)/2 features (the density dimension stated in
-                                    section "REANN Architecture"); fp32 networks and N_phi = 8 only
-                                    (REANN_ERR_UNSUPPORTED otherwise).  The messages c keep one value per
-                                    (n, l) in both forms. */
+                                    section "REANN Architecture"); N_phi = 8, L = 2 and equal hidden
+                                    widths only (REANN_ERR_UNSUPPORTED otherwise).  The messages c keep
+                                    one value per (n, l) in both forms. */
 } reann_config;
 
 /*

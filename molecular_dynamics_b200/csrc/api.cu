@@ -309,7 +309,7 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
 
 // One energy+force evaluation on the internal positions d_pos.
 reann_status run_ef(reann_ctx *c, cudaStream_t s) {
-    const bool tc = c->cfg.mlp_precision == 1;
+    const bool tc = c->cfg.mlp_precision == 1, pair = c->cfg.density_form == 1;
     const int64_t cstride = c->n_slots * c->D;
     // domain-decomposed mode: ghost positions follow their owners
     if (c->dd) CK(dd_gather_rows(c, reinterpret_cast<float *>(c->d_pos), 4, s));
@@ -317,7 +317,8 @@ reann_status run_ef(reann_ctx *c, cudaStream_t s) {
     for (int t = 0; t < c->T; ++t) {
         CK(launch_density_fwd(c, t, s));
         if (t + 1 < c->T) {
-            CK(tc ? launch_mlp_tc_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s));
+            CK(tc ? (pair ? launch_mlp_tc_pair_coef_fwd(c, t, s) : launch_mlp_tc_coef_fwd(c, t, s))
+                  : launch_mlp_coef_fwd(c, t, s));
             // the per-layer message sync: ghost c^{t+1} from the owners (or, as
             // a negative control, the ghosts keep c^0)
             if (c->dd) {
@@ -326,12 +327,13 @@ reann_status run_ef(reann_ctx *c, cudaStream_t s) {
             }
         }
     }
-    CK(tc ? launch_mlp_tc_energy(c, s) : launch_mlp_energy(c, s));
+    CK(tc ? (pair ? launch_mlp_tc_pair_energy(c, s) : launch_mlp_tc_energy(c, s)) : launch_mlp_energy(c, s));
     if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
     for (int t = c->T - 1; t >= 0; --t) {
         CK(launch_edge_bwd(c, t, t != c->T - 1, s));
         if (t >= 1) {
-            CK(tc ? launch_mlp_tc_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s));
+            CK(tc ? (pair ? launch_mlp_tc_pair_coef_bwd(c, t, s) : launch_mlp_tc_coef_bwd(c, t, s))
+                  : launch_mlp_coef_bwd(c, t, s));
             if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
         }
     }
@@ -474,9 +476,9 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
         if (cfg->dd_stale_ghosts < 0 || cfg->dd_stale_ghosts > 1) return fail(nullptr, REANN_ERR_ARG, "dd_stale_ghosts");
     }
     if (cfg->density_form < 0 || cfg->density_form > 1) return fail(nullptr, REANN_ERR_ARG, "density_form is 0 or 1");
-    if (cfg->density_form == 1 && (cfg->mlp_precision != 0 || cfg->n_radial != 8 || cfg->l_max != 2))
+    if (cfg->density_form == 1 && (cfg->n_radial != 8 || cfg->l_max != 2 || cfg->hidden[0] != cfg->hidden[1]))
         return fail(nullptr, REANN_ERR_UNSUPPORTED,
-                    "the pair-product density form is built for fp32 networks, N_phi = 8 and L = 2");
+                    "the pair-product density form is built for N_phi = 8, L = 2 and equal hidden widths");
     reann_ctx *c = new reann_ctx();
     c->cfg = *cfg;
     c->device = device;

@@ -42,6 +42,11 @@ bool tc_supported(const reann_ctx *c);
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
 cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
+// tensor-core networks for the pair-product density form (mlp_tc_pair.cu)
+bool tc_pair_supported(const reann_ctx *c);
+cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
+cudaError_t launch_mlp_tc_pair_energy(reann_ctx *c, cudaStream_t s);
+cudaError_t launch_mlp_tc_pair_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
 
 // reductions, gathers and the integrator (md.cu)
 cudaError_t launch_pos_from_caller(reann_ctx *c, const float *d_pos_caller, cudaStream_t s);

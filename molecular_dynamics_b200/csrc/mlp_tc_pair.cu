@@ -1,0 +1,401 @@
+// Tensor-core atomic networks for the pair-product density form
+// (density_form = 1, N_phi = 8, L = 2: 108 density features per atom, the
+// dimension N_phi (N_phi+1)(L+1)/2 stated in section "REANN Architecture" of
+// "Efficient Parallelization of Message Passing Neural Network Potentials for
+// Large-Scale Molecular Dynamics").  Same networks, split-bf16 operands and
+// fp32 TMEM accumulators as mlp_tc.cu; what differs is the width of the first
+// layer (K = 112, the 108 features padded) and of the input-gradient product
+// (N = 112), which no longer fit two tiles in flight per SM.  So one 512-thread
+// block per SM works on one 128-atom tile at a time: warp w reads TMEM lanes
+// 32 (w % 4) .. + 31, and warp group w / 4 takes one 32-column chunk of every
+// 128-wide accumulator.
+//
+// Inputs: the next tile's 108-wide rho rows are prefetched into registers in
+// element order (coalesced) while the current tile computes, and each thread
+// then writes its elements, standardised and split into bf16 hi + lo, straight
+// into the K-major operand tile.  Outputs leave through idle buffers: the
+// coefficient rows through the input tile (consumed by the first product), the
+// 108-wide dE/drho rows through the activation tile (consumed by the last).
+// dE/dA (Eq. 4 for the pair form):
+//   G_{n,tau} = l!/tau! sum_m (1 + [m = n]) A_{m,tau} dE/drho_(min(n,m), max(n,m), l),
+// one element per thread and step in the edge kernels' lane-interleaved order.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace reann {
+namespace {
+
+constexpr int PT = 512;       // threads per block
+constexpr int PNP = 8;        // N_phi
+constexpr int PP = PNP * (PNP + 1) / 2;   // radial pairs
+constexpr int DIN = 3 * PP;   // 108 density features
+constexpr int KIN = 112;      // padded to a multiple of 16
+constexpr int PD = 3 * PNP;   // 24 coefficients
+constexpr int PNA = PNP * NT; // 80 A values per atom
+constexpr int GXS = DIN + 1;  // padded fp32 row stride of dE/drho rows
+constexpr int YS = PD + 1;    // padded fp32 row stride of output rows
+
+template <int MODE>
+struct PairLayout {
+    static constexpr int W1 = 0;                                  // [128][KIN]
+    static constexpr int W2 = W1 + 128 * KIN * 2;                 // [128][128]
+    static constexpr int W3 = W2 + 128 * 128 * 2;                 // [KPAD][128]
+    static constexpr int X = W3 + KPAD * 128 * 2;                 // [TM][KIN] x 2
+    static constexpr int DY = X + 2 * TM * KIN * 2;               // [TM][KPAD] x 2 (BWD)
+    static constexpr int ACT = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][128] x 2
+    static constexpr int F32 = ACT + 2 * TM * 128 * 2;
+    static constexpr int nf32 = 128 + 128 + KPAD + 2 * KIN + 128 + 4 * TM;   // b1, b2, b3, shift, 1/scale, w3, e parts
+    static constexpr int BAR = F32 + nf32 * 4;
+    static constexpr int bytes = BAR + 32;
+    static constexpr int C_Z1 = 0, C_Z2 = 128, C_P = 256, C_OUT = 384;
+    static_assert(TM * GXS * 4 <= 2 * TM * 128 * 2, "dE/drho rows fit the activation tile");
+    static_assert(TM * YS * 4 <= (KIN / 8 - 1) * TM * 16, "output rows leave the input tile's padding chunk alone");
+    static_assert(X % 16 == 0 && DY % 16 == 0 && ACT % 16 == 0 && F32 % 16 == 0, "16-byte aligned tiles");
+};
+
+// one value as a bf16 pair (hi = bf16(v), lo = bf16(v - hi)) at (r, k) of two K-major tiles
+__device__ __forceinline__ void st_elem2(unsigned char *hi, unsigned char *lo, int R, int r, int k, float v) {
+    const uint32_t a = __float_as_uint(v) + 0x8000u;
+    const float l = v - __uint_as_float(a & 0xFFFF0000u);
+    const uint32_t off = kmaj(r, k, R);
+    *reinterpret_cast<unsigned short *>(hi + off) = (unsigned short)(a >> 16);
+    *reinterpret_cast<unsigned short *>(lo + off) = (unsigned short)((__float_as_uint(l) + 0x8000u) >> 16);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(PT, 1)
+    k_mlp_tc_pair(const int4 *__restrict__ tiles, int n_tiles, const float *__restrict__ w, TcNets nets,
+                  const float *__restrict__ X, float *__restrict__ Y, const float *__restrict__ dY,
+                  float *__restrict__ Ei, const float *__restrict__ A, float *__restrict__ Gout,
+                  int *__restrict__ status) {
+    using L = PairLayout<MODE>;
+    constexpr int DOUT = MODE == TC_ENERGY ? 1 : PD;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    float *f32 = reinterpret_cast<float *>(sm + L::F32);
+    float *sb1 = f32, *sb2 = sb1 + 128, *sb3 = sb2 + 128, *sshift = sb3 + KPAD, *sinv = sshift + KIN,
+          *sw3 = sinv + KIN, *se = sw3 + 128;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
+    unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KIN * 2;
+    unsigned char *dy_hi = sm + L::DY, *dy_lo = dy_hi + TM * KPAD * 2;
+    unsigned char *act_hi = sm + L::ACT, *act_lo = act_hi + TM * 128 * 2;
+    float *ystage = reinterpret_cast<float *>(x_hi);     // output rows (forward), after the first product
+    float *gxs = reinterpret_cast<float *>(act_hi);      // dE/drho rows, after the last product
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & (TM - 1);
+    const int qc = tid / TM;
+    const int c = 32 * qc;
+    const uint32_t base = smem_u32(sm);
+    auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // operand tiles start at zero: the padding columns (features 108..111,
+    // upstream gradients 24..31) are never written again
+    for (int k = tid; k < (2 * TM * KIN * 2) / 16; k += PT)
+        reinterpret_cast<uint4 *>(x_hi)[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (MODE == TC_BWD)
+        for (int k = tid; k < (2 * TM * KPAD * 2) / 16; k += PT)
+            reinterpret_cast<uint4 *>(dy_hi)[k] = make_uint4(0u, 0u, 0u, 0u);
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    uint32_t phase = 0;
+    bool failed = false;
+    int cur = -1;
+
+    auto wait_mma = [&]() -> bool {
+        bool ok = bar_wait(bar, phase);
+        phase ^= 1u;
+        fence_after();
+        return !__syncthreads_or(!ok);
+    };
+    auto handoff = [&]() {
+        fence_smem_to_async();
+        fence_before();
+        __syncthreads();
+    };
+
+    // the next tile's raw rows in element order (coalesced); the descriptor is
+    // read one tile further ahead so the addresses are known when the loads issue
+    constexpr int NXR = (TM * DIN + PT - 1) / PT;   // 27
+    constexpr int NDR = (TM * PD + PT - 1) / PT;    // 6
+    float xr[NXR], dr[NDR];
+    int4 tl = make_int4(0, 0, 0, 0);
+    int4 tl2 = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);
+    auto prefetch = [&](int t2) {
+        tl = tl2;
+        const float *xg = X + (int64_t)tl.y * DIN;
+        const int cnt = tl.z * DIN;
+#pragma unroll
+        for (int u = 0; u < NXR; ++u) {
+            const int k = tid + u * PT;
+            xr[u] = k < cnt ? xg[k] : 0.f;
+        }
+        if (MODE == TC_BWD) {
+            const float *dg = dY + (int64_t)tl.y * PD;
+            const int cd = tl.z * PD;
+#pragma unroll
+            for (int u = 0; u < NDR; ++u) {
+                const int k = tid + u * PT;
+                dr[u] = k < cd ? dg[k] : 0.f;
+            }
+        }
+        const int t3 = t2 + gridDim.x;
+        tl2 = t3 < n_tiles ? tiles[t3] : make_int4(0, 0, 0, 0);
+    };
+    prefetch(blockIdx.x);
+
+    for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
+        const int4 tile = tl;
+        const int e = tile.x, r0 = tile.y, rows = tile.z;
+        if (e != cur) {
+            const NetOffsets &o = nets.net[e];
+            for (int k = tid; k < 128 * KIN; k += PT) {
+                const int n = k / KIN, f = k % KIN;
+                st_elem(sm + L::W1, 128, n, f, f < DIN ? w[o.W1 + (int64_t)n * DIN + f] : 0.f);
+            }
+            for (int k = tid; k < 128 * 128; k += PT) st_elem(sm + L::W2, 128, k / 128, k % 128, w[o.W2 + k]);
+            for (int k = tid; k < KPAD * 128; k += PT) {
+                const int n = k / 128, h = k % 128;
+                st_elem(sm + L::W3, KPAD, n, h, n < DOUT ? w[o.W3 + (int64_t)n * 128 + h] : 0.f);
+            }
+            for (int k = tid; k < 128; k += PT) {
+                sb1[k] = w[o.b1 + k];
+                sb2[k] = w[o.b2 + k];
+                sw3[k] = MODE == TC_ENERGY ? w[o.W3 + k] : 0.f;
+            }
+            for (int k = tid; k < KPAD; k += PT) sb3[k] = k < DOUT ? w[o.b3 + k] : 0.f;
+            for (int k = tid; k < KIN; k += PT) {
+                sshift[k] = k < DIN ? w[o.shift + k] : 0.f;
+                sinv[k] = k < DIN ? 1.0f / w[o.scale + k] : 0.f;
+            }
+            cur = e;
+            __syncthreads();
+        }
+        if (MODE != TC_FWD && tid == 0) prefetch_l2(A + (int64_t)r0 * PNA, (uint32_t)(rows * PNA * 4));
+        // this thread's elements of the tile: standardised, split bf16, into the operand tiles
+#pragma unroll
+        for (int u = 0; u < NXR; ++u) {
+            const int k = tid + u * PT;
+            if (k < rows * DIN) {
+                const int rk = k / DIN, f = k - rk * DIN;
+                st_elem2(x_hi, x_lo, TM, rk, f, (xr[u] - sshift[f]) * sinv[f]);
+            }
+        }
+        if (MODE == TC_BWD) {
+#pragma unroll
+            for (int u = 0; u < NDR; ++u) {
+                const int k = tid + u * PT;
+                if (k < rows * PD) {
+                    const int rk = k / PD, f = k - rk * PD;
+                    st_elem2(dy_hi, dy_lo, TM, rk, f, dr[u]);
+                }
+            }
+        }
+        prefetch(ti + gridDim.x);
+        handoff();
+
+        if (tid == 0) {
+            fence_after();
+            gemm2<128, KIN, false, 0>(tmem + L::C_Z1, sa(x_hi), sa(x_lo), base + L::W1);
+            if (MODE == TC_BWD) gemm2<128, KPAD, true, KPAD>(tmem + L::C_P, sa(dy_hi), sa(dy_lo), base + L::W3);
+            mma_commit(bar);
+        }
+        if (!wait_mma()) { failed = true; break; }
+        {
+            float v[32];
+            tmem_ld32(lane_base + L::C_Z1 + c, v);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb1[c + u]);
+#pragma unroll
+            for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
+        }
+        handoff();
+        if (tid == 0) {
+            fence_after();
+            gemm2<128, 128, false, 0>(tmem + L::C_Z2, sa(act_hi), sa(act_lo), base + L::W2);
+            mma_commit(bar);
+        }
+        if (!wait_mma()) { failed = true; break; }
+
+        if (MODE == TC_FWD) {
+            {
+                float v[32];
+                tmem_ld32(lane_base + L::C_Z2 + c, v);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = tanh_fast(v[u] + sb2[c + u]);
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
+            }
+            handoff();
+            if (tid == 0) {
+                fence_after();
+                gemm2<KPAD, 128, false, 0>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W3);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            {
+                float v[8];
+                tmem_ld8(lane_base + L::C_OUT + 8 * qc, v);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int f = 8 * qc + u;
+                    if (f < PD) ystage[row * YS + f] = v[u] + sb3[f];
+                }
+            }
+            __syncthreads();
+            float *yo = Y + (int64_t)r0 * PD;
+            for (int k = tid; k < rows * PD; k += PT) {
+                const int rk = k / PD;
+                yo[k] = ystage[rk * YS + (k - rk * PD)];
+            }
+        } else {
+            {
+                float z[32], up[32];
+                tmem_ld32(lane_base + L::C_Z2 + c, z);
+                if (MODE == TC_BWD) tmem_ld32(lane_base + L::C_P + c, up);
+                float e_row = 0.f;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const float a = tanh_fast(z[u] + sb2[c + u]);
+                    const float g = MODE == TC_ENERGY ? sw3[c + u] : up[u];
+                    if (MODE == TC_ENERGY) e_row = fmaf(sw3[c + u], a, e_row);
+                    z[u] = g * (1.f - a * a);
+                }
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &z[u]);
+                if (MODE == TC_ENERGY) se[qc * TM + row] = e_row;
+            }
+            handoff();
+            if (MODE == TC_ENERGY && qc == 0 && row < rows)
+                Ei[r0 + row] = ((se[row] + se[TM + row]) + (se[2 * TM + row] + se[3 * TM + row])) + sb3[0];
+            if (tid == 0) {
+                fence_after();
+                gemm2<128, 128, true, 128>(tmem + L::C_P, sa(act_hi), sa(act_lo), base + L::W2);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            {
+                float p[32], z[32];
+                tmem_ld32(lane_base + L::C_P + c, p);
+                tmem_ld32(lane_base + L::C_Z1 + c, z);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const float a = tanh_fast(z[u] + sb1[c + u]);
+                    p[u] *= 1.f - a * a;
+                }
+#pragma unroll
+                for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &p[u]);
+            }
+            handoff();
+            // dE/dx = g1 W1 (MN-major view of W1): the 112 padded input columns
+            if (tid == 0) {
+                fence_after();
+                gemm2<KIN, 128, true, 128>(tmem + L::C_OUT, sa(act_hi), sa(act_lo), base + L::W1);
+                mma_commit(bar);
+            }
+            if (!wait_mma()) { failed = true; break; }
+            // dE/drho rows through the activation tile (consumed by the last product)
+            {
+                float v[32];
+                tmem_ld32(lane_base + L::C_OUT + c, v);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int f = c + u;
+                    if (f < DIN) gxs[row * GXS + f] = v[u] * sinv[f];
+                }
+            }
+            __syncthreads();
+            float *go = Gout + (int64_t)r0 * PNA;
+            const float *ag = A + (int64_t)r0 * PNA;
+            for (int k = tid; k < rows * PNA; k += PT) {
+                const int rk = k / PNA, q = k - rk * PNA;
+                const int src = g_slot_source(q, PNP), nn = src / NT, u = src - nn * NT;
+                const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
+                const float *g = gxs + rk * GXS + l * PP;
+                const float *ar = ag + (int64_t)rk * PNA + u;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < PNP; ++m) {
+                    const int lo = m < nn ? m : nn, hi = m < nn ? nn : m;
+                    const float f = (m == nn ? 2.f : 1.f) * g[lo * PNP - lo * (lo - 1) / 2 + (hi - lo)];
+                    acc = fmaf(f, ar[m * NT], acc);
+                }
+                go[k] = (u >= 7 ? 2.f : 1.f) * acc;
+            }
+        }
+        fence_before();
+        __syncthreads();
+    }
+
+    if (failed && tid == 0) atomicOr(status, ST_TIMEOUT);
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+}
+
+template <int MODE>
+cudaError_t run_pair(reann_ctx *c, const TcNets &nets, const float *X, float *Y, const float *dY, float *Ei,
+                     const float *A, float *G, cudaStream_t s) {
+    using L = PairLayout<MODE>;
+    static_assert(L::bytes > 116 * 1024 && L::bytes <= 227 * 1024, "one block per SM keeps TMEM allocation safe");
+    static bool configured[64] = {};
+    auto kern = k_mlp_tc_pair<MODE>;
+    if (c->device < 0 || c->device >= 64) return cudaErrorInvalidDevice;
+    if (!configured[c->device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::bytes);
+        if (e) return e;
+        configured[c->device] = true;
+    }
+    if (c->n_tiles128 == 0) return cudaSuccess;
+    const int grid = c->sm_count < c->n_tiles128 ? c->sm_count : c->n_tiles128;
+    REANN_TIMED(c, MODE == TC_FWD ? REANN_K_MLP_FWD : (MODE == TC_ENERGY ? REANN_K_MLP_ENERGY : REANN_K_MLP_BWD), s);
+    kern<<<grid, PT, L::bytes, s>>>(c->d_tiles128, c->n_tiles128, c->d_w, nets, X, Y, dY, Ei, A, G, c->d_status);
+    return cudaGetLastError();
+}
+
+TcNets pair_nets(const std::vector<NetOffsets> &v, int first, int ne) {
+    TcNets m;
+    for (int e = 0; e < ne; ++e) m.net[e] = v[first + e];
+    return m;
+}
+
+}  // namespace
+
+bool tc_pair_supported(const reann_ctx *c) {
+    return c->cfg.density_form == 1 && c->NP == PNP && c->DR == DIN && c->H1 == 128 && c->H2 == 128;
+}
+
+cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
+    const int64_t nR = c->n * c->DR;
+    return run_pair<TC_FWD>(c, pair_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nR,
+                            c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
+}
+
+cudaError_t launch_mlp_tc_pair_energy(reann_ctx *c, cudaStream_t s) {
+    const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
+    const int t = c->T - 1;
+    return run_pair<TC_ENERGY>(c, pair_nets(c->energy_nets, 0, c->ne), c->d_rho + t * nR, nullptr, nullptr, c->d_Ei,
+                               c->d_A + t * nA, c->d_G, s);
+}
+
+cudaError_t launch_mlp_tc_pair_coef_bwd(reann_ctx *c, int t, cudaStream_t s) {
+    const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
+    return run_pair<TC_BWD>(c, pair_nets(c->coef_nets, (t - 1) * c->ne, c->ne), c->d_rho + (t - 1) * nR, nullptr,
+                            c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
+}
+
+}  // namespace reann

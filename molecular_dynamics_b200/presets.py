@@ -136,9 +136,9 @@ PRESETS = {
         kind="fcc", ncell=4, a=4.09, sigma=0.05, density_form=1),
     "ag1mp": Preset(
         key="ag1mp", index=7,
-        description="Ag FCC 64x64x64 cells (1,048,576 atoms), a=4.09 A, sigma=0.05 A, pair-product densities, "
-                    "fp32 networks; 200 velocity-Verlet steps of 1 fs",
-        elements=("Ag",), T=3, r_cut=6.0, n_radial=8, hidden=(128, 128),
+        description="Ag FCC 64x64x64 cells (1,048,576 atoms), a=4.09 A, sigma=0.05 A, pair-product densities; "
+                    "200 velocity-Verlet steps of 1 fs",
+        elements=("Ag",), T=3, r_cut=6.0, n_radial=8, hidden=(128, 128), mlp_precision=1,
         kind="fcc", ncell=64, a=4.09, sigma=0.05, md_steps=200, dt_fs=1.0, density_form=1, stats_ncell=16),
 }
 

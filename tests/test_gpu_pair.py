@@ -61,6 +61,19 @@ def test_pair_larger_lattice_parity():
         assert_forces_close(F, ref.forces)
 
 
+@pytest.mark.parametrize("ncell", [8, 7])
+def test_pair_tensor_core_networks_parity(ncell):
+    # bf16 tensor-core networks (split activations, bf16-valued weights): the
+    # bf16 force tolerance; tiles of 128 rows, ragged at 1,372 atoms
+    p = presets.scaled("ag1mp", ncell=ncell)
+    pos, types, box = synth.make_structure(p)
+    _, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=1)
+    ref = oracle_eval(p, pos, types, box)
+    _energy_close(E, ref.energy, len(pos))
+    _atoms_close(Ei, ref.atom_energy)
+    assert_forces_close(F, ref.forces, 1)
+
+
 def test_pair_domain_decomposed_bit_identical():
     torch = torch_cuda()
     p = presets.scaled("ag1mp", ncell=8)
@@ -94,14 +107,16 @@ def test_pair_md_anchored_steps():
     assert abs(st.e_pot - ep[-1]) / len(pos) < 1e-5
 
 
-def test_pair_full_size_sampled():
-    # the 1M-atom pair workload: sampled forces and atomic energies against the
-    # oracle on the cluster of every atom within 2 T r_c; zero net force
+@pytest.mark.parametrize("prec", [1, 0])
+def test_pair_full_size_sampled(prec):
+    # the 1M-atom pair workload (its bf16 tensor-core networks, and fp32 ones):
+    # sampled forces and atomic energies against the oracle on the cluster of
+    # every atom within 2 T r_c; zero net force
     p = presets.get("ag1mp")
     pos, types, box = synth.make_structure(p)
     n = len(pos)
     w = synth.weight_blob(p)
-    _, E, F, Ei = gpu_eval(p, pos, types, box, weights=w)
+    _, E, F, Ei = gpu_eval(p, pos, types, box, weights=w, mlp_precision=prec)
     assert np.abs(F.sum(0)).max() <= 1e-4 * np.sqrt(n) + 1e-3
     assert abs(Ei.sum() - E) <= 1e-6 * n + 1e-4 * abs(E)
     radius = 2 * p.T * p.r_cut + 0.5
@@ -109,14 +124,14 @@ def test_pair_full_size_sampled():
     for k in rng.choice(n, size=3, replace=False):
         cpos, ctypes_, cbox, _ = cluster_around(pos, types, box, k, radius)
         ref = oracle_eval(p, cpos, ctypes_, cbox, weights=w)
-        assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[0], (k, F[k], ref.forces[0])
+        assert np.abs(F[k] - ref.forces[0]).max() <= F_TOL[prec], (k, F[k], ref.forces[0])
         rel = abs(Ei[k] - ref.atom_energy[0]) / max(float(np.sqrt(np.mean(Ei ** 2))), 0.1)
-        assert rel <= 10 * E_TOL[0], (k, Ei[k], ref.atom_energy[0])
+        assert rel <= 10 * E_TOL[prec], (k, Ei[k], ref.atom_energy[0])
 
 
 def test_pair_form_rejects_unsupported_configs():
     p = presets.get("ag256p")
-    for spec in (reann.ModelSpec.from_preset(p, mlp_precision=1),
+    for spec in (reann.ModelSpec.from_preset(p.with_(hidden=(64, 128))),
                  reann.ModelSpec.from_preset(p.with_(n_radial=10))):
         with pytest.raises(reann.ReannError):
             reann.Context(spec, np.zeros(10, np.float32))
