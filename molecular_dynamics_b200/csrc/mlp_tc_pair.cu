@@ -10,15 +10,16 @@
 // 32 (w % 4) .. + 31, and warp group w / 4 takes one 32-column chunk of every
 // 128-wide accumulator.
 //
-// Inputs: the next tile's 108-wide rho rows are prefetched into registers in
-// element order (coalesced) while the current tile computes, and each thread
-// then writes its elements, standardised and split into bf16 hi + lo, straight
-// into the K-major operand tile.  Outputs leave through idle buffers: the
+// Inputs: the next tile's 108-wide rho rows are prefetched into L2 (one bulk
+// prefetch) while the current tile computes; each tile loads its rows in
+// element order (coalesced) and each thread writes its elements, standardised
+// and split into bf16 hi + lo, straight into the K-major operand tile.  Outputs leave through idle buffers: the
 // coefficient rows through the input tile (consumed by the first product), the
 // 108-wide dE/drho rows through the activation tile (consumed by the last).
 // dE/dA (Eq. 4 for the pair form):
 //   G_{n,tau} = l!/tau! sum_m (1 + [m = n]) A_{m,tau} dE/drho_(min(n,m), max(n,m), l),
-// one element per thread and step in the edge kernels' lane-interleaved order.
+// four threads per atom, each owning two radial indices and writing its 20
+// values as five float4 in the edge kernels' lane-interleaved order.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -127,39 +128,16 @@ __global__ void __launch_bounds__(PT, 1)
         __syncthreads();
     };
 
-    // the next tile's raw rows in element order (coalesced); the descriptor is
-    // read one tile further ahead so the addresses are known when the loads issue
+    // raw rows: the next tile's (contiguous) rows are prefetched into L2 while
+    // the current tile computes; each tile then loads its own rows from L2 in
+    // element order (coalesced), so no registers stay live across a tile
     constexpr int NXR = (TM * DIN + PT - 1) / PT;   // 27
     constexpr int NDR = (TM * PD + PT - 1) / PT;    // 6
-    float xr[NXR], dr[NDR];
-    int4 tl = make_int4(0, 0, 0, 0);
-    int4 tl2 = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);
-    auto prefetch = [&](int t2) {
-        tl = tl2;
-        const float *xg = X + (int64_t)tl.y * DIN;
-        const int cnt = tl.z * DIN;
-#pragma unroll
-        for (int u = 0; u < NXR; ++u) {
-            const int k = tid + u * PT;
-            xr[u] = k < cnt ? xg[k] : 0.f;
-        }
-        if (MODE == TC_BWD) {
-            const float *dg = dY + (int64_t)tl.y * PD;
-            const int cd = tl.z * PD;
-#pragma unroll
-            for (int u = 0; u < NDR; ++u) {
-                const int k = tid + u * PT;
-                dr[u] = k < cd ? dg[k] : 0.f;
-            }
-        }
-        const int t3 = t2 + gridDim.x;
-        tl2 = t3 < n_tiles ? tiles[t3] : make_int4(0, 0, 0, 0);
-    };
-    prefetch(blockIdx.x);
-
+    int4 tl = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);
     for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
         const int4 tile = tl;
         const int e = tile.x, r0 = tile.y, rows = tile.z;
+        tl = ti + (int)gridDim.x < n_tiles ? tiles[ti + gridDim.x] : make_int4(0, 0, 0, 0);
         if (e != cur) {
             const NetOffsets &o = nets.net[e];
             for (int k = tid; k < 128 * KIN; k += PT) {
@@ -184,17 +162,39 @@ __global__ void __launch_bounds__(PT, 1)
             cur = e;
             __syncthreads();
         }
-        if (MODE != TC_FWD && tid == 0) prefetch_l2(A + (int64_t)r0 * PNA, (uint32_t)(rows * PNA * 4));
+        if (tid == 0) {
+            if (MODE != TC_FWD) prefetch_l2(A + (int64_t)r0 * PNA, (uint32_t)(rows * PNA * 4));
+            if (tl.z > 0) {
+                prefetch_l2(X + (int64_t)tl.y * DIN, (uint32_t)(tl.z * DIN * 4));
+                if (MODE == TC_BWD) prefetch_l2(dY + (int64_t)tl.y * PD, (uint32_t)(tl.z * PD * 4));
+            }
+        }
         // this thread's elements of the tile: standardised, split bf16, into the operand tiles
+        {
+            const float *xg = X + (int64_t)r0 * DIN;
+            float xr[NXR];
 #pragma unroll
-        for (int u = 0; u < NXR; ++u) {
-            const int k = tid + u * PT;
-            if (k < rows * DIN) {
-                const int rk = k / DIN, f = k - rk * DIN;
-                st_elem2(x_hi, x_lo, TM, rk, f, (xr[u] - sshift[f]) * sinv[f]);
+            for (int u = 0; u < NXR; ++u) {
+                const int k = tid + u * PT;
+                xr[u] = k < rows * DIN ? xg[k] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < NXR; ++u) {
+                const int k = tid + u * PT;
+                if (k < rows * DIN) {
+                    const int rk = k / DIN, f = k - rk * DIN;
+                    st_elem2(x_hi, x_lo, TM, rk, f, (xr[u] - sshift[f]) * sinv[f]);
+                }
             }
         }
         if (MODE == TC_BWD) {
+            const float *dg = dY + (int64_t)r0 * PD;
+            float dr[NDR];
+#pragma unroll
+            for (int u = 0; u < NDR; ++u) {
+                const int k = tid + u * PT;
+                dr[u] = k < rows * PD ? dg[k] : 0.f;
+            }
 #pragma unroll
             for (int u = 0; u < NDR; ++u) {
                 const int k = tid + u * PT;
@@ -204,7 +204,6 @@ __global__ void __launch_bounds__(PT, 1)
                 }
             }
         }
-        prefetch(ti + gridDim.x);
         handoff();
 
         if (tid == 0) {
@@ -318,22 +317,54 @@ __global__ void __launch_bounds__(PT, 1)
                 }
             }
             __syncthreads();
-            float *go = Gout + (int64_t)r0 * PNA;
-            const float *ag = A + (int64_t)r0 * PNA;
-            for (int k = tid; k < rows * PNA; k += PT) {
-                const int rk = k / PNA, q = k - rk * PNA;
-                const int src = g_slot_source(q, PNP), nn = src / NT, u = src - nn * NT;
-                const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
-                const float *g = gxs + rk * GXS + l * PP;
-                const float *ar = ag + (int64_t)rk * PNA + u;
-                float acc = 0.f;
+            // G = dE/dA: thread (atom rk, part) takes radial indices n = 2 part, 2 part + 1.  Per l it
+            // forms the coupling rows M_{n,m} = (1 + [m = n]) dE/drho_(min, max of n m, l) once and
+            // streams the atom's A_{m,tau}; its 20 results are the lane-interleaved positions
+            // 16 q + 4 part + e (q < 5, e < 4), i.e. five float4 stores.
+            {
+                const int rk = tid >> 2, part = tid & 3;
+                if (rk < rows) {
+                    const float *g = gxs + rk * GXS;
+                    const float *ar = A + (int64_t)(r0 + rk) * PNA;
+                    float acc[2][NT];
 #pragma unroll
-                for (int m = 0; m < PNP; ++m) {
-                    const int lo = m < nn ? m : nn, hi = m < nn ? nn : m;
-                    const float f = (m == nn ? 2.f : 1.f) * g[lo * PNP - lo * (lo - 1) / 2 + (hi - lo)];
-                    acc = fmaf(f, ar[m * NT], acc);
+                    for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                        for (int u = 0; u < NT; ++u) acc[s2][u] = 0.f;
+#pragma unroll
+                    for (int l = 0; l < 3; ++l) {
+                        float M[2][PNP];
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int n = 2 * part + s2;
+#pragma unroll
+                            for (int m = 0; m < PNP; ++m) {
+                                const int lo = m < n ? m : n, hi = m < n ? n : m;
+                                M[s2][m] = (m == n ? 2.f : 1.f) * g[l * PP + lo * PNP - lo * (lo - 1) / 2 + (hi - lo)];
+                            }
+                        }
+                        constexpr int T0[3] = {0, 1, 4}, T1[3] = {1, 4, 10};
+#pragma unroll
+                        for (int u = T0[l]; u < T1[l]; ++u)
+#pragma unroll
+                            for (int m = 0; m < PNP; ++m) {
+                                const float a = ar[m * NT + u];
+                                acc[0][u] = fmaf(M[0][m], a, acc[0][u]);
+                                acc[1][u] = fmaf(M[1][m], a, acc[1][u]);
+                            }
+                    }
+                    float4 *go4 = reinterpret_cast<float4 *>(Gout + (int64_t)(r0 + rk) * PNA);
+#pragma unroll
+                    for (int q = 0; q < 5; ++q) {
+                        float v[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int idx = 4 * q + e2, s2 = idx / NT, u = idx % NT;
+                            v[e2] = (u >= 7 ? 2.f : 1.f) * acc[s2][u];   // l!/tau!
+                        }
+                        go4[4 * q + part] = make_float4(v[0], v[1], v[2], v[3]);
+                    }
                 }
-                go[k] = (u >= 7 ? 2.f : 1.f) * acc;
             }
         }
         fence_before();
