@@ -98,3 +98,44 @@ def test_host_state_equals_device_state():
     sh = _ctx(p, pos, types, box).reann_md_step(6, 0.5, xh, vh, p.masses)
     assert np.array_equal(xd.cpu().numpy(), xh) and np.array_equal(vd.cpu().numpy(), vh)
     assert sd.e_pot == sh.e_pot
+
+
+def _gpu_run(ctx, x, v, dt, n, p):
+    torch = torch_cuda()
+    xd = torch.from_numpy(x.copy()).cuda()
+    vd = torch.from_numpy(v.copy()).cuda()
+    st = ctx.reann_md_step(n, dt, xd, vd, p.masses)
+    return xd.cpu().numpy(), vd.cpu().numpy(), st
+
+
+def test_time_reversal_on_gpu():
+    # k steps forward, negate v, k steps: velocity Verlet returns to the start;
+    # with fp32 forces the return is exact up to their rounding
+    p, pos, types, box = small("water")
+    v0 = synth.maxwell_boltzmann(p, types, temperature=100.0)
+    x0 = pos.astype(np.float64)
+    ctx = _ctx(p, pos, types, box)
+    x1, v1, _ = _gpu_run(ctx, x0, v0, 0.25, 20, p)
+    x2, v2, _ = _gpu_run(ctx, x1, -v1, 0.25, 20, p)
+    assert np.abs(_min_image(x2 - x0, box)).max() < 1e-5
+    assert np.abs(v2 + v0).max() < 1e-5
+
+
+def test_energy_error_is_second_order_on_gpu():
+    # the NVE total-energy error over a fixed time shrinks about fourfold when dt halves
+    p, pos, types, box = small("water")
+    v0 = synth.maxwell_boltzmann(p, types, temperature=100.0)
+    x0 = pos.astype(np.float64)
+    errs = []
+    for dt, n in ((0.4, 10), (0.2, 20)):
+        ctx = _ctx(p, pos, types, box)
+        et = []
+        x, v = x0, v0
+        for _ in range(n):
+            x, v, st = _gpu_run(ctx, x, v, dt, 1, p)
+            if not et:
+                et.append(st.e_pot0 + st.e_kin0)
+            et.append(st.e_pot + st.e_kin)
+        errs.append(np.abs(np.array(et) - et[0]).max())
+    ratio = errs[0] / errs[1]
+    assert 3.0 < ratio < 5.0, (ratio, errs)
