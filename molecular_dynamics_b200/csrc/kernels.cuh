@@ -38,12 +38,10 @@ cudaError_t dd_gather_rows(reann_ctx *c, float *base, int width, cudaStream_t s)
 cudaError_t dd_stale_coef(reann_ctx *c, float *coef, cudaStream_t s);
 
 // atomic networks on tcgen05 tensor cores, bf16 operands (mlp_tc.cu)
-bool tc_supported(const reann_ctx *c);
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
 cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
 // tensor-core networks for the pair-product density form (mlp_tc_pair.cu)
-bool tc_pair_supported(const reann_ctx *c);
 cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
 cudaError_t launch_mlp_tc_pair_energy(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_mlp_tc_pair_coef_bwd(reann_ctx *c, int t, cudaStream_t s);

@@ -446,8 +446,6 @@ TcNets tc_nets(const std::vector<NetOffsets> &v, int first, int ne) {
 
 }  // namespace
 
-bool tc_supported(const reann_ctx *c) { return (c->NP == 8 || c->NP == 10) && c->H1 == 128 && c->H2 == 128; }
-
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nD = c->n * c->D;
     return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD,

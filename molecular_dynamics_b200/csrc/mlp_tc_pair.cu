@@ -406,10 +406,6 @@ TcNets pair_nets(const std::vector<NetOffsets> &v, int first, int ne) {
 
 }  // namespace
 
-bool tc_pair_supported(const reann_ctx *c) {
-    return c->cfg.density_form == 1 && c->NP == PNP && c->DR == DIN && c->H1 == 128 && c->H2 == 128;
-}
-
 cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nR = c->n * c->DR;
     return run_pair<TC_FWD>(c, pair_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nR,
