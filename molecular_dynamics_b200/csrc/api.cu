@@ -5,12 +5,16 @@
 // Large-Scale Molecular Dynamics":
 //   forward  (section "REANN Architecture", Eqs. 1-2)
 //     t = 0 .. T-1:  A^t, rho^t from c^t (c^0 = element table)   [edge.cu]
-//                    c^{t+1} = M^t(rho^t) for t < T-1            [mlp.cu]
-//     E_i = N(rho^{T-1}) and G^{T-1} = dE/dA^{T-1}                [mlp.cu]
+//                    c^{t+1} = M^t(rho^t) for t < T-1            [mlp*.cu]
+//     E_i = N(rho^{T-1}) and G^{T-1} = dE/dA^{T-1}                [mlp*.cu]
 //   backward (section "Parallelization Algorithm", Eqs. 3-5)
 //     t = T-1 .. 0:  F += edge VJP, dE/dc^t                      [edge.cu]
-//                    G^{t-1} from M^{t-1}'s VJP (Eq. 5)          [mlp.cu]
+//                    G^{t-1} from M^{t-1}'s VJP (Eq. 5)          [mlp*.cu]
 //   E = sum_i E_i (deterministic fp64 tree)                      [md.cu]
+// The networks run on the tensor cores (mlp_tc.cu; mlp_tc_pair.cu for the
+// pair-product densities) or, with fp32 networks, on the CUDA cores (mlp.cu).
+// reann_md_step replays each step's evaluation and closing half kick as a
+// CUDA graph captured once per neighbour list (ef_and_kick).
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>

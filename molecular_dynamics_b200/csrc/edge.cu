@@ -26,6 +26,9 @@
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
+// With pair-product densities (density_form = 1) the density pass writes A
+// only and k_rho_pair forms rho_(n,m,l) = sum_tau l!/tau! A_{n,tau} A_{m,tau};
+// the backward pass is the same in both forms (it consumes G = dE/dA).
 #include <algorithm>
 
 #include "common.cuh"

@@ -17,27 +17,26 @@
 // canonical K-major layout (one activation buffer, reused by every layer once
 // the product that read it has completed), and one thread issues the next MMA.
 //
-// Block: 512 threads, one per SM (shared memory > half an SM), persistent over
-// the tiles.  Warp w reads TMEM lanes 32 (w % 4) .. + 31; warp group w / 4
-// takes one 32-column chunk of every 128-wide accumulator, so a tile row is
-// shared by four threads.  The epilogue is bound by the tanh unit: bf16
-// rounding of the split operands is done with integer instructions so that
-// the special-function pipe only evaluates tanh.
+// Block: 512 threads, one per SM (shared memory > half an SM), working through
+// a contiguous range of one element's tiles (the element's weights are loaded
+// once).  The block runs two independent groups of 256 threads, each on every
+// other tile of the range with its own 256 TMEM columns, operand buffers,
+// MMA-completion mbarrier and named barrier, so one group's epilogue overlaps
+// the other's products.  In a group, warp w reads TMEM lanes 32 (w % 4) .. + 31
+// and half (w / 4) % 2 takes 64 columns of every 128-wide accumulator.  The
+// epilogue is bound by the tanh unit: bf16 rounding of the split operands is
+// done with integer instructions so that the special-function pipe only
+// evaluates tanh.  The coefficient backward recomputes the first layer's
+// pre-activation (one small product) instead of keeping it, to fit 256 columns.
 //
-// Global traffic is contiguous: the next tile's raw inputs are prefetched in
-// element order while the current tile computes and transposed to rows through
-// the idle activation buffer; forward outputs leave through the idle input
-// buffer; for the energy network and the coefficient backward the tile's A rows
-// arrive by one bulk copy (cp.async.bulk, completion on an mbarrier) issued at
-// the start of the tile, and dE/dA = 2 w_tau A dE/drho is written one warp per
-// row in the edge kernels' lane-interleaved order.  All waits (MMA completion,
-// bulk copy) are bounded: a wait that gives up sets ST_TIMEOUT, the block waits
-// once more for a copy still in flight, frees its tensor memory and returns.
-//
-// Shared-memory operand layout (K-major, no swizzle): an R x K bf16 tile keeps
-// element (r, k) at byte (k/8) R 16 + (r/8) 128 + (r%8) 16 + (k%8) 2, i.e.
-// 8-row x 16-byte core matrices, 128 B between 8-row groups (SBO) and R*16 B
-// between 16-byte K chunks (LBO).
+// Global traffic is contiguous: each tile's raw inputs are loaded in element
+// order and transposed to rows through the idle activation buffer; forward
+// outputs leave the same way; for the energy network and the coefficient
+// backward the tile's A rows are prefetched into L2 at the start of the tile,
+// and dE/dA = 2 w_tau A dE/drho is written one warp per row in the edge
+// kernels' lane-interleaved order.  All MMA-completion waits are bounded: a wait
+// that gives up sets ST_TIMEOUT, and the block frees its tensor memory and
+// returns.  The shared-memory operand layout is described in tc_common.cuh.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
