@@ -139,3 +139,25 @@ def test_energy_error_is_second_order_on_gpu():
         errs.append(np.abs(np.array(et) - et[0]).max())
     ratio = errs[0] / errs[1]
     assert 3.0 < ratio < 5.0, (ratio, errs)
+
+
+def test_graph_replay_matches_eager_launches(monkeypatch):
+    # reann_md_step replays each step's evaluation as a CUDA graph; with
+    # REANN_GRAPHS=0 at context creation it launches eagerly.  Same trajectory
+    # bit for bit, same kernel-launch count.
+    torch = torch_cuda()
+    p, pos, types, box = small("water")
+    v0 = synth.maxwell_boltzmann(p, types)
+    out = []
+    for graphs in ("1", "0"):
+        monkeypatch.setenv("REANN_GRAPHS", graphs)
+        ctx = _ctx(p, pos, types, box)
+        x = torch.from_numpy(pos.astype(np.float64)).cuda()
+        v = torch.from_numpy(v0.copy()).cuda()
+        k0 = ctx.reann_get_counters().kernel_launches
+        st = ctx.reann_md_step(30, p.dt_fs, x, v, p.masses)
+        out.append((x.cpu().numpy(), v.cpu().numpy(), st.e_pot, ctx.reann_get_counters().kernel_launches - k0,
+                    st.rebuilds))
+    assert np.array_equal(out[0][0], out[1][0]) and np.array_equal(out[0][1], out[1][1])
+    assert out[0][2] == out[1][2]
+    assert out[0][3] == out[1][3] and out[0][4] == out[1][4]
