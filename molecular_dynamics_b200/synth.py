@@ -223,6 +223,15 @@ def maxwell_boltzmann(p: Preset, types: np.ndarray, seed: Optional[int] = None,
     return v * np.sqrt(Tk / t_now)
 
 
+def thermostat_noise(n_atoms: int, nsteps: int, seed: int) -> np.ndarray:
+    """The random numbers of stochastic velocity rescaling, two per step:
+    R1 ~ N(0, 1) and S = a sum of Nf - 1 squared standard normals
+    (Nf = 3 n - 3), drawn as a chi-squared variate; [nsteps][2]."""
+    rng = np.random.default_rng(seed)
+    nf = 3 * n_atoms - 3
+    return np.stack([rng.standard_normal(nsteps), rng.chisquare(nf - 1, nsteps)], axis=1)
+
+
 # ----------------------------------------------------------------------------
 # weights
 

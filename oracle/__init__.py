@@ -94,6 +94,8 @@ def _bind_signatures(cdll):
     cdll.oracle_energy_forces.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, P, P, P, P, P, P]
     cdll.oracle_rho_pairwise.argtypes = [P, C.c_int64, P, P, P, P, P, P]
     cdll.oracle_md_verlet.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, C.c_double, C.c_int32, P, P]
+    cdll.oracle_md_nvt.argtypes = [P, P, C.c_int64, C.c_int64, P, P, P, P, P, C.c_double, C.c_int32, P, P, P, P,
+                                   P]
     cdll.oracle_weight_count.argtypes = [P]
     cdll.oracle_weight_count.restype = C.c_int64
     cdll.oracle_num_threads.restype = C.c_int
@@ -250,6 +252,25 @@ def md_verlet(model: Model, x, v, types, box, masses, dt: float, nsteps: int):
     _check(lib().oracle_md_verlet(C.byref(cfg), _p(model.weights), len(model.weights), len(x), _p(x), _p(v),
                                   _p(types), _p(box), _p(m), dt, nsteps, _p(ep), _p(ek)), "md_verlet")
     return x, v, ep, ek
+
+
+def md_nvt(model: Model, x, v, types, box, masses, dt: float, nsteps: int, temperature: float, tau: float,
+           noise):
+    """Velocity Verlet with stochastic velocity rescaling (see reann_oracle.c);
+    noise [nsteps][2] = (R1, S) per step.  Returns (x, v, epot, ekin, work),
+    each energy array of length nsteps + 1."""
+    x, v, box = _f64(x).copy(), _f64(v).copy(), _f64(box)
+    types = np.ascontiguousarray(types, dtype=np.int32)
+    m = _f64(masses)
+    noise = _f64(noise).reshape(-1)
+    if len(noise) < 2 * nsteps:
+        raise ValueError("noise needs two numbers per step")
+    ep, ek, wk = np.zeros(nsteps + 1), np.zeros(nsteps + 1), np.zeros(nsteps + 1)
+    thermo = np.array([temperature, tau], np.float64)
+    cfg = model.cfg()
+    _check(lib().oracle_md_nvt(C.byref(cfg), _p(model.weights), len(model.weights), len(x), _p(x), _p(v), _p(types),
+                               _p(box), _p(m), dt, nsteps, _p(thermo), _p(noise), _p(ep), _p(ek), _p(wk)), "md_nvt")
+    return x, v, ep, ek, wk
 
 
 def pairs_as_set(row, col) -> np.ndarray:

@@ -730,14 +730,25 @@ static int brute_csr(int64_t n, const double *x, const double *box, double r_cut
  * recorded for s = 0..nsteps (s = 0 is the initial state).  The unit of
  * acceleration is 1 eV/(A amu) = 1/103.6426965 A/fs^2.
  */
-int oracle_md_verlet(const oracle_cfg *c, const float *weights, int64_t weight_count, int64_t n, double *x,
-                     double *v, const int32_t *types, const double *box, const double *mass, double dt,
-                     int32_t nsteps, double *epot, double *ekin) {
-    const double conv = 1.0 / 103.6426965;
+/*
+ * Velocity Verlet (NVE) and, with a thermostat, canonical sampling by
+ * stochastic velocity rescaling (Bussi, Donadio and Parrinello, J. Chem. Phys.
+ * 126, 014101 (2007)): after each step the kinetic energy K is replaced by
+ *   K' = K + (1 - c) (Kt (R1^2 + S) / Nf - K) + 2 R1 sqrt(c (1 - c) K Kt / Nf),
+ * c = exp(-dt / tau), Kt = Nf kB T / 2, Nf = 3 n - 3, by scaling every velocity
+ * by sqrt(K' / K).  R1 (standard normal) and S (a sum of Nf - 1 squared
+ * standard normals) are inputs, two per step, so that any two implementations
+ * given the same numbers take the same steps.  work[s] accumulates K' - K, the
+ * energy the thermostat has added up to step s.
+ */
+static int md_run(const oracle_cfg *c, const float *weights, int64_t weight_count, int64_t n, double *x, double *v,
+                  const int32_t *types, const double *box, const double *mass, double dt, int32_t nsteps,
+                  const double *thermo, const double *noise, double *epot, double *ekin, double *work) {
+    const double conv = 1.0 / 103.6426965, kB = 8.617333262e-5;
     double *F = (double *)malloc(sizeof(double) * 3 * n + 1);
     int64_t *row = NULL;
     int32_t *col = NULL;
-    double E = 0.0;
+    double E = 0.0, W = 0.0;
     int rc = brute_csr(n, x, box, c->r_cut, c->skin, &row, &col);
     if (rc) { free(F); return rc; }
     rc = oracle_energy_forces(c, weights, weight_count, n, x, types, box, row, col, &E, NULL, F, NULL, NULL, NULL);
@@ -763,9 +774,37 @@ int oracle_md_verlet(const oracle_cfg *c, const float *weights, int64_t weight_c
         double K = 0.0;
         for (int64_t i = 0; i < n; ++i)
             for (int a = 0; a < 3; ++a) K += 0.5 * mass[types[i]] * v[3 * i + a] * v[3 * i + a];
+        K *= 103.6426965;   /* eV */
+        if (thermo && s > 0 && K > 0.0) {
+            const double T = thermo[0], tau = thermo[1];
+            const double Nf = (double)(3 * n - 3), Kt = 0.5 * Nf * kB * T;
+            const double cc = tau > 0.0 ? exp(-dt / tau) : 0.0;
+            const double R1 = noise[2 * (s - 1)], S = noise[2 * (s - 1) + 1];
+            const double Kn =
+                K + (1.0 - cc) * (Kt * (R1 * R1 + S) / Nf - K) + 2.0 * R1 * sqrt(cc * (1.0 - cc) * K * Kt / Nf);
+            const double alpha = sqrt(Kn / K);
+            for (int64_t i = 0; i < 3 * n; ++i) v[i] *= alpha;
+            W += Kn - K;
+            K = Kn;
+        }
         if (epot) epot[s] = E;
-        if (ekin) ekin[s] = K * 103.6426965;
+        if (ekin) ekin[s] = K;
+        if (work) work[s] = W;
     }
     free(F);
     return ORACLE_OK;
+}
+
+int oracle_md_verlet(const oracle_cfg *c, const float *weights, int64_t weight_count, int64_t n, double *x,
+                     double *v, const int32_t *types, const double *box, const double *mass, double dt,
+                     int32_t nsteps, double *epot, double *ekin) {
+    return md_run(c, weights, weight_count, n, x, v, types, box, mass, dt, nsteps, NULL, NULL, epot, ekin, NULL);
+}
+
+/* thermo = {T (K), tau (fs; +inf: no coupling, 0: full resampling)}, noise [nsteps][2] */
+int oracle_md_nvt(const oracle_cfg *c, const float *weights, int64_t weight_count, int64_t n, double *x, double *v,
+                  const int32_t *types, const double *box, const double *mass, double dt, int32_t nsteps,
+                  const double *thermo, const double *noise, double *epot, double *ekin, double *work) {
+    if (!thermo || !noise || n < 2 || !(thermo[0] > 0.0) || !(thermo[1] >= 0.0)) return ORACLE_ERR_ARG;
+    return md_run(c, weights, weight_count, n, x, v, types, box, mass, dt, nsteps, thermo, noise, epot, ekin, work);
 }

@@ -54,3 +54,49 @@ def test_first_step_is_taylor_update():
     d = x1 - expect
     d -= box * np.rint(d / box)
     assert np.abs(d).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# NVT: stochastic velocity rescaling (Bussi, Donadio and Parrinello, J. Chem.
+# Phys. 126, 014101 (2007)) with the per-step random numbers given as inputs.
+
+def test_nvt_without_coupling_is_nve():
+    # tau = infinity: c = 1, the rescaling factor is exactly 1 and the run is the
+    # NVE run (to the oracle's run-to-run rounding: its threaded force sums are
+    # reduced in schedule order)
+    p, m, x0, v0, types, box = _setup()
+    noise = synth.thermostat_noise(len(x0), 10, seed=5)
+    xa, va, epa, eka = oracle.md_verlet(m, x0, v0, types, box, p.masses, 0.25, 10)
+    xb, vb, epb, ekb, wk = oracle.md_nvt(m, x0, v0, types, box, p.masses, 0.25, 10, 300.0, np.inf, noise)
+    assert np.abs(xa - xb).max() < 1e-12 and np.abs(va - vb).max() < 1e-12
+    assert np.abs(epa - epb).max() < 1e-10 and np.abs(eka - ekb).max() < 1e-12
+    assert np.all(wk == 0.0)
+
+
+def test_nvt_effective_energy_is_conserved():
+    # E_pot + E_kin minus the thermostat's accumulated work is conserved to the
+    # integrator's own error (the NVE run with the same dt sets the scale)
+    p, m, x0, v0, types, box = _setup()
+    n = 80
+    noise = synth.thermostat_noise(len(x0), n, seed=6)
+    _, _, ep, ek, wk = oracle.md_nvt(m, x0, v0, types, box, p.masses, 0.2, n, 300.0, 20.0, noise)
+    h = ep + ek - wk
+    _, _, ep0, ek0 = oracle.md_verlet(m, x0, v0, types, box, p.masses, 0.2, n)
+    nve = np.abs((ep0 + ek0) - (ep0[0] + ek0[0])).max()
+    assert np.abs(h - h[0]).max() <= 3.0 * nve + 1e-9
+    assert np.abs(wk).max() > 10.0 * nve           # the thermostat did work
+
+
+def test_nvt_temperature_relaxes_to_target():
+    p, pos, types, box = small("ag256")
+    m = model_for(p)
+    x0 = pos.astype(np.float64)
+    v0 = synth.maxwell_boltzmann(p, types, temperature=300.0)
+    n, target = 300, 600.0
+    noise = synth.thermostat_noise(len(x0), n, seed=7)
+    _, _, ep, ek, wk = oracle.md_nvt(m, x0, v0, types, box, p.masses, 1.0, n, target, 10.0, noise)
+    nf = 3 * len(x0) - 3
+    temp = 2.0 * ek / (nf * 8.617333262e-5)
+    # kinetic temperature fluctuates by sqrt(2 / Nf) ~ 5 % per sample; over the
+    # last half of the run its mean is within a few percent of the target
+    assert abs(temp[n // 2:].mean() - target) < 0.1 * target, temp[n // 2:].mean()

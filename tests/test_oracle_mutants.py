@@ -14,6 +14,7 @@ import pytest
 import oracle
 import test_oracle_density as dens
 import test_oracle_forces as forc
+import test_oracle_md as md
 import test_oracle_pair_density as pairden
 import test_oracle_pairs as pairs
 
@@ -49,6 +50,12 @@ MUTANTS = [
     ("pair form: diagonal factor 2 dropped in the backward",
      "s += (mm == nn ? 2.0 : 1.0) * At[i * nA + mm * ntau + tau] *", "s += 1.0 * At[i * nA + mm * ntau + tau] *",
      lambda: pairden.test_pair_forces_match_central_differences()),
+    ("thermostat: coupling factor (1 - c) dropped from the cross term",
+     "sqrt(cc * (1.0 - cc) * K * Kt / Nf)", "sqrt(cc * K * Kt / Nf)",
+     lambda: md.test_nvt_without_coupling_is_nve()),
+    ("thermostat: work accumulated with the wrong sign",
+     "W += Kn - K;", "W -= Kn - K;",
+     lambda: md.test_nvt_effective_energy_is_conserved()),
     ("pair form: second factor taken from the same radial index",
      "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[mm * ntau + tau];",
      "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[nn * ntau + tau];",
