@@ -273,6 +273,10 @@ def main():
     ap.add_argument("--dd-grid", default="8x8x8")
     ap.add_argument("--ncell", type=int, default=0,
                     help="FCC workloads: cells per axis (smaller lattices for profiling captures)")
+    ap.add_argument("--ensemble", default="nve", choices=("nve", "nvt"),
+                    help="nvt: stochastic velocity rescaling after every step (reann_md_step_nvt)")
+    ap.add_argument("--temperature", type=float, default=300.0, help="NVT target temperature, K")
+    ap.add_argument("--tau", type=float, default=100.0, help="NVT coupling time, fs")
     args = ap.parse_args()
 
     info = RankInfo.from_env()
@@ -302,8 +306,21 @@ def main():
     v = torch.from_numpy(v0.copy()).cuda()
     ctx.reann_build_neighbors(torch.from_numpy(pos).cuda(), torch.from_numpy(types).cuda(), box)
 
+    # the MD call of the chosen ensemble; NVT draws every step's two random
+    # numbers up front on the host (the library takes them as inputs)
+    total_steps = args.warmup + args.steps + min(args.steps, 20) + (0 if args.no_e2e else args.steps + 1)
+    noise = synth.thermostat_noise(n, total_steps, seed=2024) if args.ensemble == "nvt" else None
+    cursor = [0]
+
+    def md(k, xx, vv):
+        if noise is None:
+            return ctx.reann_md_step(k, dt_fs, xx, vv, p.masses)
+        z = noise[cursor[0]:cursor[0] + k]
+        cursor[0] += k
+        return ctx.reann_md_step_nvt(k, dt_fs, args.temperature, args.tau, z, xx, vv, p.masses)
+
     # warm-up (the first call also evaluates the entry forces)
-    ctx.reann_md_step(args.warmup, dt_fs, x, v, p.masses)
+    md(args.warmup, x, v)
     torch.cuda.synchronize()
 
     # ---- device-resident timed region: K steps in one call (a continuation);
@@ -311,8 +328,7 @@ def main():
     clocks = ClockSampler(info.local)
     launches0 = ctx.reann_get_counters().kernel_launches
     clocks.start()
-    run = timed_region(group, lambda: ctx.reann_md_step(args.steps, dt_fs, x, v, p.masses), clock,
-                       n * args.steps)
+    run = timed_region(group, lambda: md(args.steps, x, v), clock, n * args.steps)
     clk = clocks.stop()
     st = run.result
     t_ms = run.ms
@@ -322,7 +338,7 @@ def main():
     # ---- kernel breakdown: a separate call with per-launch CUDA events (eager launches)
     prof_steps = min(args.steps, 20)
     ctx.reann_profile(True)
-    ctx.reann_md_step(prof_steps, dt_fs, x, v, p.masses)
+    md(prof_steps, x, v)
     torch.cuda.synchronize()
     prof = ctx.reann_profile_read()
     ctx.reann_profile(False)
@@ -335,16 +351,17 @@ def main():
         vh = torch.empty((n, 3), dtype=torch.float64).pin_memory()
         xh.copy_(x.cpu())
         vh.copy_(v.cpu())
-        ctx.reann_md_step(1, dt_fs, xh.numpy(), vh.numpy(), p.masses)      # warm the host path
+        md(1, xh.numpy(), vh.numpy())      # warm the host path
 
         def host_steps():
             for _ in range(args.steps):
-                ctx.reann_md_step(1, dt_fs, xh.numpy(), vh.numpy(), p.masses)
+                md(1, xh.numpy(), vh.numpy())
 
         run_e = timed_region(group, host_steps, clock, n * args.steps)
         e2e = {"value": run_e.throughput, "unit": UNIT,
                "h2d_bytes_per_step": 2 * 3 * 8 * n, "d2h_bytes_per_step": 2 * 3 * 8 * n,
-               "note": "reann_md_step(1) per step with pinned host x, v: x and v copied in and out every step"}
+               "note": f"{'reann_md_step_nvt' if noise is not None else 'reann_md_step'}(1) per step with pinned "
+                       "host x, v: x and v copied in and out every step"}
 
     if info.rank != 0:
         group.close()
@@ -368,6 +385,8 @@ def main():
                    "n_radial": p.n_radial, "l_max": p.l_max, "hidden": list(p.hidden), "dt_fs": dt_fs,
                    "networks": "bf16 tcgen05, fp32 accumulate" if p.mlp_precision else "fp32 CUDA-core",
                    "launch": "energy+forces and half kick replayed as one CUDA graph per step",
+                   "ensemble": "NVE (velocity Verlet)" if noise is None else
+                               f"NVT (stochastic velocity rescaling, {args.temperature:g} K, tau {args.tau:g} fs)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"working set > L2 ({n * (p.T * (10 * p.n_radial + 6 * p.n_radial) * 4) / 1e9:.1f} GB of "
                          f"per-layer activations vs 126 MB L2); no flush needed"},

@@ -108,6 +108,7 @@ typedef struct {
     double e_kin0;      /* kinetic energy at entry, eV */
     int64_t rebuilds;   /* neighbour-list rebuilds during the call */
     int64_t steps;      /* steps completed */
+    double e_thermostat; /* energy the thermostat added during the call, eV (0 for reann_md_step) */
 } reann_md_stats;
 
 typedef struct {
@@ -208,6 +209,30 @@ reann_status reann_energy_forces(reann_ctx *ctx, const float *pos, double *energ
  */
 reann_status reann_md_step(reann_ctx *ctx, int32_t nsteps, double dt_fs, double *x, double *v,
                            const double *mass_amu, reann_md_stats *stats, reann_stream stream);
+
+/*
+ * nsteps of canonical (NVT) MD, the ensemble of the capsid production run on
+ * the Tessera page (abstract): the reann_md_step update, and after each
+ * step's closing half kick stochastic velocity rescaling (Bussi, Donadio and
+ * Parrinello, J. Chem. Phys. 126, 014101 (2007)).  With K the kinetic energy,
+ * Nf = 3n - 3, Kt = Nf kB T / 2 and c = exp(-dt / tau), every velocity is
+ * scaled by sqrt(K' / K),
+ *   K' = K + (1 - c) (Kt (R1^2 + S) / Nf - K) + 2 R1 sqrt(c (1 - c) K Kt / Nf),
+ * computed on the device from the device-side K (no synchronisation).
+ * temperature_K > 0; tau_fs >= 0 (0: K drawn afresh each step; +inf: NVE).
+ * noise: HOST double [nsteps][2], the step's (R1, S): R1 a standard normal
+ * number and S >= 0 a sum of Nf - 1 squared standard normals, drawn by the
+ * caller, so that the run is reproducible and comparable with any other
+ * implementation given the same numbers.  stats->e_thermostat receives the
+ * summed K' - K (the conserved quantity is E_pot + E_kin - e_thermostat).
+ * Continuations, allocation, synchronisation and errors as reann_md_step;
+ * also REANN_ERR_ARG for fewer than two atoms, a device noise pointer or a
+ * non-finite (or negative S) noise entry.  Three kernel launches per step
+ * beyond reann_md_step's.
+ */
+reann_status reann_md_step_nvt(reann_ctx *ctx, int32_t nsteps, double dt_fs, double temperature_K, double tau_fs,
+                               const double *noise, double *x, double *v, const double *mass_amu,
+                               reann_md_stats *stats, reann_stream stream);
 
 /* Copies the counters of the context into *out (host).  Synchronises nothing. */
 reann_status reann_get_counters(const reann_ctx *ctx, reann_counters *out);

@@ -530,7 +530,7 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
         (e = cudaMalloc(&c->d_E, sizeof(double) * 4)) ||
         (e = cudaMallocHost(&c->h_status, sizeof(int) * 4)) ||
         (e = cudaMallocHost(&c->h_i64, sizeof(int64_t) * 8)) ||
-        (e = cudaMallocHost(&c->h_E, sizeof(double) * 4)) ||
+        (e = cudaMallocHost(&c->h_E, sizeof(double) * 6)) ||
         (e = cudaMallocHost(&c->h_seg, sizeof(int) * (MAX_ELEMENTS + 1)))) {
         std::string msg = std::string("CUDA initialisation failed: ") + cudaGetErrorString(e);
         cudaGetLastError();
@@ -644,12 +644,38 @@ extern "C" reann_status reann_energy_forces(reann_ctx *c, const float *pos, doub
     return check_status(c, *c->h_status);
 }
 
-extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v,
-                                      const double *mass_amu, reann_md_stats *stats, reann_stream stream) {
+constexpr double KB_EV = 8.617333262e-5;   // Boltzmann constant, eV/K (CODATA 2018)
+
+// Canonical sampling by stochastic velocity rescaling: target temperature,
+// coupling time and the caller's two random numbers per step (host).
+struct NvtArgs {
+    double temperature, tau;
+    const double *noise;
+};
+
+// Velocity Verlet, with the thermostat applied after each step's closing half
+// kick when nvt is given.  The d_E slots: [0] energy, [1] kinetic energy,
+// [2] the step's rescaling factor, [3] thermostat work of this call.
+static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, const double *mass_amu,
+                           reann_md_stats *stats, reann_stream stream, const NvtArgs *nvt) {
     if (!c) return REANN_ERR_ARG;
     if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
     if (nsteps < 0 || !std::isfinite(dt_fs) || !mass_amu || (c->n > 0 && (!x || !v)))
         return fail(c, REANN_ERR_ARG, "invalid arguments");
+    BussiParams B{};
+    if (nvt) {
+        if (!(nvt->temperature > 0) || !std::isfinite(nvt->temperature) || !(nvt->tau >= 0))
+            return fail(c, REANN_ERR_ARG, "temperature must be positive and finite, tau non-negative");
+        if (c->n < 2) return fail(c, REANN_ERR_ARG, "the thermostat needs at least two atoms");
+        if (nsteps > 0 && (!nvt->noise || is_device_ptr(nvt->noise)))
+            return fail(c, REANN_ERR_ARG, "noise must be a host array of two numbers per step");
+        for (int64_t k = 0; k < 2 * (int64_t)nsteps; ++k)
+            if (!std::isfinite(nvt->noise[k]) || (k % 2 == 1 && nvt->noise[k] < 0))
+                return fail(c, REANN_ERR_ARG, "noise must be finite, with S >= 0");
+        B.nf = (double)(3 * c->n - 3);
+        B.kt = 0.5 * B.nf * KB_EV * nvt->temperature;
+        B.c = nvt->tau > 0 ? std::exp(-dt_fs / nvt->tau) : 0.0;
+    }
     double inv_mass[MAX_ELEMENTS], mass[MAX_ELEMENTS];
     for (int e = 0; e < c->ne; ++e) {
         if (!(mass_amu[e] > 0) || !std::isfinite(mass_amu[e])) return fail(c, REANN_ERR_ARG, "masses must be positive");
@@ -693,6 +719,7 @@ extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs
     }
     CK(launch_kinetic(c, mass, c->d_E + 1, s));
     CK(cudaMemcpyAsync(c->h_E + 2, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemsetAsync(c->d_E + 3, 0, sizeof(double), s));
     for (int32_t step = 0; step < nsteps; ++step) {
         CK(launch_md_kick_drift(c, dt_fs, inv_mass, c->d_status + 1, s));
         CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int) * 2, cudaMemcpyDeviceToHost, s));
@@ -706,10 +733,16 @@ extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs
             ++rebuilds;
         }
         if ((st = ef_and_kick(c, dt_fs, inv_mass, s))) return st;
+        if (nvt) {
+            B.r1 = nvt->noise[2 * step];
+            B.s = nvt->noise[2 * step + 1];
+            CK(launch_thermostat(c, mass, B, c->d_E + 2, s));
+        }
         ++done;
     }
     CK(launch_kinetic(c, mass, c->d_E + 1, s));
     CK(cudaMemcpyAsync(c->h_E, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_E + 4, c->d_E + 3, sizeof(double), cudaMemcpyDeviceToHost, s));
     if (n > 0) {
         // final state in caller order: kept for continuation checks, then copied out
         CK(launch_md_scatter(c, c->d_last_x, c->d_last_v, nullptr, s));
@@ -731,8 +764,21 @@ extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs
         stats->e_kin0 = c->h_E[3];
         stats->rebuilds = rebuilds;
         stats->steps = done;
+        stats->e_thermostat = c->h_E[4];
     }
     return check_status(c, c->h_status[0] & ~ST_SKIN);
+}
+
+extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v,
+                                      const double *mass_amu, reann_md_stats *stats, reann_stream stream) {
+    return md_run(c, nsteps, dt_fs, x, v, mass_amu, stats, stream, nullptr);
+}
+
+extern "C" reann_status reann_md_step_nvt(reann_ctx *c, int32_t nsteps, double dt_fs, double temperature_K,
+                                          double tau_fs, const double *noise, double *x, double *v,
+                                          const double *mass_amu, reann_md_stats *stats, reann_stream stream) {
+    const NvtArgs nvt{temperature_K, tau_fs, noise};
+    return md_run(c, nsteps, dt_fs, x, v, mass_amu, stats, stream, &nvt);
 }
 
 extern "C" reann_status reann_get_counters(const reann_ctx *c, reann_counters *out) {

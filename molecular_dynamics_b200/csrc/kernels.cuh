@@ -56,6 +56,12 @@ cudaError_t launch_md_scatter(reann_ctx *c, double *d_x_caller, double *d_v_call
 cudaError_t launch_md_kick_drift(reann_ctx *c, double dt, const double *inv_mass, int *flag, cudaStream_t s);
 cudaError_t launch_md_kick(reann_ctx *c, double dt, const double *inv_mass, cudaStream_t s);
 cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cudaStream_t s);
+// One step of stochastic velocity rescaling: d_state[0] <- the factor, d_state[1] += K' - K.
+struct BussiParams {
+    double c, kt, nf, r1, s;   // exp(-dt/tau), Kt (eV), Nf, the step's normal and chi-square numbers
+};
+cudaError_t launch_thermostat(reann_ctx *c, const double *mass, const BussiParams &B, double *d_state,
+                              cudaStream_t s);
 cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s);
 cudaError_t launch_wrap_state(reann_ctx *c, double *d_x_caller, float *d_pos_caller, cudaStream_t s);
 cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s);

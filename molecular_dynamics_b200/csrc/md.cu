@@ -301,4 +301,46 @@ cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cuda
     return cudaGetLastError();
 }
 
+// Stochastic velocity rescaling (Bussi, Donadio and Parrinello, J. Chem. Phys.
+// 126, 014101 (2007)), the thermostat of the NVT runs named on the Tessera
+// page (abstract): K' = K + (1 - c)(Kt (R1^2 + S)/Nf - K) + 2 R1 sqrt(c (1 - c)
+// K Kt / Nf), every velocity scaled by sqrt(K' / K).  One block sums the
+// kinetic-energy partials in the fixed tree order of k_sum_partials, takes the
+// factor and adds K' - K to the work accumulator; the next kernel scales.
+// K' is a sum of squares in exact arithmetic; a rounding below zero is
+// clamped to it.
+__global__ void k_bussi_factor(int np, const double *__restrict__ part, BussiParams B, double *__restrict__ state) {
+    double v = 0.0;
+    for (int k = threadIdx.x; k < np; k += RED_THREADS) v += part[k];
+    double K = block_sum(v);
+    if (threadIdx.x == 0) {
+        double alpha = 1.0, Kn = K;
+        if (K > 0.0) {
+            Kn = K + (1.0 - B.c) * (B.kt * (B.r1 * B.r1 + B.s) / B.nf - K) +
+                 2.0 * B.r1 * sqrt(B.c * (1.0 - B.c) * K * B.kt / B.nf);
+            Kn = fmax(Kn, 0.0);
+            alpha = sqrt(Kn / K);
+        }
+        state[0] = alpha;
+        state[1] += Kn - K;
+    }
+}
+
+__global__ void k_scale_velocities(int64_t m, double *__restrict__ v, const double *__restrict__ alpha) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < m) v[i] *= *alpha;
+}
+
+cudaError_t launch_thermostat(reann_ctx *c, const double *mass, const BussiParams &B, double *d_state,
+                              cudaStream_t s) {
+    MdParams M = md_params(c, 0.0, mass);
+    int np = (int)blocks(c->n, RED_THREADS);
+    if (c->n == 0) return cudaSuccess;
+    REANN_TIMED(c, REANN_K_INTEGRATE, s, 3);
+    k_kinetic_partial<<<np, RED_THREADS, 0, s>>>(c->n, c->d_v, c->d_pos, M, c->d_Epart);
+    k_bussi_factor<<<1, RED_THREADS, 0, s>>>(np, c->d_Epart, B, d_state);
+    k_scale_velocities<<<blocks(3 * c->n, 256), 256, 0, s>>>(3 * c->n, c->d_v, d_state);
+    return cudaGetLastError();
+}
+
 }  // namespace reann

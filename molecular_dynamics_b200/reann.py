@@ -23,7 +23,7 @@ STATUS = {
 }
 
 EXPORTS = ("reann_create", "reann_destroy", "reann_build_neighbors", "reann_energy_forces", "reann_md_step",
-           "reann_get_counters", "reann_last_error", "reann_get_neighbors", "reann_get_features", "reann_profile",
+           "reann_md_step_nvt", "reann_get_counters", "reann_last_error", "reann_get_neighbors", "reann_get_features", "reann_profile",
            "reann_profile_read", "reann_pair_list_noalloc")
 
 KERNEL_GROUPS = ("active", "density", "mlp_fwd", "mlp_energy", "edge_bwd", "mlp_bwd", "energy_sum", "integrate",
@@ -45,7 +45,7 @@ class Config(C.Structure):
 
 class MdStats(C.Structure):
     _fields_ = [("e_pot", C.c_double), ("e_kin", C.c_double), ("e_pot0", C.c_double), ("e_kin0", C.c_double),
-                ("rebuilds", C.c_int64), ("steps", C.c_int64)]
+                ("rebuilds", C.c_int64), ("steps", C.c_int64), ("e_thermostat", C.c_double)]
 
 
 class Counters(C.Structure):
@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH):
     lib.reann_build_neighbors.argtypes = [P, I64, P, P, C.POINTER(D), P]
     lib.reann_energy_forces.argtypes = [P, P, C.POINTER(D), P, P, P]
     lib.reann_md_step.argtypes = [P, I32, D, P, P, C.POINTER(D), C.POINTER(MdStats), P]
+    lib.reann_md_step_nvt.argtypes = [P, I32, D, D, D, C.POINTER(D), P, P, C.POINTER(D), C.POINTER(MdStats), P]
     lib.reann_get_counters.argtypes = [P, C.POINTER(Counters)]
     lib.reann_last_error.argtypes = [P]
     lib.reann_last_error.restype = C.c_char_p
@@ -222,6 +223,19 @@ class Context:
         st = MdStats()
         self._check(self.lib.reann_md_step(self.h, int(nsteps), float(dt_fs), _ptr(x), _ptr(v), m, C.byref(st),
                                            _stream(stream)))
+        return st
+
+    def reann_md_step_nvt(self, nsteps: int, dt_fs: float, temperature: float, tau_fs: float, noise, x, v, masses,
+                          stream=None) -> MdStats:
+        """noise: host array [nsteps][2] of (R1, S) per step (synth.thermostat_noise draws them)."""
+        m = (C.c_double * self.spec.n_elements)(*[float(a) for a in masses])
+        z = np.ascontiguousarray(np.asarray(noise, np.float64).reshape(-1))
+        if len(z) < 2 * int(nsteps):
+            raise ValueError("noise needs two numbers per step")
+        st = MdStats()
+        self._check(self.lib.reann_md_step_nvt(self.h, int(nsteps), float(dt_fs), float(temperature), float(tau_fs),
+                                               z.ctypes.data_as(C.POINTER(C.c_double)), _ptr(x), _ptr(v), m,
+                                               C.byref(st), _stream(stream)))
         return st
 
     def reann_get_counters(self) -> Counters:
