@@ -200,7 +200,8 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         }
         const float r = g.w;
         const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
-        const float *cj = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
+        // first layer: c^0 by element (no lookup with a single element)
+        const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
         float c[3][2];
 #pragma unroll
         for (int l = 0; l < 3; ++l) {
@@ -279,15 +280,17 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             }
         }
         const int q0 = row[i], q1 = q0 + act_cnt[i];
-        int j_next = q0 < q1 ? act_col[q0] : 0;
-        float4 geo_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 1.f);
+        // the edge list is read once per launch: streaming loads (evict first)
+        // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
+        int j_next = q0 < q1 ? __ldcs(act_col + q0) : 0;
+        float4 geo_next = q0 < q1 ? __ldcs(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; ++q) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
             if (q + 1 < q1) {
-                j_next = act_col[q + 1];
-                geo_next = act_geo[q + 1];
+                j_next = __ldcs(act_col + q + 1);
+                geo_next = __ldcs(act_geo + q + 1);
             }
             const float3 d = make_float3(geo.x, geo.y, geo.z);
             const float r = geo.w;
