@@ -51,7 +51,7 @@ FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without d
 # DRAM read + write of one k_edge_bwd launch from the ncu capture summarised in
 # profiles/k_edge_bwd_ag256k.md (256,000 atoms), scaled to the atom count of the
 # run; None when the kernel has changed since that capture
-EDGE_BWD_TRAFFIC_PER_ATOM = (446.554112e6 + 25.812736e6) / 256000
+EDGE_BWD_TRAFFIC_PER_ATOM = (780.347648e6 + 19.375104e6) / 256000
 EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom capture scaled by the atom count"
 
 
