@@ -20,9 +20,10 @@
 //
 // The backward pass uses the SFU intrinsics (__expf, __sincosf, __fdividef):
 // their arguments are bounded (sine/cosine argument in [0, pi), exponent <= 0)
-// and only forces depend on them.  The forward pass keeps the accurate
-// expf/cospif: the densities feed standardised network inputs, where the
-// intrinsics' ~1e-7 errors showed up as 1e-5-level per-atom energy errors.
+// and only forces depend on them.  The forward pass keeps an accurate expf and
+// evaluates the cutoff as a polynomial accurate to fp32 rounding: the densities
+// feed standardised network inputs, where the intrinsics' ~1e-7 errors showed
+// up as 1e-5-level per-atom energy errors.
 //
 // Tuple order inside one radial index n: (000); (100)(010)(001);
 // (200)(020)(002)(110)(101)(011).  Feature (n, l) sits at index l*N_phi + n.
@@ -156,6 +157,22 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
 // neighbour's coefficients and dE/dA row as contiguous runs, and each lane
 // keeps only its own radial indices' accumulators, so the forward needs no
 // cross-lane reduction and the backward only a sum of the force over the slot.
+// f_c(r) = (cos(pi r / r_c) + 1) / 2 = cos^2(theta), theta = pi r / (2 r_c) in
+// [0, pi/2): the Taylor series of cos to theta^14 in Horner form (truncation
+// below theta^16 / 16! < 7e-11), squared.
+__device__ __forceinline__ float cutoff_cos2(float theta) {
+    const float z = theta * theta;
+    float c = -1.0f / 87178291200.0f;
+    c = fmaf(c, z, 1.0f / 479001600.0f);
+    c = fmaf(c, z, -1.0f / 3628800.0f);
+    c = fmaf(c, z, 1.0f / 40320.0f);
+    c = fmaf(c, z, -1.0f / 720.0f);
+    c = fmaf(c, z, 1.0f / 24.0f);
+    c = fmaf(c, z, -0.5f);
+    c = fmaf(c, z, 1.0f);
+    return c * c;
+}
+
 template <int NP>
 struct Lanes {
     static constexpr int LPE = NP / 2;
@@ -199,7 +216,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             g_next = act_geo[q + 1];
         }
         const float r = g.w;
-        const float fc = 0.5f * (cospif(r * (1.0f / P.r_cut)) + 1.0f);
+        const float fc = cutoff_cos2(r * (0.5f * P.pi_over_rc));
         // first layer: c^0 by element (no lookup with a single element)
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
         float c[3][2];
