@@ -205,7 +205,10 @@ reann_status reann_energy_forces(reann_ctx *ctx, const float *pos, double *energ
  * reann_build_neighbors for the same atoms and types (positions may have
  * moved; the list is rebuilt at entry).  Allocates only if the neighbour
  * list outgrows its capacity.  Synchronises the stream once per step (to
- * read the rebuild flag) and at the end.  Errors: as reann_energy_forces.
+ * read the rebuild flag) and at the end.  The final x is copied out on a
+ * library stream during the last step's force evaluation; every return,
+ * error returns included, waits for that copy, so x and v are not written
+ * after the call returns.  Errors: as reann_energy_forces.
  */
 reann_status reann_md_step(reann_ctx *ctx, int32_t nsteps, double dt_fs, double *x, double *v,
                            const double *mass_amu, reann_md_stats *stats, reann_stream stream);

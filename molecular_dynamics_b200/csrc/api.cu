@@ -563,6 +563,9 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     for (auto ev : c->g_ev)
         if (ev) cudaEventDestroy(ev);
     if (c->g_stream) cudaStreamDestroy(c->g_stream);
+    for (auto ev : c->o_ev)
+        if (ev) cudaEventDestroy(ev);
+    if (c->o_stream) cudaStreamDestroy(c->o_stream);
     delete c;
     return REANN_OK;
 }
@@ -720,6 +723,20 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
     CK(launch_kinetic(c, mass, c->d_E + 1, s));
     CK(cudaMemcpyAsync(c->h_E + 2, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
     CK(cudaMemsetAsync(c->d_E + 3, 0, sizeof(double), s));
+    // the positions are final after the last step's drift (and list check):
+    // they go out on the copy stream while that step's forces are evaluated.
+    // Every return after that waits for the copy (the caller's buffer must
+    // not be written after the call returns).
+    struct CopyWait {
+        cudaStream_t s = nullptr;
+        ~CopyWait() {
+            if (s) cudaStreamSynchronize(s);
+        }
+    } x_wait;
+    if (nsteps > 0 && n > 0 && !c->o_stream) {
+        CK(cudaStreamCreateWithFlags(&c->o_stream, cudaStreamNonBlocking));
+        for (auto &ev : c->o_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    }
     for (int32_t step = 0; step < nsteps; ++step) {
         CK(launch_md_kick_drift(c, dt_fs, inv_mass, c->d_status + 1, s));
         CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int) * 2, cudaMemcpyDeviceToHost, s));
@@ -731,6 +748,15 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
             CK(launch_md_gather(c, c->d_stage_x, c->d_stage_v, s));
             CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
             ++rebuilds;
+        }
+        if (step == nsteps - 1 && n > 0) {
+            CK(launch_md_scatter(c, c->d_last_x, nullptr, nullptr, s));
+            CK(cudaEventRecord(c->o_ev[0], s));
+            CK(cudaStreamWaitEvent(c->o_stream, c->o_ev[0], 0));
+            x_wait.s = c->o_stream;
+            CK(cudaMemcpyAsync(x, c->d_last_x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                               c->o_stream));
+            CK(cudaEventRecord(c->o_ev[1], c->o_stream));
         }
         if ((st = ef_and_kick(c, dt_fs, inv_mass, s))) return st;
         if (nvt) {
@@ -745,9 +771,13 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
     CK(cudaMemcpyAsync(c->h_E + 4, c->d_E + 3, sizeof(double), cudaMemcpyDeviceToHost, s));
     if (n > 0) {
         // final state in caller order: kept for continuation checks, then copied out
-        CK(launch_md_scatter(c, c->d_last_x, c->d_last_v, nullptr, s));
-        CK(cudaMemcpyAsync(x, c->d_last_x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, s));
+        const bool x_out = x_wait.s != nullptr;
+        CK(launch_md_scatter(c, x_out ? nullptr : c->d_last_x, c->d_last_v, nullptr, s));
+        if (!x_out)
+            CK(cudaMemcpyAsync(x, c->d_last_x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
+                               s));
         CK(cudaMemcpyAsync(v, c->d_last_v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost, s));
+        if (x_out) CK(cudaStreamWaitEvent(s, c->o_ev[1], 0));
     }
     CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
     CK(cudaMemcpyAsync(c->h_i64 + 3, c->d_i64 + 3, sizeof(int64_t), cudaMemcpyDeviceToHost, s));

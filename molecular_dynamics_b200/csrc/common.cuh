@@ -173,6 +173,10 @@ struct reann_ctx {
     double g_dt = 0.0;
     double g_inv_mass[reann::MAX_ELEMENTS] = {};
     int64_t g_launches = 0;   // kernels one replay runs
+    // the final positions of an MD call are copied out on this stream while
+    // the last step's forces are evaluated
+    cudaStream_t o_stream = nullptr;
+    cudaEvent_t o_ev[2] = {nullptr, nullptr};
     bool g_disabled = false;  // REANN_GRAPHS=0 in the environment
 
     // status
