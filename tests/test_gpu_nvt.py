@@ -9,7 +9,8 @@ random numbers are inputs, so both sides take the same steps.
   * tau = +inf is the NVE step bit for bit, with zero work;
   * the effective energy E_pot + E_kin - W is conserved;
   * a split call equals one call (continuation with the noise split);
-  * invalid thermostat arguments are rejected.
+  * invalid thermostat arguments are rejected;
+  * the domain-decomposed checking mode runs the same NVT trajectory bit for bit.
 """
 import ctypes as C
 
@@ -147,3 +148,25 @@ def test_invalid_thermostat_arguments_are_rejected():
     rc = ctx.lib.reann_md_step_nvt(ctx.h, 2, 0.5, 300.0, 10.0, C.cast(z.data_ptr(), C.POINTER(C.c_double)),
                                    x.data_ptr(), v.data_ptr(), m, C.byref(st), None)
     assert rc == 1
+
+
+def test_domain_decomposed_nvt_is_bit_identical():
+    # the single-GPU domain-decomposed mode gives the monolithic forces bit for
+    # bit, and the thermostat reduces the same velocities in the same order
+    torch = torch_cuda()
+    from molecular_dynamics_b200 import presets
+    p = presets.scaled("ag1m", ncell=8)
+    pos, types, box = synth.make_structure(p)
+    v0 = synth.maxwell_boltzmann(p, types)
+    noise = synth.thermostat_noise(len(pos), 8, seed=21)
+    out = []
+    for grid in ((0, 0, 0), (2, 2, 2)):
+        spec = reann.ModelSpec.from_preset(p, mlp_precision=0, dd_grid=grid)
+        ctx = reann.Context(spec, synth.weight_blob(p))
+        ctx.reann_build_neighbors(pos, types, box)
+        x = torch.from_numpy(pos.astype(np.float64)).cuda()
+        v = torch.from_numpy(v0.copy()).cuda()
+        st = ctx.reann_md_step_nvt(8, 1.0, 500.0, 10.0, noise, x, v, p.masses)
+        out.append((x.cpu().numpy(), v.cpu().numpy(), st.e_pot, st.e_kin, st.e_thermostat))
+    assert np.array_equal(out[0][0], out[1][0]) and np.array_equal(out[0][1], out[1][1])
+    assert out[0][2:] == out[1][2:]
