@@ -64,6 +64,20 @@ def test_create_rejects_unsupported_and_invalid_configs(lib):
 def test_null_context_is_rejected(lib):
     assert lib.reann_destroy(None) == 0
     assert lib.reann_get_counters(None, None) == 1
+    m = (C.c_double * 1)(107.8682)
+    noise = (C.c_double * 2)(0.0, 1.0)
+    assert lib.reann_md_step(None, 1, 1.0, None, None, m, None, None) == 1
+    assert lib.reann_md_step_nvt(None, 1, 1.0, 300.0, 10.0, noise, None, None, m, None, None) == 1
+
+
+def test_md_stats_layout_matches_the_header():
+    # the ctypes mirror of reann_md_stats has the header's fields in order
+    import re
+    from pathlib import Path
+    hdr = (Path(__file__).resolve().parent.parent / "include" / "reann.h").read_text()
+    block = re.search(r"typedef struct \{([^}]*)\} reann_md_stats;", hdr).group(1)
+    names = re.findall(r"^\s*(?:double|int64_t)\s+(\w+);", block, re.M)
+    assert names == [f[0] for f in reann.MdStats._fields_]
 
 
 def test_blob_layout_matches_the_header(lib):
