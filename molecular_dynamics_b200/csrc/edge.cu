@@ -324,12 +324,21 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                     const float4 v = __ldg(g4 + q2 * LPE + sub);
                     gj[4 * q2] = v.x; gj[4 * q2 + 1] = v.y; gj[4 * q2 + 2] = v.z; gj[4 * q2 + 3] = v.w;
                 }
-                const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
+                if (!HAS_DC && ne == 1) {
+                    // first layer, one element: every atom carries the same c^0
 #pragma unroll
-                for (int l = 0; l < 3; ++l) {
-                    const float2 v = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
-                    cj[l][0] = v.x;
-                    cj[l][1] = v.y;
+                    for (int l = 0; l < 3; ++l) {
+                        cj[l][0] = ck[l][0];
+                        cj[l][1] = ck[l][1];
+                    }
+                } else {
+                    const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
+#pragma unroll
+                    for (int l = 0; l < 3; ++l) {
+                        const float2 v = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+                        cj[l][0] = v.x;
+                        cj[l][1] = v.y;
+                    }
                 }
             }
             const float xx = d.x * d.x, yy = d.y * d.y, zz = d.z * d.z;
