@@ -212,50 +212,74 @@ def network_flop_per_atom(group, d_in, d_out, hidden):
     return {"mlp_fwd": fwd(d_out), "mlp_energy": 2 * fwd(1), "mlp_bwd": 2 * fwd(d_out)}[group]
 
 
-def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None):
-    """Roofline entry of the dominant kernel group: algorithmic operations per
-    launch over its mean CUDA-event launch time.  Edge passes and fp32
+KERNEL_NAMES = {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd", "active": "k_active"}
+NETWORK_NAMES = {"mlp_fwd": " (coefficient networks)", "mlp_energy": " (energy network + VJP)",
+                 "mlp_bwd": " (coefficient-network VJP)"}
+
+
+def kernel_roofline(group, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None, nnz=None):
+    """Roofline entry of one kernel group: algorithmic operations (or bytes)
+    per launch over its mean CUDA-event launch time.  Edge passes and fp32
     networks: FP32 FMA peak of the SM count at clocks.max.sm; bf16 tensor-core
-    networks: the measured sustained bf16 peak.  `net` = (d_in, d_out, hidden,
-    mlp_precision) of the workload's networks."""
-    shares = {k: v_[0] for k, v_ in prof.items()}
-    dominant = max(shares, key=shares.get)
+    networks: the measured sustained bf16 peak; the active-pair compaction:
+    the measured HBM copy bandwidth, with the bytes it must move (full-list
+    columns and row offsets read, positions read once, active columns and
+    geometry and counts written).  `net` = (d_in, d_out, hidden,
+    mlp_precision) of the workload's networks; `nnz` the full-list length.
+    None for a group without an algorithmic count or launches."""
+    if group not in prof or not prof[group][1]:
+        return None
+    ms, launches = prof[group]
+    launch_s = ms / launches * 1e-3
+    smax = pk.get("sm_max_mhz", 1965.0)
+    clock_mhz = clk.get("sm_mhz") or smax
+    fp32_peak = sm_count * 128 * 2 * smax * 1e6 / 1e12
+    fp32_note = (f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {smax:.0f} MHz "
+                 f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz")
+    if group == "active":
+        if nnz is None:
+            return None
+        work = 4.0 * nnz + 4.0 * (n_atoms + 1) + 16.0 * n_atoms + 20.0 * active_pairs + 4.0 * n_atoms
+        peak = pk.get("hbm_gbs", 6650.0)
+        achieved = work / launch_s / 1e9
+        return {"kernel": "k_active", "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "bytes_per_launch": work, "launch_ms": launch_s * 1e3,
+                "peak_note": f"HBM copy bandwidth ({pk_kind})"}
     tensor = False
-    if dominant == "edge_bwd":
-        flop_per_launch = active_pairs * (FLOP_EDGE_BWD_PER_PAIR[NP][0] + (T - 1) * FLOP_EDGE_BWD_PER_PAIR[NP][1]) / T
-    elif dominant == "density":
-        flop_per_launch = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
-    elif dominant.startswith("mlp_") and net is not None:
+    if group == "edge_bwd":
+        work = active_pairs * (FLOP_EDGE_BWD_PER_PAIR[NP][0] + (T - 1) * FLOP_EDGE_BWD_PER_PAIR[NP][1]) / T
+    elif group == "density":
+        work = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
+    elif group.startswith("mlp_") and net is not None:
         d_in, d_out, hidden, prec = net
-        flop_per_launch = n_atoms * network_flop_per_atom(dominant, d_in, d_out, hidden)
+        work = n_atoms * network_flop_per_atom(group, d_in, d_out, hidden)
         tensor = prec == 1
     else:
         return None
-    ms_dom, n_dom = prof[dominant]
-    if not n_dom:
-        return None
-    smax = pk.get("sm_max_mhz", 1965.0)
-    clock_mhz = clk.get("sm_mhz") or smax
-    achieved = flop_per_launch / (ms_dom / n_dom * 1e-3) / 1e12
-    traffic = None
-    if dominant == "edge_bwd" and EDGE_BWD_TRAFFIC_PER_ATOM is not None:
-        traffic = EDGE_BWD_TRAFFIC_PER_ATOM * n_atoms
-    kernel = {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd"}.get(
-        dominant, ("k_mlp_tc" if tensor else "k_mlp") + {"mlp_fwd": " (coefficient networks)",
-                                                          "mlp_energy": " (energy network + VJP)",
-                                                          "mlp_bwd": " (coefficient-network VJP)"}.get(dominant, ""))
+    achieved = work / launch_s / 1e12
     if tensor:
-        peak_tf = pk.get("bf16_tflops_sustained", 1400.0)
-        peak_note = f"bf16 dense, sustained ({pk_kind})"
+        peak, note = pk.get("bf16_tflops_sustained", 1400.0), f"bf16 dense, sustained ({pk_kind})"
     else:
-        peak_tf = sm_count * 128 * 2 * smax * 1e6 / 1e12
-        peak_note = (f"FP32 FMA peak {sm_count} SMs x 128 lanes x 2 flop x {smax:.0f} MHz "
-                     f"(clocks.max.sm, {pk_kind}); median SM clock during the run {clock_mhz} MHz")
-    return {"kernel": kernel, "bound": "tensor" if tensor else "alu",
-            "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-            "traffic": traffic,
-            "traffic_note": EDGE_BWD_TRAFFIC_NOTE if traffic is not None else "no DRAM capture of this kernel",
-            "peak_note": peak_note, "flop_per_launch": flop_per_launch, "launch_ms": ms_dom / n_dom}
+        peak, note = fp32_peak, fp32_note
+    kernel = KERNEL_NAMES.get(group) or ("k_mlp_tc" if tensor else "k_mlp") + NETWORK_NAMES.get(group, "")
+    return {"kernel": kernel, "bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "flop_per_launch": work, "launch_ms": launch_s * 1e3,
+            "peak_note": note}
+
+
+def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None):
+    """Roofline entry of the dominant kernel group (largest share of the
+    profiled time), with its DRAM traffic per launch where an ncu capture of
+    that kernel exists."""
+    shares = {k: v_[0] for k, v_ in prof.items()}
+    dominant = max(shares, key=shares.get)
+    r = kernel_roofline(dominant, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net)
+    if r is None:
+        return None
+    traffic = EDGE_BWD_TRAFFIC_PER_ATOM * n_atoms if dominant == "edge_bwd" and EDGE_BWD_TRAFFIC_PER_ATOM else None
+    r["traffic"] = traffic
+    r["traffic_note"] = EDGE_BWD_TRAFFIC_NOTE if traffic is not None else "no DRAM capture of this kernel"
+    return r
 
 
 def main():
@@ -373,8 +397,14 @@ def main():
     sm_count = torch.cuda.get_device_properties(info.local).multi_processor_count
     shares = {k: v_[0] for k, v_ in prof.items()}
     total = sum(shares.values()) or 1.0
-    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk,
-                    net=(p.DR, p.D, tuple(p.hidden), p.mlp_precision))
+    net = (p.DR, p.D, tuple(p.hidden), p.mlp_precision)
+    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net)
+    per_kernel = {}
+    for g in ("edge_bwd", "density", "mlp_bwd", "mlp_fwd", "mlp_energy", "active"):
+        r = kernel_roofline(g, prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net,
+                            nnz=cnt.nnz)
+        if r is not None:
+            per_kernel[g] = {k: r[k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac", "launch_ms")}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -398,6 +428,7 @@ def main():
         "kernel_profile_note": f"per-launch CUDA events over a separate {prof_steps}-step call with eager launches",
         "kernel_share": {k: v_ / total for k, v_ in shares.items() if v_},
         "roofline": roof,
+        "kernel_roofline": per_kernel,
     }
     if e2e is not None:
         line["e2e"] = e2e

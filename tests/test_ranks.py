@@ -115,3 +115,24 @@ def test_roofline_arithmetic():
     r3 = bench.roofline({"mlp_fwd": (8.0, 2)}, pairs, 8, 3, 1000, 148, {"bf16_tflops_sustained": 1382.5}, "measured",
                         {}, net=(24, 24, (128, 128), 1))
     assert r3["bound"] == "tensor" and r3["peak"] == 1382.5
+
+
+def test_per_kernel_roofline_arithmetic():
+    import bench
+    prof = {"active": (2.0, 4), "density": (6.0, 3), "mlp_fwd": (1.0, 2), "energy_sum": (0.1, 1)}
+    pk = {"hbm_gbs": 6500.0, "sm_max_mhz": 2000.0, "bf16_tflops_sustained": 1400.0}
+    n, pairs, nnz = 1000, 54_000, 78_000
+    a = bench.kernel_roofline("active", prof, pairs, 8, 3, n, 148, pk, "measured", {}, nnz=nnz)
+    bytes_ = 4 * nnz + 4 * (n + 1) + 16 * n + 20 * pairs + 4 * n
+    assert a["bound"] == "hbm" and a["unit"] == "GB/s"
+    assert a["achieved"] == pytest.approx(bytes_ / 0.5e-3 / 1e9)
+    assert a["frac"] == pytest.approx(a["achieved"] / 6500.0)
+    d = bench.kernel_roofline("density", prof, pairs, 8, 3, n, 148, pk, "measured", {})
+    assert d["achieved"] == pytest.approx(pairs * bench.FLOP_DENSITY_PER_PAIR[8] / 2e-3 / 1e12)
+    m = bench.kernel_roofline("mlp_fwd", prof, pairs, 8, 3, n, 148, pk, "measured", {}, net=(24, 24, (128, 128), 1))
+    assert m["bound"] == "tensor" and m["peak"] == 1400.0
+    assert m["achieved"] == pytest.approx(n * bench.network_flop_per_atom("mlp_fwd", 24, 24, (128, 128)) / 0.5e-3 / 1e12)
+    # groups without an algorithmic count, or absent, have no entry
+    assert bench.kernel_roofline("energy_sum", prof, pairs, 8, 3, n, 148, pk, "measured", {}) is None
+    assert bench.kernel_roofline("edge_bwd", prof, pairs, 8, 3, n, 148, pk, "measured", {}) is None
+    assert bench.kernel_roofline("active", prof, pairs, 8, 3, n, 148, pk, "measured", {}) is None
