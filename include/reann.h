@@ -24,7 +24,8 @@
  *             order.  Any array pointer may point to device memory or to
  *             host memory (pinned or pageable); the library detects which
  *             with cudaPointerGetAttributes and copies host arrays through
- *             its own device buffers on the given stream.  The caller owns
+ *             its own device buffers on the given stream (the thermostat's
+ *             random numbers are the one host-only array).  The caller owns
  *             every array it passes; the library owns the context and all
  *             workspaces.
  *   streams   work is enqueued on the caller's stream; calls that return a
