@@ -132,11 +132,32 @@ def cpu_sample(steps: int):
                       f"{dt:.1f} s"}, dt
 
 
+def oracle_breakdown():
+    """The oracle's parts on the same 6,912-atom sample: the O(N^2) pair
+    search, the cell-list pair search, and one energy+force evaluation given
+    the pair list (ms each)."""
+    import oracle
+    base = presets.get("ag1m")
+    p = base.with_(ncell=12)
+    pos, types, box = synth.make_structure(p)
+    model = oracle.Model.from_preset(base, synth.weight_blob(base))
+    t0 = time.perf_counter()
+    pairs = oracle.pairs_brute(pos, box, p.r_cut, p.skin)
+    t1 = time.perf_counter()
+    oracle.pairs_cells(pos, box, p.r_cut, p.skin)
+    t2 = time.perf_counter()
+    oracle.energy_forces(model, pos, types, box, pairs)
+    t3 = time.perf_counter()
+    return {"atoms": len(pos), "pairs_brute_ms": 1e3 * (t1 - t0), "pairs_cells_ms": 1e3 * (t2 - t1),
+            "energy_forces_given_pairs_ms": 1e3 * (t3 - t2)}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     _, dt_w = cpu_sample(args.warmup) if args.warmup > 0 else (None, 0.0)
     cb, dt = cpu_sample(args.steps)
+    parts = oracle_breakdown()
     line = {
         "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
@@ -145,6 +166,7 @@ def run_reference(args, rank, world):
                                "1 fs velocity Verlet (oracle timed on a 12^3-cell sample of it)"},
         "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
         "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "oracle_breakdown": parts,
     }
     print(json.dumps(line), flush=True)
     return 0
