@@ -100,3 +100,25 @@ def test_nvt_temperature_relaxes_to_target():
     # kinetic temperature fluctuates by sqrt(2 / Nf) ~ 5 % per sample; over the
     # last half of the run its mean is within a few percent of the target
     assert abs(temp[n // 2:].mean() - target) < 0.1 * target, temp[n // 2:].mean()
+
+
+def test_nvt_kinetic_energy_is_canonical():
+    # the thermostat samples the canonical ensemble, where the kinetic energy
+    # follows a Gamma distribution: mean Kt = Nf kB T / 2 and relative spread
+    # sqrt(2 / Nf), whatever the potential.  Strong coupling (tau = dt) keeps
+    # the correlation time to a few steps, so 800 samples after a 200-step
+    # burn-in pin both moments; a wrong weight of either random term moves the
+    # spread (halving the cross term gives ~0.77 of it)
+    p, pos, types, box = small("ag256")
+    m = model_for(p)
+    x0 = pos.astype(np.float64)
+    v0 = synth.maxwell_boltzmann(p, types, temperature=300.0)
+    n = len(x0)
+    nf = 3 * n - 3
+    kt = 0.5 * nf * 8.617333262e-5 * 300.0
+    noise = synth.thermostat_noise(n, 1000, seed=8)
+    _, _, ep, ek, wk = oracle.md_nvt(m, x0, v0, types, box, p.masses, 1.0, 1000, 300.0, 1.0, noise)
+    K = ek[200:]
+    assert abs(K.mean() / kt - 1.0) < 0.01, K.mean() / kt
+    ratio = K.std() / kt / np.sqrt(2.0 / nf)
+    assert 0.85 < ratio < 1.15, ratio

@@ -53,6 +53,9 @@ MUTANTS = [
     ("thermostat: coupling factor (1 - c) dropped from the cross term",
      "sqrt(cc * (1.0 - cc) * K * Kt / Nf)", "sqrt(cc * K * Kt / Nf)",
      lambda: md.test_nvt_without_coupling_is_nve()),
+    ("thermostat: cross term halved",
+     "2.0 * R1 * sqrt(cc * (1.0 - cc) * K * Kt / Nf)", "1.0 * R1 * sqrt(cc * (1.0 - cc) * K * Kt / Nf)",
+     lambda: md.test_nvt_kinetic_energy_is_canonical()),
     ("thermostat: work accumulated with the wrong sign",
      "W += Kn - K;", "W -= Kn - K;",
      lambda: md.test_nvt_effective_energy_is_conserved()),
