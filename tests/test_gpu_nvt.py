@@ -10,7 +10,8 @@ random numbers are inputs, so both sides take the same steps.
   * the effective energy E_pot + E_kin - W is conserved;
   * a split call equals one call (continuation with the noise split);
   * invalid thermostat arguments are rejected;
-  * the domain-decomposed checking mode runs the same NVT trajectory bit for bit.
+  * the domain-decomposed checking mode runs the same NVT trajectory bit for bit;
+  * at strong coupling the kinetic energy has the canonical moments.
 """
 import ctypes as C
 
@@ -170,3 +171,24 @@ def test_domain_decomposed_nvt_is_bit_identical():
         out.append((x.cpu().numpy(), v.cpu().numpy(), st.e_pot, st.e_kin, st.e_thermostat))
     assert np.array_equal(out[0][0], out[1][0]) and np.array_equal(out[0][1], out[1][1])
     assert out[0][2:] == out[1][2:]
+
+
+def test_kinetic_energy_is_canonical():
+    # the GPU thermostat on its own trajectory: at tau = dt the kinetic energy
+    # has the canonical (Gamma) moments, mean Nf kB T / 2 and relative spread
+    # sqrt(2 / Nf), over 800 steps after a 200-step burn-in
+    p, pos, types, box = small("ag256")
+    _, _, x, v = _state(p, pos, types)
+    n = len(pos)
+    nf = 3 * n - 3
+    kt = 0.5 * nf * KB * 300.0
+    noise = synth.thermostat_noise(n, 1000, seed=8)
+    ctx = _ctx(p, pos, types, box)
+    K = []
+    for k in range(1000):
+        st = ctx.reann_md_step_nvt(1, 1.0, 300.0, 1.0, noise[k:k + 1], x, v, p.masses)
+        K.append(st.e_kin)
+    K = np.array(K[200:])
+    assert abs(K.mean() / kt - 1.0) < 0.01, K.mean() / kt
+    ratio = K.std() / kt / np.sqrt(2.0 / nf)
+    assert 0.85 < ratio < 1.15, ratio
