@@ -8,6 +8,8 @@ must give the coordination shells fixed by geometry; rows must be symmetric,
 sorted and free of self pairs; a box smaller than twice the list radius is
 an error.
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -34,12 +36,25 @@ def test_cell_list_with_many_cells():
     assert np.array_equal(rb[0], rc[0]) and np.array_equal(rb[1], rc[1])
 
 
+def _fcc_shells():
+    """(n, sites) of the FCC neighbour shells at squared radius n a^2 / 2, from
+    the cited fixture tests/golden/fcc_shells.txt."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "fcc_shells.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    return [(int(n), int(k)) for n, k in rows]
+
+
+def _sites_within(a, r):
+    return sum(k for n, k in _fcc_shells() if n * a * a / 2.0 < r * r)
+
+
 @pytest.mark.parametrize("a,rc,listed,active", [
-    # FCC shells at a/sqrt2 (12), a (6), a*sqrt(3/2) (24), a*sqrt2 (12), a*sqrt(5/2) (24), a*sqrt3 (8)
     (4.09, 6.0, 78, 54),   # Ag: shells below 7.0 A: 12+6+24+12+24; below 6.0 A: 12+6+24+12
     (3.60, 5.5, 86, 54),   # HEA: shells below 6.5 A add the 8 at 6.235 A; below 5.5 A: 12+6+24+12
 ])
 def test_fcc_shell_counts(a, rc, listed, active):
+    # the expected counts follow from the lattice's shells (skin 1.0 A)
+    assert _sites_within(a, rc + 1.0) == listed and _sites_within(a, rc) == active
     pos, box = fcc_perfect(6, a)
     row, col = oracle.pairs_brute(pos, box, rc, 1.0)
     assert np.all(np.diff(row) == listed)
