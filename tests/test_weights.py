@@ -61,3 +61,18 @@ def test_energy_scale_multiplies_only_the_energy_output_layer():
         o, shape = net["W3"]
         m = int(np.prod(shape))
         assert np.allclose(b[o:o + m], 2 * a[o:o + m])
+
+
+def test_thermostat_noise_has_the_stated_distributions():
+    # R1 standard normal, S chi-squared with Nf - 1 = 3 n - 4 degrees of
+    # freedom; seeded, so both sides of a parity test read the same numbers
+    n, steps = 256, 20000
+    z = synth.thermostat_noise(n, steps, seed=3)
+    assert z.shape == (steps, 2)
+    assert np.array_equal(z, synth.thermostat_noise(n, steps, seed=3))
+    r1, s = z[:, 0], z[:, 1]
+    k = 3 * n - 4
+    assert abs(r1.mean()) < 4 / np.sqrt(steps) and abs(r1.std() - 1.0) < 0.02
+    assert abs(s.mean() / k - 1.0) < 4 * np.sqrt(2.0 / k / steps)
+    assert abs(s.var() / (2.0 * k) - 1.0) < 0.05
+    assert np.all(s > 0)
