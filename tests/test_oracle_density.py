@@ -100,3 +100,55 @@ def test_t1_energy_is_the_local_eann_network_on_closed_form_density():
         assert res.atom_energy[i] == pytest.approx(e, rel=1e-12)
         expect += e
     assert res.energy == pytest.approx(expect, rel=1e-12)
+
+
+def _blob_net(blob, spec):
+    """One network of the weight blob as a numpy function (row-major W, output
+    index first; input standardised as (x - shift) / scale)."""
+    g = lambda k: blob[spec[k][0]:spec[k][0] + int(np.prod(spec[k][1]))].reshape(spec[k][1]).astype(np.float64)
+
+    def f(x):
+        a1 = np.tanh(g("W1") @ ((x - g("shift")) / g("scale")) + g("b1"))
+        a2 = np.tanh(g("W2") @ a1 + g("b2"))
+        return g("W3") @ a2 + g("b3")
+    return f
+
+
+@pytest.mark.parametrize("T", [2, 3])
+@pytest.mark.parametrize("types", [(0, 1), (1, 0)])
+def test_message_passing_dimer_chain(T, types):
+    """Eq. 2 (section "REANN Architecture"): c^{t+1}_i = M^t_{Z_i}(rho^t_i), one
+    network per layer t and per element of the centre atom.  For a hetero
+    dimer every layer's density has the closed form
+    rho^t_{i,(n,l)} = (c^t_{j,(n,l)} phi_n(r))^2 r^(2l) of the partner j, so the
+    whole chain c^0 -> rho^0 -> c^1 -> ... -> rho^{T-1} -> E_i is written out
+    here with the networks read straight from the blob.  Using the networks
+    in another layer order, or the partner's element (or one element for
+    every atom), changes E_i."""
+    p = presets.get("water3k")
+    blob = synth.weight_blob(p, T=T)
+    lay = synth.blob_layout(p, T)
+    m = oracle.Model.from_preset(p, blob, T=T)
+    NP, L = p.n_radial, p.l_max
+    C0 = blob[:p.n_elements * p.D].reshape(p.n_elements, p.D).astype(np.float64)
+    r = 2.61
+    d = np.array([-0.36, 0.48, 0.8]) * r
+    x = np.array([[7.0, 7.0, 7.0], [7.0, 7.0, 7.0] + d])
+    z = np.array(types, np.int32)
+    box = np.array([22.0, 22.0, 22.0])
+    res = oracle.energy_forces(m, x, z, box, forces=False, intermediates=True)
+
+    shape = np.array([_phi(r, n, p) ** 2 * r ** (2 * l) for l in range(L + 1) for n in range(NP)])
+    c = [C0[z[0]], C0[z[1]]]
+    for t in range(T):
+        rho = [c[1] ** 2 * shape, c[0] ** 2 * shape]          # each atom's density from its partner
+        for i in range(2):
+            assert res.rho[t][i] == pytest.approx(rho[i], rel=1e-12, abs=1e-300)
+        if t + 1 < T:
+            c = [_blob_net(blob, lay["coef"][t][z[i]])(rho[i]) for i in range(2)]
+            for i in range(2):
+                assert res.coef[t + 1][i] == pytest.approx(c[i], rel=1e-12, abs=1e-14)
+    e = [float(_blob_net(blob, lay["energy"][z[i]])(rho[i])[0]) for i in range(2)]
+    for i in range(2):
+        assert res.atom_energy[i] == pytest.approx(e[i], rel=1e-12)
+    assert res.energy == pytest.approx(e[0] + e[1], rel=1e-12)

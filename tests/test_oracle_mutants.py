@@ -2,7 +2,9 @@
 the oracle's C source (a dropped term, a wrong sign, a transposed operand, a
 wrong index or layer) must each make at least one pin fail.
 
-Each case patches one expression of oracle/reann_oracle.c, compiles the copy,
+Each case patches one expression of oracle/reann_oracle.c (or several, for a
+mistake made consistently in the forward and the reverse sweep, which finite
+differences cannot see), compiles the copy,
 routes the oracle through it and runs an existing pin test expecting an
 AssertionError.  The real oracle is restored afterwards.  Everything here is
 CPU only.
@@ -59,6 +61,17 @@ MUTANTS = [
     ("thermostat: work accumulated with the wrong sign",
      "W += Kn - K;", "W -= Kn - K;",
      lambda: md.test_nvt_effective_energy_is_conserved()),
+    ("coefficient networks applied in reversed layer order (forward and backward)",
+     ("&w.coef[t * c->n_elements + types[i]]", "&w.coef[(t - 1) * c->n_elements + types[i]]"),
+     ("&w.coef[(T - 2 - t) * c->n_elements + types[i]]", "&w.coef[(T - 1 - t) * c->n_elements + types[i]]"),
+     lambda: dens.test_message_passing_dimer_chain(3, (0, 1))),
+    ("element 0's coefficient network used for every atom (forward and backward)",
+     ("&w.coef[t * c->n_elements + types[i]]", "&w.coef[(t - 1) * c->n_elements + types[i]]"),
+     ("&w.coef[t * c->n_elements + 0]", "&w.coef[(t - 1) * c->n_elements + 0]"),
+     lambda: dens.test_message_passing_dimer_chain(2, (0, 1))),
+    ("coefficient network chosen by the neighbour's element",
+     "&w.coef[t * c->n_elements + types[i]]", "&w.coef[t * c->n_elements + types[n - 1 - i]]",
+     lambda: dens.test_message_passing_dimer_chain(2, (0, 1))),
     ("pair form: second factor taken from the same radial index",
      "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[mm * ntau + tau];",
      "tuple_weight(tau) * Ai[nn * ntau + tau] * Ai[nn * ntau + tau];",
@@ -69,9 +82,12 @@ MUTANTS = [
 @pytest.mark.parametrize("name,old,new,pin", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_planted_mistake_is_caught(name, old, new, pin, tmp_path):
     src = open(oracle.SRC).read()
-    assert src.count(old) == 1, f"mutation site not found once: {old}"
+    olds, news = (old, new) if isinstance(old, tuple) else ((old,), (new,))
+    for o, n_ in zip(olds, news):
+        assert src.count(o) == 1, f"mutation site not found once: {o}"
+        src = src.replace(o, n_)
     path = tmp_path / "mutant.c"
-    path.write_text(src.replace(old, new))
+    path.write_text(src)
     lib = oracle.compile_source(str(path), str(tmp_path / "libmutant.so"))
     with oracle.use_library(lib):
         with pytest.raises(AssertionError):
