@@ -48,11 +48,22 @@ FLOP_DENSITY_PER_PAIR = {8: 240, 10: 298}
 FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without dE/dc, layers >= 1)
 
 
-# DRAM read + write of one k_edge_bwd launch from the ncu capture summarised in
-# profiles/k_edge_bwd_ag256k.md (256,000 atoms), scaled to the atom count of the
-# run; None when the kernel has changed since that capture
-EDGE_BWD_TRAFFIC_PER_ATOM = (780.347648e6 + 19.375104e6) / 256000
-EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom capture scaled by the atom count"
+# DRAM read + write (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# k_edge_bwd launch from an ncu capture on 256,000 Ag atoms, scaled to the atom
+# count of the run.  The capture belongs to the kernel source whose SHA-256
+# prefix is recorded beside it: once edge.cu or common.cuh change, the figure
+# no longer describes the kernel and the line reports null.
+EDGE_BWD_CAPTURE = {"bytes_per_atom": (780.347648e6 + 19.375104e6) / 256000, "source_sha": None}
+EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom ncu capture scaled by the atom count"
+
+
+def edge_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("edge.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "molecular_dynamics_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def peaks():
@@ -65,7 +76,7 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -79,7 +90,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -298,9 +309,11 @@ def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net
     r = kernel_roofline(dominant, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net)
     if r is None:
         return None
-    traffic = EDGE_BWD_TRAFFIC_PER_ATOM * n_atoms if dominant == "edge_bwd" and EDGE_BWD_TRAFFIC_PER_ATOM else None
+    current = dominant == "edge_bwd" and EDGE_BWD_CAPTURE["source_sha"] == edge_source_sha()
+    traffic = EDGE_BWD_CAPTURE["bytes_per_atom"] * n_atoms if current else None
     r["traffic"] = traffic
-    r["traffic_note"] = EDGE_BWD_TRAFFIC_NOTE if traffic is not None else "no DRAM capture of this kernel"
+    r["traffic_note"] = EDGE_BWD_TRAFFIC_NOTE if traffic is not None else \
+        "no DRAM capture of the current source of this kernel"
     return r
 
 

@@ -295,16 +295,20 @@ reann_status reann_profile_read(const reann_ctx *ctx, int32_t group, double *ms,
  * rows sorted by j.  pos: device float32 [n][3] (A); box: host double[3];
  * nnz: host, receives the list length.  At most 131,072 atoms: larger n is
  * rejected with REANN_ERR_CAPACITY before any GPU work; if the list outgrows
- * cap, REANN_ERR_CAPACITY is returned with *nnz set, row filled and col not
- * written.  Other errors: REANN_ERR_ARG, REANN_ERR_BOX, REANN_ERR_NONFINITE,
- * REANN_ERR_CUDA; reann_last_error(NULL) gives the message.
+ * cap, or has more than 2^31-1 entries (the int32 offsets' range),
+ * REANN_ERR_CAPACITY is returned with *nnz set and col not written (row is
+ * meaningful only when the list fits the int32 range).  Other errors:
+ * REANN_ERR_ARG, REANN_ERR_BOX, REANN_ERR_NONFINITE, REANN_ERR_CUDA;
+ * reann_last_error(NULL) gives the message.
  *
  * All calls share the scratch array and it keeps the last call's contents;
  * each call clears what must start at zero.  Calls whose GPU work overlaps
  * (two streams, or two host threads on one device) race on the array:
  * serialise them.  The first call on a device looks up the array's device
  * address with that device current (cudaGetSymbolAddress); make that first
- * call before any stream capture.  Synchronises the stream twice.
+ * call before any stream capture.  The address is kept for the rest of the
+ * process: after cudaDeviceReset on a device the array may move, so the call
+ * must not be used on that device again.  Synchronises the stream twice.
  */
 reann_status reann_pair_list_noalloc(int64_t n, const float *pos, const double box[3], double r_cut, double skin,
                                      int32_t *row, int32_t *col, int64_t cap, int64_t *nnz, reann_stream stream);

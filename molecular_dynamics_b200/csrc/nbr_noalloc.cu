@@ -23,6 +23,9 @@
 // on the array and corrupt each other's result: serialise them.  The first
 // call on a device looks up the array's device address (cudaGetSymbolAddress)
 // with that device current; make that first call before any stream capture.
+// The address is kept for the life of the process: after cudaDeviceReset on
+// a device the array may move, and this call must not be used on that device
+// again in the same process.
 #include <mutex>
 
 #include "common.cuh"
@@ -299,6 +302,11 @@ extern "C" reann_status reann_pair_list_noalloc(int64_t n, const float *pos, con
         k_na_rows<false><<<nb, 256, 0, s>>>(S, N, pos, g, nullptr, nullptr);
     }
     k_na_scan_rows<<<1, NA_SCAN_THREADS, 0, s>>>(S, N, row);
+    if ((e = cudaGetLastError()) != cudaSuccess) {
+        cudaStreamSynchronize(s);
+        cudaGetLastError();
+        return na_fail(REANN_ERR_CUDA, std::string("CUDA error: ") + cudaGetErrorString(e));
+    }
     long long total = 0;
     int status = 0;
     if ((e = cudaMemcpyAsync(&total, &S->total, sizeof(long long), cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
@@ -309,6 +317,8 @@ extern "C" reann_status reann_pair_list_noalloc(int64_t n, const float *pos, con
     }
     *nnz = total;
     if (status & ST_NONFINITE) return na_fail(REANN_ERR_NONFINITE, "non-finite position");
+    // row offsets are int32: a longer list is rejected before anything is written to col
+    if (total > INT32_MAX) return na_fail(REANN_ERR_CAPACITY, "neighbour list exceeds 2^31-1 entries");
     if (total > cap)
         return na_fail(REANN_ERR_CAPACITY, "col holds " + std::to_string(cap) + " entries, the list has " +
                                                std::to_string(total));

@@ -7,7 +7,10 @@ times, checked against the oracle on outputs it can compute one by one:
     cluster of every atom within 2 T r_c (+ margin) of the sample -- exactly
     the atoms a force depends on through T message-passing layers;
   * properties that hold at any size: zero net force, and the total energy
-    equal to the sum of the atomic energies.
+    equal to the sum of the atomic energies;
+  * the whole system against the oracle run on all N atoms (with the
+    oracle's own cell-list pair search): every force component, every atomic
+    energy and the total energy at the stated tolerances.
 Small workloads (up to 3,000 atoms) are compared in full.
 """
 import numpy as np
@@ -72,3 +75,25 @@ def test_sampled_forces_and_energies(full):
         # against the system's per-atom energy scale, as in gpu_helpers
         rel = abs(Ei[k] - ref.atom_energy[0]) / max(float(np.sqrt(np.mean(Ei ** 2))), 1e-2)
         assert rel <= 10 * E_TOL[prec], (k, Ei[k], ref.atom_energy[0])
+
+
+def test_whole_system_matches_oracle(full):
+    """Element by element at full size (108,000 / 244,000 / 1,048,576 atoms):
+    forces max-abs within 1e-4 eV/A (fp32 networks) or 5e-3 eV/A (bf16
+    networks), the total energy within 1e-5 per atom, every atomic energy
+    within 1e-4 of the RMS atomic energy."""
+    p, pos, types, box, ctx, E, F, Ei = full
+    n = len(pos)
+    if n <= 3000:
+        pytest.skip("compared in full by test_sampled_forces_and_energies")
+    pairs = oracle.pairs_cells(pos, box, p.r_cut, p.skin)
+    ref = oracle.energy_forces(oracle.Model.from_preset(p, synth.weight_blob(p)), pos, types, box, pairs)
+    prec = p.mlp_precision
+    de = abs(E - ref.energy) / n
+    dei = np.abs(Ei - ref.atom_energy).max() / max(float(np.sqrt(np.mean(ref.atom_energy ** 2))), 1e-2)
+    df = np.abs(F - ref.forces).max()
+    print(f"\n{p.key}: n={n} |dE|/N={de:.3e} eV (|E|/N={abs(ref.energy) / n:.3e}), "
+          f"max|dE_i|/rms(E_i)={dei:.3e}, max|dF|={df:.3e} eV/A (max|F|={np.abs(ref.forces).max():.2f})")
+    assert_energy_close(E, ref.energy, n, prec)
+    assert_atom_energies_close(Ei, ref.atom_energy, prec)
+    assert_forces_close(F, ref.forces, prec)
