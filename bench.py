@@ -264,6 +264,21 @@ def network_flop_per_atom(group, d_in, d_out, hidden):
     return {"mlp_fwd": fwd(d_out), "mlp_energy": 2 * fwd(1), "mlp_bwd": 2 * fwd(d_out)}[group]
 
 
+def network_kind(p) -> str:
+    """Which network kernels the library runs for this model (include/reann.h,
+    mlp_precision): bf16 tensor cores, three-pass tf32 tensor cores, or fp32
+    CUDA cores."""
+    if p.mlp_precision == 1:
+        return "bf16"
+    if p.mlp_precision == 0 and tuple(p.hidden) == (64, 64) and p.density_form == 0 and p.n_radial in (8, 10):
+        return "tf32x3"
+    return "simt"
+
+
+NETWORK_DESCRIPTION = {"bf16": "bf16 tcgen05 (split bf16 activations), fp32 accumulate",
+                       "tf32x3": "fp32-accurate tcgen05: three tf32 passes of hi/lo split operands, fp32 accumulate",
+                       "simt": "fp32 CUDA-core"}
+
 KERNEL_NAMES = {"edge_bwd": "k_edge_bwd", "density": "k_density_fwd", "active": "k_active"}
 NETWORK_NAMES = {"mlp_fwd": " (coefficient networks)", "mlp_energy": " (energy network + VJP)",
                  "mlp_bwd": " (coefficient-network VJP)"}
@@ -303,17 +318,23 @@ def kernel_roofline(group, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_
     elif group == "density":
         work = active_pairs * FLOP_DENSITY_PER_PAIR[NP]
     elif group.startswith("mlp_") and net is not None:
-        d_in, d_out, hidden, prec = net
+        d_in, d_out, hidden, kind = net
         work = n_atoms * network_flop_per_atom(group, d_in, d_out, hidden)
-        tensor = prec == 1
+        tensor = kind != "simt"
     else:
         return None
     achieved = work / launch_s / 1e12
-    if tensor:
+    if tensor and kind == "bf16":
         peak, note = pk.get("bf16_tflops_sustained", 1400.0), f"bf16 dense, sustained ({pk_kind})"
+    elif tensor:
+        # tf32 dense: the measured sustained bf16 peak x the nominal tf32/bf16 ratio (1.1 / 2.25 PFLOP/s);
+        # the three tf32 passes per product are not counted as work
+        peak = pk.get("bf16_tflops_sustained", 1400.0) * 1.1 / 2.25
+        note = f"tf32 dense = sustained bf16 ({pk_kind}) x 1.1/2.25 nominal; algorithmic flops (each product runs 3 passes)"
     else:
         peak, note = fp32_peak, fp32_note
-    kernel = KERNEL_NAMES.get(group) or ("k_mlp_tc" if tensor else "k_mlp") + NETWORK_NAMES.get(group, "")
+    kernel = KERNEL_NAMES.get(group) or {"bf16": "k_mlp_tc", "tf32x3": "k_mlp_tc32", "simt": "k_mlp"}.get(
+        kind, "k_mlp") + NETWORK_NAMES.get(group, "")
     return {"kernel": kernel, "bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak, "flop_per_launch": work, "launch_ms": launch_s * 1e3,
             "peak_note": note}
@@ -355,6 +376,8 @@ def main():
                     help="nvt: stochastic velocity rescaling after every step (reann_md_step_nvt)")
     ap.add_argument("--temperature", type=float, default=300.0, help="NVT target temperature, K")
     ap.add_argument("--tau", type=float, default=100.0, help="NVT coupling time, fs")
+    ap.add_argument("--mlp-precision", type=int, default=None, choices=(0, 1, 2),
+                    help="override the workload's network precision (2: fp32 CUDA-core networks)")
     args = ap.parse_args()
 
     info = RankInfo.from_env()
@@ -372,6 +395,8 @@ def main():
     p = presets.get(args.workload)
     if args.ncell:
         p = presets.scaled(args.workload, ncell=args.ncell)
+    if args.mlp_precision is not None:
+        p = p.with_(mlp_precision=args.mlp_precision)
     pos, types, box = synth.make_structure(p)
     v0 = synth.maxwell_boltzmann(p, types)
     n = len(pos)
@@ -466,7 +491,7 @@ def main():
     sm_count = torch.cuda.get_device_properties(info.local).multi_processor_count
     shares = {k: v_[0] for k, v_ in prof.items()}
     total = sum(shares.values()) or 1.0
-    net = (p.DR, p.D, tuple(p.hidden), p.mlp_precision)
+    net = (p.DR, p.D, tuple(p.hidden), network_kind(p))
     roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net)
     per_kernel = {}
     for g in ("edge_bwd", "density", "mlp_bwd", "mlp_fwd", "mlp_energy", "active"):
@@ -482,7 +507,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": f"{p.key}: {p.description}", "atoms": n, "T": p.T, "r_cut": p.r_cut,
                    "n_radial": p.n_radial, "l_max": p.l_max, "hidden": list(p.hidden), "dt_fs": dt_fs,
-                   "networks": "bf16 tcgen05, fp32 accumulate" if p.mlp_precision else "fp32 CUDA-core",
+                   "networks": NETWORK_DESCRIPTION[network_kind(p)],
                    "launch": "energy+forces and half kick replayed as one CUDA graph per step",
                    "ensemble": "NVE (velocity Verlet)" if noise is None else
                                f"NVT (stochastic velocity rescaling, {args.temperature:g} K, tau {args.tau:g} fs)",

@@ -79,7 +79,12 @@ typedef struct {
     double r_cut;          /* A */
     double skin;           /* A; the list radius is r_cut + skin */
     double alpha;          /* A^-2 */
-    int32_t mlp_precision; /* 0 = fp32 networks; 1 = bf16 tensor-core GEMMs, fp32 accumulate */
+    int32_t mlp_precision; /* 0 = fp32-accurate networks: on the tensor cores as three tf32 passes
+                                  (operands split hi + lo) for hidden widths [64, 64] with Eq. 1's
+                                  densities, on the CUDA cores otherwise;
+                              1 = bf16 tensor-core GEMMs (16-bit split activations), fp32 accumulate;
+                              2 = fp32 networks on the CUDA cores for every shape (a reference
+                                  for measuring the tensor-core paths) */
     int32_t dd_grid[3];    /* {0,0,0} = monolithic; else subdomains per axis (checking mode) */
     int32_t dd_stale_ghosts; /* checking mode only: 1 = skip the per-layer ghost refresh (negative control) */
     int32_t density_form;    /* 0 = Eq. 1: rho_(n,l) = sum_tau w_tau A_{n,tau}^2, D_rho = N_phi (L+1) features;
@@ -120,9 +125,12 @@ typedef struct {
     int64_t active_pairs;        /* ordered pairs within r_cut at the last evaluation */
     int64_t builds;              /* neighbour-list builds since creation */
     int64_t evaluations;         /* energy+force evaluations since creation */
-    int64_t ghost_slots;         /* domain-decomposed mode: ghost atoms over all subdomains */
-    int64_t ghost_bytes_fwd;     /* domain-decomposed mode: bytes gathered per layer, forward */
-    int64_t ghost_bytes_bwd;     /* domain-decomposed mode: bytes reduced per layer, backward */
+    int64_t ghost_slots;         /* domain-decomposed mode: ghost atoms over all subdomains;
+                                    halo plan: this process's ghost atoms */
+    int64_t ghost_bytes_fwd;     /* domain-decomposed mode: bytes gathered per layer, forward;
+                                    halo plan: coefficient bytes this process sends per layer */
+    int64_t ghost_bytes_bwd;     /* domain-decomposed mode: bytes reduced per layer, backward;
+                                    halo plan: gradient-partial bytes this process sends per layer */
     int64_t kernel_launches;     /* kernels this context has launched since creation */
     int32_t cells[3];            /* cell grid of the neighbour search */
     int32_t reserved;
@@ -240,6 +248,67 @@ reann_status reann_md_step_nvt(reann_ctx *ctx, int32_t nsteps, double dt_fs, dou
 
 /* Copies the counters of the context into *out (host).  Synchronises nothing. */
 reann_status reann_get_counters(const reann_ctx *ctx, reann_counters *out);
+
+/*
+ * One process's share of a spatial decomposition over several processes or
+ * GPUs: the per-layer halo exchange of section "Parallelization Algorithm"
+ * (Figs. 3-4, Eqs. 3-5).  The caller owns the decomposition and the transport;
+ * the library evaluates its own atoms and moves rows to and from two
+ * library-owned device buffers at the points where the method exchanges data.
+ *
+ * Atoms are in the caller's order: n_local own atoms, then n_ghost ghosts
+ * (other processes' atoms within r_cut + skin of this process's own atoms,
+ * e.g. of its region, grouped by the process that owns them).  send_index
+ * (host, [n_send]) lists the own atoms, by caller index, that are ghosts of
+ * other processes, in the order the exchange function sends them (grouped by
+ * destination); an own atom may appear several times.
+ *
+ * reann_halo_plan sets this up (allocates the exchange buffers); then
+ * reann_build_neighbors takes n = n_local + n_ghost atoms and builds rows for
+ * own atoms (all neighbours) and for ghosts (own neighbours only).  The plan
+ * stays until the next reann_halo_plan; reann_energy_forces and the MD calls
+ * refuse a context with a plan (REANN_ERR_STATE).  Errors: REANN_ERR_ARG
+ * (sizes, an entry outside [0, n_local)), REANN_ERR_STATE (domain-decomposed
+ * checking mode), REANN_ERR_CUDA.
+ */
+reann_status reann_halo_plan(reann_ctx *ctx, int64_t n_local, int64_t n_ghost, const int32_t *send_index,
+                             int64_t n_send);
+
+/*
+ * The exchange function the caller provides.  kind:
+ *   REANN_EXCHANGE_COEF (after coefficient network t-1, layer = t = 1..T-1):
+ *     send = own atoms' c^t rows in send_index order [send_rows = n_send][width = D];
+ *     recv must receive the ghosts' c^t rows in ghost order [recv_rows = n_ghost][D].
+ *   REANN_EXCHANGE_COEF_GRAD (after layer t's edge pass, layer = t = T-1..1):
+ *     send = the ghosts' partial dE/dc^t from this process's energies [n_ghost][D];
+ *     recv must receive the partials other processes computed for this
+ *     process's sent rows, in send_index order [n_send][D]; they are added.
+ *   REANN_EXCHANGE_FORCE (once, layer = 0): the same with partial forces [.][3].
+ * send and recv are library-owned device buffers (float32, row-major); the
+ * send rows are complete in `stream` order when the function is called, and
+ * the received rows must be in place, in `stream` order, before work the
+ * library enqueues on `stream` after it returns (enqueue the transfer on
+ * `stream`, or synchronise it and copy).  Return 0, or nonzero to abort the
+ * evaluation with REANN_ERR_CUDA.
+ */
+enum { REANN_EXCHANGE_COEF = 0, REANN_EXCHANGE_COEF_GRAD = 1, REANN_EXCHANGE_FORCE = 2 };
+typedef int32_t (*reann_exchange_fn)(void *user, int32_t kind, int32_t layer, const float *send, int64_t send_rows,
+                                     float *recv, int64_t recv_rows, int32_t width, reann_stream stream);
+
+/*
+ * Energy and forces of this process's own atoms under a halo plan.  pos: all
+ * n_local + n_ghost positions (float32 [n][3], caller order; the caller moves
+ * the ghosts' positions); *energy (host): the sum of the own atoms' energies;
+ * forces [n_local][3] and atom_energy [n_local] (nullable): own atoms, forces
+ * including the partials received from the other processes.  Host or device
+ * arrays as in reann_energy_forces.  Calls `exchange` 2 (T - 1) + 1 times, in
+ * the same order on every process.  Synchronises the stream at the end.
+ * Errors: REANN_ERR_STATE (no plan or no list), REANN_ERR_ARG,
+ * REANN_ERR_SKIN, REANN_ERR_NONFINITE, REANN_ERR_CUDA, REANN_ERR_TIMEOUT.
+ */
+reann_status reann_energy_forces_halo(reann_ctx *ctx, const float *pos, double *energy, float *forces,
+                                      float *atom_energy, reann_exchange_fn exchange, void *user,
+                                      reann_stream stream);
 
 /* Message of the last error on this context (or of the last failed create when ctx is NULL). */
 const char *reann_last_error(const reann_ctx *ctx);

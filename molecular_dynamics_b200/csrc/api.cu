@@ -11,8 +11,10 @@
 //     t = T-1 .. 0:  F += edge VJP, dE/dc^t                      [edge.cu]
 //                    G^{t-1} from M^{t-1}'s VJP (Eq. 5)          [mlp*.cu]
 //   E = sum_i E_i (deterministic fp64 tree)                      [md.cu]
-// The networks run on the tensor cores (mlp_tc.cu; mlp_tc_pair.cu for the
-// pair-product densities) or, with fp32 networks, on the CUDA cores (mlp.cu).
+// The networks run on the tensor cores: bf16 operands (mlp_tc.cu; mlp_tc_pair.cu
+// for the pair-product densities) or fp32-accurate three-pass tf32 for hidden
+// widths [64, 64] (mlp_tc32.cu); the other fp32 shapes, and mlp_precision 2,
+// use the CUDA cores (mlp.cu).
 // reann_md_step replays each step's evaluation and closing half kick as a
 // CUDA graph captured once per neighbour list (ef_and_kick).
 #include <algorithm>
@@ -109,7 +111,7 @@ void free_atoms(reann_ctx *c) {
     dfree(c->d_A); dfree(c->d_rho); dfree(c->d_coef); dfree(c->d_G); dfree(c->d_dc); dfree(c->d_Ei);
     dfree(c->d_F); dfree(c->d_Epart); dfree(c->d_stage_f); dfree(c->d_stage_i); dfree(c->d_stage_x);
     dfree(c->d_stage_v); dfree(c->d_stage_e); dfree(c->d_x); dfree(c->d_v); dfree(c->d_diag);
-    dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub);
+    dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub); dfree(c->d_tanhd); dfree(c->d_order);
     c->md_valid = false;
     c->slots_alloc = 0;
     c->n_alloc = 0;
@@ -129,6 +131,7 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_row, N + 1));
     CK(dalloc(&c->d_cnt, N));
     CK(dalloc(&c->d_act_cnt, N));
+    CK(dalloc(&c->d_order, N));
     CK(dalloc(&c->d_A, (size_t)c->T * N * c->NA));
     CK(dalloc(&c->d_rho, (size_t)c->T * N * c->DR));
     CK(dalloc(&c->d_coef, (size_t)c->T * N * c->D));
@@ -148,6 +151,8 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_last_x, 3 * N));
     CK(dalloc(&c->d_last_v, 3 * N));
     if (c->dd) CK(dalloc(&c->d_dd_sub, N));
+    if (c->cfg.mlp_precision == 0 && tc32_supported(c))
+        CK(dalloc(&c->d_tanhd, (size_t)std::max(c->T - 1, 1) * N * (size_t)(c->H1 + c->H2)));
     c->slots_alloc = n;
     c->n_alloc = n;
     return REANN_OK;
@@ -156,6 +161,7 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
 // slot-sized arrays (positions, coefficients, dE/dA) for n_slots >= n slots;
 // the first n positions are kept
 reann_status ensure_slots(reann_ctx *c, int64_t n_slots, cudaStream_t s) {
+    if (n_slots != c->n_slots) ++c->layout_gen;
     c->n_slots = n_slots;
     if (n_slots <= c->slots_alloc) return REANN_OK;
     float4 *pos = nullptr;
@@ -191,6 +197,7 @@ reann_status ensure_bins(reann_ctx *c) {
 
 reann_status ensure_capacity(reann_ctx *c, int64_t nnz) {
     if (nnz <= c->cap && c->d_col) return REANN_OK;
+    ++c->layout_gen;
     int64_t cap = nnz + nnz / 5 + 1024;
     if (cap > INT32_MAX) cap = INT32_MAX;
     CK(dalloc(&c->d_col, (size_t)cap));
@@ -219,7 +226,7 @@ reann_status check_status(reann_ctx *c, int st) {
 // Binning + CSR for the caller-order float positions/types already on the
 // device.  Reads nnz back (one synchronisation) and grows the list if needed.
 reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s) {
-    c->g_valid = false;   // list sizes and buffers may change: the step graph is recaptured
+    if (c->dd) ++c->layout_gen;   // the checking mode's ghost maps and slot count change with the list
     CK(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
     CK(launch_build(c, d_pos_caller, d_types_caller, s));
     CK(cudaMemcpyAsync(c->h_i64, c->d_i64, sizeof(int64_t) * 3, cudaMemcpyDeviceToHost, s));
@@ -234,6 +241,7 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
     if (nnz > INT32_MAX) return fail(c, REANN_ERR_CAPACITY, "neighbour list exceeds 2^31-1 entries");
     if ((st = ensure_capacity(c, nnz))) return st;
     CK(launch_fill(c, s));
+    CK(launch_work_order(c, s));
     c->nnz = nnz;
     c->max_row = c->h_i64[2];
     // tile tables of the atomic networks: element segments cut into 32-row
@@ -242,6 +250,7 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
     bool same = c->elem_start.size() == (size_t)c->ne + 1 &&
                 std::equal(c->elem_start.begin(), c->elem_start.end(), c->h_seg);
     if (!same) {
+        ++c->layout_gen;
         std::vector<int4> tiles, tiles128;
         for (int e = 0; e < c->ne; ++e) {
             for (int r = c->h_seg[e]; r < c->h_seg[e + 1]; r += 32)
@@ -314,6 +323,7 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
 // One energy+force evaluation on the internal positions d_pos.
 reann_status run_ef(reann_ctx *c, cudaStream_t s) {
     const bool tc = c->cfg.mlp_precision == 1, pair = c->cfg.density_form == 1;
+    const bool tc32 = c->cfg.mlp_precision == 0 && tc32_supported(c);
     const int64_t cstride = c->n_slots * c->D;
     // domain-decomposed mode: ghost positions follow their owners
     if (c->dd) CK(dd_gather_rows(c, reinterpret_cast<float *>(c->d_pos), 4, s));
@@ -322,7 +332,7 @@ reann_status run_ef(reann_ctx *c, cudaStream_t s) {
         CK(launch_density_fwd(c, t, s));
         if (t + 1 < c->T) {
             CK(tc ? (pair ? launch_mlp_tc_pair_coef_fwd(c, t, s) : launch_mlp_tc_coef_fwd(c, t, s))
-                  : launch_mlp_coef_fwd(c, t, s));
+                  : (tc32 ? launch_mlp_tc32_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s)));
             // the per-layer message sync: ghost c^{t+1} from the owners (or, as
             // a negative control, the ghosts keep c^0)
             if (c->dd) {
@@ -331,13 +341,14 @@ reann_status run_ef(reann_ctx *c, cudaStream_t s) {
             }
         }
     }
-    CK(tc ? (pair ? launch_mlp_tc_pair_energy(c, s) : launch_mlp_tc_energy(c, s)) : launch_mlp_energy(c, s));
+    CK(tc ? (pair ? launch_mlp_tc_pair_energy(c, s) : launch_mlp_tc_energy(c, s))
+          : (tc32 ? launch_mlp_tc32_energy(c, s) : launch_mlp_energy(c, s)));
     if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
     for (int t = c->T - 1; t >= 0; --t) {
         CK(launch_edge_bwd(c, t, t != c->T - 1, s));
         if (t >= 1) {
             CK(tc ? (pair ? launch_mlp_tc_pair_coef_bwd(c, t, s) : launch_mlp_tc_coef_bwd(c, t, s))
-                  : launch_mlp_coef_bwd(c, t, s));
+                  : (tc32 ? launch_mlp_tc32_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s)));
             if (c->dd) CK(dd_gather_rows(c, c->d_G, c->NA, s));
         }
     }
@@ -363,7 +374,8 @@ reann_status ef_and_kick(reann_ctx *c, double dt_fs, const double *inv_mass, cud
         CK(cudaStreamCreateWithFlags(&c->g_stream, cudaStreamNonBlocking));
         for (auto &ev : c->g_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
     }
-    const bool same = c->g_valid && c->g_dt == dt_fs && std::equal(inv_mass, inv_mass + c->ne, c->g_inv_mass);
+    const bool same = c->g_valid && c->g_gen == c->layout_gen && c->g_dt == dt_fs &&
+                      std::equal(inv_mass, inv_mass + c->ne, c->g_inv_mass);
     CK(cudaEventRecord(c->g_ev[0], s));
     CK(cudaStreamWaitEvent(c->g_stream, c->g_ev[0], 0));
     if (!same) {
@@ -389,6 +401,7 @@ reann_status ef_and_kick(reann_ctx *c, double dt_fs, const double *inv_mass, cud
         cudaGraphDestroy(g);
         CK(ei);
         c->g_valid = true;
+        c->g_gen = c->layout_gen;
         c->g_dt = dt_fs;
         std::copy(inv_mass, inv_mass + c->ne, c->g_inv_mass);
     }
@@ -399,6 +412,100 @@ reann_status ef_and_kick(reann_ctx *c, double dt_fs, const double *inv_mass, cud
     c->counters.evaluations++;
     c->have_eval = true;
     return REANN_OK;
+}
+
+// Builds the device-side step loop (see reann_ctx::l_exec) for the current
+// list, dt, masses and thermostat: a WHILE node whose body is kick-drift and
+// the gate, followed by an IF node holding energy+forces, the closing kick and
+// (NVT) the thermostat with its numbers read from d_noise.  Bodies are filled
+// by stream capture on the library stream.
+cudaError_t capture_loop(reann_ctx *c, double dt_fs, const double *inv_mass, const double *mass,
+                         const BussiParams *B) {
+    if (c->l_exec) {
+        cudaGraphExecDestroy(c->l_exec);
+        c->l_exec = nullptr;
+    }
+    c->l_valid = false;
+    const int64_t k0 = c->counters.kernel_launches, e0 = c->counters.evaluations;
+    cudaGraph_t lg = nullptr;
+    cudaError_t e = cudaGraphCreate(&lg, 0);
+    if (e) return e;
+    struct Cleanup {
+        cudaGraph_t g;
+        reann_ctx *c;
+        int64_t k0, e0;
+        ~Cleanup() {
+            if (g) cudaGraphDestroy(g);
+            c->counters.kernel_launches = k0;
+            c->counters.evaluations = e0;
+        }
+    } cleanup{lg, c, k0, e0};
+    cudaGraphConditionalHandle h_while, h_step;
+    if ((e = cudaGraphConditionalHandleCreate(&h_while, lg, 1, cudaGraphCondAssignDefault))) return e;
+    cudaGraphNodeParams wp = {};
+    wp.type = cudaGraphNodeTypeConditional;
+    wp.conditional.handle = h_while;
+    wp.conditional.type = cudaGraphCondTypeWhile;
+    wp.conditional.size = 1;
+    cudaGraphNode_t wnode;
+    if ((e = cudaGraphAddNode(&wnode, lg, nullptr, 0, &wp))) return e;
+    cudaGraph_t body = wp.conditional.phGraph_out[0];
+    if ((e = cudaGraphConditionalHandleCreate(&h_step, body, 0, cudaGraphCondAssignDefault))) return e;
+    // body: kick-drift, then the gate
+    cudaGraph_t got = nullptr;
+    if ((e = cudaStreamBeginCaptureToGraph(c->g_stream, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal)))
+        return e;
+    cudaError_t e1 = launch_md_kick_drift(c, dt_fs, inv_mass, c->d_status + 1, c->g_stream);
+    cudaError_t e2 = e1 ? e1 : launch_loop_gate(c, h_while, h_step, c->g_stream);
+    e = cudaStreamEndCapture(c->g_stream, &got);
+    if (e2) return e2;
+    if (e) return e;
+    // the gate is the body's one node without dependents
+    size_t nn = 0;
+    if ((e = cudaGraphGetNodes(body, nullptr, &nn))) return e;
+    std::vector<cudaGraphNode_t> nodes(nn);
+    if ((e = cudaGraphGetNodes(body, nodes.data(), &nn))) return e;
+    cudaGraphNode_t leaf = nullptr;
+    for (auto nd : nodes) {
+        size_t nd_out = 0;
+        if ((e = cudaGraphNodeGetDependentNodes(nd, nullptr, &nd_out))) return e;
+        if (nd_out == 0) leaf = nd;
+    }
+    if (!leaf) return cudaErrorInvalidValue;
+    cudaGraphNodeParams ip = {};
+    ip.type = cudaGraphNodeTypeConditional;
+    ip.conditional.handle = h_step;
+    ip.conditional.type = cudaGraphCondTypeIf;
+    ip.conditional.size = 1;
+    cudaGraphNode_t inode;
+    if ((e = cudaGraphAddNode(&inode, body, &leaf, 1, &ip))) return e;
+    cudaGraph_t step_body = ip.conditional.phGraph_out[0];
+    // the admitted step: energy+forces, closing kick, thermostat
+    const int64_t k1 = c->counters.kernel_launches;
+    if ((e = cudaStreamBeginCaptureToGraph(c->g_stream, step_body, nullptr, nullptr, 0,
+                                           cudaStreamCaptureModeThreadLocal)))
+        return e;
+    reann_status st = run_ef(c, c->g_stream);
+    e1 = st ? cudaSuccess : launch_md_kick(c, dt_fs, inv_mass, c->g_stream);
+    if (!st && !e1 && B) e1 = launch_thermostat(c, mass, *B, c->d_E + 2, c->g_stream, c->d_noise, c->d_loop);
+    e = cudaStreamEndCapture(c->g_stream, &got);
+    if (st) return cudaErrorInvalidValue;
+    if (e1) return e1;
+    if (e) return e;
+    c->l_step_launches = c->counters.kernel_launches - k0;
+    (void)k1;
+    if ((e = cudaGraphInstantiate(&c->l_exec, lg, 0))) {
+        c->l_exec = nullptr;
+        return e;
+    }
+    c->l_valid = true;
+    c->l_gen = c->layout_gen;
+    c->l_dt = dt_fs;
+    std::copy(inv_mass, inv_mass + c->ne, c->l_inv_mass);
+    c->l_thermo[0] = B ? B->c : -1.0;
+    c->l_thermo[1] = B ? B->kt : 0.0;
+    c->l_thermo[2] = B ? B->nf : 0.0;
+    return cudaSuccess;
 }
 
 void fill_counters(reann_ctx *c) {
@@ -465,7 +572,7 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     *out = nullptr;
     if (cfg->n_elements < 1 || cfg->n_elements > MAX_ELEMENTS || cfg->T < 1 || cfg->T > MAX_T ||
         !(cfg->r_cut > 0) || !(cfg->skin >= 0) || !(cfg->alpha > 0) || !std::isfinite(cfg->r_cut) ||
-        !std::isfinite(cfg->skin) || cfg->mlp_precision < 0 || cfg->mlp_precision > 1)
+        !std::isfinite(cfg->skin) || cfg->mlp_precision < 0 || cfg->mlp_precision > 2)
         return fail(nullptr, REANN_ERR_ARG, "invalid configuration");
     if (cfg->mlp_precision == 1 && (cfg->hidden[0] != 128 || cfg->hidden[1] != 128))
         return fail(nullptr, REANN_ERR_UNSUPPORTED, "bf16 tensor-core networks need hidden widths [128, 128]");
@@ -489,6 +596,8 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     {
         const char *gv = std::getenv("REANN_GRAPHS");
         c->g_disabled = gv && std::strcmp(gv, "0") == 0;
+        const char *lv = std::getenv("REANN_LOOP");
+        c->l_disabled = lv && std::strcmp(lv, "0") == 0;
     }
     c->NP = cfg->n_radial;
     c->D = c->NP * (cfg->l_max + 1);
@@ -559,7 +668,13 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
         cudaEventDestroy(r.b);
     }
     for (auto ev : c->prof_pool) cudaEventDestroy(ev);
+    dfree(c->d_send_caller); dfree(c->d_send_atom); dfree(c->d_send_off); dfree(c->d_send_order);
+    dfree(c->d_xsend); dfree(c->d_xrecv);
     if (c->g_exec) cudaGraphExecDestroy(c->g_exec);
+    if (c->l_exec) cudaGraphExecDestroy(c->l_exec);
+    if (c->d_loop) cudaFree(c->d_loop);
+    if (c->h_loop) cudaFreeHost(c->h_loop);
+    if (c->d_noise) cudaFree(c->d_noise);
     for (auto ev : c->g_ev)
         if (ev) cudaEventDestroy(ev);
     if (c->g_stream) cudaStreamDestroy(c->g_stream);
@@ -581,8 +696,11 @@ extern "C" reann_status reann_build_neighbors(reann_ctx *c, int64_t n, const flo
     for (int a = 0; a < 3; ++a)
         if (!(box[a] > 0) || !std::isfinite(box[a]) || box[a] < 2.0 * rl)
             return fail(c, REANN_ERR_BOX, "box edge must be finite and at least 2 (r_cut + skin)");
+    if (c->halo && n != c->n_local + c->n_ghost_plan)
+        return fail(c, REANN_ERR_ARG, "with a halo plan, n must be the plan's own plus ghost atoms");
     reann_status st;
     if ((st = ensure_atoms(c, n))) return st;
+    ++c->layout_gen;   // a caller's build may change n, the box or any buffer
     c->n = n;
     c->have_list = c->have_eval = false;
     c->md_valid = false;
@@ -593,7 +711,7 @@ extern "C" reann_status reann_build_neighbors(reann_ctx *c, int64_t n, const flo
         ncell *= c->m[a];
     }
     c->ncell = ncell;
-    c->nbins = ncell * c->ne;
+    c->nbins = ncell * c->ne * (c->halo ? 2 : 1);   // a halo plan's ghosts bin in classes of their own
     if ((st = ensure_bins(c))) return st;
     if ((st = ensure_scan_tmp(c, std::max<int64_t>(n, c->nbins)))) return st;
     const float *d_pos = pos;
@@ -612,6 +730,7 @@ extern "C" reann_status reann_energy_forces(reann_ctx *c, const float *pos, doub
                                             float *atom_energy, reann_stream stream) {
     if (!c) return REANN_ERR_ARG;
     if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if (c->halo) return fail(c, REANN_ERR_STATE, "a halo plan needs reann_energy_forces_halo");
     if (c->n > 0 && !pos) return fail(c, REANN_ERR_ARG, "null positions");
     DeviceGuard guard(c->device);
     cudaStream_t s = (cudaStream_t)stream;
@@ -663,6 +782,7 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
                            reann_md_stats *stats, reann_stream stream, const NvtArgs *nvt) {
     if (!c) return REANN_ERR_ARG;
     if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if (c->halo) return fail(c, REANN_ERR_STATE, "MD steps over a halo plan are not provided (energy+forces only)");
     if (nsteps < 0 || !std::isfinite(dt_fs) || !mass_amu || (c->n > 0 && (!x || !v)))
         return fail(c, REANN_ERR_ARG, "invalid arguments");
     BussiParams B{};
@@ -737,7 +857,85 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
         CK(cudaStreamCreateWithFlags(&c->o_stream, cudaStreamNonBlocking));
         for (auto &ev : c->o_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
     }
-    for (int32_t step = 0; step < nsteps; ++step) {
+    int32_t step = 0;
+    // all steps but the last between rebuilds on the device (one host
+    // synchronisation per stretch); the last step keeps the overlapped copy-out
+    const bool loop = !c->prof && !c->g_disabled && !c->l_disabled && n > 0 && nsteps >= 2;
+    if (loop && nvt) {
+        if (2 * (int64_t)nsteps > c->noise_alloc) {
+            if (c->d_noise) cudaFree(c->d_noise);
+            c->d_noise = nullptr;
+            c->noise_alloc = 0;
+            c->l_valid = false;   // the loop graph reads the noise through this pointer
+            CK(cudaMalloc(&c->d_noise, sizeof(double) * 2 * (size_t)nsteps));
+            c->noise_alloc = 2 * (int64_t)nsteps;
+        }
+        CK(cudaMemcpyAsync(c->d_noise, nvt->noise, sizeof(double) * 2 * (size_t)nsteps, cudaMemcpyHostToDevice, s));
+    }
+    while (loop && !c->l_disabled && step < nsteps - 1) {
+        if (!c->g_stream) {
+            CK(cudaStreamCreateWithFlags(&c->g_stream, cudaStreamNonBlocking));
+            for (auto &ev : c->g_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+        }
+        if (!c->d_loop) {
+            CK(cudaMalloc(&c->d_loop, sizeof(int) * 4));
+            CK(cudaMallocHost(&c->h_loop, sizeof(int) * 4));
+        }
+        const bool same = c->l_valid && c->l_gen == c->layout_gen && c->l_dt == dt_fs &&
+                          std::equal(inv_mass, inv_mass + c->ne, c->l_inv_mass) &&
+                          (nvt ? (c->l_thermo[0] == B.c && c->l_thermo[1] == B.kt && c->l_thermo[2] == B.nf)
+                               : c->l_thermo[0] < 0);
+        if (!same) {
+            CK(cudaStreamSynchronize(s));
+            cudaError_t el = capture_loop(c, dt_fs, inv_mass, mass, nvt ? &B : nullptr);
+            if (el) {
+                // this runtime or driver cannot build the loop graph: per-step graphs from here on
+                cudaGetLastError();
+                c->l_disabled = true;
+                break;
+            }
+        }
+        c->h_loop[0] = 0;
+        c->h_loop[1] = nsteps - 1 - step;
+        c->h_loop[2] = 0;
+        c->h_loop[3] = step;
+        CK(cudaMemcpyAsync(c->d_loop, c->h_loop, sizeof(int) * 4, cudaMemcpyHostToDevice, s));
+        CK(cudaEventRecord(c->g_ev[0], s));
+        CK(cudaStreamWaitEvent(c->g_stream, c->g_ev[0], 0));
+        CK(cudaGraphLaunch(c->l_exec, c->g_stream));
+        CK(cudaEventRecord(c->g_ev[1], c->g_stream));
+        CK(cudaStreamWaitEvent(s, c->g_ev[1], 0));
+        CK(cudaMemcpyAsync(c->h_loop, c->d_loop, sizeof(int) * 4, cudaMemcpyDeviceToHost, s));
+        CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int) * 2, cudaMemcpyDeviceToHost, s));
+        CK(sync_stream(c, s));
+        const int admitted = c->h_loop[0];
+        c->counters.kernel_launches += (int64_t)admitted * c->l_step_launches + (c->h_loop[2] == 3 ? 0 : 2);
+        c->counters.evaluations += admitted;
+        c->have_eval = c->have_eval || admitted > 0;
+        step += admitted;
+        done += admitted;
+        if (c->h_loop[2] == 2 || (st = check_status(c, c->h_status[0] & ~ST_SKIN))) {
+            if (!st) st = check_status(c, c->h_status[0]);
+            return st ? st : fail(c, REANN_ERR_CUDA, "device step loop stopped on an error");
+        }
+        if (c->h_loop[2] == 1) {
+            // step `step` has drifted and tripped the skin check: rebuild, then finish it here
+            CK(launch_md_scatter(c, c->d_stage_x, c->d_stage_v, c->d_stage_f, s));
+            if ((st = build_internal(c, c->d_stage_f, c->d_types_caller, s))) return st;
+            CK(launch_md_gather(c, c->d_stage_x, c->d_stage_v, s));
+            CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
+            ++rebuilds;
+            if ((st = ef_and_kick(c, dt_fs, inv_mass, s))) return st;
+            if (nvt) {
+                B.r1 = nvt->noise[2 * step];
+                B.s = nvt->noise[2 * step + 1];
+                CK(launch_thermostat(c, mass, B, c->d_E + 2, s));
+            }
+            ++step;
+            ++done;
+        }
+    }
+    for (; step < nsteps; ++step) {
         CK(launch_md_kick_drift(c, dt_fs, inv_mass, c->d_status + 1, s));
         CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int) * 2, cudaMemcpyDeviceToHost, s));
         CK(sync_stream(c, s));
@@ -809,6 +1007,149 @@ extern "C" reann_status reann_md_step_nvt(reann_ctx *c, int32_t nsteps, double d
                                           const double *mass_amu, reann_md_stats *stats, reann_stream stream) {
     const NvtArgs nvt{temperature_K, tau_fs, noise};
     return md_run(c, nsteps, dt_fs, x, v, mass_amu, stats, stream, &nvt);
+}
+
+// ---------------------------------------------------------------------------
+// One process's share of a spatial decomposition (halo.cu has the row moves).
+
+extern "C" reann_status reann_halo_plan(reann_ctx *c, int64_t n_local, int64_t n_ghost, const int32_t *send_index,
+                                        int64_t n_send) {
+    if (!c) return REANN_ERR_ARG;
+    if (n_local < 0 || n_ghost < 0 || n_send < 0 || (n_send > 0 && !send_index) || n_local + n_ghost >= INT32_MAX)
+        return fail(c, REANN_ERR_ARG, "invalid halo plan sizes");
+    if (c->dd) return fail(c, REANN_ERR_STATE, "a halo plan and the domain-decomposed checking mode exclude each other");
+    std::vector<int32_t> idx(send_index, send_index + n_send);
+    for (int32_t a : idx)
+        if (a < 0 || a >= n_local) return fail(c, REANN_ERR_ARG, "send_index entries must be own atoms, 0 <= i < n_local");
+    // sent rows grouped by own atom (ascending), positions ascending within an atom
+    std::vector<int32_t> order(n_send);
+    for (int64_t k = 0; k < n_send; ++k) order[k] = (int32_t)k;
+    std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return idx[x] < idx[y]; });
+    std::vector<int32_t> atoms, off;
+    for (int64_t k = 0; k < n_send; ++k) {
+        if (k == 0 || idx[order[k]] != idx[order[k - 1]]) {
+            atoms.push_back(idx[order[k]]);
+            off.push_back((int32_t)k);
+        }
+    }
+    off.push_back((int32_t)n_send);
+    DeviceGuard guard(c->device);
+    dfree(c->d_send_caller); dfree(c->d_send_atom); dfree(c->d_send_off); dfree(c->d_send_order);
+    const int width = std::max(c->D, 3);
+    const int64_t rows = std::max<int64_t>(std::max(n_send, n_ghost), 1);
+    if (rows * width > c->xbuf_alloc) {
+        dfree(c->d_xsend); dfree(c->d_xrecv);
+        c->xbuf_alloc = 0;
+        CK(dalloc(&c->d_xsend, (size_t)(rows * width)));
+        CK(dalloc(&c->d_xrecv, (size_t)(rows * width)));
+        c->xbuf_alloc = rows * width;
+    }
+    CK(dalloc(&c->d_send_caller, (size_t)std::max<int64_t>(n_send, 1)));
+    CK(dalloc(&c->d_send_order, (size_t)std::max<int64_t>(n_send, 1)));
+    CK(dalloc(&c->d_send_atom, std::max<size_t>(atoms.size(), 1)));
+    CK(dalloc(&c->d_send_off, off.size()));
+    if (n_send > 0) {
+        CK(cudaMemcpy(c->d_send_caller, idx.data(), sizeof(int32_t) * n_send, cudaMemcpyHostToDevice));
+        CK(cudaMemcpy(c->d_send_order, order.data(), sizeof(int32_t) * n_send, cudaMemcpyHostToDevice));
+        CK(cudaMemcpy(c->d_send_atom, atoms.data(), sizeof(int32_t) * atoms.size(), cudaMemcpyHostToDevice));
+    }
+    CK(cudaMemcpy(c->d_send_off, off.data(), sizeof(int32_t) * off.size(), cudaMemcpyHostToDevice));
+    c->halo = true;
+    c->n_local = n_local;
+    c->n_ghost_plan = n_ghost;
+    c->n_send = n_send;
+    c->n_send_atoms = (int64_t)atoms.size();
+    c->halo_bytes_fwd = n_send * c->D * (int64_t)sizeof(float);
+    c->halo_bytes_bwd = n_ghost * c->D * (int64_t)sizeof(float);
+    c->have_list = c->have_eval = false;   // the list must be rebuilt for the plan's atoms
+    c->md_valid = false;
+    return REANN_OK;
+}
+
+extern "C" reann_status reann_energy_forces_halo(reann_ctx *c, const float *pos, double *energy, float *forces,
+                                                 float *atom_energy, reann_exchange_fn exchange, void *user,
+                                                 reann_stream stream) {
+    if (!c) return REANN_ERR_ARG;
+    if (!c->halo) return fail(c, REANN_ERR_STATE, "reann_halo_plan must come first");
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if ((c->n > 0 && !pos) || !exchange) return fail(c, REANN_ERR_ARG, "null positions or exchange function");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n, nl = c->n_local, ng = c->n - c->n_local;
+    c->md_valid = false;
+    CK(cudaMemsetAsync(c->d_status, 0, sizeof(int), s));
+    if (n > 0) {
+        const float *d_pos = pos;
+        if (!is_device_ptr(pos)) {
+            CK(cudaMemcpyAsync(c->d_stage_f, pos, sizeof(float) * 3 * n, cudaMemcpyHostToDevice, s));
+            d_pos = c->d_stage_f;
+        }
+        CK(launch_pos_from_caller(c, d_pos, s));
+        CK(launch_skin_check(c, c->d_status, s));
+    }
+    auto call = [&](int kind, int layer, int width, int64_t send_rows, int64_t recv_rows) -> reann_status {
+        const int32_t rc = exchange(user, kind, layer, c->d_xsend, send_rows, c->d_xrecv, recv_rows, width, stream);
+        if (rc != 0) return fail(c, REANN_ERR_CUDA, "the exchange function failed (" + std::to_string(rc) + ")");
+        return REANN_OK;
+    };
+    reann_status st;
+    const bool tc = c->cfg.mlp_precision == 1, pair = c->cfg.density_form == 1;
+    const bool tc32 = c->cfg.mlp_precision == 0 && tc32_supported(c);
+    const int64_t cstride = c->n_slots * c->D;
+    // ghost rows of dE/dA are zero throughout: a ghost's energy is its owner's
+    if (ng > 0) CK(cudaMemsetAsync(c->d_G + nl * c->NA, 0, sizeof(float) * (size_t)(ng * c->NA), s));
+    CK(launch_active(c, s));
+    for (int t = 0; t < c->T; ++t) {
+        CK(launch_density_fwd(c, t, s));
+        if (t + 1 < c->T) {
+            float *coef = c->d_coef + (t + 1) * cstride;
+            CK(tc ? (pair ? launch_mlp_tc_pair_coef_fwd(c, t, s) : launch_mlp_tc_coef_fwd(c, t, s))
+                  : (tc32 ? launch_mlp_tc32_coef_fwd(c, t, s) : launch_mlp_coef_fwd(c, t, s)));
+            // forward exchange: own c^{t+1} rows out, ghost rows in
+            CK(launch_halo_pack_own(c, coef, c->D, s));
+            if ((st = call(REANN_EXCHANGE_COEF, t + 1, c->D, c->n_send, ng))) return st;
+            CK(launch_halo_unpack_ghosts(c, coef, c->D, s));
+        }
+    }
+    CK(tc ? (pair ? launch_mlp_tc_pair_energy(c, s) : launch_mlp_tc_energy(c, s))
+          : (tc32 ? launch_mlp_tc32_energy(c, s) : launch_mlp_energy(c, s)));
+    for (int t = c->T - 1; t >= 0; --t) {
+        CK(launch_edge_bwd(c, t, t != c->T - 1, s));
+        if (t >= 1) {
+            // reverse exchange: ghost partials of dE/dc^t back to their owners
+            CK(launch_halo_pack_ghosts(c, c->d_dc, c->D, s));
+            if ((st = call(REANN_EXCHANGE_COEF_GRAD, t, c->D, ng, c->n_send))) return st;
+            CK(launch_halo_add_partials(c, c->d_dc, c->D, s));
+            CK(tc ? (pair ? launch_mlp_tc_pair_coef_bwd(c, t, s) : launch_mlp_tc_coef_bwd(c, t, s))
+                  : (tc32 ? launch_mlp_tc32_coef_bwd(c, t, s) : launch_mlp_coef_bwd(c, t, s)));
+        }
+    }
+    // ghost force partials back to their owners
+    CK(launch_halo_pack_ghosts(c, c->d_F, 3, s));
+    if ((st = call(REANN_EXCHANGE_FORCE, 0, 3, ng, c->n_send))) return st;
+    CK(launch_halo_add_partials(c, c->d_F, 3, s));
+    CK(launch_energy_sum(c, s));
+    c->counters.evaluations++;
+    c->have_eval = true;
+    bool f_dev = forces && is_device_ptr(forces), e_dev = atom_energy && is_device_ptr(atom_energy);
+    float *fo = forces ? (f_dev ? forces : c->d_stage_f) : nullptr;
+    float *eo = atom_energy ? (e_dev ? atom_energy : c->d_stage_e) : nullptr;
+    CK(launch_scatter_outputs(c, fo, eo, s));
+    if (forces && !f_dev && nl > 0)
+        CK(cudaMemcpyAsync(forces, c->d_stage_f, sizeof(float) * 3 * nl, cudaMemcpyDeviceToHost, s));
+    if (atom_energy && !e_dev && nl > 0)
+        CK(cudaMemcpyAsync(atom_energy, c->d_stage_e, sizeof(float) * nl, cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_E, c->d_E, sizeof(double), cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    CK(cudaMemcpyAsync(c->h_i64 + 3, c->d_i64 + 3, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+    CK(sync_stream(c, s));
+    c->counters.active_pairs = c->h_i64[3];
+    c->counters.ghost_slots = ng;
+    c->counters.ghost_bytes_fwd = c->halo_bytes_fwd;
+    c->counters.ghost_bytes_bwd = c->halo_bytes_bwd;
+    fill_counters(c);
+    if (energy) *energy = c->h_E[0];
+    return check_status(c, *c->h_status);
 }
 
 extern "C" reann_status reann_get_counters(const reann_ctx *c, reann_counters *out) {

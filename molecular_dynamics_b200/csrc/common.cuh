@@ -31,9 +31,14 @@ struct EdgeParams {
     double inv_box[3];
     float L_hi[3], L_lo[3], inv_L[3];   // box edge as an fp32 pair L_hi + L_lo, and 1/L
     float r_cut, r_cut2;
-    float pi_over_rc;
+    // theta = pi r / (2 r_c) as r th_hi + r th_lo, and the Gaussian centres
+    // mu_n = r_c n / (N_phi - 1) as mu_hi[n] + mu_lo[n]: fp32 pairs of the fp64
+    // constants, so that no constant carries a rounding error that every
+    // atom would share (a systematic shift of the centres or of the cutoff
+    // argument biases a large system's energy)
+    float th_hi, th_lo;
     float alpha;
-    float mu_step;      // mu_n = n * mu_step
+    float mu_hi[16], mu_lo[16];
 };
 
 // offsets (in floats) of one atomic network inside the device weight blob
@@ -108,6 +113,9 @@ struct reann_ctx {
     int *d_cnt = nullptr;          // [n]
     int *d_col = nullptr;          // [cap]
     int *d_act_cnt = nullptr;      // [n]
+    int *d_order = nullptr;        // [n] centre order of the edge passes: windows of consecutive atoms
+                                   // sorted by row length, so the centres a warp walks together have
+                                   // similar neighbour counts
     int *d_act_col = nullptr;      // [cap]
     float4 *d_act_geo = nullptr;   // [cap] displacement and distance of each active entry
     int64_t nnz = 0, cap = 0, max_row = 0;
@@ -115,6 +123,22 @@ struct reann_ctx {
     size_t scan_tmp_size = 0;
     int64_t *d_i64 = nullptr;      // small scratch of int64 scalars
     int64_t *h_i64 = nullptr;      // pinned mirror
+
+    // multi-process spatial decomposition (reann_halo_plan): caller atoms
+    // [0, n_local) are this process's own, [n_local, n) ghosts from other
+    // processes; internal order keeps the own atoms in [0, n_local)
+    bool halo = false;
+    int64_t n_local = 0;           // atoms whose densities, networks and energies this process evaluates
+    int64_t n_ghost_plan = 0;
+    int64_t n_send = 0;            // rows this process sends (its own atoms that are ghosts elsewhere)
+    int *d_send_caller = nullptr;  // [n_send] caller index of each sent row
+    int64_t n_send_atoms = 0;      // distinct own atoms among them
+    int *d_send_atom = nullptr;    // [n_send_atoms] their caller indices, ascending
+    int *d_send_off = nullptr;     // [n_send_atoms + 1] offsets into d_send_order
+    int *d_send_order = nullptr;   // [n_send] sent-row positions grouped by atom, ascending
+    float *d_xsend = nullptr, *d_xrecv = nullptr;   // exchange buffers
+    int64_t xbuf_alloc = 0;        // floats in each
+    int64_t halo_bytes_fwd = 0, halo_bytes_bwd = 0; // per layer, this process's send side
 
     // domain-decomposed checking mode: slots [0, n) local atoms, [n, n_slots) ghosts
     bool dd = false;
@@ -135,6 +159,7 @@ struct reann_ctx {
     float *d_coef = nullptr;   // [T][n_slots][D]  (layer 0 unused: c^0 comes from C0)
     float *d_G = nullptr;      // [n_slots][NA]  dE/dA^t
     float *d_dc = nullptr;     // [n][D]   dE/dc^t
+    float *d_tanhd = nullptr;  // [T-1][n][2 H] tanh' of both hidden layers (three-pass tf32 networks)
     float *d_Ei = nullptr;     // [n]
     float *d_F = nullptr;      // [n][3] internal order
     double *d_Epart = nullptr; // block partial sums of E
@@ -170,6 +195,12 @@ struct reann_ctx {
     cudaEvent_t g_ev[2] = {nullptr, nullptr};
     cudaGraphExec_t g_exec = nullptr;
     bool g_valid = false;
+    // what a captured graph bakes in -- buffer addresses, sizes, the box --
+    // changes only when layout_gen does (a caller's list build, a grown
+    // buffer, new network tiles, the checking mode's ghost maps); an MD
+    // rebuild that reuses every buffer keeps the graphs
+    int64_t layout_gen = 0;
+    int64_t g_gen = -1, l_gen = -1;
     double g_dt = 0.0;
     double g_inv_mass[reann::MAX_ELEMENTS] = {};
     int64_t g_launches = 0;   // kernels one replay runs
@@ -178,6 +209,21 @@ struct reann_ctx {
     cudaStream_t o_stream = nullptr;
     cudaEvent_t o_ev[2] = {nullptr, nullptr};
     bool g_disabled = false;  // REANN_GRAPHS=0 in the environment
+    // MD calls of two or more steps replay whole stretches between neighbour
+    // rebuilds as one graph: a WHILE node whose body is one step (kick-drift,
+    // a gate kernel, then under an IF node energy+forces, the closing kick and
+    // the thermostat); the host synchronises once per launch, not per step
+    cudaGraphExec_t l_exec = nullptr;
+    bool l_valid = false;
+    bool l_disabled = false;  // REANN_LOOP=0, or the loop graph could not be built
+    double l_dt = 0.0;
+    double l_inv_mass[reann::MAX_ELEMENTS] = {};
+    double l_thermo[3] = {-1.0, 0.0, 0.0};   // thermostat c, Kt, Nf of the captured loop (c < 0: none)
+    int64_t l_step_launches = 0;              // kernels one loop iteration runs
+    int *d_loop = nullptr;    // [4]: steps admitted, steps requested, end reason, first step index
+    int *h_loop = nullptr;    // pinned mirror
+    double *d_noise = nullptr;    // NVT: the call's two numbers per step
+    int64_t noise_alloc = 0;
 
     // status
     int *d_status = nullptr;

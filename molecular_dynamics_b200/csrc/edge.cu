@@ -48,9 +48,15 @@ EdgeParams make_edge_params(const reann_ctx *c) {
     }
     P.r_cut = (float)c->cfg.r_cut;
     P.r_cut2 = (float)(c->cfg.r_cut * c->cfg.r_cut);
-    P.pi_over_rc = (float)(3.14159265358979323846 / c->cfg.r_cut);
+    const double th = 0.5 * 3.14159265358979323846 / c->cfg.r_cut;
+    P.th_hi = (float)th;
+    P.th_lo = (float)(th - (double)P.th_hi);
     P.alpha = (float)c->cfg.alpha;
-    P.mu_step = (float)(c->cfg.r_cut / (c->cfg.n_radial - 1));
+    for (int k = 0; k < 16; ++k) {
+        const double mu = k < c->cfg.n_radial ? c->cfg.r_cut * k / (double)(c->cfg.n_radial - 1) : 0.0;
+        P.mu_hi[k] = (float)mu;
+        P.mu_lo[k] = (float)(mu - (double)P.mu_hi[k]);
+    }
     return P;
 }
 
@@ -151,7 +157,8 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
 
 // ---------------------------------------------------------------------------
 // Lane decomposition shared by both edge passes: a slot of LPE = N_phi / 2
-// lanes owns one centre atom and walks its active neighbours in row order;
+// lanes owns one centre atom (taken in the build's work order, which groups
+// centres of similar row length) and walks its active neighbours in row order;
 // lane `sub` owns radial indices 2 sub and 2 sub + 1.  A warp holds
 // CPW = 32 / LPE slots (8 centres for N_phi = 8).  The slot's lanes read one
 // neighbour's coefficients and dE/dA row as contiguous runs, and each lane
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
                                                      const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
-                                                     EdgeParams P) {
+                                                     const int *__restrict__ order, EdgeParams P) {
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -195,8 +202,9 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
-    if (lane >= Ln::USED || i >= n) return;
+    const int w_idx = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    if (lane >= Ln::USED || w_idx >= n) return;
+    const int i = order[w_idx];
     const int n0 = 2 * sub;
 
     float acc[2][NT];
@@ -204,6 +212,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     for (int m = 0; m < 2; ++m)
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = 0.f;
+    const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]}, ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
     const int q0 = row[i], q1 = q0 + act_cnt[i];
     int j_next = q0 < q1 ? act_col[q0] : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -216,7 +225,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             g_next = act_geo[q + 1];
         }
         const float r = g.w;
-        const float fc = cutoff_cos2(r * (0.5f * P.pi_over_rc));
+        const float fc = cutoff_cos2(fmaf(r, P.th_hi, r * P.th_lo));
         // first layer: c^0 by element (no lookup with a single element)
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
         float c[3][2];
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         const float Y[NT] = {1.f, g.x, g.y, g.z, g.x * g.x, g.y * g.y, g.z * g.z, g.x * g.y, g.x * g.z, g.y * g.z};
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            const float t = r - (float)(n0 + m) * P.mu_step;
+            const float t = (r - mh[m]) - ml[m];
             const float phi = expf(-P.alpha * t * t) * fc;
             const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
             acc[m][0] += a0;
@@ -265,7 +274,8 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                                                   const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
-                                                  float *__restrict__ dc, bool accumulate, EdgeParams P) {
+                                                  float *__restrict__ dc, bool accumulate,
+                                                  const int *__restrict__ order, EdgeParams P) {
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -273,8 +283,9 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
-    const bool live = lane < Ln::USED && i < n;
+    const int w_idx = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const bool live = lane < Ln::USED && w_idx < n;
+    const int i = live ? order[w_idx] : 0;
     const int n0 = 2 * sub;
 
     float fx = 0.f, fy = 0.f, fz = 0.f;
@@ -296,6 +307,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                 ck[l][1] = v.y;
             }
         }
+        const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]}, ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
         const int q0 = row[i], q1 = q0 + act_cnt[i];
         // the edge list is read once per launch: streaming loads (evict first)
         // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
@@ -313,9 +325,9 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             const float r = geo.w;
             const float inv_r = __fdividef(1.0f, r);
             float sn, cs;
-            __sincosf(r * P.pi_over_rc, &sn, &cs);   // argument in [0, pi)
+            __sincosf(2.f * fmaf(r, P.th_hi, r * P.th_lo), &sn, &cs);   // 2 theta in [0, pi)
             const float fc = 0.5f * (cs + 1.0f);
-            const float dfc = -0.5f * P.pi_over_rc * sn;
+            const float dfc = -fmaf(P.th_hi, sn, P.th_lo * sn);
             float gj[2 * NT], cj[3][2];
             {
                 const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)j * NA);
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             const float xy = d.x * d.y, xz = d.x * d.z, yz = d.y * d.z;
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
-                const float t = r - (float)(n0 + m) * P.mu_step;
+                const float t = (r - mh[m]) - ml[m];
                 const float g = __expf(-P.alpha * t * t);
                 const float phi = g * fc;
                 const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
@@ -442,7 +454,8 @@ __global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict
 // host wrappers
 
 cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
-    if (c->n == 0) return cudaSuccess;
+    const int64_t nc = centres(c);
+    if (nc == 0) return cudaSuccess;
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
@@ -452,19 +465,21 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     if (pair) {
         if (c->NP != 8) return cudaErrorInvalidValue;
         const int64_t threads = c->n * (8 * 9 / 2);
-        k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, nullptr,
-            P);
+        k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, nullptr,
+            c->d_order, P);
         k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>((int)c->n, A,
                                                                         c->d_rho + (int64_t)t * c->n * c->DR);
         return cudaGetLastError();
     }
     if (c->NP == 8)
-        k_density_fwd<8><<<(unsigned)((c->n + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
+        k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
+            c->d_order, P);
     else if (c->NP == 10)
-        k_density_fwd<10><<<(unsigned)((c->n + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
-            (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, P);
+        k_density_fwd<10><<<(unsigned)((nc + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
+            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
+            c->d_order, P);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
@@ -479,7 +494,7 @@ cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s
 #define REANN_EDGE_BWD(NPV, DC)                                                                                  \
     k_edge_bwd<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
         (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, c->d_G, c->d_F, \
-        c->d_dc, accumulate, P)
+        c->d_dc, accumulate, c->d_order, P)
     if (c->NP == 8) {
         if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
     } else if (c->NP == 10) {

@@ -10,6 +10,11 @@ struct BinParams {
     int m[3];
     int ncell;
     int ne;
+    // bin classes: the ne elements, and with a halo plan (multi-process
+    // decomposition) ne more for the ghost atoms, caller indices >= n_local;
+    // ghost rows list only the process's own atoms
+    int nclass;
+    int64_t n_local;
     double thr;  // (r_cut + skin)^2
 };
 
@@ -20,6 +25,7 @@ EdgeParams make_edge_params(const reann_ctx *c);
 cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s);
 cudaError_t launch_fill(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_skin_check(reann_ctx *c, int *flag, cudaStream_t s);
+cudaError_t launch_work_order(reann_ctx *c, cudaStream_t s);
 
 // edge kernels (edge.cu)
 cudaError_t launch_active(reann_ctx *c, cudaStream_t s);
@@ -41,10 +47,26 @@ cudaError_t dd_stale_coef(reann_ctx *c, float *coef, cudaStream_t s);
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
 cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
+// fp32-accurate networks on tcgen05 tensor cores, three tf32 passes (mlp_tc32.cu)
+bool tc32_supported(const reann_ctx *c);
+cudaError_t launch_mlp_tc32_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
+cudaError_t launch_mlp_tc32_energy(reann_ctx *c, cudaStream_t s);
+cudaError_t launch_mlp_tc32_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
 // tensor-core networks for the pair-product density form (mlp_tc_pair.cu)
 cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s);
 cudaError_t launch_mlp_tc_pair_energy(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_mlp_tc_pair_coef_bwd(reann_ctx *c, int t, cudaStream_t s);
+
+// a process's share of a multi-process decomposition (halo.cu): rows between
+// internal order and the exchange buffers
+cudaError_t launch_halo_pack_own(reann_ctx *c, const float *src, int width, cudaStream_t s);
+cudaError_t launch_halo_pack_ghosts(reann_ctx *c, const float *src, int width, cudaStream_t s);
+cudaError_t launch_halo_unpack_ghosts(reann_ctx *c, float *dst, int width, cudaStream_t s);
+cudaError_t launch_halo_add_partials(reann_ctx *c, float *dst, int width, cudaStream_t s);
+
+// atoms whose densities, networks and energies this context evaluates: all,
+// or a halo plan's own atoms (the ghosts follow them in internal order)
+inline int64_t centres(const reann_ctx *c) { return c->halo ? c->n_local : c->n; }
 
 // reductions, gathers and the integrator (md.cu)
 cudaError_t launch_pos_from_caller(reann_ctx *c, const float *d_pos_caller, cudaStream_t s);
@@ -60,8 +82,13 @@ cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cuda
 struct BussiParams {
     double c, kt, nf, r1, s;   // exp(-dt/tau), Kt (eV), Nf, the step's normal and chi-square numbers
 };
+// d_noise / d_loop (both or neither): the step's numbers come from the device
+// noise array at the device-side loop's current step instead of from B
 cudaError_t launch_thermostat(reann_ctx *c, const double *mass, const BussiParams &B, double *d_state,
-                              cudaStream_t s);
+                              cudaStream_t s, const double *d_noise = nullptr, const int *d_loop = nullptr);
+// the device-side step loop's gate (md.cu)
+cudaError_t launch_loop_gate(reann_ctx *c, cudaGraphConditionalHandle h_while, cudaGraphConditionalHandle h_step,
+                             cudaStream_t s);
 cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s);
 cudaError_t launch_wrap_state(reann_ctx *c, double *d_x_caller, float *d_pos_caller, cudaStream_t s);
 cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s);

@@ -72,10 +72,11 @@ __global__ void k_sum_partials(int np, const double *__restrict__ part, double *
 }
 
 cudaError_t launch_energy_sum(reann_ctx *c, cudaStream_t s) {
-    int np = (int)blocks(c->n, RED_THREADS);
+    const int64_t nc = centres(c);
+    int np = (int)blocks(nc, RED_THREADS);
     REANN_TIMED(c, REANN_K_ENERGY_SUM, s, 2);
-    if (c->n > 0) k_energy_partial<<<np, RED_THREADS, 0, s>>>(c->n, c->d_Ei, c->d_F, c->d_Epart, c->d_status);
-    k_sum_partials<<<1, RED_THREADS, 0, s>>>(c->n > 0 ? np : 0, c->d_Epart, c->d_E);
+    if (nc > 0) k_energy_partial<<<np, RED_THREADS, 0, s>>>(nc, c->d_Ei, c->d_F, c->d_Epart, c->d_status);
+    k_sum_partials<<<1, RED_THREADS, 0, s>>>(nc > 0 ? np : 0, c->d_Epart, c->d_E);
     return cudaGetLastError();
 }
 
@@ -93,10 +94,10 @@ __global__ void k_scatter_outputs(int64_t n, const int *__restrict__ perm, const
 }
 
 cudaError_t launch_scatter_outputs(reann_ctx *c, float *d_forces, float *d_atom_energy, cudaStream_t s) {
+    const int64_t nc = centres(c);   // own atoms sit at internal [0, nc) and caller [0, nc)
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
-    if (c->n > 0 && (d_forces || d_atom_energy))
-        k_scatter_outputs<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, c->d_F, c->d_Ei, d_forces,
-                                                            d_atom_energy);
+    if (nc > 0 && (d_forces || d_atom_energy))
+        k_scatter_outputs<<<blocks(nc, 256), 256, 0, s>>>(nc, c->d_perm, c->d_F, c->d_Ei, d_forces, d_atom_energy);
     return cudaGetLastError();
 }
 
@@ -309,11 +310,20 @@ cudaError_t launch_kinetic(reann_ctx *c, const double *mass, double *d_out, cuda
 // factor and adds K' - K to the work accumulator; the next kernel scales.
 // K' is a sum of squares in exact arithmetic; a rounding below zero is
 // clamped to it.
-__global__ void k_bussi_factor(int np, const double *__restrict__ part, BussiParams B, double *__restrict__ state) {
+// With `noise` given (the device-side step loop), the step's two numbers are
+// read at index loop[3] + loop[0] - 1: the first step of the launch plus the
+// steps the loop gate has admitted so far, minus the current one.
+__global__ void k_bussi_factor(int np, const double *__restrict__ part, BussiParams B, const double *__restrict__ noise,
+                               const int *__restrict__ loop, double *__restrict__ state) {
     double v = 0.0;
     for (int k = threadIdx.x; k < np; k += RED_THREADS) v += part[k];
     double K = block_sum(v);
     if (threadIdx.x == 0) {
+        if (noise) {
+            const int64_t step = (int64_t)loop[3] + loop[0] - 1;
+            B.r1 = noise[2 * step];
+            B.s = noise[2 * step + 1];
+        }
         double alpha = 1.0, Kn = K;
         if (K > 0.0) {
             Kn = K + (1.0 - B.c) * (B.kt * (B.r1 * B.r1 + B.s) / B.nf - K) +
@@ -332,14 +342,48 @@ __global__ void k_scale_velocities(int64_t m, double *__restrict__ v, const doub
 }
 
 cudaError_t launch_thermostat(reann_ctx *c, const double *mass, const BussiParams &B, double *d_state,
-                              cudaStream_t s) {
+                              cudaStream_t s, const double *d_noise, const int *d_loop) {
     MdParams M = md_params(c, 0.0, mass);
     int np = (int)blocks(c->n, RED_THREADS);
     if (c->n == 0) return cudaSuccess;
     REANN_TIMED(c, REANN_K_INTEGRATE, s, 3);
     k_kinetic_partial<<<np, RED_THREADS, 0, s>>>(c->n, c->d_v, c->d_pos, M, c->d_Epart);
-    k_bussi_factor<<<1, RED_THREADS, 0, s>>>(np, c->d_Epart, B, d_state);
+    k_bussi_factor<<<1, RED_THREADS, 0, s>>>(np, c->d_Epart, B, d_noise, d_loop, d_state);
     k_scale_velocities<<<blocks(3 * c->n, 256), 256, 0, s>>>(3 * c->n, c->d_v, d_state);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Device-side step loop.  After each kick-drift the gate decides on the GPU
+// whether the step may go on without the host: not when an earlier kernel
+// flagged an error (status[0]) or the skin check tripped (status[1]), which
+// need the host (error return, neighbour-list rebuild).  loop[0] counts the
+// steps admitted in this launch, loop[1] is the number requested, loop[2] the
+// reason the loop ended (1 rebuild, 2 error, 3 all steps done).  The gate sets
+// the IF handle that runs the step's energy+forces and closing kick, and the
+// WHILE handle that runs the next step.
+__global__ void k_loop_gate(const int *__restrict__ status, int *__restrict__ loop, cudaGraphConditionalHandle h_while,
+                            cudaGraphConditionalHandle h_step) {
+    if (threadIdx.x != 0) return;
+    const int err = status[0] & ~ST_SKIN, trip = status[1];
+    if (err || trip) {
+        loop[2] = err ? 2 : 1;
+        cudaGraphSetConditional(h_step, 0);
+        cudaGraphSetConditional(h_while, 0);
+        return;
+    }
+    const int d = loop[0] + 1;
+    loop[0] = d;
+    cudaGraphSetConditional(h_step, 1);
+    const bool more = d < loop[1];
+    if (!more) loop[2] = 3;
+    cudaGraphSetConditional(h_while, more ? 1u : 0u);
+}
+
+cudaError_t launch_loop_gate(reann_ctx *c, cudaGraphConditionalHandle h_while, cudaGraphConditionalHandle h_step,
+                             cudaStream_t s) {
+    REANN_TIMED(c, REANN_K_INTEGRATE, s, 1);
+    k_loop_gate<<<1, 32, 0, s>>>(c->d_status, c->d_loop, h_while, h_step);
     return cudaGetLastError();
 }
 

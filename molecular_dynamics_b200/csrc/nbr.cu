@@ -10,6 +10,11 @@
 // Internal atom order is (element, cell, caller index).  Each element's atoms
 // form one contiguous segment (the atomic networks run on contiguous rows),
 // and inside a segment atoms are in cell order (neighbour gathers stay local).
+// With a halo plan (a process's share of a spatial decomposition) the ghost
+// atoms copied from other processes follow all own atoms, in segments of
+// their own, and their rows list own atoms only: the edges a process must
+// differentiate for the partial gradients it returns to the ghosts' owners
+// (section "Parallelization Algorithm", Fig. 4).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -134,7 +139,8 @@ __global__ void k_bin_count(int64_t n, const float *__restrict__ pos, const int 
     int cx = cell_axis(x, B.box[0], B.m[0]);
     int cy = cell_axis(y, B.box[1], B.m[1]);
     int cz = cell_axis(z, B.box[2], B.m[2]);
-    int k = e * B.ncell + (cx * B.m[1] + cy) * B.m[2] + cz;
+    const int cls = a >= B.n_local ? B.ne + e : e;   // ghosts after every own atom
+    int k = cls * B.ncell + (cx * B.m[1] + cy) * B.m[2] + cz;
     key[a] = k;
     atomicAdd(&bin_count[k], 1);
 }
@@ -218,7 +224,9 @@ __global__ void __launch_bounds__(128) k_nbr(int n, const float4 *__restrict__ p
     int nz = axis_stencil(cell_axis(pi.z, B.box[2], B.m[2]), B.m[2], sz);
     int c = 0;
     int o = FILL ? row[i] : 0;
-    for (int e = 0; e < B.ne; ++e) {
+    // own atoms come first in internal order; a ghost's row lists own atoms only
+    const int ncls = i >= B.n_local ? B.ne : B.nclass;
+    for (int e = 0; e < ncls; ++e) {
         for (int a = 0; a < nx; ++a)
             for (int b = 0; b < ny; ++b)
                 for (int d = 0; d < nz; ++d) {
@@ -245,6 +253,33 @@ __global__ void k_row_max(int n, const int *__restrict__ cnt, int64_t *__restric
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
     if ((threadIdx.x & 31) == 0 && v > 0) atomicMax((unsigned long long *)out, (unsigned long long)v);
+}
+
+// Centre order of the edge passes.  A warp of an edge pass walks the rows of
+// several centres side by side, so one long row keeps the others' lanes idle;
+// in systems with uneven neighbour counts (a gas of molecules) that idles a
+// quarter of the lanes.  Each window of ORDER_WINDOW consecutive atoms (one
+// neighbourhood, so the gathers stay local) is ordered by row length, then
+// index: the centres a warp takes together have similar lengths.  Windows do
+// not cross `split` (a halo plan's first ghost), so own atoms stay first.
+constexpr int ORDER_WINDOW = 256;
+
+__global__ void k_window_order(int n, int split, const int *__restrict__ cnt, int *__restrict__ order) {
+    const int w = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    const int nw_own = (split + ORDER_WINDOW - 1) / ORDER_WINDOW;
+    const int s0 = w < nw_own ? w * ORDER_WINDOW : split + (w - nw_own) * ORDER_WINDOW;
+    if (s0 >= (w < nw_own ? split : n)) return;
+    const int s1 = min(s0 + ORDER_WINDOW, w < nw_own ? split : n);
+    for (int p = s0 + lane; p < s1; p += 32) {
+        const int len = cnt[p];
+        int rank = 0;
+        for (int q = s0; q < s1; ++q) {
+            const int lq = cnt[q];
+            rank += lq < len || (lq == len && q < p);
+        }
+        order[s0 + rank] = p;
+    }
 }
 
 // Sets ST_SKIN when any atom has moved more than skin/2 (minimum image) since
@@ -304,6 +339,14 @@ cudaError_t launch_fill(reann_ctx *c, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+cudaError_t launch_work_order(reann_ctx *c, cudaStream_t s) {
+    const int n = (int)c->n, split = (int)(c->halo ? c->n_local : c->n);
+    const int64_t windows = (split + ORDER_WINDOW - 1) / ORDER_WINDOW + (n - split + ORDER_WINDOW - 1) / ORDER_WINDOW;
+    REANN_TIMED(c, REANN_K_NEIGHBORS, s);
+    if (windows > 0) k_window_order<<<blocks(windows * 32, 256), 256, 0, s>>>(n, split, c->d_cnt, c->d_order);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_skin_check(reann_ctx *c, int *flag, cudaStream_t s) {
     BinParams B = make_bin_params(c);
     double h = 0.5 * c->cfg.skin;
@@ -321,6 +364,8 @@ BinParams make_bin_params(const reann_ctx *c) {
     }
     B.ncell = c->ncell;
     B.ne = c->ne;
+    B.nclass = c->halo ? 2 * c->ne : c->ne;
+    B.n_local = c->halo ? c->n_local : c->n;
     double rl = c->cfg.r_cut + c->cfg.skin;
     B.thr = rl * rl;
     return B;

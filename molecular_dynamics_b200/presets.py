@@ -40,7 +40,7 @@ class Preset:
     alpha: float = 1.0          # Gaussian width, A^-2
     skin: float = 1.0           # Verlet skin, A
     hidden: Tuple[int, int] = (64, 64)
-    mlp_precision: int = 0      # 0 = fp32, 1 = bf16 GEMMs with fp32 accumulate
+    mlp_precision: int = 0      # 0 = fp32 accuracy (3xTF32 tensor cores for [64,64]), 1 = bf16 GEMMs, 2 = fp32 CUDA cores
     # structure recipe
     kind: str = "fcc"           # fcc | water | chon
     ncell: int = 0              # fcc: conventional cells per axis

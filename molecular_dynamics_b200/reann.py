@@ -24,7 +24,12 @@ STATUS = {
 
 EXPORTS = ("reann_create", "reann_destroy", "reann_build_neighbors", "reann_energy_forces", "reann_md_step",
            "reann_md_step_nvt", "reann_get_counters", "reann_last_error", "reann_get_neighbors", "reann_get_features", "reann_profile",
-           "reann_profile_read", "reann_pair_list_noalloc")
+           "reann_profile_read", "reann_pair_list_noalloc", "reann_halo_plan", "reann_energy_forces_halo")
+
+# kinds of the exchange function (include/reann.h)
+EXCHANGE_COEF, EXCHANGE_COEF_GRAD, EXCHANGE_FORCE = 0, 1, 2
+ExchangeFn = C.CFUNCTYPE(C.c_int32, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_int64, C.c_void_p, C.c_int64,
+                         C.c_int32, C.c_void_p)
 
 KERNEL_GROUPS = ("active", "density", "mlp_fwd", "mlp_energy", "edge_bwd", "mlp_bwd", "energy_sum", "integrate",
                  "neighbors", "other", "ghost")
@@ -81,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.reann_profile.argtypes = [P, I32]
     lib.reann_pair_list_noalloc.argtypes = [I64, P, C.POINTER(D), D, D, P, P, I64, C.POINTER(I64), P]
     lib.reann_profile_read.argtypes = [P, I32, C.POINTER(D), C.POINTER(I64)]
+    lib.reann_halo_plan.argtypes = [P, I64, I64, P, I64]
+    lib.reann_energy_forces_halo.argtypes = [P, P, C.POINTER(D), P, P, ExchangeFn, P, P]
     for name in EXPORTS:
         if name != "reann_last_error":
             getattr(lib, name).restype = C.c_int
@@ -170,6 +177,14 @@ class ModelSpec:
         return c
 
 
+class _DeviceRows:
+    """A float32 [rows][width] device array at a raw address, for torch.as_tensor."""
+
+    def __init__(self, ptr: int, rows: int, width: int):
+        self.__cuda_array_interface__ = {"shape": (int(rows), int(width)), "typestr": "<f4",
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
 class Context:
     """One reann_ctx.  Methods mirror the C entry points."""
 
@@ -216,6 +231,43 @@ class Context:
         e = C.c_double(0.0)
         self._check(self.lib.reann_energy_forces(self.h, _ptr(pos), C.byref(e), _ptr(forces), _ptr(atom_energy),
                                                  _stream(stream)))
+        return e.value
+
+    def reann_halo_plan(self, n_local: int, n_ghost: int, send_index):
+        """send_index: own atoms (caller indices < n_local) in send order, host int array."""
+        idx = np.ascontiguousarray(np.asarray(send_index, np.int32).reshape(-1))
+        self._check(self.lib.reann_halo_plan(self.h, int(n_local), int(n_ghost), idx.ctypes.data if len(idx) else None,
+                                             len(idx)))
+
+    def reann_energy_forces_halo(self, pos, exchange, forces=None, atom_energy=None, stream=None) -> float:
+        """exchange(kind, layer, send, recv, stream): send and recv are torch
+        CUDA tensors [rows][width] viewing the library's exchange buffers; it
+        must fill recv (in stream order) and return nothing.  Exceptions abort
+        the evaluation."""
+        import torch
+
+        errors = []
+
+        def view(ptr, rows, width):
+            if rows == 0:
+                return torch.empty((0, width), dtype=torch.float32, device="cuda")
+            return torch.as_tensor(_DeviceRows(ptr, rows, width), device="cuda")
+
+        def cb(user, kind, layer, send, send_rows, recv, recv_rows, width, strm):
+            try:
+                exchange(kind, layer, view(send, send_rows, width), view(recv, recv_rows, width), strm)
+                return 0
+            except Exception as exc:   # reported after the library returns
+                errors.append(exc)
+                return 1
+
+        fn = ExchangeFn(cb)
+        e = C.c_double(0.0)
+        st = self.lib.reann_energy_forces_halo(self.h, _ptr(pos), C.byref(e), _ptr(forces), _ptr(atom_energy), fn,
+                                               None, _stream(stream))
+        if errors:
+            raise errors[0]
+        self._check(st)
         return e.value
 
     def reann_md_step(self, nsteps: int, dt_fs: float, x, v, masses, stream=None) -> MdStats:

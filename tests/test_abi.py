@@ -53,7 +53,7 @@ def test_create_rejects_unsupported_and_invalid_configs(lib):
     p = presets.get("ag256")
     w = synth.weight_blob(p)
     for field, value, expect in (("n_radial", 7, 9), ("l_max", 1, 9), ("T", 0, 1), ("n_elements", 0, 1),
-                                 ("mlp_precision", 3, 1)):
+                                 ("mlp_precision", 3, 1), ("mlp_precision", -1, 1)):
         cfg = reann.ModelSpec.from_preset(p).config()
         setattr(cfg, field, value)
         h = C.c_void_p()

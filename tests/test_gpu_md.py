@@ -150,22 +150,55 @@ def test_energy_error_is_second_order_on_gpu():
 
 
 def test_graph_replay_matches_eager_launches(monkeypatch):
-    # reann_md_step replays each step's evaluation as a CUDA graph; with
-    # REANN_GRAPHS=0 at context creation it launches eagerly.  Same trajectory
-    # bit for bit, same kernel-launch count.
+    # reann_md_step runs all steps but the last of a call as a device-side
+    # loop (one graph launch per stretch between neighbour rebuilds); with
+    # REANN_LOOP=0 it replays one graph per step, with REANN_GRAPHS=0 it
+    # launches eagerly.  Same trajectory bit for bit in all three; the loop
+    # adds its gate kernel once per looped step.
     torch = torch_cuda()
     p, pos, types, box = small("water")
     v0 = synth.maxwell_boltzmann(p, types)
     out = []
-    for graphs in ("1", "0"):
+    nsteps = 30
+    for graphs, loop in (("1", "1"), ("1", "0"), ("0", "1")):
         monkeypatch.setenv("REANN_GRAPHS", graphs)
+        monkeypatch.setenv("REANN_LOOP", loop)
         ctx = _ctx(p, pos, types, box)
         x = torch.from_numpy(pos.astype(np.float64)).cuda()
         v = torch.from_numpy(v0.copy()).cuda()
         k0 = ctx.reann_get_counters().kernel_launches
-        st = ctx.reann_md_step(30, p.dt_fs, x, v, p.masses)
+        st = ctx.reann_md_step(nsteps, p.dt_fs, x, v, p.masses)
         out.append((x.cpu().numpy(), v.cpu().numpy(), st.e_pot, ctx.reann_get_counters().kernel_launches - k0,
-                    st.rebuilds))
-    assert np.array_equal(out[0][0], out[1][0]) and np.array_equal(out[0][1], out[1][1])
-    assert out[0][2] == out[1][2]
-    assert out[0][3] == out[1][3] and out[0][4] == out[1][4]
+                    st.rebuilds, st.steps))
+    for o in out[1:]:
+        assert np.array_equal(out[0][0], o[0]) and np.array_equal(out[0][1], o[1])
+        assert out[0][2] == o[2] and out[0][4] == o[4] and o[5] == nsteps
+    assert out[1][3] == out[2][3]
+    assert out[0][3] == out[1][3] + (nsteps - 1)
+
+
+@pytest.mark.parametrize("ensemble", ["nve", "nvt"])
+def test_device_loop_across_rebuilds(monkeypatch, ensemble):
+    # a hot water sample rebuilds its list several times within one call: the
+    # device-side loop hands each rebuild to the host and resumes; trajectory,
+    # energies, thermostat work and rebuild count equal the per-step graphs'
+    torch = torch_cuda()
+    p, pos, types, box = small("water")
+    v0 = synth.maxwell_boltzmann(p, types, temperature=900.0)
+    nsteps = 150
+    noise = synth.thermostat_noise(len(pos), nsteps, seed=77)
+    out = []
+    for loop in ("1", "0"):
+        monkeypatch.setenv("REANN_LOOP", loop)
+        ctx = _ctx(p, pos, types, box)
+        x = torch.from_numpy(pos.astype(np.float64)).cuda()
+        v = torch.from_numpy(v0.copy()).cuda()
+        if ensemble == "nve":
+            st = ctx.reann_md_step(nsteps, p.dt_fs, x, v, p.masses)
+        else:
+            st = ctx.reann_md_step_nvt(nsteps, p.dt_fs, 300.0, 20.0, noise, x, v, p.masses)
+        out.append((x.cpu().numpy(), v.cpu().numpy(), st))
+    (x1, v1, s1), (x2, v2, s2) = out
+    assert s1.rebuilds >= 2 and s1.rebuilds == s2.rebuilds
+    assert np.array_equal(x1, x2) and np.array_equal(v1, v2)
+    assert s1.e_pot == s2.e_pot and s1.e_kin == s2.e_kin and s1.e_thermostat == s2.e_thermostat

@@ -49,6 +49,34 @@ def test_energy_forces_match_oracle(case):
     assert abs(Ei.sum() - E) <= 1e-4 * max(1.0, abs(E))
 
 
+@pytest.mark.parametrize("case", ["water300", "hea1372", "chon976"])
+def test_cuda_core_fp32_networks_match_oracle(case):
+    # mlp_precision 2: the fp32 networks on the CUDA cores (the reference the
+    # three-pass tf32 tensor-core networks of mlp_precision 0 are measured
+    # against) meet the same tolerances
+    p, pos, types, box = CASES[case]()
+    _, E, F, Ei = gpu_eval(p, pos, types, box, mlp_precision=2)
+    ref = oracle_eval(p, pos, types, box)
+    assert_energy_close(E, ref.energy, len(pos))
+    assert_atom_energies_close(Ei, ref.atom_energy)
+    assert_forces_close(F, ref.forces)
+
+
+@pytest.mark.parametrize("case", ["hea1372", "chon976"])
+def test_tf32_and_cuda_core_networks_agree(case):
+    # both fp32-accurate network paths on the same inputs: per-atom energies
+    # and forces agree at the fp32 level, and the tensor-core path is
+    # deterministic (fixed MMA order)
+    p, pos, types, box = CASES[case]()
+    _, E0, F0, Ei0 = gpu_eval(p, pos, types, box, mlp_precision=0)
+    _, E0b, F0b, _ = gpu_eval(p, pos, types, box, mlp_precision=0)
+    _, E2, F2, Ei2 = gpu_eval(p, pos, types, box, mlp_precision=2)
+    assert E0 == E0b and np.array_equal(F0, F0b)
+    scale = max(float(np.sqrt(np.mean(Ei2 ** 2))), 1e-2)
+    assert np.abs(Ei0 - Ei2).max() <= 2e-5 * scale
+    assert np.abs(F0 - F2).max() <= 5e-5
+
+
 @pytest.mark.parametrize("case", ["ag500", "water300", "hea1372", "chon976"])
 def test_every_layer_matches_oracle(case):
     # rho^t in the units the networks see, (rho - shift) / scale.  This is a

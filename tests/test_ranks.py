@@ -107,14 +107,19 @@ def test_roofline_arithmetic():
     json.dumps(roof)
     # dominant fp32 networks: 2 (108*128 + 128*128 + 128*24) flop per forward, doubled for the VJP launch
     r2 = bench.roofline({"mlp_bwd": (8.0, 2), "edge_bwd": (1.0, 3)}, pairs, 8, 3, 1000, 148, {"sm_max_mhz": 2000.0},
-                        "measured", {}, net=(108, 24, (128, 128), 0))
+                        "measured", {}, net=(108, 24, (128, 128), "simt"))
     assert r2["bound"] == "alu"
     assert r2["flop_per_launch"] == 1000 * 2 * 2 * (108 * 128 + 128 * 128 + 128 * 24)
     assert r2["achieved"] == pytest.approx(r2["flop_per_launch"] / 4e-3 / 1e12)
     # bf16 tensor-core networks: against the sustained bf16 peak
     r3 = bench.roofline({"mlp_fwd": (8.0, 2)}, pairs, 8, 3, 1000, 148, {"bf16_tflops_sustained": 1382.5}, "measured",
-                        {}, net=(24, 24, (128, 128), 1))
+                        {}, net=(24, 24, (128, 128), "bf16"))
     assert r3["bound"] == "tensor" and r3["peak"] == 1382.5
+    # three-pass tf32 networks: against the tf32 peak (bf16 x the nominal 1.1 / 2.25), algorithmic flops
+    r4 = bench.roofline({"mlp_fwd": (8.0, 2)}, pairs, 8, 3, 1000, 148, {"bf16_tflops_sustained": 1382.5}, "measured",
+                        {}, net=(24, 24, (64, 64), "tf32x3"))
+    assert r4["bound"] == "tensor" and r4["peak"] == pytest.approx(1382.5 * 1.1 / 2.25)
+    assert r4["flop_per_launch"] == 1000 * 2 * (24 * 64 + 64 * 64 + 64 * 24)
 
 
 def test_per_kernel_roofline_arithmetic():
@@ -129,7 +134,7 @@ def test_per_kernel_roofline_arithmetic():
     assert a["frac"] == pytest.approx(a["achieved"] / 6500.0)
     d = bench.kernel_roofline("density", prof, pairs, 8, 3, n, 148, pk, "measured", {})
     assert d["achieved"] == pytest.approx(pairs * bench.FLOP_DENSITY_PER_PAIR[8] / 2e-3 / 1e12)
-    m = bench.kernel_roofline("mlp_fwd", prof, pairs, 8, 3, n, 148, pk, "measured", {}, net=(24, 24, (128, 128), 1))
+    m = bench.kernel_roofline("mlp_fwd", prof, pairs, 8, 3, n, 148, pk, "measured", {}, net=(24, 24, (128, 128), "bf16"))
     assert m["bound"] == "tensor" and m["peak"] == 1400.0
     assert m["achieved"] == pytest.approx(n * bench.network_flop_per_atom("mlp_fwd", 24, 24, (128, 128)) / 0.5e-3 / 1e12)
     # groups without an algorithmic count, or absent, have no entry
