@@ -111,7 +111,7 @@ void free_atoms(reann_ctx *c) {
     dfree(c->d_A); dfree(c->d_rho); dfree(c->d_coef); dfree(c->d_G); dfree(c->d_dc); dfree(c->d_Ei);
     dfree(c->d_F); dfree(c->d_Epart); dfree(c->d_stage_f); dfree(c->d_stage_i); dfree(c->d_stage_x);
     dfree(c->d_stage_v); dfree(c->d_stage_e); dfree(c->d_x); dfree(c->d_v); dfree(c->d_diag);
-    dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub); dfree(c->d_tanhd); dfree(c->d_order);
+    dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub); dfree(c->d_tanhd);
     c->md_valid = false;
     c->slots_alloc = 0;
     c->n_alloc = 0;
@@ -131,7 +131,6 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_row, N + 1));
     CK(dalloc(&c->d_cnt, N));
     CK(dalloc(&c->d_act_cnt, N));
-    CK(dalloc(&c->d_order, N));
     CK(dalloc(&c->d_A, (size_t)c->T * N * c->NA));
     CK(dalloc(&c->d_rho, (size_t)c->T * N * c->DR));
     CK(dalloc(&c->d_coef, (size_t)c->T * N * c->D));
@@ -203,6 +202,7 @@ reann_status ensure_capacity(reann_ctx *c, int64_t nnz) {
     CK(dalloc(&c->d_col, (size_t)cap));
     CK(dalloc(&c->d_act_col, (size_t)cap));
     CK(dalloc(&c->d_act_geo, (size_t)cap));
+    if (c->cfg.mlp_precision != 1) CK(dalloc(&c->d_act_dr, (size_t)cap));
     c->cap = cap;
     return REANN_OK;
 }
@@ -241,7 +241,6 @@ reann_status build_internal(reann_ctx *c, const float *d_pos_caller, const int *
     if (nnz > INT32_MAX) return fail(c, REANN_ERR_CAPACITY, "neighbour list exceeds 2^31-1 entries");
     if ((st = ensure_capacity(c, nnz))) return st;
     CK(launch_fill(c, s));
-    CK(launch_work_order(c, s));
     c->nnz = nnz;
     c->max_row = c->h_i64[2];
     // tile tables of the atomic networks: element segments cut into 32-row
@@ -627,11 +626,24 @@ extern "C" reann_status reann_create(const reann_config *cfg, const void *weight
     for (int e = 0; e < c->ne; ++e) c->energy_nets.push_back(bind_net(c, off, 1));
     c->n_w = expect;
     c->h_C0.assign((const float *)weights, (const float *)weights + (size_t)c->ne * c->D);
+    // shifts out of the blob (see reann_ctx::d_shift)
+    std::vector<float> blob((const float *)weights, (const float *)weights + expect);
+    c->h_shift.assign((size_t)c->T * c->ne * c->DR, 0.f);
+    for (int t = 0; t < c->T; ++t)
+        for (int e = 0; e < c->ne; ++e) {
+            const NetOffsets &o = t + 1 < c->T ? c->coef_nets[t * c->ne + e] : c->energy_nets[e];
+            for (int f = 0; f < c->DR; ++f) {
+                c->h_shift[((size_t)t * c->ne + e) * c->DR + f] = blob[o.shift + f];
+                blob[o.shift + f] = 0.f;
+            }
+        }
     cudaError_t e;
     cudaDeviceProp prop;
     if ((e = cudaGetDeviceProperties(&prop, device)) ||
         (e = cudaMalloc(&c->d_w, nbytes)) ||
-        (e = cudaMemcpy(c->d_w, weights, nbytes, cudaMemcpyHostToDevice)) ||
+        (e = cudaMemcpy(c->d_w, blob.data(), nbytes, cudaMemcpyHostToDevice)) ||
+        (e = cudaMalloc(&c->d_shift, sizeof(float) * c->h_shift.size())) ||
+        (e = cudaMemcpy(c->d_shift, c->h_shift.data(), sizeof(float) * c->h_shift.size(), cudaMemcpyHostToDevice)) ||
         (e = cudaMalloc(&c->d_status, sizeof(int) * 4)) ||
         (e = cudaMemset(c->d_status, 0, sizeof(int) * 4)) ||
         (e = cudaMalloc(&c->d_i64, sizeof(int64_t) * 8)) ||
@@ -655,9 +667,9 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     if (!c) return REANN_OK;
     DeviceGuard guard(c->device);
     free_atoms(c);
-    dfree(c->d_w); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
+    dfree(c->d_w); dfree(c->d_shift); dfree(c->d_bin_count); dfree(c->d_bin_start); dfree(c->d_bin_fill); dfree(c->d_col);
     dfree(c->d_dd_bits); dfree(c->d_dd_prefix); dfree(c->d_dd_cnt); dfree(c->d_dd_owner); dfree(c->d_col_dd);
-    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
+    dfree(c->d_act_col); dfree(c->d_act_geo); dfree(c->d_act_dr); dfree(c->d_tiles); dfree(c->d_tiles128); dfree(c->d_status); dfree(c->d_i64); dfree(c->d_E);
     if (c->d_scan_tmp) cudaFree(c->d_scan_tmp);
     if (c->h_status) cudaFreeHost(c->h_status);
     if (c->h_i64) cudaFreeHost(c->h_i64);
@@ -1198,9 +1210,17 @@ extern "C" reann_status reann_get_features(reann_ctx *c, int32_t t, float *rho, 
     const int64_t n = c->n, nD = n * c->D, nR = n * c->DR;
     if (n == 0) return REANN_OK;
     if (rho) {
+        // stored as rho - shift of the atom's element: the shift is added back here
         CK(launch_to_caller_rows(c, c->d_rho + t * nR, c->DR, c->d_diag, s));
-        CK(cudaMemcpyAsync(rho, c->d_diag, sizeof(float) * nR, cudaMemcpyDefault, s));
+        std::vector<float> h((size_t)nR);
+        std::vector<int> types(n);
+        CK(cudaMemcpyAsync(h.data(), c->d_diag, sizeof(float) * nR, cudaMemcpyDeviceToHost, s));
+        CK(cudaMemcpyAsync(types.data(), c->d_types_caller, sizeof(int) * n, cudaMemcpyDeviceToHost, s));
         CK(sync_stream(c, s));
+        for (int64_t a = 0; a < n; ++a)
+            for (int f = 0; f < c->DR; ++f)
+                h[a * c->DR + f] += c->h_shift[((size_t)t * c->ne + types[a]) * c->DR + f];
+        CK(cudaMemcpy(rho, h.data(), sizeof(float) * nR, cudaMemcpyDefault));
     }
     if (coef) {
         if (t == 0) {

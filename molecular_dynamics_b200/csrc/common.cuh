@@ -80,8 +80,13 @@ struct reann_ctx {
     int NP = 0, D = 0, NA = 0, T = 0, ne = 0, H1 = 0, H2 = 0;
     int DR = 0;   // density features per atom (network input width): D, or N_phi (N_phi+1)(L+1)/2 in the pair form
 
-    // weights
+    // weights.  The networks' input shifts live apart from the blob: the
+    // density kernels subtract them in fp64 before rounding to fp32 (d_rho
+    // holds rho - shift), so a feature close to its shift keeps its relative
+    // precision; the device blob's shift entries are zero.
     float *d_w = nullptr;
+    float *d_shift = nullptr;          // [T][ne][DR]: layer t feeds M^t (t < T-1) or the energy network
+    std::vector<float> h_shift;
     int64_t n_w = 0;
     std::vector<reann::NetOffsets> coef_nets;  // [(T-1) * ne]
     std::vector<reann::NetOffsets> energy_nets;  // [ne]
@@ -113,11 +118,10 @@ struct reann_ctx {
     int *d_cnt = nullptr;          // [n]
     int *d_col = nullptr;          // [cap]
     int *d_act_cnt = nullptr;      // [n]
-    int *d_order = nullptr;        // [n] centre order of the edge passes: windows of consecutive atoms
-                                   // sorted by row length, so the centres a warp walks together have
-                                   // similar neighbour counts
     int *d_act_col = nullptr;      // [cap]
     float4 *d_act_geo = nullptr;   // [cap] displacement and distance of each active entry
+    float *d_act_dr = nullptr;     // [cap] fp32-accurate paths: r - fp32(r) of each active entry, from the
+                                   // exact displacement (the densities are stiff in r: Gaussian slopes 2 alpha t)
     int64_t nnz = 0, cap = 0, max_row = 0;
     void *d_scan_tmp = nullptr;
     size_t scan_tmp_size = 0;

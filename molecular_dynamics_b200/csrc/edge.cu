@@ -88,7 +88,8 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
-                                                EdgeParams P, unsigned long long *__restrict__ total) {
+                                                float *__restrict__ act_dr, EdgeParams P,
+                                                unsigned long long *__restrict__ total) {
     // one warp per row: lanes test consecutive entries, a ballot compacts the
     // active ones in row order and the writes stay contiguous.  Warps stride
     // over the rows (the next row's position and bounds are loaded while the
@@ -129,7 +130,19 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
                 if (act) {
                     const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
                     act_col[o] = j[b];
-                    act_geo[o] = make_float4(d.x, d.y, d.z, sqrtf(r2));
+                    float r = sqrtf(r2);
+                    if (act_dr) {
+                        // the fp32-accurate paths: r from the exact displacement of the
+                        // fp32 positions, correctly rounded, and its rounding residual
+                        double e[3] = {(double)pj[b].x - (double)pi.x, (double)pj[b].y - (double)pi.y,
+                                       (double)pj[b].z - (double)pi.z};
+#pragma unroll
+                        for (int a = 0; a < 3; ++a) e[a] -= P.box[a] * rint(e[a] * P.inv_box[a]);
+                        const double r64 = sqrt(e[0] * e[0] + e[1] * e[1] + e[2] * e[2]);
+                        r = (float)r64;
+                        act_dr[o] = (float)(r64 - (double)r);
+                    }
+                    act_geo[o] = make_float4(d.x, d.y, d.z, r);
                 }
                 k += __popc(mask);
             }
@@ -150,15 +163,14 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     const unsigned grid = (unsigned)std::min<int64_t>((c->n + 3) / 4, (int64_t)c->sm_count * 8);
     k_active<<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row,
                                                         c->dd ? c->d_col_dd : c->d_col, c->d_act_cnt,
-                                                            c->d_act_col, c->d_act_geo, P,
+                                                            c->d_act_col, c->d_act_geo, c->d_act_dr, P,
                                                             (unsigned long long *)(c->d_i64 + 3));
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
 // Lane decomposition shared by both edge passes: a slot of LPE = N_phi / 2
-// lanes owns one centre atom (taken in the build's work order, which groups
-// centres of similar row length) and walks its active neighbours in row order;
+// lanes owns one centre atom and walks its active neighbours in row order;
 // lane `sub` owns radial indices 2 sub and 2 sub + 1.  A warp holds
 // CPW = 32 / LPE slots (8 centres for N_phi = 8).  The slot's lanes read one
 // neighbour's coefficients and dE/dA row as contiguous runs, and each lane
@@ -194,7 +206,8 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
                                                      const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
-                                                     const int *__restrict__ order, EdgeParams P) {
+                                                     const float *__restrict__ shift, const float *__restrict__ act_dr,
+                                                     EdgeParams P) {
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -202,9 +215,8 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int w_idx = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
-    if (lane >= Ln::USED || w_idx >= n) return;
-    const int i = order[w_idx];
+    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    if (lane >= Ln::USED || i >= n) return;
     const int n0 = 2 * sub;
 
     float acc[2][NT];
@@ -216,13 +228,16 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     const int q0 = row[i], q1 = q0 + act_cnt[i];
     int j_next = q0 < q1 ? act_col[q0] : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float dr_next = (act_dr && q0 < q1) ? act_dr[q0] : 0.f;
     for (int q = q0; q < q1; ++q) {
         // the next edge's index and geometry are in flight while this one computes
         const int j = j_next;
         const float4 g = g_next;         // dx, dy, dz, r
+        const float dr = dr_next;        // r - fp32(r) (fp32-accurate paths), else 0
         if (q + 1 < q1) {
             j_next = act_col[q + 1];
             g_next = act_geo[q + 1];
+            if (act_dr) dr_next = act_dr[q + 1];
         }
         const float r = g.w;
         const float fc = cutoff_cos2(fmaf(r, P.th_hi, r * P.th_lo));
@@ -238,7 +253,9 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
         const float Y[NT] = {1.f, g.x, g.y, g.z, g.x * g.x, g.y * g.y, g.z * g.z, g.x * g.y, g.x * g.z, g.y * g.z};
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            const float t = (r - mh[m]) - ml[m];
+            // the Gaussians' slope 2 alpha t makes them the part of the density most
+            // sensitive to r: t carries r's rounding residual
+            const float t = ((r - mh[m]) - ml[m]) + dr;
             const float phi = expf(-P.alpha * t * t) * fc;
             const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
             acc[m][0] += a0;
@@ -256,10 +273,17 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(v[u], v[u + 1]);
         if (!rho_out) continue;   // pair form: rho from A in k_rho_pair
+        // rho - shift in fp64 (the networks see (rho - shift) / scale, which the
+        // fp32 rounding of rho itself would blur when rho is close to its shift)
         float *ro = rho_out + (int64_t)i * D;
-        ro[nn] = v[0] * v[0];
-        ro[NP + nn] = v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
-        ro[2 * NP + nn] = v[4] * v[4] + v[5] * v[5] + v[6] * v[6] + 2.f * (v[7] * v[7] + v[8] * v[8] + v[9] * v[9]);
+        const float *sh = shift + (ne > 1 ? __float_as_int(pos[i].w) : 0) * D;
+        double x[NT];
+#pragma unroll
+        for (int u = 0; u < NT; ++u) x[u] = (double)v[u];
+        ro[nn] = (float)(x[0] * x[0] - (double)sh[nn]);
+        ro[NP + nn] = (float)(x[1] * x[1] + x[2] * x[2] + x[3] * x[3] - (double)sh[NP + nn]);
+        ro[2 * NP + nn] = (float)(x[4] * x[4] + x[5] * x[5] + x[6] * x[6] + 2.0 * (x[7] * x[7] + x[8] * x[8] + x[9] * x[9]) -
+                                  (double)sh[2 * NP + nn]);
     }
 }
 
@@ -274,8 +298,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                                                   const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
-                                                  float *__restrict__ dc, bool accumulate,
-                                                  const int *__restrict__ order, EdgeParams P) {
+                                                  float *__restrict__ dc, bool accumulate, EdgeParams P) {
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -283,9 +306,8 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int w_idx = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
-    const bool live = lane < Ln::USED && w_idx < n;
-    const int i = live ? order[w_idx] : 0;
+    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const bool live = lane < Ln::USED && i < n;
     const int n0 = 2 * sub;
 
     float fx = 0.f, fy = 0.f, fz = 0.f;
@@ -431,7 +453,9 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
 // density dimension N_phi (N_phi+1)(L+1)/2 of section "REANN Architecture".
 // One thread per (atom, pair); the atom's A row is read from L1.
 template <int NP>
-__global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict__ A, float *__restrict__ rho) {
+__global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict__ A, float *__restrict__ rho,
+                                                  const float4 *__restrict__ pos, const float *__restrict__ shift,
+                                                  int ne) {
     constexpr int P = NP * (NP + 1) / 2, NA = NP * NT, DR = 3 * P;
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= (int64_t)n * P) return;
@@ -445,9 +469,14 @@ __global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict
     const int b = a + (p - first);
     const float *x = A + i * NA + a * NT, *y = A + i * NA + b * NT;
     float *ro = rho + i * DR;
-    ro[p] = x[0] * y[0];
-    ro[P + p] = x[1] * y[1] + x[2] * y[2] + x[3] * y[3];
-    ro[2 * P + p] = x[4] * y[4] + x[5] * y[5] + x[6] * y[6] + 2.f * (x[7] * y[7] + x[8] * y[8] + x[9] * y[9]);
+    const float *sh = shift + (ne > 1 ? __float_as_int(pos[i].w) : 0) * DR;
+    double q[NT];
+#pragma unroll
+    for (int u = 0; u < NT; ++u) q[u] = (double)x[u] * (double)y[u];
+    // rho - shift in fp64, as in the square form
+    ro[p] = (float)(q[0] - (double)sh[p]);
+    ro[P + p] = (float)(q[1] + q[2] + q[3] - (double)sh[P + p]);
+    ro[2 * P + p] = (float)(q[4] + q[5] + q[6] + 2.0 * (q[7] + q[8] + q[9]) - (double)sh[2 * P + p]);
 }
 
 // ---------------------------------------------------------------------------
@@ -461,25 +490,26 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     float *A = c->d_A + (int64_t)t * c->n * c->NA;
     const bool pair = c->cfg.density_form == 1;
     float *rho = pair ? nullptr : c->d_rho + (int64_t)t * c->n * c->D;
+    const float *shift = c->d_shift + (int64_t)t * c->ne * c->DR;
     REANN_TIMED(c, REANN_K_DENSITY, s, pair ? 2 : 1);
     if (pair) {
         if (c->NP != 8) return cudaErrorInvalidValue;
-        const int64_t threads = c->n * (8 * 9 / 2);
+        const int64_t threads = nc * (8 * 9 / 2);
         k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
             (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, nullptr,
-            c->d_order, P);
-        k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>((int)c->n, A,
-                                                                        c->d_rho + (int64_t)t * c->n * c->DR);
+            shift, c->d_act_dr, P);
+        k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+            (int)nc, A, c->d_rho + (int64_t)t * c->n * c->DR, c->d_pos, shift, c->ne);
         return cudaGetLastError();
     }
     if (c->NP == 8)
         k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
             (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
-            c->d_order, P);
+            shift, c->d_act_dr, P);
     else if (c->NP == 10)
         k_density_fwd<10><<<(unsigned)((nc + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
             (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
-            c->d_order, P);
+            shift, c->d_act_dr, P);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
@@ -494,7 +524,7 @@ cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s
 #define REANN_EDGE_BWD(NPV, DC)                                                                                  \
     k_edge_bwd<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
         (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, c->d_G, c->d_F, \
-        c->d_dc, accumulate, c->d_order, P)
+        c->d_dc, accumulate, P)
     if (c->NP == 8) {
         if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
     } else if (c->NP == 10) {

@@ -25,7 +25,6 @@ EdgeParams make_edge_params(const reann_ctx *c);
 cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s);
 cudaError_t launch_fill(reann_ctx *c, cudaStream_t s);
 cudaError_t launch_skin_check(reann_ctx *c, int *flag, cudaStream_t s);
-cudaError_t launch_work_order(reann_ctx *c, cudaStream_t s);
 
 // edge kernels (edge.cu)
 cudaError_t launch_active(reann_ctx *c, cudaStream_t s);

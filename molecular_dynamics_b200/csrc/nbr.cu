@@ -255,33 +255,6 @@ __global__ void k_row_max(int n, const int *__restrict__ cnt, int64_t *__restric
     if ((threadIdx.x & 31) == 0 && v > 0) atomicMax((unsigned long long *)out, (unsigned long long)v);
 }
 
-// Centre order of the edge passes.  A warp of an edge pass walks the rows of
-// several centres side by side, so one long row keeps the others' lanes idle;
-// in systems with uneven neighbour counts (a gas of molecules) that idles a
-// quarter of the lanes.  Each window of ORDER_WINDOW consecutive atoms (one
-// neighbourhood, so the gathers stay local) is ordered by row length, then
-// index: the centres a warp takes together have similar lengths.  Windows do
-// not cross `split` (a halo plan's first ghost), so own atoms stay first.
-constexpr int ORDER_WINDOW = 256;
-
-__global__ void k_window_order(int n, int split, const int *__restrict__ cnt, int *__restrict__ order) {
-    const int w = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-    const int lane = threadIdx.x & 31;
-    const int nw_own = (split + ORDER_WINDOW - 1) / ORDER_WINDOW;
-    const int s0 = w < nw_own ? w * ORDER_WINDOW : split + (w - nw_own) * ORDER_WINDOW;
-    if (s0 >= (w < nw_own ? split : n)) return;
-    const int s1 = min(s0 + ORDER_WINDOW, w < nw_own ? split : n);
-    for (int p = s0 + lane; p < s1; p += 32) {
-        const int len = cnt[p];
-        int rank = 0;
-        for (int q = s0; q < s1; ++q) {
-            const int lq = cnt[q];
-            rank += lq < len || (lq == len && q < p);
-        }
-        order[s0 + rank] = p;
-    }
-}
-
 // Sets ST_SKIN when any atom has moved more than skin/2 (minimum image) since
 // the list was built.
 __global__ void k_max_disp(int n, const float4 *__restrict__ pos, const float4 *__restrict__ pos_build, BinParams B,
@@ -336,14 +309,6 @@ cudaError_t launch_fill(reann_ctx *c, cudaStream_t s) {
     if (c->n > 0)
         k_nbr<true><<<blocks(c->n, 128), 128, 0, s>>>((int)c->n, c->d_pos, c->d_bin_start, B, c->d_row, nullptr,
                                                        c->d_col);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_work_order(reann_ctx *c, cudaStream_t s) {
-    const int n = (int)c->n, split = (int)(c->halo ? c->n_local : c->n);
-    const int64_t windows = (split + ORDER_WINDOW - 1) / ORDER_WINDOW + (n - split + ORDER_WINDOW - 1) / ORDER_WINDOW;
-    REANN_TIMED(c, REANN_K_NEIGHBORS, s);
-    if (windows > 0) k_window_order<<<blocks(windows * 32, 256), 256, 0, s>>>(n, split, c->d_cnt, c->d_order);
     return cudaGetLastError();
 }
 
