@@ -31,6 +31,7 @@
 // only and k_rho_pair forms rho_(n,m,l) = sum_tau l!/tau! A_{n,tau} A_{m,tau};
 // the backward pass is the same in both forms (it consumes G = dE/dA).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -200,7 +201,17 @@ struct Lanes {
     static constexpr int CPB = 4 * CPW;         // centres per 128-thread block
 };
 
-template <int NP>
+// ACC64: the fp32-accurate paths form the orbital products c phi Y and
+// accumulate A in fp64 (phi itself stays fp32), form rho - shift in fp64, and
+// take the Gaussian centres and the cutoff factor as fp32 pairs with r's
+// rounding residual: on the stiff gas workload the fp32 rounding of these
+// products and sums left a force error of 1.1e-4 eV/A against the oracle, 8e-5
+// with them, at 1.4-1.5x the kernel time.  The bf16-network path, whose force
+// tolerance is 5e-3 eV/A, keeps the plain fp32 forms.
+template <bool ACC64>
+using acc_t = typename std::conditional<ACC64, double, float>::type;
+
+template <int NP, bool ACC64>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                      const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
@@ -219,12 +230,14 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     if (lane >= Ln::USED || i >= n) return;
     const int n0 = 2 * sub;
 
-    float acc[2][NT];
+    using R = acc_t<ACC64>;
+    R acc[2][NT];
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int u = 0; u < NT; ++u) acc[m][u] = 0.f;
-    const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]}, ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
+        for (int u = 0; u < NT; ++u) acc[m][u] = R(0);
+    const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
+    const float ml[2] = {ACC64 ? P.mu_lo[n0] : 0.f, ACC64 ? P.mu_lo[n0 + 1] : 0.f};
     const int q0 = row[i], q1 = q0 + act_cnt[i];
     int j_next = q0 < q1 ? act_col[q0] : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -240,7 +253,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             if (act_dr) dr_next = act_dr[q + 1];
         }
         const float r = g.w;
-        const float fc = cutoff_cos2(fmaf(r, P.th_hi, r * P.th_lo));
+        const float fc = cutoff_cos2(ACC64 ? fmaf(r, P.th_hi, r * P.th_lo) : r * P.th_hi);
         // first layer: c^0 by element (no lookup with a single element)
         const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
         float c[3][2];
@@ -250,40 +263,44 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             c[l][0] = v.x;
             c[l][1] = v.y;
         }
-        const float Y[NT] = {1.f, g.x, g.y, g.z, g.x * g.x, g.y * g.y, g.z * g.z, g.x * g.y, g.x * g.z, g.y * g.z};
+        const R gx = g.x, gy = g.y, gz = g.z;
+        const R Y[NT] = {R(1), gx, gy, gz, gx * gx, gy * gy, gz * gz, gx * gy, gx * gz, gy * gz};
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
             // the Gaussians' slope 2 alpha t makes them the part of the density most
-            // sensitive to r: t carries r's rounding residual
-            const float t = ((r - mh[m]) - ml[m]) + dr;
+            // sensitive to r: on the fp32-accurate paths t takes the centres' second
+            // fp32 halves and r's rounding residual
+            const float t = ACC64 ? ((r - mh[m]) - ml[m]) + dr : r - mh[m];
             const float phi = expf(-P.alpha * t * t) * fc;
-            const float a0 = c[0][m] * phi, a1 = c[1][m] * phi, a2 = c[2][m] * phi;
+            const R a0 = R(c[0][m]) * phi, a1 = R(c[1][m]) * phi, a2 = R(c[2][m]) * phi;
             acc[m][0] += a0;
 #pragma unroll
-            for (int u = 1; u < 4; ++u) acc[m][u] = fmaf(a1, Y[u], acc[m][u]);
+            for (int u = 1; u < 4; ++u) acc[m][u] = fma(a1, Y[u], acc[m][u]);
 #pragma unroll
-            for (int u = 4; u < NT; ++u) acc[m][u] = fmaf(a2, Y[u], acc[m][u]);
+            for (int u = 4; u < NT; ++u) acc[m][u] = fma(a2, Y[u], acc[m][u]);
         }
     }
     float *Ao = A_out + (int64_t)i * NA;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
         const int nn = n0 + m;
-        const float *v = acc[m];
+        const R *v = acc[m];
 #pragma unroll
-        for (int u = 0; u < NT; u += 2) *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2(v[u], v[u + 1]);
+        for (int u = 0; u < NT; u += 2)
+            *reinterpret_cast<float2 *>(Ao + nn * NT + u) = make_float2((float)v[u], (float)v[u + 1]);
         if (!rho_out) continue;   // pair form: rho from A in k_rho_pair
         // rho - shift in fp64 (the networks see (rho - shift) / scale, which the
         // fp32 rounding of rho itself would blur when rho is close to its shift)
+        // (on the bf16-network path in fp32)
         float *ro = rho_out + (int64_t)i * D;
         const float *sh = shift + (ne > 1 ? __float_as_int(pos[i].w) : 0) * D;
-        double x[NT];
+        R x[NT];
 #pragma unroll
-        for (int u = 0; u < NT; ++u) x[u] = (double)v[u];
-        ro[nn] = (float)(x[0] * x[0] - (double)sh[nn]);
-        ro[NP + nn] = (float)(x[1] * x[1] + x[2] * x[2] + x[3] * x[3] - (double)sh[NP + nn]);
-        ro[2 * NP + nn] = (float)(x[4] * x[4] + x[5] * x[5] + x[6] * x[6] + 2.0 * (x[7] * x[7] + x[8] * x[8] + x[9] * x[9]) -
-                                  (double)sh[2 * NP + nn]);
+        for (int u = 0; u < NT; ++u) x[u] = ACC64 ? v[u] : R((float)v[u]);
+        ro[nn] = (float)(x[0] * x[0] - (R)sh[nn]);
+        ro[NP + nn] = (float)(x[1] * x[1] + x[2] * x[2] + x[3] * x[3] - (R)sh[NP + nn]);
+        ro[2 * NP + nn] = (float)(x[4] * x[4] + x[5] * x[5] + x[6] * x[6] + R(2) * (x[7] * x[7] + x[8] * x[8] + x[9] * x[9]) -
+                                  (R)sh[2 * NP + nn]);
     }
 }
 
@@ -329,7 +346,9 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                 ck[l][1] = v.y;
             }
         }
-        const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]}, ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
+        // the backward takes the constants' fp32 values: its rounding shifts forces by
+        // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
+        const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
         const int q0 = row[i], q1 = q0 + act_cnt[i];
         // the edge list is read once per launch: streaming loads (evict first)
         // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
@@ -347,9 +366,9 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             const float r = geo.w;
             const float inv_r = __fdividef(1.0f, r);
             float sn, cs;
-            __sincosf(2.f * fmaf(r, P.th_hi, r * P.th_lo), &sn, &cs);   // 2 theta in [0, pi)
+            __sincosf(r * (2.f * P.th_hi), &sn, &cs);   // 2 theta in [0, pi)
             const float fc = 0.5f * (cs + 1.0f);
-            const float dfc = -fmaf(P.th_hi, sn, P.th_lo * sn);
+            const float dfc = -P.th_hi * sn;
             float gj[2 * NT], cj[3][2];
             {
                 const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)j * NA);
@@ -379,7 +398,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             const float xy = d.x * d.y, xz = d.x * d.z, yz = d.y * d.z;
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
-                const float t = (r - mh[m]) - ml[m];
+                const float t = r - mh[m];
                 const float g = __expf(-P.alpha * t * t);
                 const float phi = g * fc;
                 const float dphi = g * (-2.0f * P.alpha * t * fc + dfc);
@@ -491,27 +510,35 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const bool pair = c->cfg.density_form == 1;
     float *rho = pair ? nullptr : c->d_rho + (int64_t)t * c->n * c->D;
     const float *shift = c->d_shift + (int64_t)t * c->ne * c->DR;
+    const bool acc64 = c->cfg.mlp_precision != 1;   // the fp32-accurate paths
     REANN_TIMED(c, REANN_K_DENSITY, s, pair ? 2 : 1);
     if (pair) {
         if (c->NP != 8) return cudaErrorInvalidValue;
         const int64_t threads = nc * (8 * 9 / 2);
-        k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, nullptr,
-            shift, c->d_act_dr, P);
+        if (acc64)
+            k_density_fwd<8, true><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+                (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A,
+                nullptr, shift, c->d_act_dr, P);
+        else
+            k_density_fwd<8, false><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
+                (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A,
+                nullptr, shift, c->d_act_dr, P);
         k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
             (int)nc, A, c->d_rho + (int64_t)t * c->n * c->DR, c->d_pos, shift, c->ne);
         return cudaGetLastError();
     }
-    if (c->NP == 8)
-        k_density_fwd<8><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
-            shift, c->d_act_dr, P);
-    else if (c->NP == 10)
-        k_density_fwd<10><<<(unsigned)((nc + Lanes<10>::CPB - 1) / Lanes<10>::CPB), 128, 0, s>>>(
-            (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho,
-            shift, c->d_act_dr, P);
-    else
+#define REANN_DENSITY(NPV, ACC)                                                                                 \
+    k_density_fwd<NPV, ACC><<<(unsigned)((nc + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(               \
+        (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, shift,    \
+        c->d_act_dr, P)
+    if (c->NP == 8) {
+        if (acc64) REANN_DENSITY(8, true); else REANN_DENSITY(8, false);
+    } else if (c->NP == 10) {
+        if (acc64) REANN_DENSITY(10, true); else REANN_DENSITY(10, false);
+    } else {
         return cudaErrorInvalidValue;
+    }
+#undef REANN_DENSITY
     return cudaGetLastError();
 }
 

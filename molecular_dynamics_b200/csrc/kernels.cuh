@@ -7,6 +7,7 @@ namespace reann {
 
 struct BinParams {
     double box[3];
+    double inv_box[3];
     int m[3];
     int ncell;
     int ne;

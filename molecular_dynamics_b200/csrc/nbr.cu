@@ -187,12 +187,17 @@ __global__ void k_gather_pos(int64_t n, const float *__restrict__ pos, const int
 
 // Minimum-image squared distance in fp64 with every operation rounded
 // separately (no contraction), exactly as the list definition states:
-// d = x_j - x_i; d -= L rint(d / L); r2 = (dx dx + dy dy) + dz dz.
+// d = x_j - x_i; d -= L k with k = rint(d / L); r2 = (dx dx + dy dy) + dz dz.
+// k is taken as rint(d (1/L)): the product can differ from the quotient only
+// in the last bit, which changes k only when d / L is within an ulp of a
+// half-integer -- a pair half a box apart, never closer than r_cut + skin
+// (the box is at least twice that) -- so every listed pair gets the same k,
+// the same d and the same r2 as with the division.
 __device__ __forceinline__ double list_r2(float4 pi, float4 pj, const BinParams &B) {
     double d[3] = {__dsub_rn((double)pj.x, (double)pi.x), __dsub_rn((double)pj.y, (double)pi.y),
                    __dsub_rn((double)pj.z, (double)pi.z)};
 #pragma unroll
-    for (int a = 0; a < 3; ++a) d[a] = __dsub_rn(d[a], __dmul_rn(B.box[a], rint(__ddiv_rn(d[a], B.box[a]))));
+    for (int a = 0; a < 3; ++a) d[a] = __dsub_rn(d[a], __dmul_rn(B.box[a], rint(d[a] * B.inv_box[a])));
     return __dadd_rn(__dadd_rn(__dmul_rn(d[0], d[0]), __dmul_rn(d[1], d[1])), __dmul_rn(d[2], d[2]));
 }
 
@@ -325,6 +330,7 @@ BinParams make_bin_params(const reann_ctx *c) {
     BinParams B;
     for (int a = 0; a < 3; ++a) {
         B.box[a] = c->box[a];
+        B.inv_box[a] = 1.0 / c->box[a];
         B.m[a] = c->m[a];
     }
     B.ncell = c->ncell;

@@ -133,10 +133,14 @@ def test_depths_other_than_the_preset(key, T):
     n = len(pos)
     tol_E = 1e-5 * max(abs(ref.energy) / n, 1e-2)
     tol_F = 1e-4
+    stated = (tol_E, tol_F)
     if T > 3:
         dE, dF = _rounding_sensitivity(p, pos, types, box, T, w, ref)
         tol_E = max(tol_E, ROUNDING_FACTOR * dE)
         tol_F = max(tol_F, ROUNDING_FACTOR * dF)
+        print(f"\n{key} T={T}: |dE|/N={abs(E - ref.energy) / n:.3e} (stated {stated[0]:.3e}), "
+              f"max|dF|={np.abs(F - ref.forces).max():.3e} (stated {stated[1]:.1e}); oracle response to "
+              f"2^-24 position noise: dE/N {dE:.3e}, dF {dF:.3e}")
     assert abs(E - ref.energy) / n <= tol_E, (abs(E - ref.energy) / n, tol_E)
     assert np.abs(F - ref.forces).max() <= tol_F, (np.abs(F - ref.forces).max(), tol_F)
 
