@@ -49,11 +49,11 @@ FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without d
 
 
 # DRAM read + write (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# k_edge_bwd launch (a layer >= 1 launch) from an ncu capture on 256,000 Ag
-# atoms, scaled to the atom count of the run.  The capture belongs to the kernel
-# source whose SHA-256 prefix is recorded beside it (the text of the k_edge_bwd
-# kernel in edge.cu): once that text changes, the figure no longer describes the
-# kernel and the line reports null.
+# k_edge_bwd launch (a layer >= 1 launch: the scalar kernel) from an ncu
+# capture on 256,000 Ag atoms, scaled to the atom count of the run.  The capture
+# belongs to the kernel source whose SHA-256 prefix is recorded beside it (the
+# text of the scalar k_edge_bwd kernel in edge.cu): once that text changes, the
+# figure no longer describes the kernel and the line reports null.
 EDGE_BWD_CAPTURE = {"bytes_per_atom": (772.892160e6 + 18.705664e6) / 256000, "source_sha": "cd5bc3ff23f61b1f"}
 EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom ncu capture scaled by the atom count"
 
@@ -63,7 +63,7 @@ def edge_source_sha() -> str:
     with open(os.path.join(ROOT, "molecular_dynamics_b200", "csrc", "edge.cu")) as f:
         src = f.read()
     a = src.index("k_edge_bwd(int n")
-    b = src.index("\n// ----", a)
+    b = src.index("\n// Packed form of the backward", a)
     return hashlib.sha256(src[a:b].encode()).hexdigest()[:16]
 
 

@@ -38,6 +38,7 @@ struct EdgeParams {
     // argument biases a large system's energy)
     float th_hi, th_lo;
     float alpha;
+    float neg_alpha_log2e;   // -alpha log2(e): exp(-alpha t^2) = 2^(t^2 neg_alpha_log2e)
     float mu_hi[16], mu_lo[16];
 };
 
@@ -51,16 +52,35 @@ struct NetOffsets {
 // works on one edge, lane `sub` of the slot owning radial indices 2 sub and
 // 2 sub + 1.  dE/dA rows (G) are stored lane-interleaved so that a slot's
 // loads of one neighbour's row are contiguous: the 20 values of lane `sub`
-// (index m*10 + tau for its radial index 2 sub + m) sit at
-//   p = (idx / 4) * 4 LPE + 4 sub + idx % 4.
-__host__ __device__ constexpr int g_slot_index(int n, int tau, int NP) {
-    return ((((n % 2) * NT + tau) / 4) * 4 * (NP / 2)) + 4 * (n / 2) + (((n % 2) * NT + tau) % 4);
+// sit at
+//   p = (idx / 4) * 4 LPE + 4 sub + idx % 4,
+// with idx = 2 tau + m for radial index 2 sub + m in the pair order, where
+// each float4 holds two tuples' (m = 0, m = 1) pairs for packed fp32
+// arithmetic, and idx = 10 m + tau in the radial-major order.  The backward
+// pass of layer t takes the pair order except for N_phi = 8 at t >= 1 (see
+// the edge kernels), and the networks write each layer's rows in its order.
+__host__ __device__ constexpr bool g_pairs(int NP, int layer) { return !(NP == 8 && layer >= 1); }
+__host__ __device__ constexpr int g_lane_index(int m, int tau, bool pairs) {
+    return pairs ? 2 * tau + m : m * NT + tau;
 }
-// inverse: the (radial index, tuple) stored at position p
-__host__ __device__ constexpr int g_slot_source(int p, int NP) {
-    return (2 * ((p % (4 * (NP / 2))) / 4) + ((p / (4 * (NP / 2))) * 4 + p % 4) / NT) * NT +
-           ((p / (4 * (NP / 2))) * 4 + p % 4) % NT;
+__host__ __device__ constexpr int g_slot_index(int n, int tau, int NP, bool pairs) {
+    return (g_lane_index(n % 2, tau, pairs) / 4) * 4 * (NP / 2) + 4 * (n / 2) + g_lane_index(n % 2, tau, pairs) % 4;
 }
+// inverse: the (radial index, tuple) stored at position p, as n * 10 + tau
+__host__ __device__ constexpr int g_slot_source(int p, int NP, bool pairs) {
+    return (2 * ((p % (4 * (NP / 2))) / 4) +
+            (pairs ? ((p / (4 * (NP / 2))) * 4 + p % 4) % 2 : ((p / (4 * (NP / 2))) * 4 + p % 4) / NT)) * NT +
+           (pairs ? ((p / (4 * (NP / 2))) * 4 + p % 4) / 2 : ((p / (4 * (NP / 2))) * 4 + p % 4) % NT);
+}
+constexpr bool g_slot_roundtrip(int NP, bool pairs) {
+    for (int n = 0; n < NP; ++n)
+        for (int t = 0; t < NT; ++t)
+            if (g_slot_source(g_slot_index(n, t, NP, pairs), NP, pairs) != n * NT + t) return false;
+    return true;
+}
+static_assert(g_slot_roundtrip(8, true) && g_slot_roundtrip(10, true) && g_slot_roundtrip(8, false) &&
+                  g_slot_roundtrip(10, false),
+              "dE/dA lane orders are permutations");
 
 struct Ctx;
 

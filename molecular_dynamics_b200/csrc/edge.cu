@@ -53,6 +53,7 @@ EdgeParams make_edge_params(const reann_ctx *c) {
     P.th_hi = (float)th;
     P.th_lo = (float)(th - (double)P.th_hi);
     P.alpha = (float)c->cfg.alpha;
+    P.neg_alpha_log2e = (float)(-c->cfg.alpha * 1.44269504088896340736);
     for (int k = 0; k < 16; ++k) {
         const double mu = k < c->cfg.n_radial ? c->cfg.r_cut * k / (double)(c->cfg.n_radial - 1) : 0.0;
         P.mu_hi[k] = (float)mu;
@@ -193,6 +194,20 @@ __device__ __forceinline__ float cutoff_cos2(float theta) {
     return c * c;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction applies the
+// same operation to a lane's two radial indices.
+__device__ __forceinline__ float2 bc2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// 2^x per component on the SFU (x <= 0 here)
+__device__ __forceinline__ float2 exp2_sfu(float2 x) {
+    float2 y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y.x) : "f"(x.x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y.y) : "f"(x.y));
+    return y;
+}
+
 template <int NP>
 struct Lanes {
     static constexpr int LPE = NP / 2;
@@ -237,47 +252,89 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = R(0);
     const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
-    const float ml[2] = {ACC64 ? P.mu_lo[n0] : 0.f, ACC64 ? P.mu_lo[n0 + 1] : 0.f};
     const int q0 = row[i], q1 = q0 + act_cnt[i];
     int j_next = q0 < q1 ? act_col[q0] : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
-    float dr_next = (act_dr && q0 < q1) ? act_dr[q0] : 0.f;
-    for (int q = q0; q < q1; ++q) {
-        // the next edge's index and geometry are in flight while this one computes
-        const int j = j_next;
-        const float4 g = g_next;         // dx, dy, dz, r
-        const float dr = dr_next;        // r - fp32(r) (fp32-accurate paths), else 0
-        if (q + 1 < q1) {
-            j_next = act_col[q + 1];
-            g_next = act_geo[q + 1];
-            if (act_dr) dr_next = act_dr[q + 1];
+    if constexpr (!ACC64) {
+        // fp32 sums: the lane's two radial indices as packed pairs (m = 0, m = 1)
+        float2 acc2[NT];
+#pragma unroll
+        for (int u = 0; u < NT; ++u) acc2[u] = bc2(0.f);
+        const float2 NMU = make_float2(-mh[0], -mh[1]);
+        for (int q = q0; q < q1; ++q) {
+            const int j = j_next;
+            const float4 g = g_next;
+            if (q + 1 < q1) {
+                j_next = act_col[q + 1];
+                g_next = act_geo[q + 1];
+            }
+            const float r = g.w;
+            const float fc = cutoff_cos2(r * P.th_hi);
+            const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
+            float2 C[3];
+#pragma unroll
+            for (int l = 0; l < 3; ++l) C[l] = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
+            const float2 t = add2(bc2(r), NMU);
+            const float2 e = mul2(mul2(t, t), bc2(-P.alpha));
+            const float2 phi = mul2(make_float2(expf(e.x), expf(e.y)), bc2(fc));
+            const float2 a0 = mul2(C[0], phi), a1 = mul2(C[1], phi), a2 = mul2(C[2], phi);
+            const float2 DX = bc2(g.x), DY = bc2(g.y), DZ = bc2(g.z);
+            acc2[0] = add2(acc2[0], a0);
+            acc2[1] = fma2(a1, DX, acc2[1]);
+            acc2[2] = fma2(a1, DY, acc2[2]);
+            acc2[3] = fma2(a1, DZ, acc2[3]);
+            acc2[4] = fma2(a2, mul2(DX, DX), acc2[4]);
+            acc2[5] = fma2(a2, mul2(DY, DY), acc2[5]);
+            acc2[6] = fma2(a2, mul2(DZ, DZ), acc2[6]);
+            acc2[7] = fma2(a2, mul2(DX, DY), acc2[7]);
+            acc2[8] = fma2(a2, mul2(DX, DZ), acc2[8]);
+            acc2[9] = fma2(a2, mul2(DY, DZ), acc2[9]);
         }
-        const float r = g.w;
-        const float fc = cutoff_cos2(ACC64 ? fmaf(r, P.th_hi, r * P.th_lo) : r * P.th_hi);
-        // first layer: c^0 by element (no lookup with a single element)
-        const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
-        float c[3][2];
 #pragma unroll
-        for (int l = 0; l < 3; ++l) {
-            const float2 v = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
-            c[l][0] = v.x;
-            c[l][1] = v.y;
+        for (int u = 0; u < NT; ++u) {
+            acc[0][u] = acc2[u].x;
+            acc[1][u] = acc2[u].y;
         }
-        const R gx = g.x, gy = g.y, gz = g.z;
-        const R Y[NT] = {R(1), gx, gy, gz, gx * gx, gy * gy, gz * gz, gx * gy, gx * gz, gy * gz};
+    } else {
+        const float ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
+        float dr_next = act_dr && q0 < q1 ? act_dr[q0] : 0.f;
+        for (int q = q0; q < q1; ++q) {
+            // the next edge's index and geometry are in flight while this one computes
+            const int j = j_next;
+            const float4 g = g_next;         // dx, dy, dz, r
+            const float dr = dr_next;        // r - fp32(r)
+            if (q + 1 < q1) {
+                j_next = act_col[q + 1];
+                g_next = act_geo[q + 1];
+                if (act_dr) dr_next = act_dr[q + 1];
+            }
+            const float r = g.w;
+            const float fc = cutoff_cos2(fmaf(r, P.th_hi, r * P.th_lo));
+            // first layer: c^0 by element (no lookup with a single element)
+            const float *cj = coef ? coef + (int64_t)j * D : sC0 + (ne > 1 ? __float_as_int(pos[j].w) * D : 0);
+            float c[3][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            // the Gaussians' slope 2 alpha t makes them the part of the density most
-            // sensitive to r: on the fp32-accurate paths t takes the centres' second
-            // fp32 halves and r's rounding residual
-            const float t = ACC64 ? ((r - mh[m]) - ml[m]) + dr : r - mh[m];
-            const float phi = expf(-P.alpha * t * t) * fc;
-            const R a0 = R(c[0][m]) * phi, a1 = R(c[1][m]) * phi, a2 = R(c[2][m]) * phi;
-            acc[m][0] += a0;
+            for (int l = 0; l < 3; ++l) {
+                const float2 v = *reinterpret_cast<const float2 *>(cj + l * NP + n0);
+                c[l][0] = v.x;
+                c[l][1] = v.y;
+            }
+            const R gx = g.x, gy = g.y, gz = g.z;
+            const R Y[NT] = {R(1), gx, gy, gz, gx * gx, gy * gy, gz * gz, gx * gy, gx * gz, gy * gz};
 #pragma unroll
-            for (int u = 1; u < 4; ++u) acc[m][u] = fma(a1, Y[u], acc[m][u]);
+            for (int m = 0; m < 2; ++m) {
+                // the Gaussians' slope 2 alpha t makes them the part of the density most
+                // sensitive to r: t takes the centres' second fp32 halves and r's
+                // rounding residual
+                const float t = ((r - mh[m]) - ml[m]) + dr;
+                const float phi = expf(-P.alpha * t * t) * fc;
+                const R a0 = R(c[0][m]) * phi, a1 = R(c[1][m]) * phi, a2 = R(c[2][m]) * phi;
+                acc[m][0] += a0;
 #pragma unroll
-            for (int u = 4; u < NT; ++u) acc[m][u] = fma(a2, Y[u], acc[m][u]);
+                for (int u = 1; u < 4; ++u) acc[m][u] = fma(a1, Y[u], acc[m][u]);
+#pragma unroll
+                for (int u = 4; u < NT; ++u) acc[m][u] = fma(a2, Y[u], acc[m][u]);
+            }
         }
     }
     float *Ao = A_out + (int64_t)i * NA;
@@ -306,8 +363,8 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 
 // backward: same slots and lanes.  Lane `sub` keeps G_k and c_k of its two
 // radial indices in registers and reads the neighbour's 20 interleaved dE/dA
-// values as five float4 (the slot's four lanes read 64 contiguous bytes per
-// load).  dE/dc_k of the lane's radial indices needs no reduction; the force
+// values (radial-major lane order) as five float4 (the slot's four lanes read
+// 64 contiguous bytes per load).  dE/dc_k of the lane's radial indices needs no reduction; the force
 // is summed over the slot's lanes in a fixed order.
 template <int NP, bool HAS_DC>
 __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restrict__ row,
@@ -316,6 +373,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
                                                   float *__restrict__ dc, bool accumulate, EdgeParams P) {
+    static_assert(!g_pairs(NP, HAS_DC ? 1 : 0), "scalar backward reads the radial-major lane order");
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -465,6 +523,194 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
     }
 }
 
+// Packed form of the backward pass for rows in the pair lane order: each
+// float4 of a dE/dA row holds two tuples' (m = 0, m = 1) pairs, and the
+// per-edge arithmetic runs on those pairs with packed fp32 instructions
+// (sm_100 f32x2), half the instructions of the scalar form.  With the
+// coefficient gradient at N_phi = 8 the pairs' extra live registers spill at
+// the 80 registers that six blocks per SM allow and the scalar form above is
+// faster (1M-atom Ag: first layer 1.96 -> 1.66 ms packed, later layers 2.16
+// -> 2.41 ms); for N_phi = 10 the packed form is faster in every layer (108k
+// atoms: 0.49 -> 0.45 ms and 0.33 -> 0.29 ms).
+template <int NP, bool HAS_DC>
+__global__ void __launch_bounds__(128, 6) k_edge_bwd_pk(int n, const int *__restrict__ row,
+                                                     const int *__restrict__ act_cnt, const int *__restrict__ act_col,
+                                                     const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
+                                                     const float *__restrict__ coef, const float *__restrict__ C0,
+                                                     int ne, const float *__restrict__ G, float *__restrict__ F,
+                                                     float *__restrict__ dc, bool accumulate, EdgeParams P) {
+    static_assert(g_pairs(NP, HAS_DC ? 1 : 0), "packed backward reads the pair lane order");
+    using Ln = Lanes<NP>;
+    constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
+    __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
+    for (int k = threadIdx.x; k < ne * D; k += blockDim.x) sC0[k] = C0[k];
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = lane / LPE, sub = lane % LPE;
+    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const bool live = lane < Ln::USED && i < n;
+    const int n0 = 2 * sub;
+
+    // force and dE/dc_k partials as (m = 0, m = 1) pairs
+    float2 fx = bc2(0.f), fy = bc2(0.f), fz = bc2(0.f);
+    // dE/dc_k: sum phi G_j Y per l (l = 1 without its sign)
+    float2 dck[3] = {bc2(0.f), bc2(0.f), bc2(0.f)};
+    if (live) {
+        // gk[2 tau + m]: dE/dA of the centre for radial index n0 + m;
+        // ck[l]: its coefficients (n0, n0 + 1), l = 1 held with its parity sign
+        float gk[2 * NT];
+        float2 ck[3];
+        {
+            const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)i * NA);
+#pragma unroll
+            for (int q = 0; q < 5; ++q) {
+                const float4 v = g4[q * LPE + sub];
+                gk[4 * q] = v.x; gk[4 * q + 1] = v.y; gk[4 * q + 2] = v.z; gk[4 * q + 3] = v.w;
+            }
+            const float *cp = coef ? coef + (int64_t)i * D : sC0 + __float_as_int(pos[i].w) * D;
+#pragma unroll
+            for (int l = 0; l < 3; ++l) ck[l] = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+            ck[1] = make_float2(-ck[1].x, -ck[1].y);
+        }
+        // the backward takes the constants' fp32 values: its rounding shifts forces by
+        // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
+        const float2 nmu = make_float2(-P.mu_hi[n0], -P.mu_hi[n0 + 1]);
+        const int q0 = row[i], q1 = q0 + act_cnt[i];
+        // the edge list is read once per launch: streaming loads (evict first)
+        // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
+        int j_next = q0 < q1 ? __ldcs(act_col + q0) : 0;
+        float4 geo_next = q0 < q1 ? __ldcs(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
+        for (int q = q0; q < q1; ++q) {
+            // the next edge's index and geometry are in flight while this one computes
+            const int j = j_next;
+            const float4 geo = geo_next;
+            if (q + 1 < q1) {
+                j_next = __ldcs(act_col + q + 1);
+                geo_next = __ldcs(act_geo + q + 1);
+            }
+            const float r = geo.w;
+            const float inv_r = __fdividef(1.0f, r);
+            float sn, cs;
+            __sincosf(r * (2.f * P.th_hi), &sn, &cs);   // 2 theta in [0, pi)
+            const float fc = 0.5f * (cs + 1.0f);
+            const float dfc = -P.th_hi * sn;
+            float gj[2 * NT];
+            float2 cj[3];
+            {
+                const float4 *g4 = reinterpret_cast<const float4 *>(G + (int64_t)j * NA);
+#pragma unroll
+                for (int q2 = 0; q2 < 5; ++q2) {
+                    const float4 v = __ldg(g4 + q2 * LPE + sub);
+                    gj[4 * q2] = v.x; gj[4 * q2 + 1] = v.y; gj[4 * q2 + 2] = v.z; gj[4 * q2 + 3] = v.w;
+                }
+                if (!HAS_DC && ne == 1) {
+                    // first layer, one element: every atom carries the same c^0
+                    cj[0] = ck[0];
+                    cj[1] = make_float2(-ck[1].x, -ck[1].y);
+                    cj[2] = ck[2];
+                } else {
+                    const float *cp = coef ? coef + (int64_t)j * D : sC0 + __float_as_int(pos[j].w) * D;
+#pragma unroll
+                    for (int l = 0; l < 3; ++l) cj[l] = *reinterpret_cast<const float2 *>(cp + l * NP + n0);
+                }
+            }
+            // phi_n = g_n fc and phi_n' / r = g_n (-2 alpha t_n fc + fc') / r, t_n = r - mu_n;
+            // H_tau = G_k c_j + (-1)^l G_j c_k, folded tuple by tuple into
+            //   Pv = sum_tau H_tau Y_tau and Q = sum_tau H_tau grad Y_tau,
+            // and (layers >= 1) S_l = sum_{|tau|=l} G_j Y_tau
+#define GK2(u) make_float2(gk[2 * (u)], gk[2 * (u) + 1])
+#define GJ2(u) make_float2(gj[2 * (u)], gj[2 * (u) + 1])
+            const float2 DX = bc2(geo.x), DY = bc2(geo.y), DZ = bc2(geo.z);
+            const float2 t = add2(bc2(r), nmu);
+            const float2 g = exp2_sfu(mul2(mul2(t, t), bc2(P.neg_alpha_log2e)));
+            const float2 phi = mul2(g, bc2(fc));
+            const float2 dphir = mul2(g, fma2(t, bc2(-2.0f * P.alpha * fc * inv_r), bc2(dfc * inv_r)));
+            float2 Pv, Qx, Qy, Qz, S1, S2, Y2, H;
+            Pv = fma2(GK2(0), cj[0], mul2(GJ2(0), ck[0]));
+            Qx = fma2(GK2(1), cj[1], mul2(GJ2(1), ck[1]));
+            Pv = fma2(Qx, DX, Pv);
+            Qy = fma2(GK2(2), cj[1], mul2(GJ2(2), ck[1]));
+            Pv = fma2(Qy, DY, Pv);
+            Qz = fma2(GK2(3), cj[1], mul2(GJ2(3), ck[1]));
+            Pv = fma2(Qz, DZ, Pv);
+            if (HAS_DC) S1 = fma2(GJ2(3), DZ, fma2(GJ2(2), DY, mul2(GJ2(1), DX)));
+            Y2 = mul2(DX, DX);
+            H = fma2(GK2(4), cj[2], mul2(GJ2(4), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qx = fma2(H, add2(DX, DX), Qx);
+            if (HAS_DC) S2 = mul2(GJ2(4), Y2);
+            Y2 = mul2(DY, DY);
+            H = fma2(GK2(5), cj[2], mul2(GJ2(5), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qy = fma2(H, add2(DY, DY), Qy);
+            if (HAS_DC) S2 = fma2(GJ2(5), Y2, S2);
+            Y2 = mul2(DZ, DZ);
+            H = fma2(GK2(6), cj[2], mul2(GJ2(6), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qz = fma2(H, add2(DZ, DZ), Qz);
+            if (HAS_DC) S2 = fma2(GJ2(6), Y2, S2);
+            Y2 = mul2(DX, DY);
+            H = fma2(GK2(7), cj[2], mul2(GJ2(7), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qx = fma2(H, DY, Qx);
+            Qy = fma2(H, DX, Qy);
+            if (HAS_DC) S2 = fma2(GJ2(7), Y2, S2);
+            Y2 = mul2(DX, DZ);
+            H = fma2(GK2(8), cj[2], mul2(GJ2(8), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qx = fma2(H, DZ, Qx);
+            Qz = fma2(H, DX, Qz);
+            if (HAS_DC) S2 = fma2(GJ2(8), Y2, S2);
+            Y2 = mul2(DY, DZ);
+            H = fma2(GK2(9), cj[2], mul2(GJ2(9), ck[2]));
+            Pv = fma2(H, Y2, Pv);
+            Qy = fma2(H, DZ, Qy);
+            Qz = fma2(H, DY, Qz);
+            if (HAS_DC) S2 = fma2(GJ2(9), Y2, S2);
+            const float2 sv = mul2(dphir, Pv);
+            fx = fma2(sv, DX, fma2(phi, Qx, fx));
+            fy = fma2(sv, DY, fma2(phi, Qy, fy));
+            fz = fma2(sv, DZ, fma2(phi, Qz, fz));
+            if (HAS_DC) {
+                dck[0] = fma2(phi, GJ2(0), dck[0]);
+                dck[1] = fma2(phi, S1, dck[1]);
+                dck[2] = fma2(phi, S2, dck[2]);
+            }
+#undef GK2
+#undef GJ2
+        }
+    }
+    // force: the lane's pair, then the slot's lanes (sub 0 .. LPE-1), in a fixed order
+    const float lx = fx.x + fx.y, ly = fy.x + fy.y, lz = fz.x + fz.y;
+    const int base = (lane / LPE) * LPE;
+    float sx = 0.f, sy = 0.f, sz = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < LPE; ++s2) {
+        const int src = base + s2 < 32 ? base + s2 : lane;
+        sx += __shfl_sync(0xffffffffu, lx, src);
+        sy += __shfl_sync(0xffffffffu, ly, src);
+        sz += __shfl_sync(0xffffffffu, lz, src);
+    }
+    if (!live) return;
+    if (sub == 0) {
+        float *Fo = F + 3 * (int64_t)i;
+        if (accumulate) {
+            sx += Fo[0];
+            sy += Fo[1];
+            sz += Fo[2];
+        }
+        Fo[0] = sx;
+        Fo[1] = sy;
+        Fo[2] = sz;
+    }
+    if (HAS_DC) {
+        float *o = dc + (int64_t)i * D;
+        *reinterpret_cast<float2 *>(o + n0) = dck[0];
+        *reinterpret_cast<float2 *>(o + NP + n0) = make_float2(-dck[1].x, -dck[1].y);
+        *reinterpret_cast<float2 *>(o + 2 * NP + n0) = dck[2];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Pair-product densities (density_form = 1): rho_(n,m,l) = sum_{|tau|=l}
 // l!/tau! A_{n,tau} A_{m,tau} for n <= m, at index l P + pair(n, m) with
@@ -548,14 +794,15 @@ cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     const bool has_dc = t >= 1;
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
-#define REANN_EDGE_BWD(NPV, DC)                                                                                  \
-    k_edge_bwd<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
+#define REANN_EDGE_BWD(K, NPV, DC)                                                                               \
+    K<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
         (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, c->d_G, c->d_F, \
         c->d_dc, accumulate, P)
+    // the kernel reads the lane order the networks wrote for this layer (g_pairs)
     if (c->NP == 8) {
-        if (has_dc) REANN_EDGE_BWD(8, true); else REANN_EDGE_BWD(8, false);
+        if (has_dc) REANN_EDGE_BWD(k_edge_bwd, 8, true); else REANN_EDGE_BWD(k_edge_bwd_pk, 8, false);
     } else if (c->NP == 10) {
-        if (has_dc) REANN_EDGE_BWD(10, true); else REANN_EDGE_BWD(10, false);
+        if (has_dc) REANN_EDGE_BWD(k_edge_bwd_pk, 10, true); else REANN_EDGE_BWD(k_edge_bwd_pk, 10, false);
     } else {
         return cudaErrorInvalidValue;
     }

@@ -26,6 +26,7 @@ constexpr int MLP_THREADS = 256;
 
 struct MlpNets {
     NetOffsets net[MAX_ELEMENTS];
+    int g_pairs;   // lane order of the dE/dA rows written (g_pairs of their layer)
 };
 
 enum { MODE_FWD = 0, MODE_ENERGY = 1, MODE_BWD = 2 };
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(MLP_THREADS) k_mlp(const int4 *__restrict__ ti
             // G rows are stored in the edge kernels' lane-interleaved order
             for (int k = tid; k < rows * NA; k += MLP_THREADS) {
                 const int r = k / NA, q = k % NA;
-                const int src = g_slot_source(q, NP);
+                const int src = g_slot_source(q, NP, nets.g_pairs);
                 const int nn = src / NT, u = src % NT;
                 const int l = u == 0 ? 0 : (u < 4 ? 1 : 2);
                 const int64_t rb = (int64_t)(r0 + r) * NA;
@@ -258,30 +259,31 @@ static cudaError_t dispatch(reann_ctx *c, const MlpNets &nets, const float *X, f
     return cudaErrorInvalidValue;
 }
 
-static MlpNets nets_of(const std::vector<NetOffsets> &v, int first, int ne) {
+static MlpNets nets_of(const std::vector<NetOffsets> &v, int first, int ne, int NP, int layer) {
     MlpNets m;
+    m.g_pairs = g_pairs(NP, layer);
     for (int e = 0; e < ne; ++e) m.net[e] = v[first + e];
     return m;
 }
 
 cudaError_t launch_mlp_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nR = c->n * c->DR;
-    return dispatch<MODE_FWD>(c, nets_of(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nR,
+    return dispatch<MODE_FWD>(c, nets_of(c->coef_nets, t * c->ne, c->ne, c->NP, 0), c->d_rho + t * nR,
                               c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_mlp_energy(reann_ctx *c, cudaStream_t s) {
     const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
     const int t = c->T - 1;
-    return dispatch<MODE_ENERGY>(c, nets_of(c->energy_nets, 0, c->ne), c->d_rho + t * nR, nullptr, nullptr, c->d_Ei,
-                                 c->d_A + t * nA, c->d_G, s);
+    return dispatch<MODE_ENERGY>(c, nets_of(c->energy_nets, 0, c->ne, c->NP, c->T - 1), c->d_rho + t * nR, nullptr,
+                                 nullptr, c->d_Ei, c->d_A + t * nA, c->d_G, s);
 }
 
 cudaError_t launch_mlp_coef_bwd(reann_ctx *c, int t, cudaStream_t s) {
     // network M^{t-1}: input rho^{t-1}, upstream gradient dE/dc^t, output G^{t-1}
     const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
-    return dispatch<MODE_BWD>(c, nets_of(c->coef_nets, (t - 1) * c->ne, c->ne), c->d_rho + (t - 1) * nR, nullptr,
-                              c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
+    return dispatch<MODE_BWD>(c, nets_of(c->coef_nets, (t - 1) * c->ne, c->ne, c->NP, t - 1), c->d_rho + (t - 1) * nR,
+                              nullptr, c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
 }
 
 }  // namespace reann

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
         const int pk = (tid & 31) + 32 * j;
-        const int src = g_slot_source(pk < NA ? pk : 0, NP), nn = src / NT, u = src - nn * NT;
+        const int src = g_slot_source(pk < NA ? pk : 0, NP, nets.g_pairs), nn = src / NT, u = src - nn * NT;
         const int gi = (u == 0 ? 0 : (u < 4 ? 1 : 2)) * NP + nn;
         posj[j] = src | (gi << 8) | ((u >= 7 ? 1 : 0) << 16);
     }
@@ -437,8 +437,9 @@ cudaError_t dispatch_tc(reann_ctx *c, const TcNets &nets, const float *X, float 
     return cudaErrorInvalidValue;
 }
 
-TcNets tc_nets(const std::vector<NetOffsets> &v, int first, int ne) {
+TcNets tc_nets(const std::vector<NetOffsets> &v, int first, int ne, int NP, int layer) {
     TcNets m;
+    m.g_pairs = g_pairs(NP, layer);
     for (int e = 0; e < ne; ++e) m.net[e] = v[first + e];
     return m;
 }
@@ -447,21 +448,21 @@ TcNets tc_nets(const std::vector<NetOffsets> &v, int first, int ne) {
 
 cudaError_t launch_mlp_tc_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nD = c->n * c->D;
-    return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nD,
+    return dispatch_tc<TC_FWD>(c, tc_nets(c->coef_nets, t * c->ne, c->ne, c->NP, 0), c->d_rho + t * nD,
                                c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_mlp_tc_energy(reann_ctx *c, cudaStream_t s) {
     const int64_t nD = c->n * c->D, nA = c->n * c->NA;
     const int t = c->T - 1;
-    return dispatch_tc<TC_ENERGY>(c, tc_nets(c->energy_nets, 0, c->ne), c->d_rho + t * nD, nullptr, nullptr, c->d_Ei,
-                                  c->d_A + t * nA, c->d_G, s);
+    return dispatch_tc<TC_ENERGY>(c, tc_nets(c->energy_nets, 0, c->ne, c->NP, c->T - 1), c->d_rho + t * nD, nullptr,
+                                  nullptr, c->d_Ei, c->d_A + t * nA, c->d_G, s);
 }
 
 cudaError_t launch_mlp_tc_coef_bwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nD = c->n * c->D, nA = c->n * c->NA;
-    return dispatch_tc<TC_BWD>(c, tc_nets(c->coef_nets, (t - 1) * c->ne, c->ne), c->d_rho + (t - 1) * nD, nullptr,
-                               c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
+    return dispatch_tc<TC_BWD>(c, tc_nets(c->coef_nets, (t - 1) * c->ne, c->ne, c->NP, t - 1), c->d_rho + (t - 1) * nD,
+                               nullptr, c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
 }
 
 }  // namespace reann

@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(PT, 1)
                         float v[4];
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
-                            const int idx = 4 * q + e2, s2 = idx / NT, u = idx % NT;
+                            const int idx = 4 * q + e2;   // g_lane_index order
+                            const int s2 = nets.g_pairs ? idx % 2 : idx / NT, u = nets.g_pairs ? idx / 2 : idx % NT;
                             v[e2] = (u >= 7 ? 2.f : 1.f) * acc[s2][u];   // l!/tau!
                         }
                         go4[4 * q + part] = make_float4(v[0], v[1], v[2], v[3]);
@@ -398,8 +399,9 @@ cudaError_t run_pair(reann_ctx *c, const TcNets &nets, const float *X, float *Y,
     return cudaGetLastError();
 }
 
-TcNets pair_nets(const std::vector<NetOffsets> &v, int first, int ne) {
+TcNets pair_nets(const std::vector<NetOffsets> &v, int first, int ne, int NP, int layer) {
     TcNets m;
+    m.g_pairs = g_pairs(NP, layer);
     for (int e = 0; e < ne; ++e) m.net[e] = v[first + e];
     return m;
 }
@@ -408,21 +410,21 @@ TcNets pair_nets(const std::vector<NetOffsets> &v, int first, int ne) {
 
 cudaError_t launch_mlp_tc_pair_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nR = c->n * c->DR;
-    return run_pair<TC_FWD>(c, pair_nets(c->coef_nets, t * c->ne, c->ne), c->d_rho + t * nR,
+    return run_pair<TC_FWD>(c, pair_nets(c->coef_nets, t * c->ne, c->ne, c->NP, 0), c->d_rho + t * nR,
                             c->d_coef + (t + 1) * c->n_slots * c->D, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 cudaError_t launch_mlp_tc_pair_energy(reann_ctx *c, cudaStream_t s) {
     const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
     const int t = c->T - 1;
-    return run_pair<TC_ENERGY>(c, pair_nets(c->energy_nets, 0, c->ne), c->d_rho + t * nR, nullptr, nullptr, c->d_Ei,
-                               c->d_A + t * nA, c->d_G, s);
+    return run_pair<TC_ENERGY>(c, pair_nets(c->energy_nets, 0, c->ne, c->NP, c->T - 1), c->d_rho + t * nR, nullptr,
+                               nullptr, c->d_Ei, c->d_A + t * nA, c->d_G, s);
 }
 
 cudaError_t launch_mlp_tc_pair_coef_bwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nR = c->n * c->DR, nA = c->n * c->NA;
-    return run_pair<TC_BWD>(c, pair_nets(c->coef_nets, (t - 1) * c->ne, c->ne), c->d_rho + (t - 1) * nR, nullptr,
-                            c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
+    return run_pair<TC_BWD>(c, pair_nets(c->coef_nets, (t - 1) * c->ne, c->ne, c->NP, t - 1), c->d_rho + (t - 1) * nR,
+                            nullptr, c->d_dc, nullptr, c->d_A + (t - 1) * nA, c->d_G, s);
 }
 
 }  // namespace reann

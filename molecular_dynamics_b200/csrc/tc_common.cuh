@@ -148,6 +148,7 @@ __device__ __forceinline__ void st_elem(unsigned char *tile, int R, int r, int k
 
 struct TcNets {
     NetOffsets net[MAX_ELEMENTS];
+    int g_pairs;   // lane order of the dE/dA rows written (g_pairs of their layer)
 };
 
 // 8 consecutive fp32 TMEM columns of this thread's lane
