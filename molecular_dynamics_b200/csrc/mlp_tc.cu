@@ -210,6 +210,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // energy and backward: the tile's A rows are read at the end; start
         // moving them into L2 now
         if (MODE != TC_FWD && gt == 0) prefetch_l2(A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4));
+        // the group's next tile: its input rows into L2 while this one computes
+        if (gt == 0 && ti + 2 < rg.y) {
+            const int4 nx = tiles[ti + 2];
+            prefetch_l2_span(X + (int64_t)nx.y * D, (size_t)nx.z * D * 4);
+            if (MODE == TC_BWD) prefetch_l2_span(dY + (int64_t)nx.y * D, (size_t)nx.z * D * 4);
+        }
         // input tile: contiguous raw rows -> padded fp32 rows in ACT, then the
         // standardised rho (and the upstream gradient) split bf16
         {

@@ -167,6 +167,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
+// L2 prefetch of the whole 16-byte units inside [p, p + bytes) (the bulk
+// prefetch takes 16-byte aligned spans)
+__device__ __forceinline__ void prefetch_l2_span(const void *p, size_t bytes) {
+    const uintptr_t a = ((uintptr_t)p + 15) & ~(uintptr_t)15, e = ((uintptr_t)p + bytes) & ~(uintptr_t)15;
+    if (e > a) prefetch_l2(reinterpret_cast<const void *>(a), (uint32_t)(e - a));
+}
 
 }  // namespace
 }  // namespace reann
