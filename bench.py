@@ -50,11 +50,13 @@ FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without d
 
 # DRAM read + write (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # k_edge_bwd launch (a layer >= 1 launch: the scalar kernel) from an ncu
-# capture on 256,000 Ag atoms, scaled to the atom count of the run.  The capture
+# capture on 256,000 Ag atoms of the 1M-atom Ag model, scaled to the atom count
+# of the run; other models (other densities, cut-offs, radial counts) report null.  The capture
 # belongs to the kernel source whose SHA-256 prefix is recorded beside it (the
 # text of the scalar k_edge_bwd kernel in edge.cu): once that text changes, the
 # figure no longer describes the kernel and the line reports null.
-EDGE_BWD_CAPTURE = {"bytes_per_atom": (772.892160e6 + 18.705664e6) / 256000, "source_sha": "cd5bc3ff23f61b1f"}
+EDGE_BWD_CAPTURE = {"bytes_per_atom": (770.977280e6 + 18.616064e6) / 256000, "source_sha": "6b6ae64692141468",
+                    "workload": "ag1m"}
 EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom ncu capture scaled by the atom count"
 
 
@@ -341,7 +343,7 @@ def kernel_roofline(group, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_
             "peak_note": note}
 
 
-def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None):
+def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net=None, workload=None):
     """Roofline entry of the dominant kernel group (largest share of the
     profiled time), with its DRAM traffic per launch where an ncu capture of
     that kernel exists."""
@@ -350,11 +352,12 @@ def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net
     r = kernel_roofline(dominant, prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net)
     if r is None:
         return None
-    current = dominant == "edge_bwd" and EDGE_BWD_CAPTURE["source_sha"] == edge_source_sha()
+    current = (dominant == "edge_bwd" and EDGE_BWD_CAPTURE["source_sha"] == edge_source_sha()
+               and workload == EDGE_BWD_CAPTURE["workload"])
     traffic = EDGE_BWD_CAPTURE["bytes_per_atom"] * n_atoms if current else None
     r["traffic"] = traffic
     r["traffic_note"] = EDGE_BWD_TRAFFIC_NOTE if traffic is not None else \
-        "no DRAM capture of the current source of this kernel"
+        "no DRAM capture of the current source of this kernel on this model"
     return r
 
 
@@ -493,7 +496,7 @@ def main():
     shares = {k: v_[0] for k, v_ in prof.items()}
     total = sum(shares.values()) or 1.0
     net = (p.DR, p.D, tuple(p.hidden), network_kind(p))
-    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net)
+    roof = roofline(prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net, workload=p.key)
     per_kernel = {}
     for g in ("edge_bwd", "density", "mlp_bwd", "mlp_fwd", "mlp_energy", "active"):
         r = kernel_roofline(g, prof, cnt.active_pairs, p.n_radial, p.T, n, sm_count, pk, pk_kind, clk, net=net,

@@ -138,9 +138,12 @@ def test_depths_other_than_the_preset(key, T):
         dE, dF = _rounding_sensitivity(p, pos, types, box, T, w, ref)
         tol_E = max(tol_E, ROUNDING_FACTOR * dE)
         tol_F = max(tol_F, ROUNDING_FACTOR * dF)
+        # relative condition number of the forces: relative response per unit relative input change
+        kappa = dF / float(np.sqrt((ref.forces ** 2).mean())) / 2.0 ** -24
         print(f"\n{key} T={T}: |dE|/N={abs(E - ref.energy) / n:.3e} (stated {stated[0]:.3e}), "
               f"max|dF|={np.abs(F - ref.forces).max():.3e} (stated {stated[1]:.1e}); oracle response to "
-              f"2^-24 position noise: dE/N {dE:.3e}, dF {dF:.3e}")
+              f"2^-24 position noise: dE/N {dE:.3e}, dF {dF:.3e}; rms F {np.sqrt((ref.forces ** 2).mean()):.3f}, "
+              f"force condition number {kappa:.0f}")
     assert abs(E - ref.energy) / n <= tol_E, (abs(E - ref.energy) / n, tol_E)
     assert np.abs(F - ref.forces).max() <= tol_F, (np.abs(F - ref.forces).max(), tol_F)
 
