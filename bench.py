@@ -530,7 +530,9 @@ def main():
         "gpu_launches": launches,
         "clocks": clk,
         "kernel_ms_per_step": {k: v_[0] / prof_steps for k, v_ in prof.items() if v_[1]},
-        "kernel_profile_note": f"per-launch CUDA events over a separate {prof_steps}-step call with eager launches",
+        "kernel_profile_note": (f"per-launch CUDA events over a separate {prof_steps}-step call with eager launches; "
+                                f"their sum {total / prof_steps:.4g} ms per step against the timed (graph-replayed) "
+                                f"step's {t_ms / args.steps:.4g} ms"),
         "kernel_share": {k: v_ / total for k, v_ in shares.items() if v_},
         "roofline": roof,
         "kernel_roofline": per_kernel,
