@@ -530,15 +530,16 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
 // coefficient gradient at N_phi = 8 the pairs' extra live registers spill at
 // the 80 registers that six blocks per SM allow and the scalar form above is
 // faster (1M-atom Ag: first layer 1.96 -> 1.66 ms packed, later layers 2.16
-// -> 2.41 ms); for N_phi = 10 the packed form is faster in every layer (108k
-// atoms: 0.49 -> 0.45 ms and 0.33 -> 0.29 ms).
+// -> 2.41 ms, 2.71 ms at five blocks per SM without spills); for N_phi = 10 the
+// packed form is faster in every layer (108k atoms: 0.49 -> 0.45 ms, and 0.40
+// ms at five blocks per SM, where its 96 registers do not spill; first layer
+// 0.33 -> 0.29 ms at six).
 template <int NP, bool HAS_DC>
-__global__ void __launch_bounds__(128, 6) k_edge_bwd_pk(int n, const int *__restrict__ row,
-                                                     const int *__restrict__ act_cnt, const int *__restrict__ act_col,
-                                                     const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
-                                                     const float *__restrict__ coef, const float *__restrict__ C0,
-                                                     int ne, const float *__restrict__ G, float *__restrict__ F,
-                                                     float *__restrict__ dc, bool accumulate, EdgeParams P) {
+__global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
+    k_edge_bwd_pk(int n, const int *__restrict__ row, const int *__restrict__ act_cnt, const int *__restrict__ act_col,
+                  const float4 *__restrict__ act_geo, const float4 *__restrict__ pos, const float *__restrict__ coef,
+                  const float *__restrict__ C0, int ne, const float *__restrict__ G, float *__restrict__ F,
+                  float *__restrict__ dc, bool accumulate, EdgeParams P) {
     static_assert(g_pairs(NP, HAS_DC ? 1 : 0), "packed backward reads the pair lane order");
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
