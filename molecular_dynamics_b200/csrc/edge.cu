@@ -408,17 +408,18 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
         const int q0 = row[i], q1 = q0 + act_cnt[i];
-        // the edge list is read once per launch: streaming loads (evict first)
-        // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
-        int j_next = q0 < q1 ? __ldcs(act_col + q0) : 0;
-        float4 geo_next = q0 < q1 ? __ldcs(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
+        // the edge list takes ordinary cached loads: its 16-byte entries share
+        // 32-byte sectors with the next edge's, and evict-first loads made the
+        // second read of a sector go back to DRAM (1.6x the traffic, no faster)
+        int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
+        float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; ++q) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
             if (q + 1 < q1) {
-                j_next = __ldcs(act_col + q + 1);
-                geo_next = __ldcs(act_geo + q + 1);
+                j_next = __ldg(act_col + q + 1);
+                geo_next = __ldg(act_geo + q + 1);
             }
             const float3 d = make_float3(geo.x, geo.y, geo.z);
             const float r = geo.w;
@@ -577,17 +578,18 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float2 nmu = make_float2(-P.mu_hi[n0], -P.mu_hi[n0 + 1]);
         const int q0 = row[i], q1 = q0 + act_cnt[i];
-        // the edge list is read once per launch: streaming loads (evict first)
-        // leave L1 to the neighbours' dE/dA and coefficient rows, which are reused
-        int j_next = q0 < q1 ? __ldcs(act_col + q0) : 0;
-        float4 geo_next = q0 < q1 ? __ldcs(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
+        // the edge list takes ordinary cached loads: its 16-byte entries share
+        // 32-byte sectors with the next edge's, and evict-first loads made the
+        // second read of a sector go back to DRAM (1.6x the traffic, no faster)
+        int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
+        float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; ++q) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
             if (q + 1 < q1) {
-                j_next = __ldcs(act_col + q + 1);
-                geo_next = __ldcs(act_geo + q + 1);
+                j_next = __ldg(act_col + q + 1);
+                geo_next = __ldg(act_geo + q + 1);
             }
             const float r = geo.w;
             const float inv_r = __fdividef(1.0f, r);
