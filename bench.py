@@ -79,9 +79,13 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 20 ms, started
+    before the warm-up so that samples flow when the timed region begins;
+    stop() keeps the samples taken between mark_begin() and mark_end() (for a
+    region shorter than the sampling interval, the nearest sample on each
+    side)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -89,11 +93,20 @@ class ClockSampler:
         self.index = index
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_begin(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        import datetime
+        self.t1 = datetime.datetime.now()
 
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -108,23 +121,34 @@ class ClockSampler:
             self.proc.kill()
         self.file.flush()
         self.file.seek(0)
-        sm, smax, reasons = [], [], set()
+        import datetime
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        rows = []
         for line in self.file.read().strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[1]), float(parts[2]),
+                             {n for n, v in zip(names, parts[5:9]) if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
         os.unlink(self.file.name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        nearest = False
+        if not inside and rows and self.t0 is not None:
+            before = [r for r in rows if r[0] < self.t0]
+            after = [r for r in rows if r[0] > self.t1]
+            inside = before[-1:] + after[:1]
+            nearest = True
+        sm = [r[1] for r in inside]
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+               "reasons": sorted(set().union(*[r[3] for r in inside])) if inside else [], "samples": len(sm)}
+        if nearest:
+            out["note"] = "timed region shorter than the 20 ms sampling interval: the nearest sample on each side"
+        return out
 
 
 def cpu_sample_preset(p):
@@ -441,16 +465,24 @@ def main():
         cursor[0] += k
         return ctx.reann_md_step_nvt(k, dt_fs, args.temperature, args.tau, z, xx, vv, p.masses)
 
-    # warm-up (the first call also evaluates the entry forces)
+    # warm-up (the first call also evaluates the entry forces); the clock
+    # sampler starts before it so that samples flow through the timed region
+    clocks = ClockSampler(info.local)
+    clocks.start()
     md(args.warmup, x, v)
     torch.cuda.synchronize()
 
     # ---- device-resident timed region: K steps in one call (a continuation);
     # each step's energy+forces and half kick replay as one CUDA graph
-    clocks = ClockSampler(info.local)
     launches0 = ctx.reann_get_counters().kernel_launches
-    clocks.start()
-    run = timed_region(group, lambda: md(args.steps, x, v), clock, n * args.steps)
+
+    def timed_steps():
+        clocks.mark_begin()
+        out = md(args.steps, x, v)   # returns after its stream has synchronised
+        clocks.mark_end()
+        return out
+
+    run = timed_region(group, timed_steps, clock, n * args.steps)
     clk = clocks.stop()
     st = run.result
     t_ms = run.ms
