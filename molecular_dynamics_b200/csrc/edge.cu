@@ -18,9 +18,10 @@
 // folded into the row of k because the list is symmetric; the parity (-1)^l
 // comes from Y_tau(-d) = (-1)^l Y_tau(d).
 //
-// The backward pass uses the SFU intrinsics (__expf, __sincosf, __fdividef):
-// their arguments are bounded (sine/cosine argument in [0, pi), exponent <= 0)
-// and only forces depend on them.  The forward pass keeps an accurate expf and
+// The backward pass uses the special-function unit (__sincosf, __fdividef, and
+// the exponential as __expf or as ex2.approx of t^2 (-alpha log2 e)): the
+// arguments are bounded (sine/cosine argument in [0, pi), exponent <= 0) and
+// only forces depend on them.  The forward pass keeps an accurate expf and
 // evaluates the cutoff as a polynomial accurate to fp32 rounding: the densities
 // feed standardised network inputs, where the intrinsics' ~1e-7 errors showed
 // up as 1e-5-level per-atom energy errors.
