@@ -515,7 +515,9 @@ def main():
         e2e = {"value": run_e.throughput, "unit": UNIT,
                "h2d_bytes_per_step": 2 * 3 * 8 * n, "d2h_bytes_per_step": 2 * 3 * 8 * n,
                "note": f"{'reann_md_step_nvt' if noise is not None else 'reann_md_step'}(1) per step with pinned "
-                       "host x, v: x and v copied in and out every step"}
+                       "host x, v: x and v copied in and out every step (the library moves them in and checks "
+                       "them against its resident state while the step runs; x goes out during the step's "
+                       "force evaluation)"}
 
     if info.rank != 0:
         group.close()

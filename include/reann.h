@@ -210,7 +210,13 @@ reann_status reann_energy_forces(reann_ctx *ctx, const float *pos, double *energ
  * previous one (x and v bitwise equal to what the previous reann_md_step
  * on this context returned, same dt and masses, no other call in between),
  * in which case the resident state, list and forces are reused and the
- * trajectory is identical to one longer call.  Requires a prior
+ * trajectory is identical to one longer call.  Whether a call continues is
+ * decided while it runs: when the previous call left a valid state with the
+ * same dt and masses, the steps start from that state at once, and x and v
+ * are moved in and compared with it on a library stream meanwhile; if they
+ * differ, that run is discarded and the call starts again from the x and v
+ * it read in (x and v are written only after the comparison, or, for the
+ * discarded run's x, overwritten by the result of the restart).  Requires a prior
  * reann_build_neighbors for the same atoms and types (positions may have
  * moved; the list is rebuilt at entry).  Allocates only if the neighbour
  * list outgrows its capacity.  Synchronises the stream once per step (to

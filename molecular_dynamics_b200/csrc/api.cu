@@ -112,6 +112,7 @@ void free_atoms(reann_ctx *c) {
     dfree(c->d_F); dfree(c->d_Epart); dfree(c->d_stage_f); dfree(c->d_stage_i); dfree(c->d_stage_x);
     dfree(c->d_stage_v); dfree(c->d_stage_e); dfree(c->d_x); dfree(c->d_v); dfree(c->d_diag);
     dfree(c->d_last_x); dfree(c->d_last_v); dfree(c->d_dd_sub); dfree(c->d_tanhd);
+    dfree(c->d_last_x_alt); dfree(c->d_last_v_alt); dfree(c->d_in_x); dfree(c->d_in_v);
     c->md_valid = false;
     c->slots_alloc = 0;
     c->n_alloc = 0;
@@ -149,6 +150,10 @@ reann_status ensure_atoms(reann_ctx *c, int64_t n) {
     CK(dalloc(&c->d_diag, N * (size_t)std::max(c->DR, c->NA)));
     CK(dalloc(&c->d_last_x, 3 * N));
     CK(dalloc(&c->d_last_v, 3 * N));
+    CK(dalloc(&c->d_last_x_alt, 3 * N));
+    CK(dalloc(&c->d_last_v_alt, 3 * N));
+    CK(dalloc(&c->d_in_x, 3 * N));
+    CK(dalloc(&c->d_in_v, 3 * N));
     if (c->dd) CK(dalloc(&c->d_dd_sub, N));
     if (c->cfg.mlp_precision == 0 && tc32_supported(c))
         CK(dalloc(&c->d_tanhd, (size_t)std::max(c->T - 1, 1) * N * (size_t)(c->H1 + c->H2)));
@@ -693,6 +698,9 @@ extern "C" reann_status reann_destroy(reann_ctx *c) {
     for (auto ev : c->o_ev)
         if (ev) cudaEventDestroy(ev);
     if (c->o_stream) cudaStreamDestroy(c->o_stream);
+    for (auto ev : c->i_ev)
+        if (ev) cudaEventDestroy(ev);
+    if (c->i_stream) cudaStreamDestroy(c->i_stream);
     delete c;
     return REANN_OK;
 }
@@ -790,56 +798,18 @@ struct NvtArgs {
 // Velocity Verlet, with the thermostat applied after each step's closing half
 // kick when nvt is given.  The d_E slots: [0] energy, [1] kinetic energy,
 // [2] the step's rescaling factor, [3] thermostat work of this call.
-static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, const double *mass_amu,
-                           reann_md_stats *stats, reann_stream stream, const NvtArgs *nvt) {
-    if (!c) return REANN_ERR_ARG;
-    if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
-    if (c->halo) return fail(c, REANN_ERR_STATE, "MD steps over a halo plan are not provided (energy+forces only)");
-    if (nsteps < 0 || !std::isfinite(dt_fs) || !mass_amu || (c->n > 0 && (!x || !v)))
-        return fail(c, REANN_ERR_ARG, "invalid arguments");
-    BussiParams B{};
-    if (nvt) {
-        if (!(nvt->temperature > 0) || !std::isfinite(nvt->temperature) || !(nvt->tau >= 0))
-            return fail(c, REANN_ERR_ARG, "temperature must be positive and finite, tau non-negative");
-        if (c->n < 2) return fail(c, REANN_ERR_ARG, "the thermostat needs at least two atoms");
-        if (nsteps > 0 && (!nvt->noise || is_device_ptr(nvt->noise)))
-            return fail(c, REANN_ERR_ARG, "noise must be a host array of two numbers per step");
-        for (int64_t k = 0; k < 2 * (int64_t)nsteps; ++k)
-            if (!std::isfinite(nvt->noise[k]) || (k % 2 == 1 && nvt->noise[k] < 0))
-                return fail(c, REANN_ERR_ARG, "noise must be finite, with S >= 0");
-        B.nf = (double)(3 * c->n - 3);
-        B.kt = 0.5 * B.nf * KB_EV * nvt->temperature;
-        B.c = nvt->tau > 0 ? std::exp(-dt_fs / nvt->tau) : 0.0;
-    }
-    double inv_mass[MAX_ELEMENTS], mass[MAX_ELEMENTS];
-    for (int e = 0; e < c->ne; ++e) {
-        if (!(mass_amu[e] > 0) || !std::isfinite(mass_amu[e])) return fail(c, REANN_ERR_ARG, "masses must be positive");
-        mass[e] = mass_amu[e];
-        inv_mass[e] = 1.0 / mass_amu[e];
-    }
-    DeviceGuard guard(c->device);
-    cudaStream_t s = (cudaStream_t)stream;
+// The steps of one MD call, from the resident state (resume) or from the
+// caller-order state in d_stage_x / d_stage_v; results to the caller's x, v.
+// spec: the caller's x and v are being read in and compared on i_stream (a
+// continuing call); writes to them wait for that.
+static reann_status md_steps(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, bool x_dev, bool v_dev,
+                             const double *mass, const double *inv_mass, reann_md_stats *stats, cudaStream_t s,
+                             const NvtArgs *nvt, BussiParams B, bool resume, bool spec) {
     const int64_t n = c->n;
     const size_t bytes3 = sizeof(double) * 3 * (size_t)n;
-    bool x_dev = is_device_ptr(x), v_dev = is_device_ptr(v);
     reann_status st;
     int64_t rebuilds = 0;
     int32_t done = 0;
-    bool resume = false;
-    if (n > 0) {
-        CK(cudaMemcpyAsync(c->d_stage_x, x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
-        CK(cudaMemcpyAsync(c->d_stage_v, v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
-        if (c->md_valid) {
-            // a continuation: the caller passes back exactly the state the last
-            // call returned, so the resident internal state and forces are reused
-            CK(cudaMemsetAsync(c->d_status + 2, 0, sizeof(int), s));
-            CK(launch_md_compare(c, c->d_stage_x, c->d_stage_v, c->d_status + 2, s));
-            CK(cudaMemcpyAsync(c->h_status + 2, c->d_status + 2, sizeof(int), cudaMemcpyDeviceToHost, s));
-            CK(sync_stream(c, s));
-            resume = c->h_status[2] == 0 && c->md_dt == dt_fs &&
-                     std::equal(mass, mass + c->ne, c->md_mass);
-        }
-    }
     c->md_valid = false;
     CK(cudaMemsetAsync(c->d_status, 0, sizeof(int) * 2, s));
     if (!resume) {
@@ -963,6 +933,8 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
             CK(launch_md_scatter(c, c->d_last_x, nullptr, nullptr, s));
             CK(cudaEventRecord(c->o_ev[0], s));
             CK(cudaStreamWaitEvent(c->o_stream, c->o_ev[0], 0));
+            // a continuing call: the caller's x must have been read in before it is written
+            if (spec) CK(cudaStreamWaitEvent(c->o_stream, c->i_ev[1], 0));
             x_wait.s = c->o_stream;
             CK(cudaMemcpyAsync(x, c->d_last_x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyDeviceToHost,
                                c->o_stream));
@@ -979,6 +951,11 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
     CK(launch_kinetic(c, mass, c->d_E + 1, s));
     CK(cudaMemcpyAsync(c->h_E, c->d_E, sizeof(double) * 2, cudaMemcpyDeviceToHost, s));
     CK(cudaMemcpyAsync(c->h_E + 4, c->d_E + 3, sizeof(double), cudaMemcpyDeviceToHost, s));
+    if (spec) {
+        // a continuing call: the caller's x and v are read in and compared before they are written
+        CK(cudaStreamWaitEvent(s, c->i_ev[2], 0));
+        CK(cudaMemcpyAsync(c->h_status + 2, c->d_status + 2, sizeof(int), cudaMemcpyDeviceToHost, s));
+    }
     if (n > 0) {
         // final state in caller order: kept for continuation checks, then copied out
         const bool x_out = x_wait.s != nullptr;
@@ -1007,6 +984,94 @@ static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x
         stats->e_thermostat = c->h_E[4];
     }
     return check_status(c, c->h_status[0] & ~ST_SKIN);
+}
+
+static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, const double *mass_amu,
+                           reann_md_stats *stats, reann_stream stream, const NvtArgs *nvt) {
+    if (!c) return REANN_ERR_ARG;
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "reann_build_neighbors must come first");
+    if (c->halo) return fail(c, REANN_ERR_STATE, "MD steps over a halo plan are not provided (energy+forces only)");
+    if (nsteps < 0 || !std::isfinite(dt_fs) || !mass_amu || (c->n > 0 && (!x || !v)))
+        return fail(c, REANN_ERR_ARG, "invalid arguments");
+    BussiParams B{};
+    if (nvt) {
+        if (!(nvt->temperature > 0) || !std::isfinite(nvt->temperature) || !(nvt->tau >= 0))
+            return fail(c, REANN_ERR_ARG, "temperature must be positive and finite, tau non-negative");
+        if (c->n < 2) return fail(c, REANN_ERR_ARG, "the thermostat needs at least two atoms");
+        if (nsteps > 0 && (!nvt->noise || is_device_ptr(nvt->noise)))
+            return fail(c, REANN_ERR_ARG, "noise must be a host array of two numbers per step");
+        for (int64_t k = 0; k < 2 * (int64_t)nsteps; ++k)
+            if (!std::isfinite(nvt->noise[k]) || (k % 2 == 1 && nvt->noise[k] < 0))
+                return fail(c, REANN_ERR_ARG, "noise must be finite, with S >= 0");
+        B.nf = (double)(3 * c->n - 3);
+        B.kt = 0.5 * B.nf * KB_EV * nvt->temperature;
+        B.c = nvt->tau > 0 ? std::exp(-dt_fs / nvt->tau) : 0.0;
+    }
+    double inv_mass[MAX_ELEMENTS], mass[MAX_ELEMENTS];
+    for (int e = 0; e < c->ne; ++e) {
+        if (!(mass_amu[e] > 0) || !std::isfinite(mass_amu[e])) return fail(c, REANN_ERR_ARG, "masses must be positive");
+        mass[e] = mass_amu[e];
+        inv_mass[e] = 1.0 / mass_amu[e];
+    }
+    DeviceGuard guard(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n = c->n;
+    const size_t bytes3 = sizeof(double) * 3 * (size_t)n;
+    const bool x_dev = is_device_ptr(x), v_dev = is_device_ptr(v);
+    // A continuation -- the caller passes back exactly the state the last call
+    // returned, with the same time step and masses -- starts from the resident
+    // state and forces at once; the caller's x and v are moved in and compared
+    // with that state on a second stream meanwhile, and the call starts again
+    // from them if they differ.
+    const bool spec = n > 0 && c->md_valid && c->md_dt == dt_fs && std::equal(mass, mass + c->ne, c->md_mass);
+    struct StreamWait {
+        cudaStream_t s = nullptr;
+        ~StreamWait() {
+            if (s) cudaStreamSynchronize(s);
+        }
+    } in_wait;
+    if (spec) {
+        if (!c->i_stream) {
+            CK(cudaStreamCreateWithFlags(&c->i_stream, cudaStreamNonBlocking));
+            for (auto &ev : c->i_ev) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+        }
+        CK(cudaMemsetAsync(c->d_status + 2, 0, sizeof(int), s));
+        CK(cudaEventRecord(c->i_ev[0], s));
+        CK(cudaStreamWaitEvent(c->i_stream, c->i_ev[0], 0));
+        in_wait.s = c->i_stream;
+        CK(cudaMemcpyAsync(c->d_in_x, x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                           c->i_stream));
+        CK(cudaEventRecord(c->i_ev[1], c->i_stream));
+        CK(cudaMemcpyAsync(c->d_in_v, v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                           c->i_stream));
+        CK(launch_md_compare(c, c->d_in_x, c->d_in_v, c->d_last_x, c->d_last_v, c->d_status + 2, c->i_stream));
+        CK(cudaEventRecord(c->i_ev[2], c->i_stream));
+        // this call's result goes to the other buffer pair; the comparison reads the last one
+        std::swap(c->d_last_x, c->d_last_x_alt);
+        std::swap(c->d_last_v, c->d_last_v_alt);
+    } else if (n > 0) {
+        CK(cudaMemcpyAsync(c->d_stage_x, x, bytes3, x_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
+        CK(cudaMemcpyAsync(c->d_stage_v, v, bytes3, v_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, s));
+    }
+    const reann_counters counters0 = c->counters;
+    reann_status st = md_steps(c, nsteps, dt_fs, x, v, x_dev, v_dev, mass, inv_mass, stats, s, nvt, B, spec, spec);
+    if (!spec) return st;
+    CK(cudaStreamSynchronize(c->i_stream));
+    in_wait.s = nullptr;
+    if (st == REANN_OK && c->h_status[2] == 0) return st;
+    if (st != REANN_OK) {
+        // the steps stopped early: was the resident state the caller's?
+        CK(cudaMemcpyAsync(c->h_status + 2, c->d_status + 2, sizeof(int), cudaMemcpyDeviceToHost, c->i_stream));
+        CK(cudaStreamSynchronize(c->i_stream));
+        if (c->h_status[2] == 0) return st;
+    }
+    // the caller's state differs from the resident one: start again from the copy read in
+    // (the caller's x may already hold the discarded run's positions)
+    c->counters = counters0;
+    c->md_valid = false;
+    CK(cudaMemcpyAsync(c->d_stage_x, c->d_in_x, bytes3, cudaMemcpyDeviceToDevice, s));
+    CK(cudaMemcpyAsync(c->d_stage_v, c->d_in_v, bytes3, cudaMemcpyDeviceToDevice, s));
+    return md_steps(c, nsteps, dt_fs, x, v, x_dev, v_dev, mass, inv_mass, stats, s, nvt, B, false, false);
 }
 
 extern "C" reann_status reann_md_step(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v,

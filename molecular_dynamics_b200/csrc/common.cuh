@@ -207,8 +207,16 @@ struct reann_ctx {
     float *d_diag = nullptr;       // [n][max(D, NA)] diagnostics scratch
     // MD state in internal order
     double *d_x = nullptr, *d_v = nullptr;  // [n][3]
-    // state returned by the last MD call (caller order), for continuation checks
+    // state returned by the last MD call (caller order), for continuation checks,
+    // and the buffer pair the next call writes (swapped per continuing call, so a
+    // call's comparison reads the previous result while its own steps run)
     double *d_last_x = nullptr, *d_last_v = nullptr;
+    double *d_last_x_alt = nullptr, *d_last_v_alt = nullptr;
+    // a continuing call's copy of the caller's x and v, moved in and compared on
+    // i_stream while the steps run (i_ev: start, caller's x read, comparison done)
+    double *d_in_x = nullptr, *d_in_v = nullptr;
+    cudaStream_t i_stream = nullptr;
+    cudaEvent_t i_ev[3] = {nullptr, nullptr, nullptr};
     bool md_valid = false;
     double md_dt = 0.0;
     double md_mass[reann::MAX_ELEMENTS] = {};

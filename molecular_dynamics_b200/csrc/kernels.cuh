@@ -89,7 +89,8 @@ cudaError_t launch_thermostat(reann_ctx *c, const double *mass, const BussiParam
 // the device-side step loop's gate (md.cu)
 cudaError_t launch_loop_gate(reann_ctx *c, cudaGraphConditionalHandle h_while, cudaGraphConditionalHandle h_step,
                              cudaStream_t s);
-cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s);
+cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, const double *lx, const double *lv,
+                              int *flag, cudaStream_t s);
 cudaError_t launch_wrap_state(reann_ctx *c, double *d_x_caller, float *d_pos_caller, cudaStream_t s);
 cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s);
 

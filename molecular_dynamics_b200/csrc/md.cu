@@ -171,13 +171,14 @@ __global__ void k_md_compare(int64_t m, const unsigned long long *__restrict__ x
     if (__any_sync(0xffffffffu, diff) && (threadIdx.x & 31) == 0) atomicOr(flag, 1);
 }
 
-cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, int *flag, cudaStream_t s) {
+cudaError_t launch_md_compare(reann_ctx *c, const double *x, const double *v, const double *lx, const double *lv,
+                              int *flag, cudaStream_t s) {
     int64_t m = 3 * c->n;
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (m > 0)
         k_md_compare<<<blocks(m, 256), 256, 0, s>>>(m, (const unsigned long long *)x, (const unsigned long long *)v,
-                                                    (const unsigned long long *)c->d_last_x,
-                                                    (const unsigned long long *)c->d_last_v, flag);
+                                                    (const unsigned long long *)lx, (const unsigned long long *)lv,
+                                                    flag);
     return cudaGetLastError();
 }
 

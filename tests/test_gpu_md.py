@@ -94,6 +94,48 @@ def test_split_run_equals_single_run():
     assert torch.equal(x1, x2) and torch.equal(v1, v2)
 
 
+def test_split_run_with_host_state_equals_single_run():
+    # a continuing call starts from the resident state while the caller's host
+    # arrays are moved in and compared on a second stream
+    p, pos, types, box = small("hea")
+    v0 = synth.maxwell_boltzmann(p, types)
+    x1, v1 = pos.astype(np.float64).copy(), v0.copy()
+    _ctx(p, pos, types, box).reann_md_step(8, 1.0, x1, v1, p.masses)
+    x2, v2 = pos.astype(np.float64).copy(), v0.copy()
+    ctx = _ctx(p, pos, types, box)
+    for k in (3, 1, 4):
+        ctx.reann_md_step(k, 1.0, x2, v2, p.masses)
+    assert np.array_equal(x1, x2) and np.array_equal(v1, v2)
+
+
+@pytest.mark.parametrize("changed", ["x", "v"])
+@pytest.mark.parametrize("where", ["host", "device"])
+def test_continuation_with_a_changed_state_starts_from_it(changed, where):
+    # the caller passes back a state other than the one the last call returned:
+    # the call must run from the caller's state, as a fresh context does
+    torch = torch_cuda()
+    p, pos, types, box = small("chon")
+    v0 = synth.maxwell_boltzmann(p, types)
+    ctx = _ctx(p, pos, types, box)
+    x, v = pos.astype(np.float64).copy(), v0.copy()
+    ctx.reann_md_step(3, 0.5, x, v, p.masses)
+    if changed == "x":
+        x[7] += np.array([0.013, -0.021, 0.008])
+    else:
+        v[11] *= -1.0
+    xr, vr = x.copy(), v.copy()
+    fresh = _ctx(p, xr.astype(np.float32), types, box)
+    fresh.reann_md_step(4, 0.5, xr, vr, p.masses)
+    if where == "host":
+        ctx.reann_md_step(4, 0.5, x, v, p.masses)
+        xo, vo = x, v
+    else:
+        xd, vd = torch.from_numpy(x).cuda(), torch.from_numpy(v).cuda()
+        ctx.reann_md_step(4, 0.5, xd, vd, p.masses)
+        xo, vo = xd.cpu().numpy(), vd.cpu().numpy()
+    assert np.array_equal(xo, xr) and np.array_equal(vo, vr)
+
+
 def test_host_state_equals_device_state():
     torch = torch_cuda()
     p, pos, types, box = small("chon")
