@@ -88,6 +88,7 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 // front of the row's slot (same offsets as the full list), each with its
 // displacement and distance (dx, dy, dz, r), which every edge pass of the
 // evaluation then reads instead of recomputing.
+template <bool DR>   // DR: also the distance rounding residuals (fp32-accurate paths)
 __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
                     const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
                     act_col[o] = j[b];
                     float r = sqrtf(r2);
-                    if (act_dr) {
+                    if (DR) {
                         // the fp32-accurate paths: r from the exact displacement of the
                         // fp32 positions, correctly rounded, and its rounding residual
                         double e[3] = {(double)pj[b].x - (double)pi.x, (double)pj[b].y - (double)pi.y,
@@ -164,10 +165,14 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     REANN_TIMED(c, REANN_K_ACTIVE, s);
     // one resident wave (8 blocks of 128 threads per SM at <= 64 registers)
     const unsigned grid = (unsigned)std::min<int64_t>((c->n + 3) / 4, (int64_t)c->sm_count * 8);
-    k_active<<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row,
-                                                        c->dd ? c->d_col_dd : c->d_col, c->d_act_cnt,
-                                                            c->d_act_col, c->d_act_geo, c->d_act_dr, P,
-                                                            (unsigned long long *)(c->d_i64 + 3));
+    const int *col = c->dd ? c->d_col_dd : c->d_col;
+    unsigned long long *total = (unsigned long long *)(c->d_i64 + 3);
+    if (c->d_act_dr)
+        k_active<true><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt, c->d_act_col,
+                                            c->d_act_geo, c->d_act_dr, P, total);
+    else
+        k_active<false><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt, c->d_act_col,
+                                             c->d_act_geo, nullptr, P, total);
     return cudaGetLastError();
 }
 
