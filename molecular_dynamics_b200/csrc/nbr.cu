@@ -216,12 +216,25 @@ __device__ __forceinline__ int axis_stencil(int c, int m, int out[3]) {
     return 3;
 }
 
-template <bool FILL>
+// Rows of the list, one thread per atom walking the stencil cells (e, x, y, z
+// ascending) and, inside a cell, ascending j.  Small systems, whose atoms
+// alone leave most of the GPU idle, take a group of GL lanes per atom instead:
+// the group tests GL candidates of a cell at once (a cell's atoms are
+// contiguous in internal order), and a ballot counts the hits and, in the fill
+// pass, places them in candidate order -- the same columns in the same order.
+// (Measured per build: 3,000 water molecules' atoms 0.63 -> 0.12 ms with 32
+// lanes; on the 108k-1M-atom systems one thread per atom is fastest.)
+template <bool FILL, int GL>
 __global__ void __launch_bounds__(128) k_nbr(int n, const float4 *__restrict__ pos, const int *__restrict__ bin_start,
                                              BinParams B, const int *__restrict__ row, int *__restrict__ cnt,
                                              int *__restrict__ col) {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    static_assert(GL >= 1 && GL <= 32 && (32 % GL) == 0, "lane groups tile a warp");
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i = t / GL, sub = t % GL;
+    // a group's lanes share i, so a group is either entirely in range or entirely out
     if (i >= n) return;
+    const int gbase = (threadIdx.x & 31) & ~(GL - 1);
+    const unsigned gmask = GL == 32 ? 0xffffffffu : (((1u << GL) - 1u) << gbase);
     float4 pi = pos[i];
     int sx[3], sy[3], sz[3];
     int nx = axis_stencil(cell_axis(pi.x, B.box[0], B.m[0]), B.m[0], sx);
@@ -236,21 +249,30 @@ __global__ void __launch_bounds__(128) k_nbr(int n, const float4 *__restrict__ p
             for (int b = 0; b < ny; ++b)
                 for (int d = 0; d < nz; ++d) {
                     int k = e * B.ncell + (sx[a] * B.m[1] + sy[b]) * B.m[2] + sz[d];
-                    int j1 = bin_start[k + 1];
-                    for (int j = bin_start[k]; j < j1; ++j) {
-                        if (j == i) continue;
-                        if (list_r2(pi, pos[j], B) < B.thr) {
-                            if (FILL) col[o + c] = j;
-                            ++c;
+                    const int j1 = bin_start[k + 1];
+                    if (GL == 1) {
+                        for (int j = bin_start[k]; j < j1; ++j) {
+                            if (j == i) continue;
+                            if (list_r2(pi, pos[j], B) < B.thr) {
+                                if (FILL) col[o + c] = j;
+                                ++c;
+                            }
                         }
+                        continue;
+                    }
+                    for (int base = bin_start[k]; base < j1; base += GL) {
+                        const int j = base + sub;
+                        const bool hit = j < j1 && j != i && list_r2(pi, pos[j], B) < B.thr;
+                        const unsigned gb = GL == 32 ? __ballot_sync(gmask, hit)
+                                                     : (__ballot_sync(gmask, hit) >> gbase) & ((1u << GL) - 1u);
+                        if (FILL && hit) col[o + c + __popc(gb & ((1u << sub) - 1u))] = j;
+                        c += __popc(gb);
                     }
                 }
     }
-    if (!FILL) cnt[i] = c;
+    if (!FILL && sub == 0) cnt[i] = c;
 }
 
-template __global__ void k_nbr<false>(int, const float4 *, const int *, BinParams, const int *, int *, int *);
-template __global__ void k_nbr<true>(int, const float4 *, const int *, BinParams, const int *, int *, int *);
 
 __global__ void k_row_max(int n, const int *__restrict__ cnt, int64_t *__restrict__ out) {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -282,6 +304,30 @@ __global__ void k_max_disp(int n, const float4 *__restrict__ pos, const float4 *
 
 static inline unsigned blocks(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
 
+// lanes per atom of the list kernels: enough threads for about 512 per SM
+static int nbr_lanes(const reann_ctx *c, int64_t n) {
+    int gl = 1;
+    while (gl < 32 && n * gl < (int64_t)c->sm_count * 512) gl *= 2;
+    return gl;
+}
+
+template <bool FILL>
+static void launch_nbr(const reann_ctx *c, int64_t n, const BinParams &B, const int *row, int *cnt, int *col,
+                       cudaStream_t s) {
+    const int gl = nbr_lanes(c, n);
+#define REANN_NBR(GLV) \
+    k_nbr<FILL, GLV><<<blocks(n * GLV, 128), 128, 0, s>>>((int)n, c->d_pos, c->d_bin_start, B, row, cnt, col)
+    switch (gl) {
+        case 1: REANN_NBR(1); break;
+        case 2: REANN_NBR(2); break;
+        case 4: REANN_NBR(4); break;
+        case 8: REANN_NBR(8); break;
+        case 16: REANN_NBR(16); break;
+        default: REANN_NBR(32); break;
+    }
+#undef REANN_NBR
+}
+
 cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_types_caller, cudaStream_t s) {
     BinParams B = make_bin_params(c);
     int64_t n = c->n;
@@ -300,7 +346,7 @@ cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_t
                                                                        c->d_perm);
         k_gather_pos<<<blocks(n, 256), 256, 0, s>>>(n, d_pos_caller, d_types_caller, c->d_perm, c->d_pos,
                                                     c->d_pos_build, c->d_inv);
-        k_nbr<false><<<blocks(n, 128), 128, 0, s>>>((int)n, c->d_pos, c->d_bin_start, B, nullptr, c->d_cnt, nullptr);
+        launch_nbr<false>(c, n, B, nullptr, c->d_cnt, nullptr, s);
     }
     if ((e = scan_exclusive(c->d_cnt, c->d_row, n, c->d_i64 + 1, c->d_scan_tmp, s))) return e;
     if ((e = cudaMemsetAsync(c->d_i64 + 2, 0, sizeof(int64_t), s))) return e;
@@ -312,8 +358,7 @@ cudaError_t launch_fill(reann_ctx *c, cudaStream_t s) {
     BinParams B = make_bin_params(c);
     REANN_TIMED(c, REANN_K_NEIGHBORS, s);
     if (c->n > 0)
-        k_nbr<true><<<blocks(c->n, 128), 128, 0, s>>>((int)c->n, c->d_pos, c->d_bin_start, B, c->d_row, nullptr,
-                                                       c->d_col);
+        launch_nbr<true>(c, c->n, B, c->d_row, nullptr, c->d_col, s);
     return cudaGetLastError();
 }
 
