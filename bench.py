@@ -95,6 +95,18 @@ class ClockSampler:
         self.proc = None
         self.t0 = self.t1 = None
 
+    def wait_ready(self, timeout: float = 5.0):
+        """Block until the sampler has written its first sample (nvidia-smi takes
+        a moment to start), so that short timed regions are covered."""
+        if self.proc is None:
+            return
+        t_end = time.time() + timeout
+        while time.time() < t_end:
+            self.file.flush()
+            if os.path.getsize(self.file.name) > 0:
+                return
+            time.sleep(0.02)
+
     def mark_begin(self):
         import datetime
         self.t0 = datetime.datetime.now()
@@ -469,6 +481,7 @@ def main():
     # sampler starts before it so that samples flow through the timed region
     clocks = ClockSampler(info.local)
     clocks.start()
+    clocks.wait_ready()
     md(args.warmup, x, v)
     torch.cuda.synchronize()
 

@@ -214,6 +214,17 @@ __device__ __forceinline__ float2 exp2_sfu(float2 x) {
     return y;
 }
 
+// Row splitting for small systems (SPLIT): a centre's row is walked by S
+// adjacent slots of one warp (part p takes entries p, p + S, ...), whose
+// partial sums are then added in a fixed butterfly over the slots' lanes, so a
+// system with too few atoms to fill the GPU still does.  S is a power of two
+// with S * LPE <= 32 (N_phi = 8 only); S = 1 is the plain one-slot walk.
+template <class T>
+__device__ __forceinline__ T parts_sum(T v, int lpe, int S) {
+    for (int off = lpe; off < lpe * S; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
 template <int NP>
 struct Lanes {
     static constexpr int LPE = NP / 2;
@@ -232,14 +243,14 @@ struct Lanes {
 template <bool ACC64>
 using acc_t = typename std::conditional<ACC64, double, float>::type;
 
-template <int NP, bool ACC64>
+template <int NP, bool ACC64, bool SPLIT>
 __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restrict__ row,
                                                      const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                      const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                      const float *__restrict__ coef, const float *__restrict__ C0,
                                                      int ne, float *__restrict__ A_out, float *__restrict__ rho_out,
                                                      const float *__restrict__ shift, const float *__restrict__ act_dr,
-                                                     EdgeParams P) {
+                                                     EdgeParams P, int S) {
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
     __shared__ __align__(16) float sC0[MAX_ELEMENTS * D];
@@ -247,8 +258,10 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
-    if (lane >= Ln::USED || i >= n) return;
+    const int gs = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const int i = SPLIT ? gs / S : gs, part = SPLIT ? gs - i * S : 0, stride = SPLIT ? S : 1;
+    const bool live = lane < Ln::USED && i < n;
+    if (!SPLIT && !live) return;   // split rows: every lane takes part in the parts' sum
     const int n0 = 2 * sub;
 
     using R = acc_t<ACC64>;
@@ -258,7 +271,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = R(0);
     const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
-    const int q0 = row[i], q1 = q0 + act_cnt[i];
+    const int q0 = live ? row[i] + part : 0, q1 = live ? row[i] + act_cnt[i] : 0;
     int j_next = q0 < q1 ? act_col[q0] : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (!ACC64) {
@@ -267,12 +280,12 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc2[u] = bc2(0.f);
         const float2 NMU = make_float2(-mh[0], -mh[1]);
-        for (int q = q0; q < q1; ++q) {
+        for (int q = q0; q < q1; q += stride) {
             const int j = j_next;
             const float4 g = g_next;
-            if (q + 1 < q1) {
-                j_next = act_col[q + 1];
-                g_next = act_geo[q + 1];
+            if (q + stride < q1) {
+                j_next = act_col[q + stride];
+                g_next = act_geo[q + stride];
             }
             const float r = g.w;
             const float fc = cutoff_cos2(r * P.th_hi);
@@ -304,15 +317,15 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
     } else {
         const float ml[2] = {P.mu_lo[n0], P.mu_lo[n0 + 1]};
         float dr_next = act_dr && q0 < q1 ? act_dr[q0] : 0.f;
-        for (int q = q0; q < q1; ++q) {
+        for (int q = q0; q < q1; q += stride) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 g = g_next;         // dx, dy, dz, r
             const float dr = dr_next;        // r - fp32(r)
-            if (q + 1 < q1) {
-                j_next = act_col[q + 1];
-                g_next = act_geo[q + 1];
-                if (act_dr) dr_next = act_dr[q + 1];
+            if (q + stride < q1) {
+                j_next = act_col[q + stride];
+                g_next = act_geo[q + stride];
+                if (act_dr) dr_next = act_dr[q + stride];
             }
             const float r = g.w;
             const float fc = cutoff_cos2(fmaf(r, P.th_hi, r * P.th_lo));
@@ -343,6 +356,13 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             }
         }
     }
+    if (SPLIT) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int u = 0; u < NT; ++u) acc[m][u] = parts_sum(acc[m][u], LPE, S);
+        if (!live || part != 0) return;
+    }
     float *Ao = A_out + (int64_t)i * NA;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
@@ -372,13 +392,13 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 // values (radial-major lane order) as five float4 (the slot's four lanes read
 // 64 contiguous bytes per load).  dE/dc_k of the lane's radial indices needs no reduction; the force
 // is summed over the slot's lanes in a fixed order.
-template <int NP, bool HAS_DC>
+template <int NP, bool HAS_DC, bool SPLIT>
 __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restrict__ row,
                                                   const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                                                   const float4 *__restrict__ act_geo, const float4 *__restrict__ pos,
                                                   const float *__restrict__ coef, const float *__restrict__ C0, int ne,
                                                   const float *__restrict__ G, float *__restrict__ F,
-                                                  float *__restrict__ dc, bool accumulate, EdgeParams P) {
+                                                  float *__restrict__ dc, bool accumulate, EdgeParams P, int S) {
     static_assert(!g_pairs(NP, HAS_DC ? 1 : 0), "scalar backward reads the radial-major lane order");
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
@@ -387,7 +407,8 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const int gs = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const int i = SPLIT ? gs / S : gs, part = SPLIT ? gs - i * S : 0, stride = SPLIT ? S : 1;
     const bool live = lane < Ln::USED && i < n;
     const int n0 = 2 * sub;
 
@@ -413,19 +434,19 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
         // the backward takes the constants' fp32 values: its rounding shifts forces by
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
-        const int q0 = row[i], q1 = q0 + act_cnt[i];
+        const int q0 = row[i] + part, q1 = row[i] + act_cnt[i];
         // the edge list takes ordinary cached loads: its 16-byte entries share
         // 32-byte sectors with the next edge's, and evict-first loads made the
         // second read of a sector go back to DRAM (1.6x the traffic, no faster)
         int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
         float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
-        for (int q = q0; q < q1; ++q) {
+        for (int q = q0; q < q1; q += stride) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
-            if (q + 1 < q1) {
-                j_next = __ldg(act_col + q + 1);
-                geo_next = __ldg(act_geo + q + 1);
+            if (q + stride < q1) {
+                j_next = __ldg(act_col + q + stride);
+                geo_next = __ldg(act_geo + q + stride);
             }
             const float3 d = make_float3(geo.x, geo.y, geo.z);
             const float r = geo.w;
@@ -501,6 +522,15 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
             }
         }
     }
+    if (SPLIT) {
+        fx = parts_sum(fx, LPE, S);
+        fy = parts_sum(fy, LPE, S);
+        fz = parts_sum(fz, LPE, S);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int l = 0; l < 3; ++l) dck[m][l] = parts_sum(dck[m][l], LPE, S);
+    }
     // force: sum over the slot's lanes (sub 0 .. LPE-1) in a fixed order
     const int base = (lane / LPE) * LPE;
     float sx = 0.f, sy = 0.f, sz = 0.f;
@@ -511,7 +541,7 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
         sy += __shfl_sync(0xffffffffu, fy, src);
         sz += __shfl_sync(0xffffffffu, fz, src);
     }
-    if (!live) return;
+    if (!live || part != 0) return;
     if (sub == 0) {
         float *Fo = F + 3 * (int64_t)i;
         if (accumulate) {
@@ -541,12 +571,12 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
 // packed form is faster in every layer (108k atoms: 0.49 -> 0.45 ms, and 0.40
 // ms at five blocks per SM, where its 96 registers do not spill; first layer
 // 0.33 -> 0.29 ms at six).
-template <int NP, bool HAS_DC>
+template <int NP, bool HAS_DC, bool SPLIT>
 __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
     k_edge_bwd_pk(int n, const int *__restrict__ row, const int *__restrict__ act_cnt, const int *__restrict__ act_col,
                   const float4 *__restrict__ act_geo, const float4 *__restrict__ pos, const float *__restrict__ coef,
                   const float *__restrict__ C0, int ne, const float *__restrict__ G, float *__restrict__ F,
-                  float *__restrict__ dc, bool accumulate, EdgeParams P) {
+                  float *__restrict__ dc, bool accumulate, EdgeParams P, int S) {
     static_assert(g_pairs(NP, HAS_DC ? 1 : 0), "packed backward reads the pair lane order");
     using Ln = Lanes<NP>;
     constexpr int D = 3 * NP, NA = NP * NT, LPE = Ln::LPE;
@@ -555,7 +585,8 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slot = lane / LPE, sub = lane % LPE;
-    const int i = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const int gs = blockIdx.x * Ln::CPB + warp * Ln::CPW + slot;
+    const int i = SPLIT ? gs / S : gs, part = SPLIT ? gs - i * S : 0, stride = SPLIT ? S : 1;
     const bool live = lane < Ln::USED && i < n;
     const int n0 = 2 * sub;
 
@@ -583,19 +614,19 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
         // the backward takes the constants' fp32 values: its rounding shifts forces by
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float2 nmu = make_float2(-P.mu_hi[n0], -P.mu_hi[n0 + 1]);
-        const int q0 = row[i], q1 = q0 + act_cnt[i];
+        const int q0 = row[i] + part, q1 = row[i] + act_cnt[i];
         // the edge list takes ordinary cached loads: its 16-byte entries share
         // 32-byte sectors with the next edge's, and evict-first loads made the
         // second read of a sector go back to DRAM (1.6x the traffic, no faster)
         int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
         float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
-        for (int q = q0; q < q1; ++q) {
+        for (int q = q0; q < q1; q += stride) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
-            if (q + 1 < q1) {
-                j_next = __ldg(act_col + q + 1);
-                geo_next = __ldg(act_geo + q + 1);
+            if (q + stride < q1) {
+                j_next = __ldg(act_col + q + stride);
+                geo_next = __ldg(act_geo + q + stride);
             }
             const float r = geo.w;
             const float inv_r = __fdividef(1.0f, r);
@@ -689,8 +720,16 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
 #undef GJ2
         }
     }
-    // force: the lane's pair, then the slot's lanes (sub 0 .. LPE-1), in a fixed order
-    const float lx = fx.x + fx.y, ly = fy.x + fy.y, lz = fz.x + fz.y;
+    // force: the lane's pair, then (split rows) the parts, then the slot's lanes
+    // (sub 0 .. LPE-1), in a fixed order
+    float lx = fx.x + fx.y, ly = fy.x + fy.y, lz = fz.x + fz.y;
+    if (SPLIT) {
+        lx = parts_sum(lx, LPE, S);
+        ly = parts_sum(ly, LPE, S);
+        lz = parts_sum(lz, LPE, S);
+#pragma unroll
+        for (int l = 0; l < 3; ++l) dck[l] = make_float2(parts_sum(dck[l].x, LPE, S), parts_sum(dck[l].y, LPE, S));
+    }
     const int base = (lane / LPE) * LPE;
     float sx = 0.f, sy = 0.f, sz = 0.f;
 #pragma unroll
@@ -700,7 +739,7 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
         sy += __shfl_sync(0xffffffffu, ly, src);
         sz += __shfl_sync(0xffffffffu, lz, src);
     }
-    if (!live) return;
+    if (!live || part != 0) return;
     if (sub == 0) {
         float *Fo = F + 3 * (int64_t)i;
         if (accumulate) {
@@ -756,6 +795,15 @@ __global__ void __launch_bounds__(256) k_rho_pair(int n, const float *__restrict
 // ---------------------------------------------------------------------------
 // host wrappers
 
+// parts per centre row (row splitting): 1 unless the centres alone would give
+// fewer than four 128-thread blocks per SM (N_phi = 8 only)
+static int edge_parts(const reann_ctx *c, int64_t centres) {
+    if (c->NP != 8) return 1;
+    int S = 1;
+    while (S < 8 && (centres * S + Lanes<8>::CPB - 1) / Lanes<8>::CPB < 4 * (int64_t)c->sm_count) S *= 2;
+    return S;
+}
+
 cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     const int64_t nc = centres(c);
     if (nc == 0) return cudaSuccess;
@@ -766,34 +814,31 @@ cudaError_t launch_density_fwd(reann_ctx *c, int t, cudaStream_t s) {
     float *rho = pair ? nullptr : c->d_rho + (int64_t)t * c->n * c->D;
     const float *shift = c->d_shift + (int64_t)t * c->ne * c->DR;
     const bool acc64 = c->cfg.mlp_precision != 1;   // the fp32-accurate paths
+    const int S = edge_parts(c, nc);
     REANN_TIMED(c, REANN_K_DENSITY, s, pair ? 2 : 1);
-    if (pair) {
-        if (c->NP != 8) return cudaErrorInvalidValue;
-        const int64_t threads = nc * (8 * 9 / 2);
-        if (acc64)
-            k_density_fwd<8, true><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-                (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A,
-                nullptr, shift, c->d_act_dr, P);
-        else
-            k_density_fwd<8, false><<<(unsigned)((nc + Lanes<8>::CPB - 1) / Lanes<8>::CPB), 128, 0, s>>>(
-                (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A,
-                nullptr, shift, c->d_act_dr, P);
-        k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
-            (int)nc, A, c->d_rho + (int64_t)t * c->n * c->DR, c->d_pos, shift, c->ne);
-        return cudaGetLastError();
-    }
-#define REANN_DENSITY(NPV, ACC)                                                                                 \
-    k_density_fwd<NPV, ACC><<<(unsigned)((nc + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(               \
-        (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, rho, shift,    \
-        c->d_act_dr, P)
+    if (pair && c->NP != 8) return cudaErrorInvalidValue;
+#define REANN_DENSITY(NPV, ACC, SPL, RHO)                                                                        \
+    k_density_fwd<NPV, ACC, SPL><<<(unsigned)((nc * S + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(     \
+        (int)nc, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, A, RHO, shift,    \
+        c->d_act_dr, P, S)
     if (c->NP == 8) {
-        if (acc64) REANN_DENSITY(8, true); else REANN_DENSITY(8, false);
+        if (S > 1) {
+            if (acc64) REANN_DENSITY(8, true, true, rho); else REANN_DENSITY(8, false, true, rho);
+        } else {
+            if (acc64) REANN_DENSITY(8, true, false, rho); else REANN_DENSITY(8, false, false, rho);
+        }
     } else if (c->NP == 10) {
-        if (acc64) REANN_DENSITY(10, true); else REANN_DENSITY(10, false);
+        if (acc64) REANN_DENSITY(10, true, false, rho); else REANN_DENSITY(10, false, false, rho);
     } else {
         return cudaErrorInvalidValue;
     }
 #undef REANN_DENSITY
+    if (pair) {
+        // rho from A in k_rho_pair (the density pass wrote A only)
+        const int64_t threads = nc * (8 * 9 / 2);
+        k_rho_pair<8><<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+            (int)nc, A, c->d_rho + (int64_t)t * c->n * c->DR, c->d_pos, shift, c->ne);
+    }
     return cudaGetLastError();
 }
 
@@ -802,16 +847,22 @@ cudaError_t launch_edge_bwd(reann_ctx *c, int t, bool accumulate, cudaStream_t s
     EdgeParams P = make_edge_params(c);
     const float *coef = t == 0 ? nullptr : c->d_coef + (int64_t)t * c->n_slots * c->D;
     const bool has_dc = t >= 1;
+    const int S = edge_parts(c, c->n);
     REANN_TIMED(c, REANN_K_EDGE_BWD, s);
-#define REANN_EDGE_BWD(K, NPV, DC)                                                                               \
-    K<NPV, DC><<<(unsigned)((c->n + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(            \
+#define REANN_EDGE_BWD(K, NPV, DC, SPL)                                                                          \
+    K<NPV, DC, SPL><<<(unsigned)((c->n * S + Lanes<NPV>::CPB - 1) / Lanes<NPV>::CPB), 128, 0, s>>>(                 \
         (int)c->n, c->d_row, c->d_act_cnt, c->d_act_col, c->d_act_geo, c->d_pos, coef, c->d_w, c->ne, c->d_G, c->d_F, \
-        c->d_dc, accumulate, P)
+        c->d_dc, accumulate, P, S)
     // the kernel reads the lane order the networks wrote for this layer (g_pairs)
     if (c->NP == 8) {
-        if (has_dc) REANN_EDGE_BWD(k_edge_bwd, 8, true); else REANN_EDGE_BWD(k_edge_bwd_pk, 8, false);
+        if (S > 1) {
+            if (has_dc) REANN_EDGE_BWD(k_edge_bwd, 8, true, true); else REANN_EDGE_BWD(k_edge_bwd_pk, 8, false, true);
+        } else {
+            if (has_dc) REANN_EDGE_BWD(k_edge_bwd, 8, true, false); else REANN_EDGE_BWD(k_edge_bwd_pk, 8, false, false);
+        }
     } else if (c->NP == 10) {
-        if (has_dc) REANN_EDGE_BWD(k_edge_bwd_pk, 10, true); else REANN_EDGE_BWD(k_edge_bwd_pk, 10, false);
+        if (has_dc) REANN_EDGE_BWD(k_edge_bwd_pk, 10, true, false);
+        else REANN_EDGE_BWD(k_edge_bwd_pk, 10, false, false);
     } else {
         return cudaErrorInvalidValue;
     }
