@@ -219,8 +219,12 @@ reann_status reann_energy_forces(reann_ctx *ctx, const float *pos, double *energ
  * discarded run's x, overwritten by the result of the restart).  Requires a prior
  * reann_build_neighbors for the same atoms and types (positions may have
  * moved; the list is rebuilt at entry).  Allocates only if the neighbour
- * list outgrows its capacity.  Synchronises the stream once per step (to
- * read the rebuild flag) and at the end.  The final x is copied out on a
+ * list outgrows its capacity.  The steps between list rebuilds, but the last
+ * one, run as one device-side graph loop (a WHILE node that stops at a
+ * rebuild or an error), so the stream is synchronised once per such stretch,
+ * once per rebuild, and at the end; with the loop unavailable (eager launches
+ * for profiling, or a runtime without conditional graph nodes) once per step.
+ * The final x is copied out on a
  * library stream during the last step's force evaluation; every return,
  * error returns included, waits for that copy, so x and v are not written
  * after the call returns.  Errors: as reann_energy_forces.
