@@ -79,10 +79,11 @@ def test_tf32_and_cuda_core_networks_agree(case):
 
 @pytest.mark.parametrize("case", ["ag500", "water300", "hea1372", "chon976"])
 def test_every_layer_matches_oracle(case):
-    # rho^t in the units the networks see, (rho - shift) / scale.  This is a
-    # layout/indexing check (a wrong index gives O(1) errors); precision is
-    # asserted on energies and forces.  fp32 rounding of c^t, amplified by the
-    # cancelling odd-l sums of near-perfect crystals, reaches a few 1e-4 here.
+    # rho^t in the units the networks see, (rho - shift) / scale, and c^t
+    # relative to each feature's largest value.  With fp64 orbital sums, rho
+    # formed as rho - shift in fp64 and fp32-pair constants (fp32-accurate
+    # paths) the layers stay within 4.3e-5 (rho) and 5.4e-6 (c); the
+    # bf16-network Ag case within 9.0e-5 and 6.6e-6.  The bounds keep about 2x.
     p, pos, types, box = CASES[case]()
     ctx, _, _, _ = gpu_eval(p, pos, types, box)
     ref = oracle_eval(p, pos, types, box, intermediates=True)
@@ -90,9 +91,11 @@ def test_every_layer_matches_oracle(case):
     for t in range(p.T):
         rho, coef = ctx.reann_get_features(t)
         err_x = np.abs(rho - ref.rho[t]) / scale[t][types]
-        assert err_x.max() <= 1e-3, (t, err_x.max())
         scale_c = np.abs(ref.coef[t]).max(axis=0) + 1e-6
-        assert (np.abs(coef - ref.coef[t]) / scale_c).max() <= 2e-5, t
+        err_c = (np.abs(coef - ref.coef[t]) / scale_c).max()
+        print(f"\n{case} t={t}: rho err (standardised) {err_x.max():.3e}, c err (relative) {err_c:.3e}")
+        assert err_x.max() <= 2e-4, (t, err_x.max())
+        assert err_c <= 1.5e-5, (t, err_c)
 
 
 def _rounding_sensitivity(p, pos, types, box, T, w, ref, draws=8):
