@@ -795,13 +795,13 @@ struct NvtArgs {
     const double *noise;
 };
 
-// Velocity Verlet, with the thermostat applied after each step's closing half
-// kick when nvt is given.  The d_E slots: [0] energy, [1] kinetic energy,
-// [2] the step's rescaling factor, [3] thermostat work of this call.
-// The steps of one MD call, from the resident state (resume) or from the
-// caller-order state in d_stage_x / d_stage_v; results to the caller's x, v.
-// spec: the caller's x and v are being read in and compared on i_stream (a
-// continuing call); writes to them wait for that.
+// The steps of one MD call (velocity Verlet, with the thermostat applied after
+// each step's closing half kick when nvt is given), from the resident state
+// (resume) or from the caller-order state in d_stage_x / d_stage_v; results to
+// the caller's x, v.  spec: the caller's x and v are being read in and
+// compared on i_stream (a continuing call); writes to them wait for that.
+// The d_E slots: [0] energy, [1] kinetic energy, [2] the step's rescaling
+// factor, [3] thermostat work of this call.
 static reann_status md_steps(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, bool x_dev, bool v_dev,
                              const double *mass, const double *inv_mass, reann_md_stats *stats, cudaStream_t s,
                              const NvtArgs *nvt, BussiParams B, bool resume, bool spec) {
@@ -986,6 +986,9 @@ static reann_status md_steps(reann_ctx *c, int32_t nsteps, double dt_fs, double 
     return check_status(c, c->h_status[0] & ~ST_SKIN);
 }
 
+// One MD call: argument checks, the continuation decision and the caller's
+// state moved in (overlapped with the steps when the call continues), then
+// md_steps.
 static reann_status md_run(reann_ctx *c, int32_t nsteps, double dt_fs, double *x, double *v, const double *mass_amu,
                            reann_md_stats *stats, reann_stream stream, const NvtArgs *nvt) {
     if (!c) return REANN_ERR_ARG;
