@@ -399,17 +399,18 @@ def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
-    ap.add_argument("--workload", default="ag1m", choices=presets.ALL)
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one process per GPU under torchrun; replicas)")
+    ap.add_argument("--steps", type=int, default=100, help="timed MD steps (one call, device-resident)")
+    ap.add_argument("--warmup", type=int, default=3, help="untimed MD steps before the timed region")
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"),
+                    help="reference: the fp64 oracle on a bounded sample of the workload, host cores")
+    ap.add_argument("--workload", default="ag1m", choices=presets.ALL, help="synthetic system and model")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-array end-to-end timing")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle baseline sample")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU time of the oracle baseline sample")
     ap.add_argument("--dd-sweep", action="store_true",
                     help="monolithic vs domain-decomposed E+F for T = 1..6 (one JSON line per T)")
-    ap.add_argument("--dd-grid", default="8x8x8")
+    ap.add_argument("--dd-grid", default="8x8x8", help="subdomain grid of --dd-sweep")
     ap.add_argument("--ncell", type=int, default=0,
                     help="FCC workloads: cells per axis (smaller lattices for profiling captures)")
     ap.add_argument("--ensemble", default="nve", choices=("nve", "nvt"),
