@@ -136,6 +136,30 @@ def test_continuation_with_a_changed_state_starts_from_it(changed, where):
     assert np.array_equal(xo, xr) and np.array_equal(vo, vr)
 
 
+def test_zero_steps_return_the_state():
+    # a call of zero steps returns the state it was given (wrapped into the
+    # box), both as a continuation and after the caller changed it
+    p, pos, types, box = small("water")
+    v0 = synth.maxwell_boltzmann(p, types)
+    ctx = _ctx(p, pos, types, box)
+    x, v = pos.astype(np.float64).copy(), v0.copy()
+    ctx.reann_md_step(2, 0.5, x, v, p.masses)
+    x1, v1 = x.copy(), v.copy()
+    st = ctx.reann_md_step(0, 0.5, x, v, p.masses)
+    assert np.array_equal(x, x1) and np.array_equal(v, v1) and st.steps == 0
+    x[3] += 0.01
+    x2 = x - np.asarray(box) * np.floor(x / np.asarray(box))   # wrapped into [0, L)
+    v2 = v.copy()
+    ctx.reann_md_step(0, 0.5, x, v, p.masses)
+    assert np.array_equal(x, x2) and np.array_equal(v, v2)
+    # and the next call continues from it like a fresh context would
+    xr, vr = x.copy(), v.copy()
+    fresh = _ctx(p, xr.astype(np.float32), types, box)
+    fresh.reann_md_step(3, 0.5, xr, vr, p.masses)
+    ctx.reann_md_step(3, 0.5, x, v, p.masses)
+    assert np.array_equal(x, xr) and np.array_equal(v, vr)
+
+
 def test_host_state_equals_device_state():
     torch = torch_cuda()
     p, pos, types, box = small("chon")
