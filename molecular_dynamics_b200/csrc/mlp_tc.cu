@@ -32,11 +32,14 @@
 // Global traffic is contiguous: each tile's raw inputs are loaded in element
 // order and transposed to rows through the idle activation buffer; forward
 // outputs leave the same way; for the energy network and the coefficient
-// backward the tile's A rows are prefetched into L2 at the start of the tile,
-// and dE/dA = 2 w_tau A dE/drho is written one warp per row in the edge
-// kernels' lane-interleaved order.  All MMA-completion waits are bounded: a wait
-// that gives up sets ST_TIMEOUT, and the block frees its tensor memory and
-// returns.  The shared-memory operand layout is described in tc_common.cuh.
+// backward the tile's A rows are prefetched into L2 at the start of the tile
+// and loaded into registers while the tile's last product runs, and dE/dA =
+// 2 w_tau A dE/drho is written one warp per row in the edge kernels'
+// lane-interleaved order.  Tile descriptors are read one tile ahead.  All
+// MMA-completion waits are bounded: a wait that gives up is recorded, the group
+// learns of it at its next barrier (a barrier with an OR over its threads, so
+// all leave together), sets ST_TIMEOUT, frees its tensor memory and returns.
+// The shared-memory operand layout is described in tc_common.cuh.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -175,20 +178,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t tmem = *tmem_slot + (uint32_t)(256 * g);
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t phase = 0;
-    bool failed = false;
+    bool failed = false, bad = false;
 
-    // completion of the MMA group the group's thread 0 committed, awaited by the group
-    auto wait_mma = [&]() -> bool {
-        bool ok = bar_wait(bar, phase);
+    // completion of the MMA group the group's thread 0 committed; a wait that
+    // gave up is recorded and acted on at the group's next barrier (the TMEM
+    // values read meanwhile are discarded)
+    auto wait_mma = [&]() {
+        bad |= !bar_wait(bar, phase);
         phase ^= 1u;
         fence_after();
-        return !group_or(g, !ok);
     };
-    // operand stores (generic proxy) and TMEM reads done -> next MMA may start
-    auto handoff = [&]() {
+    // operand stores (generic proxy) and TMEM reads done -> next MMA may
+    // start; true if a wait of the group gave up
+    auto handoff = [&]() -> bool {
         fence_smem_to_async();
         fence_before();
-        group_sync(g);
+        return group_or(g, bad);
     };
 
     // dE/dA positions of this lane (element pk = lane + 32 j of a row, in the
@@ -204,24 +209,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         posj[j] = src | (gi << 8) | ((u >= 7 ? 1 : 0) << 16);
     }
 
+    // tile descriptors are loaded one tile ahead, off the tile's critical path
+    int next_r0 = 0, next_rows = 0;
+    if (rg.x + g < rg.y) next_r0 = tiles[rg.x + g].y, next_rows = tiles[rg.x + g].z;
     for (int ti = rg.x + g; ti < rg.y && !failed; ti += 2) {
-        const int4 tile = tiles[ti];
-        const int r0 = tile.y, rows = tile.z;
+        const int r0 = next_r0, rows = next_rows;
+        if (ti + 2 < rg.y) next_r0 = tiles[ti + 2].y, next_rows = tiles[ti + 2].z;
         // energy and backward: the tile's A rows are read at the end; start
         // moving them into L2 now
         if (MODE != TC_FWD && gt == 0) prefetch_l2(A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4));
-        // the group's next tile: its input rows into L2 while this one computes
-        if (gt == 0 && ti + 2 < rg.y) {
-            const int4 nx = tiles[ti + 2];
-            prefetch_l2_span(X + (int64_t)nx.y * D, (size_t)nx.z * D * 4);
-            if (MODE == TC_BWD) prefetch_l2_span(dY + (int64_t)nx.y * D, (size_t)nx.z * D * 4);
-        }
         // input tile: contiguous raw rows -> padded fp32 rows in ACT, then the
-        // standardised rho (and the upstream gradient) split bf16
+        // standardised rho (and the upstream gradient) split bf16 (the group's
+        // next tile's rows are moved into L2 meanwhile)
         {
             float *xs = stage, *ds = stage + TM * RS;
             const float *xg = X + (int64_t)r0 * D;
             const float *dg = MODE == TC_BWD ? dY + (int64_t)r0 * D : nullptr;
+            if (gt == 0 && ti + 2 < rg.y) {
+                prefetch_l2_span(X + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
+                if (MODE == TC_BWD) prefetch_l2_span(dY + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
+            }
             for (int k = gt; k < rows * D; k += TC_GROUP) {
                 const int rk = k / D, f = k - rk * D;
                 xs[rk * RS + f] = xg[k];
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, 16 * h + c8, gv);
             }
         }
-        handoff();
+        if (handoff()) { failed = true; break; }
 
         // layer 1 (and, for the coefficient backward, dE/da2 = dY W3 via the MN-major view of W3)
         if (gt == 0) {
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (MODE == TC_BWD) gemm2<H2, KPAD, true, KPAD>(tmem + L::C_B, sa(dy_hi), sa(dy_lo), base + L::W3);
             mma_commit(bar);
         }
-        if (!wait_mma()) { failed = true; break; }
+        wait_mma();
         // a1 = tanh(z1 + b1)
 #pragma unroll 1
         for (int c = 64 * h; c < 64 * h + 64; c += 32) {
@@ -263,7 +270,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
         }
-        handoff();
+        if (handoff()) { failed = true; break; }
         // z2 = a1 W2^T: into B (forward, energy) or over z1 in A (backward, whose B holds dY W3)
         constexpr int C_Z2 = MODE == TC_BWD ? L::C_A : L::C_B;
         if (gt == 0) {
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             gemm2<H2, H1, false, 0>(tmem + C_Z2, sa(act_hi), sa(act_lo), base + L::W2);
             mma_commit(bar);
         }
-        if (!wait_mma()) { failed = true; break; }
+        wait_mma();
 
         if (MODE == TC_FWD) {
             // a2 = tanh(z2 + b2), then y = a2 W3^T + b3 (into A)
@@ -284,13 +291,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &v[u]);
             }
-            handoff();
+            if (handoff()) { failed = true; break; }
             if (gt == 0) {
                 fence_after();
                 gemm2<KPAD, H2, false, 0>(tmem + L::C_A, sa(act_hi), sa(act_lo), base + L::W3);
                 mma_commit(bar);
             }
-            if (!wait_mma()) { failed = true; break; }
+            wait_mma();
             // y rows through ACT (the last product has consumed it), then contiguous stores
 #pragma unroll
             for (int c8 = 0; c8 < 16; c8 += 8) {
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &z[u]);
             }
             if (MODE == TC_ENERGY) se[h * TM + row] = e_row;
-            handoff();
+            if (handoff()) { failed = true; break; }
             if (MODE == TC_ENERGY && h == 0 && row < rows) Ei[r0 + row] = (se[row] + se[TM + row]) + sb3[0];
             // p1 = g2 W2 (MN-major view of W2) into B; the backward recomputes z1
             // = x W1^T into A (its first copy was overwritten by z2)
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (MODE == TC_BWD) gemm2<H1, KPAD, false, 0>(tmem + L::C_A, sa(x_hi), sa(x_lo), base + L::W1);
                 mma_commit(bar);
             }
-            if (!wait_mma()) { failed = true; break; }
+            wait_mma();
             // g1 = p1 (1 - tanh^2(z1 + b1)), tanh' from the fp32 pre-activation in TMEM
 #pragma unroll 1
             for (int c = 64 * h; c < 64 * h + 64; c += 32) {
@@ -352,14 +359,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 32; u += 8) st_chunk2(act_hi, act_lo, TM, row, c + u, &p[u]);
             }
-            handoff();
+            if (handoff()) { failed = true; break; }
             // dE/dx = g1 W1 (MN-major view of W1), into A
             if (gt == 0) {
                 fence_after();
                 gemm2<KPAD, H1, true, H1>(tmem + L::C_A, sa(act_hi), sa(act_lo), base + L::W1);
                 mma_commit(bar);
             }
-            if (!wait_mma()) { failed = true; break; }
+            // while the product runs: this warp's A rows for G = dE/dA = 2 w_tau A
+            // dE/drho (warp per row, lanes along the row in the edge kernels'
+            // lane-interleaved order, contiguous stores), RQ rows per pass
+            constexpr int WARPS = TC_GROUP / 32, RQ = 8;
+            const float *ag = A + (int64_t)r0 * NA;
+            float *go = Gout + (int64_t)r0 * NA;
+            float av[RQ][NJ];
+            auto load_rows = [&](int rb) {
+#pragma unroll
+                for (int q = 0; q < RQ; ++q) {
+                    const int rk = rb + q * WARPS;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int pk = (tid & 31) + 32 * j;
+                        av[q][j] = (rk < rows && pk < NA) ? ag[(int64_t)rk * NA + (posj[j] & 255)] : 0.f;
+                    }
+                }
+            };
+            load_rows(gw);
+            wait_mma();
             // dE/drho = (g1 W1) / scale, rows through ACT (consumed by the last product)
             float *gxs = stage;
 #pragma unroll
@@ -370,25 +396,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int u = 0; u < 8; ++u) gxs[row * L::GXS + 16 * h + c8 + u] = v[u] * sinv[16 * h + c8 + u];
             }
             group_sync(g);
-            // G = dE/dA = 2 w_tau A dE/drho, warp per row, lanes along the row in the
-            // edge kernels' lane-interleaved order (contiguous stores); four rows'
-            // A values are loaded before any is used
-            const float *ag = A + (int64_t)r0 * NA;
-            float *go = Gout + (int64_t)r0 * NA;
-            for (int rb = gw; rb < rows; rb += 4 * (TC_GROUP / 32)) {
-                float av[4][NJ];
+            for (int rb = gw; rb < rows; rb += RQ * WARPS) {
+                if (rb != gw) load_rows(rb);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int rk = rb + q * (TC_GROUP / 32);
-#pragma unroll
-                    for (int j = 0; j < NJ; ++j) {
-                        const int pk = (tid & 31) + 32 * j;
-                        av[q][j] = (rk < rows && pk < NA) ? ag[(int64_t)rk * NA + (posj[j] & 255)] : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int rk = rb + q * (TC_GROUP / 32);
+                for (int q = 0; q < RQ; ++q) {
+                    const int rk = rb + q * WARPS;
                     if (rk >= rows) break;
 #pragma unroll
                     for (int j = 0; j < NJ; ++j) {
@@ -403,7 +415,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         // the next tile's input staging overwrites ACT: all of this tile's reads are done
         fence_before();
-        group_sync(g);
+        if (group_or(g, bad)) { failed = true; break; }
     }
 
     if (failed && gt == 0) atomicOr(status, ST_TIMEOUT);
