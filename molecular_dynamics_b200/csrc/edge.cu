@@ -88,20 +88,25 @@ __device__ __forceinline__ float3 displacement(float4 pi, float4 pj, const EdgeP
 // front of the row's slot (same offsets as the full list), each with its
 // displacement and distance (dx, dy, dz, r), which every edge pass of the
 // evaluation then reads instead of recomputing.
-template <bool DR>   // DR: also the distance rounding residuals (fp32-accurate paths)
+template <bool DR, int LPR, int B>   // DR: also the distance rounding residuals (fp32-accurate paths)
 __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restrict__ pos, const int *__restrict__ row,
-                                                const int *__restrict__ col, int *__restrict__ act_cnt,
-                                                int *__restrict__ act_col, float4 *__restrict__ act_geo,
-                                                float *__restrict__ act_dr, EdgeParams P,
-                                                unsigned long long *__restrict__ total) {
-    // one warp per row: lanes test consecutive entries, a ballot compacts the
-    // active ones in row order and the writes stay contiguous.  Warps stride
-    // over the rows (the next row's position and bounds are loaded while the
-    // current one is tested) and add their count of active pairs to the total once.
-    const int lane = threadIdx.x & 31;
+                                                 const int *__restrict__ col, int *__restrict__ act_cnt,
+                                                 int *__restrict__ act_col, float4 *__restrict__ act_geo,
+                                                 float *__restrict__ act_dr, EdgeParams P,
+                                                 unsigned long long *__restrict__ total) {
+    // LPR lanes per row (32 / LPR rows per warp): the lanes of a row test
+    // consecutive entries, B per lane with their loads issued together, and a
+    // ballot over the row's lanes compacts the active ones in row order, so the
+    // writes stay contiguous.  Warps stride over the rows (the next row's
+    // position and bounds are loaded while the current one is tested) and add
+    // their count of active pairs to the total once.
+    static_assert(LPR == 8 || LPR == 16 || LPR == 32, "rows of 8, 16 or 32 lanes");
+    constexpr int RPW = 32 / LPR;
+    const int lane = threadIdx.x & 31, sl = lane % LPR;
+    const unsigned rmask = LPR == 32 ? 0xffffffffu : ((1u << LPR) - 1u) << (lane - sl);
     unsigned long long tot = 0;
-    int i = blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int stride = gridDim.x * 4;
+    int i = (blockIdx.x * 4 + (threadIdx.x >> 5)) * RPW + lane / LPR;
+    const int stride = gridDim.x * 4 * RPW;
     float4 pi_n = i < n ? pos[i] : make_float4(0.f, 0.f, 0.f, 0.f);
     int q0_n = i < n ? row[i] : 0, q1_n = i < n ? row[i + 1] : 0;
     for (; i < n; i += stride) {
@@ -113,24 +118,23 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
             q1_n = row[i + stride + 1];
         }
         int k = 0;
-        constexpr int B = 4;   // entries per lane whose loads are issued together
-        for (int base = q0; base < q1; base += 32 * B) {
+        for (int base = q0; base < q1; base += LPR * B) {
             int j[B];
             float4 pj[B];
 #pragma unroll
             for (int b = 0; b < B; ++b) {
-                const int q = base + 32 * b + lane;
+                const int q = base + LPR * b + sl;
                 j[b] = q < q1 ? col[q] : -1;
             }
 #pragma unroll
             for (int b = 0; b < B; ++b) pj[b] = j[b] >= 0 ? pos[j[b]] : pi;
 #pragma unroll
             for (int b = 0; b < B; ++b) {
-                if (base + 32 * b >= q1) break;
+                if (base + LPR * b >= q1) break;
                 const float3 d = displacement(pi, pj[b], P);
                 const float r2 = d.x * d.x + d.y * d.y + d.z * d.z;
                 const bool act = j[b] >= 0 && r2 < P.r_cut2;
-                const unsigned mask = __ballot_sync(0xffffffffu, act);
+                const unsigned mask = __ballot_sync(rmask, act) & rmask;
                 if (act) {
                     const int o = q0 + k + __popc(mask & ((1u << lane) - 1u));
                     act_col[o] = j[b];
@@ -151,10 +155,10 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
                 k += __popc(mask);
             }
         }
-        if (lane == 0) act_cnt[i] = k;
+        if (sl == 0) act_cnt[i] = k;
         tot += (unsigned long long)k;
     }
-    if (lane == 0 && tot) atomicAdd(total, tot);
+    if (sl == 0 && tot) atomicAdd(total, tot);
 }
 
 cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
@@ -163,16 +167,19 @@ cudaError_t launch_active(reann_ctx *c, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(c->d_i64 + 3, 0, sizeof(int64_t), s);
     if (e) return e;
     REANN_TIMED(c, REANN_K_ACTIVE, s);
+    // two rows per warp, 16 lanes x 4 entries each (a whole warp per row left most
+    // lanes idle on rows of ~80 entries and kept half as many gathers in flight)
+    constexpr int LPR = 16, B = 4, RPB = 4 * (32 / LPR);   // rows per block and pass
     // one resident wave (8 blocks of 128 threads per SM at <= 64 registers)
-    const unsigned grid = (unsigned)std::min<int64_t>((c->n + 3) / 4, (int64_t)c->sm_count * 8);
+    const unsigned grid = (unsigned)std::min<int64_t>((c->n + RPB - 1) / RPB, (int64_t)c->sm_count * 8);
     const int *col = c->dd ? c->d_col_dd : c->d_col;
     unsigned long long *total = (unsigned long long *)(c->d_i64 + 3);
     if (c->d_act_dr)
-        k_active<true><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt, c->d_act_col,
-                                            c->d_act_geo, c->d_act_dr, P, total);
+        k_active<true, LPR, B><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt, c->d_act_col,
+                                                    c->d_act_geo, c->d_act_dr, P, total);
     else
-        k_active<false><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt, c->d_act_col,
-                                             c->d_act_geo, nullptr, P, total);
+        k_active<false, LPR, B><<<grid, 128, 0, s>>>((int)c->n, c->d_pos, c->d_row, col, c->d_act_cnt,
+                                                     c->d_act_col, c->d_act_geo, nullptr, P, total);
     return cudaGetLastError();
 }
 
