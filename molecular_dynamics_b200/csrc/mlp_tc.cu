@@ -29,12 +29,16 @@
 // evaluates tanh.  The coefficient backward recomputes the first layer's
 // pre-activation (one small product) instead of keeping it, to fit 256 columns.
 //
-// Global traffic is contiguous: each tile's raw inputs are loaded in element
-// order and transposed to rows through the idle activation buffer; forward
-// outputs leave the same way; for the energy network and the coefficient
-// backward the tile's A rows are prefetched into L2 at the start of the tile
-// and loaded into registers while the tile's last product runs, and dE/dA =
-// 2 w_tau A dE/drho is written one warp per row in the edge kernels'
+// Global traffic: the forward and energy networks' raw input rows arrive by
+// one bulk copy per tile (issued by thread 0 into the group's X buffer as soon
+// as the previous tile's first product has read it), or, for rows that are not
+// whole 16-byte units, are loaded in element order and transposed to rows
+// through the idle activation buffer; the coefficient backward loads each
+// row's rho and upstream gradient per thread; forward outputs leave through
+// the activation buffer as contiguous stores; for the energy network and the
+// coefficient backward the tile's A rows are prefetched into L2 at the start of
+// the tile and loaded into registers while the tile's last product runs, and
+// dE/dA = 2 w_tau A dE/drho is written one warp per row in the edge kernels'
 // lane-interleaved order.  Tile descriptors are read one tile ahead.  All
 // MMA-completion waits are bounded: a wait that gives up is recorded, the group
 // learns of it at its next barrier (a barrier with an OR over its threads, so
@@ -84,7 +88,8 @@ struct TcLayout {
     //   ACT  [TM][128] bf16 hi + lo: the operand of layers 2 and 3 (and of the
     //        VJP products), reused by every layer once the product that read it
     //        has completed; between products it also holds the raw input rows
-    //        (fp32 [TM][RS], x then dY), the dY operand (hi + lo at ACT_DY),
+    //        of the forward and energy networks (fp32 [TM][RS]), the dY
+    //        operand of the backward (hi + lo at ACT_DY),
     //        the output rows and the dE/drho rows
     //   X    [TM][KPAD] bf16 hi + lo, kept for the whole tile (the backward
     //        recomputes layer 1 from it)
@@ -93,10 +98,15 @@ struct TcLayout {
     static constexpr int X = ACT + 2 * TM * 128 * 2;
     static constexpr int SE = X + 2 * TM * KPAD * 2;             // energy partials [2][TM] fp32
     static constexpr int BAR = SE + 2 * TM * 4;                  // MMA-completion mbarrier
+    static constexpr int CBAR = BAR + 8;                         // input-copy mbarrier
     static constexpr int GROUP_BYTES = BAR + 16;
+    // forward and energy: the next tile's raw rows are copied into X (a bulk
+    // copy, 16-byte units) once the current tile's first product has read X
+    static constexpr bool BULK = MODE != TC_BWD && (D * 4) % 16 == 0;
+    static_assert(TM * D * 4 <= 2 * TM * KPAD * 2, "raw input rows fit the X operand buffer");
     static constexpr int SLOT = GRP + 2 * GROUP_BYTES;           // TMEM base address
     static constexpr int bytes = SLOT + 16;
-    static_assert(2 * TM * RS * 4 <= ACT_DY && ACT_DY + 2 * TM * KPAD * 2 <= X, "input staging fits the ACT buffer");
+    static_assert(TM * RS * 4 <= ACT_DY && ACT_DY + 2 * TM * KPAD * 2 <= X, "input staging fits the ACT buffer");
     static_assert(TM * GXS * 4 <= X && TM * RS * 4 <= X, "output staging fits the ACT buffer");
     static_assert(GRP % 16 == 0 && GROUP_BYTES % 16 == 0, "16-byte aligned operand tiles");
     // TMEM columns of a group (its base is 256 g): two 128-column accumulators
@@ -136,6 +146,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     float *stage = reinterpret_cast<float *>(gs + L::ACT);
     float *se = reinterpret_cast<float *>(gs + L::SE);
     uint64_t *bar = reinterpret_cast<uint64_t *>(gs + L::BAR);
+    uint64_t *cbar = reinterpret_cast<uint64_t *>(gs + L::CBAR);
     const uint32_t base = smem_u32(sm);
     auto sa = [&](const unsigned char *p) { return base + (uint32_t)(p - sm); };
 
@@ -147,6 +158,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if (gt == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(cbar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     {
@@ -212,42 +224,103 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // tile descriptors are loaded one tile ahead, off the tile's critical path
     int next_r0 = 0, next_rows = 0;
     if (rg.x + g < rg.y) next_r0 = tiles[rg.x + g].y, next_rows = tiles[rg.x + g].z;
+    // raw rows of a tile -> X by one bulk copy (thread 0), completion on cbar
+    uint32_t cphase = 0;
+    bool copy_pending = false;
+    auto copy_rows = [&](int rr0, int rrows) {
+        if (gt == 0) {
+            const uint32_t nb = (uint32_t)(rrows * D * 4);
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(cbar)), "r"(nb)
+                         : "memory");
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         ::"r"(sa(x_hi)), "l"(X + (int64_t)rr0 * D), "r"(nb), "r"(smem_u32(cbar))
+                         : "memory");
+        }
+        copy_pending = true;
+    };
+    if (L::BULK && rg.x + g < rg.y) copy_rows(next_r0, next_rows);
     for (int ti = rg.x + g; ti < rg.y && !failed; ti += 2) {
         const int r0 = next_r0, rows = next_rows;
         if (ti + 2 < rg.y) next_r0 = tiles[ti + 2].y, next_rows = tiles[ti + 2].z;
         // energy and backward: the tile's A rows are read at the end; start
         // moving them into L2 now
         if (MODE != TC_FWD && gt == 0) prefetch_l2(A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4));
-        // input tile: contiguous raw rows -> padded fp32 rows in ACT, then the
-        // standardised rho (and the upstream gradient) split bf16 (the group's
-        // next tile's rows are moved into L2 meanwhile)
-        {
-            float *xs = stage, *ds = stage + TM * RS;
-            const float *xg = X + (int64_t)r0 * D;
-            const float *dg = MODE == TC_BWD ? dY + (int64_t)r0 * D : nullptr;
+        // input tile, standardised rho (and the upstream gradient) split into
+        // bf16 hi/lo.  Coefficient backward: each thread loads its own row's 16
+        // features of both (columns 16 h .. 16 h + 15, zero past D) as float2
+        // pairs straight into registers.  Forward and energy with 16-byte rows:
+        // the raw rows were copied into X while the previous tile computed.
+        // Otherwise: contiguous raw rows -> padded fp32 rows in ACT.  Where the
+        // rows are loaded here, the group's next tile's rows are moved into L2
+        // meanwhile.
+        const bool live = row < rows;
+        if (MODE == TC_BWD) {
+            const int64_t atom = r0 + (live ? row : 0);
+            const float *xr = X + atom * D, *dr = dY + atom * D;
+            float v[16], gv[16];
+#pragma unroll
+            for (int u = 0; u < 16; u += 2) {
+                const int f = 16 * h + u;
+                const bool ok = live && f < D;
+                const float2 t = ok ? *reinterpret_cast<const float2 *>(xr + f) : make_float2(0.f, 0.f);
+                const float2 q = ok ? *reinterpret_cast<const float2 *>(dr + f) : make_float2(0.f, 0.f);
+                v[u] = t.x, v[u + 1] = t.y, gv[u] = q.x, gv[u + 1] = q.y;
+            }
             if (gt == 0 && ti + 2 < rg.y) {
                 prefetch_l2_span(X + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
-                if (MODE == TC_BWD) prefetch_l2_span(dY + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
+                prefetch_l2_span(dY + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
             }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int f = 16 * h + u;
+                v[u] = live ? (v[u] - sshift[f]) * sinv[f] : 0.f;
+            }
+            st_chunk2(x_hi, x_lo, TM, row, 16 * h, v);
+            st_chunk2(x_hi, x_lo, TM, row, 16 * h + 8, v + 8);
+            st_chunk2(dy_hi, dy_lo, TM, row, 16 * h, gv);
+            st_chunk2(dy_hi, dy_lo, TM, row, 16 * h + 8, gv + 8);
+        } else if (L::BULK) {
+            // this tile's raw rows arrived in X by the bulk copy; each thread
+            // takes its row's 16 features (16-byte loads), then, once the group
+            // has read them all, overwrites X with the bf16 operand
+            const bool landed = bar_wait(cbar, cphase);
+            bad |= !landed;
+            cphase ^= 1u;
+            copy_pending = !landed;
+            const float *xs = reinterpret_cast<const float *>(x_hi) + row * D;
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; u += 4) {
+                const int f = 16 * h + u;
+                const float4 t = live && f < D ? *reinterpret_cast<const float4 *>(xs + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[u] = t.x, v[u + 1] = t.y, v[u + 2] = t.z, v[u + 3] = t.w;
+            }
+            group_sync(g);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int f = 16 * h + u;
+                v[u] = live && f < D ? (v[u] - sshift[f]) * sinv[f] : 0.f;
+            }
+            st_chunk2(x_hi, x_lo, TM, row, 16 * h, v);
+            st_chunk2(x_hi, x_lo, TM, row, 16 * h + 8, v + 8);
+        } else {
+            if (gt == 0 && ti + 2 < rg.y) prefetch_l2_span(X + (int64_t)next_r0 * D, (size_t)next_rows * D * 4);
+            float *xs = stage;
+            const float *xg = X + (int64_t)r0 * D;
             for (int k = gt; k < rows * D; k += TC_GROUP) {
                 const int rk = k / D, f = k - rk * D;
                 xs[rk * RS + f] = xg[k];
-                if (MODE == TC_BWD) ds[rk * RS + f] = dg[k];
             }
             group_sync(g);
-            const bool live = row < rows;
 #pragma unroll
             for (int c8 = 0; c8 < 16; c8 += 8) {
-                float v[8], gv[8];
+                float v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int f = 16 * h + c8 + u;
-                    const bool ok = live && f < D;
-                    v[u] = ok ? (xs[row * RS + f] - sshift[f]) * sinv[f] : 0.f;
-                    gv[u] = (MODE == TC_BWD && ok) ? ds[row * RS + f] : 0.f;
+                    v[u] = live && f < D ? (xs[row * RS + f] - sshift[f]) * sinv[f] : 0.f;
                 }
                 st_chunk2(x_hi, x_lo, TM, row, 16 * h + c8, v);
-                if (MODE == TC_BWD) st_chunk2(dy_hi, dy_lo, TM, row, 16 * h + c8, gv);
             }
         }
         if (handoff()) { failed = true; break; }
@@ -260,6 +333,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mma_commit(bar);
         }
         wait_mma();
+        // X has been read by the product: the group's next tile's raw rows may land there
+        if (L::BULK && ti + 2 < rg.y) copy_rows(next_r0, next_rows);
         // a1 = tanh(z1 + b1)
 #pragma unroll 1
         for (int c = 64 * h; c < 64 * h + 64; c += 32) {
@@ -418,6 +493,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (group_or(g, bad)) { failed = true; break; }
     }
 
+    // a copy still in flight (a group that left early) lands before the block exits
+    if (copy_pending) bar_wait(cbar, cphase & 1u);
     if (failed && gt == 0) atomicOr(status, ST_TIMEOUT);
     fence_before();
     __syncthreads();
