@@ -55,7 +55,7 @@ FLOP_EDGE_BWD_PER_PAIR = {8: (754, 930), 10: (938, 1158)}   # (layer 0 without d
 # belongs to the kernel source whose SHA-256 prefix is recorded beside it (the
 # text of the scalar k_edge_bwd kernel in edge.cu): once that text changes, the
 # figure no longer describes the kernel and the line reports null.
-EDGE_BWD_CAPTURE = {"bytes_per_atom": (448.149376e6 + 24.650496e6) / 256000, "source_sha": "62ad35946708c7d9",
+EDGE_BWD_CAPTURE = {"bytes_per_atom": (448.216192e6 + 23.258240e6) / 256000, "source_sha": "73c818a4f0abbb25",
                     "workload": "ag1m"}
 EDGE_BWD_TRAFFIC_NOTE = "bytes per launch: DRAM read+write of a 256,000-atom ncu capture scaled by the atom count"
 

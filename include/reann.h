@@ -60,7 +60,8 @@ typedef enum {
     REANN_ERR_STATE = 6,     /* call out of order, e.g. forces before a neighbour list */
     REANN_ERR_CUDA = 7,      /* a CUDA runtime call failed */
     REANN_ERR_TIMEOUT = 8,   /* a bounded device wait gave up */
-    REANN_ERR_UNSUPPORTED = 9
+    REANN_ERR_UNSUPPORTED = 9,
+    REANN_ERR_INDEX = 10     /* checked builds: an internal index was outside its array */
 } reann_status;
 
 /*
@@ -391,6 +392,29 @@ reann_status reann_profile_read(const reann_ctx *ctx, int32_t group, double *ms,
  */
 reann_status reann_pair_list_noalloc(int64_t n, const float *pos, const double box[3], double r_cut, double skin,
                                      int32_t *row, int32_t *col, int64_t cap, int64_t *nnz, reann_stream stream);
+
+/*
+ * Checked builds.  libreann_checked.so is this library compiled with
+ * REANN_CHECKED: every index that a kernel reads from a neighbour list, a
+ * permutation, a ghost map or a halo list (and every row end of a list) is
+ * tested against the length of the array it indexes before use.  One out of
+ * range is replaced by 0, so the access stays inside the array; the call
+ * that ran the kernel then returns REANN_ERR_INDEX, its outputs not valid.
+ * No device trap is used.  Valid inputs give the same results as the
+ * unchecked build.  Returns 1 in a checked build, 0 otherwise.
+ */
+int32_t reann_checked(void);
+
+/*
+ * Fault injection for the checked build, on the host side (nothing is made
+ * to fault on the device): writes j into entry k (0 <= k < nnz, the list's
+ * internal order) of the neighbour list the next energy+force call reads, as
+ * a damaged list would hold it.  With j outside [0, n) that call returns
+ * REANN_ERR_INDEX; reann_build_neighbors rebuilds the list.  Synchronises the
+ * device.  Errors: REANN_ERR_UNSUPPORTED (unchecked build), REANN_ERR_STATE
+ * (no list), REANN_ERR_ARG (k outside the list), REANN_ERR_CUDA.
+ */
+reann_status reann_debug_set_neighbor(reann_ctx *ctx, int64_t k, int32_t j);
 
 #ifdef __cplusplus
 }

@@ -1,6 +1,8 @@
-"""Builds libreann.so in-tree with nvcc for sm_100a.
+"""Builds libreann.so in-tree with nvcc for sm_100a, and with --checked the
+checked build libreann_checked.so (REANN_CHECKED: every internal index tested
+before use, see include/reann.h).
 
-    python -m molecular_dynamics_b200.build [--force] [--verbose]
+    python -m molecular_dynamics_b200.build [--force] [--verbose] [--checked]
 """
 from __future__ import annotations
 
@@ -13,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libreann.so")
+LIB_CHECKED = os.path.join(HERE, "libreann_checked.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -32,17 +35,20 @@ def headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in sources() + headers() + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not stale():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+def build(force: bool = False, verbose: bool = False, extra=(), checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not stale(lib):
+        return lib
+    if checked:
+        extra = ("-DREANN_CHECKED", *extra)
+    objdir = os.path.join(HERE, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     procs = []
@@ -63,13 +69,12 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for " + ", ".join(os.path.basename(f) for f in failed))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp,
                            "-lcudart"])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv))

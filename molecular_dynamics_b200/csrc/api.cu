@@ -220,6 +220,7 @@ cudaError_t sync_stream(reann_ctx *c, cudaStream_t s) {
 
 // status word -> API status
 reann_status check_status(reann_ctx *c, int st) {
+    if (st & ST_INDEX) return fail(c, REANN_ERR_INDEX, "an internal index was outside its array (checked build)");
     if (st & ST_BADTYPE) return fail(c, REANN_ERR_ARG, "atom type outside [0, n_elements)");
     if (st & ST_NONFINITE) return fail(c, REANN_ERR_NONFINITE, "non-finite position, energy or force");
     if (st & ST_CAPACITY) return fail(c, REANN_ERR_CAPACITY, "neighbour capacity exceeded");
@@ -1266,6 +1267,20 @@ extern "C" reann_status reann_get_neighbors(reann_ctx *c, int64_t *row, int32_t 
     }
     CK(cudaMemcpy(row, orow.data(), sizeof(int64_t) * (n + 1), cudaMemcpyDefault));
     if (c->nnz > 0) CK(cudaMemcpy(col, ocol.data(), sizeof(int32_t) * c->nnz, cudaMemcpyDefault));
+    return REANN_OK;
+}
+
+extern "C" int32_t reann_checked(void) { return kChecked ? 1 : 0; }
+
+extern "C" reann_status reann_debug_set_neighbor(reann_ctx *c, int64_t k, int32_t j) {
+    if (!c) return REANN_ERR_ARG;
+    if (!kChecked) return fail(c, REANN_ERR_UNSUPPORTED, "fault injection needs the checked build");
+    if (!c->have_list) return fail(c, REANN_ERR_STATE, "no neighbour list");
+    if (k < 0 || k >= c->nnz) return fail(c, REANN_ERR_ARG, "entry outside the neighbour list");
+    DeviceGuard guard(c->device);
+    CK(cudaDeviceSynchronize());
+    int *col = c->dd ? c->d_col_dd : c->d_col;
+    CK(cudaMemcpy(col + k, &j, sizeof(int32_t), cudaMemcpyHostToDevice));
     return REANN_OK;
 }
 

@@ -23,7 +23,39 @@ enum : int {
     ST_SKIN = 4,
     ST_BADTYPE = 8,
     ST_TIMEOUT = 16,
+    ST_INDEX = 32,      // checked builds: an index outside its array
 };
+
+// Checked builds (compiled with REANN_CHECKED): every index read from a
+// neighbour list, permutation, ghost map or halo list is tested against the
+// length of the array it indexes before use.  One out of range or-s ST_INDEX
+// into the status word and is replaced by 0, so the access stays inside the
+// array; the results of that call are then wrong and the call reports
+// REANN_ERR_INDEX.  Other builds: no test, the index is used as read.
+#ifdef REANN_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+__device__ __forceinline__ int64_t checked(int64_t j, int64_t n, int *status) {
+    if constexpr (kChecked) {
+        if (j < 0 || j >= n) {
+            atomicOr(status, ST_INDEX);
+            return 0;
+        }
+    }
+    return j;
+}
+// a row's end offset, tested against the list's length the same way
+__device__ __forceinline__ int checked_end(int q1, int64_t len, int *status) {
+    if constexpr (kChecked) {
+        if (q1 < 0 || q1 > len) {
+            atomicOr(status, ST_INDEX);
+            return 0;
+        }
+    }
+    return q1;
+}
 
 // geometry and model constants passed by value to the edge kernels
 struct EdgeParams {
@@ -40,6 +72,9 @@ struct EdgeParams {
     float alpha;
     float neg_alpha_log2e;   // -alpha log2(e): exp(-alpha t^2) = 2^(t^2 neg_alpha_log2e)
     float mu_hi[16], mu_lo[16];
+    int64_t n_rows;   // rows (atoms and ghost slots) a neighbour index may name
+    int64_t n_list;   // entries of the neighbour list (its capacity)
+    int *status;      // device status word (checked builds)
 };
 
 // offsets (in floats) of one atomic network inside the device weight blob

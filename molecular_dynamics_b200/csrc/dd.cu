@@ -56,12 +56,13 @@ __global__ void k_dd_subdomain(int n, const float4 *__restrict__ pos, DDGrid g, 
 
 // bit (s, j) set when atom j of another subdomain is a list neighbour of a local atom of s
 __global__ void k_dd_mark(int n, const int *__restrict__ row, const int *__restrict__ col, const int *__restrict__ sub,
-                          int64_t words, unsigned *__restrict__ bits) {
+                          int64_t words, unsigned *__restrict__ bits, int64_t n_list, int *__restrict__ status) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const int s = sub[i];
-    for (int q = row[i]; q < row[i + 1]; ++q) {
-        const int j = col[q];
+    const int q1 = checked_end(row[i + 1], n_list, status);
+    for (int q = row[i]; q < q1; ++q) {
+        const int j = (int)checked(col[q], n, status);
         if (sub[j] != s) atomicOr(&bits[(int64_t)s * words + (j >> 5)], 1u << (j & 31));
     }
 }
@@ -95,38 +96,43 @@ __device__ __forceinline__ int dd_ghost_slot(int s, int j, int64_t words, int n,
 
 __global__ void k_dd_remap(int n, const int *__restrict__ row, const int *__restrict__ col,
                            const int *__restrict__ sub, int64_t words, const unsigned *__restrict__ bits,
-                           const int *__restrict__ prefix, int *__restrict__ dd_col) {
+                           const int *__restrict__ prefix, int *__restrict__ dd_col, int64_t n_list,
+                           int *__restrict__ status) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const int s = sub[i];
-    for (int q = row[i]; q < row[i + 1]; ++q) {
-        const int j = col[q];
+    const int q1 = checked_end(row[i + 1], n_list, status);
+    for (int q = row[i]; q < q1; ++q) {
+        const int j = (int)checked(col[q], n, status);
         dd_col[q] = sub[j] == s ? j : dd_ghost_slot(s, j, words, n, bits, prefix);
     }
 }
 
 // rows of `width` floats: dst[n + g] = src[owner[g]]
-__global__ void k_dd_gather(int64_t n_ghost, int width, int n, const int *__restrict__ owner, float *__restrict__ base) {
+__global__ void k_dd_gather(int64_t n_ghost, int width, int n, const int *__restrict__ owner, float *__restrict__ base,
+                            int *__restrict__ status) {
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= n_ghost * width) return;
     const int64_t g = k / width, f = k % width;
-    base[((int64_t)n + g) * width + f] = base[(int64_t)owner[g] * width + f];
+    base[((int64_t)n + g) * width + f] = base[checked(owner[g], n, status) * width + f];
 }
 
 // negative control: ghost coefficient rows keep the element's initial c^0
 __global__ void k_dd_stale(int64_t n_ghost, int D, int n, const int *__restrict__ owner,
-                           const float4 *__restrict__ pos, const float *__restrict__ C0, float *__restrict__ coef) {
+                           const float4 *__restrict__ pos, const float *__restrict__ C0, float *__restrict__ coef,
+                           int *__restrict__ status) {
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= n_ghost * D) return;
     const int64_t g = k / D, f = k % D;
-    const int e = __float_as_int(pos[owner[g]].w);
+    const int e = __float_as_int(pos[checked(owner[g], n, status)].w);
     coef[((int64_t)n + g) * D + f] = C0[e * D + f];
 }
 
 cudaError_t dd_gather_rows(reann_ctx *c, float *base, int width, cudaStream_t s) {
     if (c->dd_ghosts == 0) return cudaSuccess;
     REANN_TIMED(c, REANN_K_GHOST, s);
-    k_dd_gather<<<blocks(c->dd_ghosts * width, 256), 256, 0, s>>>(c->dd_ghosts, width, (int)c->n, c->d_dd_owner, base);
+    k_dd_gather<<<blocks(c->dd_ghosts * width, 256), 256, 0, s>>>(c->dd_ghosts, width, (int)c->n, c->d_dd_owner, base,
+                                                                  c->d_status);
     return cudaGetLastError();
 }
 
@@ -134,7 +140,7 @@ cudaError_t dd_stale_coef(reann_ctx *c, float *coef, cudaStream_t s) {
     if (c->dd_ghosts == 0) return cudaSuccess;
     REANN_TIMED(c, REANN_K_GHOST, s);
     k_dd_stale<<<blocks(c->dd_ghosts * c->D, 256), 256, 0, s>>>(c->dd_ghosts, c->D, (int)c->n, c->d_dd_owner,
-                                                                  c->d_pos, c->d_w, coef);
+                                                                  c->d_pos, c->d_w, coef, c->d_status);
     return cudaGetLastError();
 }
 
@@ -175,7 +181,8 @@ cudaError_t dd_plan(reann_ctx *c, cudaStream_t s, int64_t *n_ghost) {
         REANN_TIMED(c, REANN_K_GHOST, s, 7);
         k_dd_subdomain<<<blocks(n, 256), 256, 0, s>>>((int)n, c->d_pos, g, c->d_dd_sub);
         if ((e = cudaMemsetAsync(c->d_dd_bits, 0, sizeof(unsigned) * (size_t)total_words, s))) return e;
-        k_dd_mark<<<blocks(n, 128), 128, 0, s>>>((int)n, c->d_row, c->d_col, c->d_dd_sub, words, c->d_dd_bits);
+        k_dd_mark<<<blocks(n, 128), 128, 0, s>>>((int)n, c->d_row, c->d_col, c->d_dd_sub, words, c->d_dd_bits,
+                                                 c->cap, c->d_status);
         k_dd_popc<<<blocks(total_words, 256), 256, 0, s>>>(total_words, c->d_dd_bits, c->d_dd_cnt);
         if ((e = scan_exclusive(c->d_dd_cnt, c->d_dd_prefix, total_words, c->d_i64 + 5, c->d_scan_tmp, s))) return e;
     }
@@ -196,10 +203,10 @@ cudaError_t dd_finish(reann_ctx *c, cudaStream_t s) {
     k_dd_owners<<<blocks(total_words, 256), 256, 0, s>>>(total_words, words, (int)n, c->d_dd_bits, c->d_dd_prefix,
                                                          c->d_dd_owner);
     k_dd_remap<<<blocks(n, 128), 128, 0, s>>>((int)n, c->d_row, c->d_col, c->d_dd_sub, words, c->d_dd_bits,
-                                              c->d_dd_prefix, c->d_col_dd);
+                                              c->d_dd_prefix, c->d_col_dd, c->cap, c->d_status);
     // ghost positions and types for the current build
     k_dd_gather<<<blocks(c->dd_ghosts * 4, 256), 256, 0, s>>>(c->dd_ghosts, 4, (int)n, c->d_dd_owner,
-                                                              reinterpret_cast<float *>(c->d_pos));
+                                                              reinterpret_cast<float *>(c->d_pos), c->d_status);
     return cudaGetLastError();
 }
 

@@ -60,6 +60,9 @@ EdgeParams make_edge_params(const reann_ctx *c) {
         P.mu_hi[k] = (float)mu;
         P.mu_lo[k] = (float)(mu - (double)P.mu_hi[k]);
     }
+    P.n_rows = c->n_slots;
+    P.n_list = c->cap;
+    P.status = c->d_status;
     return P;
 }
 
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
     int q0_n = i < n ? row[i] : 0, q1_n = i < n ? row[i + 1] : 0;
     for (; i < n; i += stride) {
         const float4 pi = pi_n;
-        const int q0 = q0_n, q1 = q1_n;
+        const int q0 = q0_n, q1 = checked_end(q1_n, P.n_list, P.status);
         if (i + stride < n) {
             pi_n = pos[i + stride];
             q0_n = row[i + stride];
@@ -124,7 +127,7 @@ __global__ void __launch_bounds__(128, 8) k_active(int n, const float4 *__restri
 #pragma unroll
             for (int b = 0; b < B; ++b) {
                 const int q = base + LPR * b + sl;
-                j[b] = q < q1 ? col[q] : -1;
+                j[b] = q < q1 ? (int)checked(col[q], P.n_rows, P.status) : -1;
             }
 #pragma unroll
             for (int b = 0; b < B; ++b) pj[b] = j[b] >= 0 ? pos[j[b]] : pi;
@@ -278,8 +281,8 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
 #pragma unroll
         for (int u = 0; u < NT; ++u) acc[m][u] = R(0);
     const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
-    const int q0 = live ? row[i] + part : 0, q1 = live ? row[i] + act_cnt[i] : 0;
-    int j_next = q0 < q1 ? act_col[q0] : 0;
+    const int q0 = live ? row[i] + part : 0, q1 = live ? checked_end(row[i] + act_cnt[i], P.n_list, P.status) : 0;
+    int j_next = q0 < q1 ? (int)checked(act_col[q0], P.n_rows, P.status) : 0;
     float4 g_next = q0 < q1 ? act_geo[q0] : make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (!ACC64) {
         // fp32 sums: the lane's two radial indices as packed pairs (m = 0, m = 1)
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             const int j = j_next;
             const float4 g = g_next;
             if (q + stride < q1) {
-                j_next = act_col[q + stride];
+                j_next = (int)checked(act_col[q + stride], P.n_rows, P.status);
                 g_next = act_geo[q + stride];
             }
             const float r = g.w;
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(128) k_density_fwd(int n, const int *__restric
             const float4 g = g_next;         // dx, dy, dz, r
             const float dr = dr_next;        // r - fp32(r)
             if (q + stride < q1) {
-                j_next = act_col[q + stride];
+                j_next = (int)checked(act_col[q + stride], P.n_rows, P.status);
                 g_next = act_geo[q + stride];
                 if (act_dr) dr_next = act_dr[q + stride];
             }
@@ -441,18 +444,18 @@ __global__ void __launch_bounds__(128, 6) k_edge_bwd(int n, const int *__restric
         // the backward takes the constants' fp32 values: its rounding shifts forces by
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float mh[2] = {P.mu_hi[n0], P.mu_hi[n0 + 1]};
-        const int q0 = row[i] + part, q1 = row[i] + act_cnt[i];
+        const int q0 = row[i] + part, q1 = checked_end(row[i] + act_cnt[i], P.n_list, P.status);
         // the edge list takes ordinary cached loads: its 16-byte entries share
         // 32-byte sectors with the next edge's, and evict-first loads made the
         // second read of a sector go back to DRAM (1.6x the traffic, no faster)
-        int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
+        int j_next = q0 < q1 ? (int)checked(__ldg(act_col + q0), P.n_rows, P.status) : 0;
         float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; q += stride) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
             if (q + stride < q1) {
-                j_next = __ldg(act_col + q + stride);
+                j_next = (int)checked(__ldg(act_col + q + stride), P.n_rows, P.status);
                 geo_next = __ldg(act_geo + q + stride);
             }
             const float3 d = make_float3(geo.x, geo.y, geo.z);
@@ -621,18 +624,18 @@ __global__ void __launch_bounds__(128, (NP == 10 && HAS_DC) ? 5 : 6)
         // the backward takes the constants' fp32 values: its rounding shifts forces by
         // ~1e-6 eV/A, and the fp32 pairs cost 8 % of its time
         const float2 nmu = make_float2(-P.mu_hi[n0], -P.mu_hi[n0 + 1]);
-        const int q0 = row[i] + part, q1 = row[i] + act_cnt[i];
+        const int q0 = row[i] + part, q1 = checked_end(row[i] + act_cnt[i], P.n_list, P.status);
         // the edge list takes ordinary cached loads: its 16-byte entries share
         // 32-byte sectors with the next edge's, and evict-first loads made the
         // second read of a sector go back to DRAM (1.6x the traffic, no faster)
-        int j_next = q0 < q1 ? __ldg(act_col + q0) : 0;
+        int j_next = q0 < q1 ? (int)checked(__ldg(act_col + q0), P.n_rows, P.status) : 0;
         float4 geo_next = q0 < q1 ? __ldg(act_geo + q0) : make_float4(0.f, 0.f, 0.f, 1.f);
         for (int q = q0; q < q1; q += stride) {
             // the next edge's index and geometry are in flight while this one computes
             const int j = j_next;
             const float4 geo = geo_next;
             if (q + stride < q1) {
-                j_next = __ldg(act_col + q + stride);
+                j_next = (int)checked(__ldg(act_col + q + stride), P.n_rows, P.status);
                 geo_next = __ldg(act_geo + q + stride);
             }
             const float r = geo.w;

@@ -30,23 +30,25 @@ namespace {
 inline unsigned nblocks(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
 
 // dst[k] = src[inv[caller[k]]] (rows of `width` floats); caller == nullptr:
-// ghost rows, caller index n_local + k
+// ghost rows, caller index n_local + k.  n: rows of src (own atoms and ghosts)
 __global__ void k_halo_pack(int64_t rows, int width, const int *__restrict__ caller, int64_t n_local,
-                            const int *__restrict__ inv, const float *__restrict__ src, float *__restrict__ dst) {
+                            const int *__restrict__ inv, const float *__restrict__ src, float *__restrict__ dst,
+                            int64_t n, int *__restrict__ status) {
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= rows * width) return;
     const int64_t r = k / width, f = k - r * width;
-    const int64_t a = caller ? (int64_t)caller[r] : n_local + r;
-    dst[k] = src[(int64_t)inv[a] * width + f];
+    const int64_t a = caller ? checked(caller[r], n_local, status) : n_local + r;
+    dst[k] = src[checked(inv[a], n, status) * width + f];
 }
 
 // ghost rows of dst (internal order) = recv rows in ghost order
 __global__ void k_halo_unpack_ghosts(int64_t rows, int width, int64_t n_local, const int *__restrict__ inv,
-                                     const float *__restrict__ recv, float *__restrict__ dst) {
+                                     const float *__restrict__ recv, float *__restrict__ dst, int64_t n,
+                                     int *__restrict__ status) {
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= rows * width) return;
     const int64_t r = k / width, f = k - r * width;
-    dst[(int64_t)inv[n_local + r] * width + f] = recv[k];
+    dst[checked(inv[n_local + r], n, status) * width + f] = recv[k];
 }
 
 // own rows of dst += the partials received for their send-list entries, summed
@@ -54,13 +56,15 @@ __global__ void k_halo_unpack_ghosts(int64_t rows, int width, int64_t n_local, c
 __global__ void k_halo_add_partials(int64_t atoms, int width, const int *__restrict__ atom_caller,
                                     const int *__restrict__ off, const int *__restrict__ order,
                                     const int *__restrict__ inv, const float *__restrict__ recv,
-                                    float *__restrict__ dst) {
+                                    float *__restrict__ dst, int64_t n_local, int64_t n_send, int64_t n,
+                                    int *__restrict__ status) {
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= atoms * width) return;
     const int64_t u = k / width, f = k - u * width;
     float s = 0.f;
-    for (int p = off[u]; p < off[u + 1]; ++p) s += recv[(int64_t)order[p] * width + f];
-    float *d = dst + (int64_t)inv[atom_caller[u]] * width + f;
+    const int p1 = checked_end(off[u + 1], n_send, status);
+    for (int p = off[u]; p < p1; ++p) s += recv[checked(order[p], n_send, status) * width + f];
+    float *d = dst + checked(inv[checked(atom_caller[u], n_local, status)], n, status) * width + f;
     *d += s;
 }
 
@@ -70,7 +74,7 @@ cudaError_t launch_halo_pack_own(reann_ctx *c, const float *src, int width, cuda
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (c->n_send > 0)
         k_halo_pack<<<nblocks(c->n_send * width, 256), 256, 0, s>>>(c->n_send, width, c->d_send_caller, c->n_local,
-                                                                    c->d_inv, src, c->d_xsend);
+                                                                    c->d_inv, src, c->d_xsend, c->n, c->d_status);
     return cudaGetLastError();
 }
 
@@ -79,7 +83,7 @@ cudaError_t launch_halo_pack_ghosts(reann_ctx *c, const float *src, int width, c
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (ng > 0)
         k_halo_pack<<<nblocks(ng * width, 256), 256, 0, s>>>(ng, width, nullptr, c->n_local, c->d_inv, src,
-                                                             c->d_xsend);
+                                                             c->d_xsend, c->n, c->d_status);
     return cudaGetLastError();
 }
 
@@ -88,7 +92,7 @@ cudaError_t launch_halo_unpack_ghosts(reann_ctx *c, float *dst, int width, cudaS
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (ng > 0)
         k_halo_unpack_ghosts<<<nblocks(ng * width, 256), 256, 0, s>>>(ng, width, c->n_local, c->d_inv, c->d_xrecv,
-                                                                      dst);
+                                                                      dst, c->n, c->d_status);
     return cudaGetLastError();
 }
 
@@ -96,7 +100,8 @@ cudaError_t launch_halo_add_partials(reann_ctx *c, float *dst, int width, cudaSt
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (c->n_send_atoms > 0)
         k_halo_add_partials<<<nblocks(c->n_send_atoms * width, 256), 256, 0, s>>>(
-            c->n_send_atoms, width, c->d_send_atom, c->d_send_off, c->d_send_order, c->d_inv, c->d_xrecv, dst);
+            c->n_send_atoms, width, c->d_send_atom, c->d_send_off, c->d_send_order, c->d_inv, c->d_xrecv, dst,
+            c->n_local, c->n_send, c->n, c->d_status);
     return cudaGetLastError();
 }
 

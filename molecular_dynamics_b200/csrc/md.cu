@@ -21,7 +21,7 @@ __global__ void k_pos_from_caller(int64_t n, const float *__restrict__ pos, cons
                                   const int *__restrict__ types, float4 *__restrict__ pos4, int *__restrict__ status) {
     int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= n) return;
-    int64_t a = perm[s];
+    int64_t a = checked(perm[s], n, status);
     float x = pos[3 * a], y = pos[3 * a + 1], z = pos[3 * a + 2];
     if (!isfinite(x) || !isfinite(y) || !isfinite(z)) atomicOr(status, ST_NONFINITE);
     pos4[s] = make_float4(x, y, z, __int_as_float(types[a]));
@@ -81,10 +81,11 @@ cudaError_t launch_energy_sum(reann_ctx *c, cudaStream_t s) {
 }
 
 __global__ void k_scatter_outputs(int64_t n, const int *__restrict__ perm, const float *__restrict__ F,
-                                  const float *__restrict__ Ei, float *__restrict__ Fo, float *__restrict__ Eo) {
+                                  const float *__restrict__ Ei, float *__restrict__ Fo, float *__restrict__ Eo,
+                                  int *__restrict__ status) {
     int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= n) return;
-    int64_t a = perm[s];
+    int64_t a = checked(perm[s], n, status);
     if (Fo) {
         Fo[3 * a] = F[3 * s];
         Fo[3 * a + 1] = F[3 * s + 1];
@@ -97,22 +98,24 @@ cudaError_t launch_scatter_outputs(reann_ctx *c, float *d_forces, float *d_atom_
     const int64_t nc = centres(c);   // own atoms sit at internal [0, nc) and caller [0, nc)
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (nc > 0 && (d_forces || d_atom_energy))
-        k_scatter_outputs<<<blocks(nc, 256), 256, 0, s>>>(nc, c->d_perm, c->d_F, c->d_Ei, d_forces, d_atom_energy);
+        k_scatter_outputs<<<blocks(nc, 256), 256, 0, s>>>(nc, c->d_perm, c->d_F, c->d_Ei, d_forces, d_atom_energy,
+                                                          c->d_status);
     return cudaGetLastError();
 }
 
 // internal rows of `width` floats -> caller order
 __global__ void k_rows_to_caller(int64_t n, int width, const int *__restrict__ perm, const float *__restrict__ in,
-                                 float *__restrict__ out) {
+                                 float *__restrict__ out, int *__restrict__ status) {
     int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= n * width) return;
     int64_t s = k / width, f = k % width;
-    out[(int64_t)perm[s] * width + f] = in[k];
+    out[checked(perm[s], n, status) * width + f] = in[k];
 }
 
 cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int width, float *d_caller, cudaStream_t s) {
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
-    if (c->n > 0) k_rows_to_caller<<<blocks(c->n * width, 256), 256, 0, s>>>(c->n, width, c->d_perm, d_internal, d_caller);
+    if (c->n > 0) k_rows_to_caller<<<blocks(c->n * width, 256), 256, 0, s>>>(c->n, width, c->d_perm, d_internal, d_caller,
+                                                                            c->d_status);
     return cudaGetLastError();
 }
 
@@ -120,10 +123,11 @@ cudaError_t launch_to_caller_rows(reann_ctx *c, const float *d_internal, int wid
 // MD state
 
 __global__ void k_md_gather(int64_t n, const int *__restrict__ perm, const double *__restrict__ xc,
-                            const double *__restrict__ vc, double *__restrict__ x, double *__restrict__ v) {
+                            const double *__restrict__ vc, double *__restrict__ x, double *__restrict__ v,
+                            int *__restrict__ status) {
     int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= n) return;
-    int64_t a = perm[s];
+    int64_t a = checked(perm[s], n, status);
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
         x[3 * s + k] = xc[3 * a + k];
@@ -133,16 +137,17 @@ __global__ void k_md_gather(int64_t n, const int *__restrict__ perm, const doubl
 
 cudaError_t launch_md_gather(reann_ctx *c, const double *d_x_caller, const double *d_v_caller, cudaStream_t s) {
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
-    if (c->n > 0) k_md_gather<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, d_x_caller, d_v_caller, c->d_x, c->d_v);
+    if (c->n > 0) k_md_gather<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, d_x_caller, d_v_caller, c->d_x, c->d_v,
+                                                                 c->d_status);
     return cudaGetLastError();
 }
 
 __global__ void k_md_scatter(int64_t n, const int *__restrict__ perm, const double *__restrict__ x,
                              const double *__restrict__ v, double *__restrict__ xc, double *__restrict__ vc,
-                             float *__restrict__ pc) {
+                             float *__restrict__ pc, int *__restrict__ status) {
     int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= n) return;
-    int64_t a = perm[s];
+    int64_t a = checked(perm[s], n, status);
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
         double xv = x[3 * s + k];
@@ -157,7 +162,7 @@ cudaError_t launch_md_scatter(reann_ctx *c, double *d_x_caller, double *d_v_call
     REANN_TIMED(c, REANN_K_OTHER, s, 1);
     if (c->n > 0)
         k_md_scatter<<<blocks(c->n, 256), 256, 0, s>>>(c->n, c->d_perm, c->d_x, c->d_v, d_x_caller, d_v_caller,
-                                                       d_pos_caller);
+                                                       d_pos_caller, c->d_status);
     return cudaGetLastError();
 }
 

@@ -172,10 +172,10 @@ __global__ void k_bin_sort(int nbins, const int *__restrict__ bin_start, const i
 
 __global__ void k_gather_pos(int64_t n, const float *__restrict__ pos, const int *__restrict__ types,
                              const int *__restrict__ perm, float4 *__restrict__ pos4, float4 *__restrict__ pos_build,
-                             int *__restrict__ inv) {
+                             int *__restrict__ inv, int *__restrict__ status) {
     int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= n) return;
-    int a = perm[s];
+    int a = (int)checked(perm[s], n, status);
     float4 p = make_float4(pos[3 * (int64_t)a], pos[3 * (int64_t)a + 1], pos[3 * (int64_t)a + 2], __int_as_float(types[a]));
     pos4[s] = p;
     pos_build[s] = p;
@@ -345,7 +345,7 @@ cudaError_t launch_build(reann_ctx *c, const float *d_pos_caller, const int *d_t
         k_bin_sort<<<blocks((int64_t)c->nbins * 32, 256), 256, 0, s>>>(c->nbins, c->d_bin_start, c->d_perm_tmp,
                                                                        c->d_perm);
         k_gather_pos<<<blocks(n, 256), 256, 0, s>>>(n, d_pos_caller, d_types_caller, c->d_perm, c->d_pos,
-                                                    c->d_pos_build, c->d_inv);
+                                                    c->d_pos_build, c->d_inv, c->d_status);
         launch_nbr<false>(c, n, B, nullptr, c->d_cnt, nullptr, s);
     }
     if ((e = scan_exclusive(c->d_cnt, c->d_row, n, c->d_i64 + 1, c->d_scan_tmp, s))) return e;

@@ -16,15 +16,18 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libreann.so")
+CHECKED_LIB_PATH = os.path.join(HERE, "libreann_checked.so")   # built with `build --checked`
 
 STATUS = {
     0: "REANN_OK", 1: "REANN_ERR_ARG", 2: "REANN_ERR_BOX", 3: "REANN_ERR_CAPACITY", 4: "REANN_ERR_NONFINITE",
     5: "REANN_ERR_SKIN", 6: "REANN_ERR_STATE", 7: "REANN_ERR_CUDA", 8: "REANN_ERR_TIMEOUT", 9: "REANN_ERR_UNSUPPORTED",
+    10: "REANN_ERR_INDEX",
 }
 
 EXPORTS = ("reann_create", "reann_destroy", "reann_build_neighbors", "reann_energy_forces", "reann_md_step",
            "reann_md_step_nvt", "reann_get_counters", "reann_last_error", "reann_get_neighbors", "reann_get_features", "reann_profile",
-           "reann_profile_read", "reann_pair_list_noalloc", "reann_halo_plan", "reann_energy_forces_halo")
+           "reann_profile_read", "reann_pair_list_noalloc", "reann_halo_plan", "reann_energy_forces_halo",
+           "reann_checked", "reann_debug_set_neighbor")
 
 # kinds of the exchange function (include/reann.h)
 EXCHANGE_COEF, EXCHANGE_COEF_GRAD, EXCHANGE_FORCE = 0, 1, 2
@@ -88,6 +91,8 @@ def load(path: str = LIB_PATH):
     lib.reann_profile_read.argtypes = [P, I32, C.POINTER(D), C.POINTER(I64)]
     lib.reann_halo_plan.argtypes = [P, I64, I64, P, I64]
     lib.reann_energy_forces_halo.argtypes = [P, P, C.POINTER(D), P, P, ExchangeFn, P, P]
+    lib.reann_checked.argtypes = []
+    lib.reann_debug_set_neighbor.argtypes = [P, I64, I32]
     for name in EXPORTS:
         if name != "reann_last_error":
             getattr(lib, name).restype = C.c_int
@@ -120,6 +125,11 @@ def _stream(stream) -> Optional[int]:
     except ImportError:
         pass
     return None
+
+
+def reann_checked() -> bool:
+    """True when the loaded library is the checked build (every internal index tested before use)."""
+    return bool(load().reann_checked())
 
 
 def reann_pair_list_noalloc(pos, box, r_cut: float, skin: float, row, col, stream=None) -> int:
@@ -305,6 +315,10 @@ class Context:
         col = np.zeros(max(nnz, 1), np.int32)
         self._check(self.lib.reann_get_neighbors(self.h, row.ctypes.data, col.ctypes.data, nnz, _stream(stream)))
         return row, col[:nnz]
+
+    def reann_debug_set_neighbor(self, k: int, j: int):
+        """Checked build only: writes j into entry k of the neighbour list (host-side fault injection)."""
+        self._check(self.lib.reann_debug_set_neighbor(self.h, int(k), int(j)))
 
     def reann_profile(self, enable: bool = True):
         self._check(self.lib.reann_profile(self.h, 1 if enable else 0))

@@ -39,6 +39,20 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(declared_functions()) == set(reann.EXPORTS)
 
 
+def test_normal_build_is_unchecked_and_refuses_fault_injection(lib):
+    assert lib.reann_checked() == 0
+    assert lib.reann_debug_set_neighbor(None, 0, 0) == 1
+
+
+def test_checked_build_exports_the_same_symbols():
+    path = build.build(checked=True)
+    clib = C.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(clib, name), name
+    clib.reann_checked.restype = C.c_int32
+    assert clib.reann_checked() == 1
+
+
 def test_create_rejects_bad_blob_size_without_touching_the_gpu(lib):
     p = presets.get("ag256")
     w = synth.weight_blob(p)
