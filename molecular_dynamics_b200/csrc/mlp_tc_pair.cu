@@ -10,12 +10,13 @@
 // 32 (w % 4) .. + 31, and warp group w / 4 takes one 32-column chunk of every
 // 128-wide accumulator.
 //
-// Inputs: the next tile's 108-wide rho rows are prefetched into L2 (one bulk
-// prefetch) while the current tile computes; each tile loads its rows in
-// element order (coalesced) and each thread writes its elements, standardised
-// and split into bf16 hi + lo, straight into the K-major operand tile.  Outputs leave through idle buffers: the
-// coefficient rows through the input tile (consumed by the first product), the
-// 108-wide dE/drho rows through the activation tile (consumed by the last).
+// Inputs: the next tile's 108-wide rho rows (432-byte rows, whole 16-byte
+// units) are copied into the input operand buffer by one bulk copy, issued by
+// thread 0 as soon as the current tile's first product has read that buffer,
+// so the copy runs behind the rest of the tile; each thread then converts 8
+// features of a row at a time, standardised and split into bf16 hi + lo, in
+// place.  Outputs leave through the activation tile once the last product has
+// read it: the coefficient rows, or the 108-wide dE/drho rows.
 // dE/dA (Eq. 4 for the pair form):
 //   G_{n,tau} = l!/tau! sum_m (1 + [m = n]) A_{m,tau} dE/drho_(min(n,m), max(n,m), l),
 // four threads per atom, each owning two radial indices and writing its 20
@@ -47,11 +48,13 @@ struct PairLayout {
     static constexpr int ACT = DY + (MODE == TC_BWD ? 2 * TM * KPAD * 2 : 0);  // [TM][128] x 2
     static constexpr int F32 = ACT + 2 * TM * 128 * 2;
     static constexpr int nf32 = 128 + 128 + KPAD + 2 * KIN + 128 + 4 * TM;   // b1, b2, b3, shift, 1/scale, w3, e parts
-    static constexpr int BAR = F32 + nf32 * 4;
+    static constexpr int BAR = F32 + nf32 * 4;   // MMA-completion mbarrier; input-copy mbarrier at BAR + 8
     static constexpr int bytes = BAR + 32;
     static constexpr int C_Z1 = 0, C_Z2 = 128, C_P = 256, C_OUT = 384;
     static_assert(TM * GXS * 4 <= 2 * TM * 128 * 2, "dE/drho rows fit the activation tile");
-    static_assert(TM * YS * 4 <= (KIN / 8 - 1) * TM * 16, "output rows leave the input tile's padding chunk alone");
+    static_assert(TM * YS * 4 <= 2 * TM * 128 * 2, "output rows fit the activation tile");
+    static_assert(TM * DIN * 4 <= 2 * TM * KIN * 2 && (DIN * 4) % 16 == 0, "raw rows fit the input tile, 16-byte rows");
+    static_assert(BAR % 16 == 0, "aligned barriers");
     static_assert(X % 16 == 0 && DY % 16 == 0 && ACT % 16 == 0 && F32 % 16 == 0, "16-byte aligned tiles");
 };
 
@@ -77,11 +80,12 @@ __global__ void __launch_bounds__(PT, 1)
     float *sb1 = f32, *sb2 = sb1 + 128, *sb3 = sb2 + 128, *sshift = sb3 + KPAD, *sinv = sshift + KIN,
           *sw3 = sinv + KIN, *se = sw3 + 128;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint64_t *cbar = reinterpret_cast<uint64_t *>(sm + L::BAR + 8);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
     unsigned char *x_hi = sm + L::X, *x_lo = x_hi + TM * KIN * 2;
     unsigned char *dy_hi = sm + L::DY, *dy_lo = dy_hi + TM * KPAD * 2;
     unsigned char *act_hi = sm + L::ACT, *act_lo = act_hi + TM * 128 * 2;
-    float *ystage = reinterpret_cast<float *>(x_hi);     // output rows (forward), after the first product
+    float *ystage = reinterpret_cast<float *>(act_hi);   // output rows (forward), after the last product
     float *gxs = reinterpret_cast<float *>(act_hi);      // dE/drho rows, after the last product
 
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -98,12 +102,12 @@ __global__ void __launch_bounds__(PT, 1)
     }
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(cbar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // operand tiles start at zero: the padding columns (features 108..111,
-    // upstream gradients 24..31) are never written again
-    for (int k = tid; k < (2 * TM * KIN * 2) / 16; k += PT)
-        reinterpret_cast<uint4 *>(x_hi)[k] = make_uint4(0u, 0u, 0u, 0u);
+    // the upstream-gradient operand starts at zero: its padding columns
+    // (24..31) are never written again (the input operand's padding, features
+    // 108..111, is rewritten with every tile)
     if (MODE == TC_BWD)
         for (int k = tid; k < (2 * TM * KPAD * 2) / 16; k += PT)
             reinterpret_cast<uint4 *>(dy_hi)[k] = make_uint4(0u, 0u, 0u, 0u);
@@ -131,9 +135,26 @@ __global__ void __launch_bounds__(PT, 1)
     // raw rows: the next tile's (contiguous) rows are prefetched into L2 while
     // the current tile computes; each tile then loads its own rows from L2 in
     // element order (coalesced), so no registers stay live across a tile
-    constexpr int NXR = (TM * DIN + PT - 1) / PT;   // 27
-    constexpr int NDR = (TM * PD + PT - 1) / PT;    // 6
+    constexpr int NCH = KIN / 8;                      // 14 eight-feature chunks per row
+    constexpr int NXC = (TM * NCH + PT - 1) / PT;    // 4 chunks per thread
+    constexpr int NDR = (TM * PD + PT - 1) / PT;     // 6
     int4 tl = blockIdx.x < n_tiles ? tiles[blockIdx.x] : make_int4(0, 0, 0, 0);
+    // a tile's raw rho rows -> the input operand buffer by one bulk copy
+    // (thread 0), completion on cbar
+    uint32_t cphase = 0;
+    bool copy_pending = false;
+    auto copy_rows = [&](int rr0, int rrows) {
+        if (tid == 0) {
+            const uint32_t nb = (uint32_t)(rrows * DIN * 4);
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(cbar)), "r"(nb)
+                         : "memory");
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         ::"r"(sa(x_hi)), "l"(X + (int64_t)rr0 * DIN), "r"(nb), "r"(smem_u32(cbar))
+                         : "memory");
+        }
+        copy_pending = true;
+    };
+    if (tl.z > 0) copy_rows(tl.y, tl.z);
     for (int ti = blockIdx.x; ti < n_tiles && !failed; ti += gridDim.x) {
         const int4 tile = tl;
         const int e = tile.x, r0 = tile.y, rows = tile.z;
@@ -164,26 +185,41 @@ __global__ void __launch_bounds__(PT, 1)
         }
         if (tid == 0) {
             if (MODE != TC_FWD) prefetch_l2(A + (int64_t)r0 * PNA, (uint32_t)(rows * PNA * 4));
-            if (tl.z > 0) {
-                prefetch_l2(X + (int64_t)tl.y * DIN, (uint32_t)(tl.z * DIN * 4));
-                if (MODE == TC_BWD) prefetch_l2(dY + (int64_t)tl.y * PD, (uint32_t)(tl.z * PD * 4));
-            }
+            if (MODE == TC_BWD && tl.z > 0) prefetch_l2(dY + (int64_t)tl.y * PD, (uint32_t)(tl.z * PD * 4));
         }
-        // this thread's elements of the tile: standardised, split bf16, into the operand tiles
+        // the tile's raw rows have arrived in the input buffer: each thread reads
+        // 8-feature chunks (chunk k / TM of row k % TM: a warp takes one chunk of
+        // 32 consecutive rows, so neither the 432-byte-strided reads nor the
+        // K-major operand stores meet a bank twice), then, once every thread has
+        // read its chunks, writes them standardised and split bf16 in place
+        // (features past 108 and rows past the tile's end as zeros)
         {
-            const float *xg = X + (int64_t)r0 * DIN;
-            float xr[NXR];
+            const bool landed = bar_wait(cbar, cphase);
+            cphase ^= 1u;
+            copy_pending = !landed;
+            if (__syncthreads_or(!landed)) { failed = true; break; }
+            const float *xs = reinterpret_cast<const float *>(x_hi);
+            float xr[NXC][8];
 #pragma unroll
-            for (int u = 0; u < NXR; ++u) {
-                const int k = tid + u * PT;
-                xr[u] = k < rows * DIN ? xg[k] : 0.f;
+            for (int u = 0; u < NXC; ++u) {
+                const int k = tid + u * PT, rk = k % TM, f0 = 8 * (k / TM);
+#pragma unroll
+                for (int h4 = 0; h4 < 8; h4 += 4) {
+                    const bool ok = k < TM * NCH && rk < rows && f0 + h4 < DIN;
+                    const float4 t = ok ? *reinterpret_cast<const float4 *>(xs + rk * DIN + f0 + h4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    xr[u][h4] = t.x, xr[u][h4 + 1] = t.y, xr[u][h4 + 2] = t.z, xr[u][h4 + 3] = t.w;
+                }
             }
+            __syncthreads();
 #pragma unroll
-            for (int u = 0; u < NXR; ++u) {
-                const int k = tid + u * PT;
-                if (k < rows * DIN) {
-                    const int rk = k / DIN, f = k - rk * DIN;
-                    st_elem2(x_hi, x_lo, TM, rk, f, (xr[u] - sshift[f]) * sinv[f]);
+            for (int u = 0; u < NXC; ++u) {
+                const int k = tid + u * PT, rk = k % TM, f0 = 8 * (k / TM);
+                if (k < TM * NCH) {
+#pragma unroll
+                    for (int e2 = 0; e2 < 8; ++e2)
+                        xr[u][e2] = rk < rows ? (xr[u][e2] - sshift[f0 + e2]) * sinv[f0 + e2] : 0.f;
+                    st_chunk2(x_hi, x_lo, TM, rk, f0, xr[u]);
                 }
             }
         }
@@ -213,6 +249,8 @@ __global__ void __launch_bounds__(PT, 1)
             mma_commit(bar);
         }
         if (!wait_mma()) { failed = true; break; }
+        // the first product has read the input buffer: the next tile's raw rows may land there
+        if (tl.z > 0) copy_rows(tl.y, tl.z);
         {
             float v[32];
             tmem_ld32(lane_base + L::C_Z1 + c, v);
@@ -372,6 +410,8 @@ __global__ void __launch_bounds__(PT, 1)
         __syncthreads();
     }
 
+    // a copy still in flight (the block left early) lands before the block exits
+    if (copy_pending) bar_wait(cbar, cphase & 1u);
     if (failed && tid == 0) atomicOr(status, ST_TIMEOUT);
     fence_before();
     __syncthreads();
