@@ -21,6 +21,8 @@
 //   G_{n,tau} = l!/tau! sum_m (1 + [m = n]) A_{m,tau} dE/drho_(min(n,m), max(n,m), l),
 // four threads per atom, each owning two radial indices and writing its 20
 // values as five float4 in the edge kernels' lane-interleaved order.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -355,54 +357,74 @@ __global__ void __launch_bounds__(PT, 1)
                 }
             }
             __syncthreads();
-            // G = dE/dA: thread (atom rk, part) takes radial indices n = 2 part, 2 part + 1.  Per l it
-            // forms the coupling rows M_{n,m} = (1 + [m = n]) dE/drho_(min, max of n m, l) once and
-            // streams the atom's A_{m,tau}; its 20 results are the lane-interleaved positions
-            // 16 q + 4 part + e (q < 5, e < 4), i.e. five float4 stores.
+            // G = dE/dA: thread (atom rk, part) takes radial indices n = 2 part, 2 part + 1.  It
+            // loads its quarter of the atom's A row (A_{m,tau} for m = 2 part, 2 part + 1: five
+            // float4) and receives the other quarters from the atom's three other lanes by warp
+            // shuffles.  Per l it forms the coupling rows M_{n,m} = (1 + [m = n])
+            // dE/drho_(min, max of n m, l) once and streams A_{m,tau}; its 20 results are the
+            // lane-interleaved positions 16 q + 4 part + e (q < 5, e < 4), i.e. five float4 stores.
             {
-                const int rk = tid >> 2, part = tid & 3;
-                if (rk < rows) {
-                    const float *g = gxs + rk * GXS;
-                    const float *ar = A + (int64_t)(r0 + rk) * PNA;
-                    float acc[2][NT];
-#pragma unroll
-                    for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                        for (int u = 0; u < NT; ++u) acc[s2][u] = 0.f;
-#pragma unroll
-                    for (int l = 0; l < 3; ++l) {
-                        float M[2][PNP];
-#pragma unroll
-                        for (int s2 = 0; s2 < 2; ++s2) {
-                            const int n = 2 * part + s2;
-#pragma unroll
-                            for (int m = 0; m < PNP; ++m) {
-                                const int lo = m < n ? m : n, hi = m < n ? n : m;
-                                M[s2][m] = (m == n ? 2.f : 1.f) * g[l * PP + lo * PNP - lo * (lo - 1) / 2 + (hi - lo)];
-                            }
-                        }
-                        constexpr int T0[3] = {0, 1, 4}, T1[3] = {1, 4, 10};
-#pragma unroll
-                        for (int u = T0[l]; u < T1[l]; ++u)
-#pragma unroll
-                            for (int m = 0; m < PNP; ++m) {
-                                const float a = ar[m * NT + u];
-                                acc[0][u] = fmaf(M[0][m], a, acc[0][u]);
-                                acc[1][u] = fmaf(M[1][m], a, acc[1][u]);
-                            }
-                    }
-                    float4 *go4 = reinterpret_cast<float4 *>(Gout + (int64_t)(r0 + rk) * PNA);
+                const int rk = tid >> 2, part = tid & 3, lead = tid & 28;
+                const bool live = rk < rows;
+                const float *g = gxs + rk * GXS;
+                float aq[2 * NT];   // A_{2 part + s, tau} at 10 s + tau
+                {
+                    const float4 *a4 =
+                        reinterpret_cast<const float4 *>(A + (int64_t)(r0 + (live ? rk : 0)) * PNA) + 5 * part;
 #pragma unroll
                     for (int q = 0; q < 5; ++q) {
-                        float v[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int idx = 4 * q + e2;   // g_lane_index order
-                            const int s2 = nets.g_pairs ? idx % 2 : idx / NT, u = nets.g_pairs ? idx / 2 : idx % NT;
-                            v[e2] = (u >= 7 ? 2.f : 1.f) * acc[s2][u];   // l!/tau!
-                        }
-                        go4[4 * q + part] = make_float4(v[0], v[1], v[2], v[3]);
+                        const float4 v = live ? __ldg(a4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        aq[4 * q] = v.x, aq[4 * q + 1] = v.y, aq[4 * q + 2] = v.z, aq[4 * q + 3] = v.w;
                     }
+                }
+                float acc[2][NT];
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                    for (int u = 0; u < NT; ++u) acc[s2][u] = 0.f;
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                    float M[2][PNP];
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int n = 2 * part + s2;
+#pragma unroll
+                        for (int m = 0; m < PNP; ++m) {
+                            const int lo = m < n ? m : n, hi = m < n ? n : m;
+                            M[s2][m] = (m == n ? 2.f : 1.f) * g[l * PP + lo * PNP - lo * (lo - 1) / 2 + (hi - lo)];
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < NT; ++u) {
+                        // the tuples of order l: u in [0, 1), [1, 4), [4, 10)
+                        if (u < (l == 0 ? 0 : (l == 1 ? 1 : 4)) || u >= (l == 0 ? 1 : (l == 1 ? 4 : 10))) continue;
+#pragma unroll
+                        for (int m = 0; m < PNP; ++m) {
+                            const float a = __shfl_sync(0xffffffffu, aq[(m & 1) * NT + u], lead + (m >> 1));
+                            acc[0][u] = fmaf(M[0][m], a, acc[0][u]);
+                            acc[1][u] = fmaf(M[1][m], a, acc[1][u]);
+                        }
+                    }
+                }
+                if (live) {
+                    float4 *go4 = reinterpret_cast<float4 *>(Gout + (int64_t)(r0 + rk) * PNA);
+                    // l!/tau! times the sums, in the layer's lane order (pairs: idx = 2 tau + s,
+                    // radial-major: idx = 10 s + tau)
+                    auto put = [&](auto pairs) {
+#pragma unroll
+                        for (int q = 0; q < 5; ++q) {
+                            float v[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const int idx = 4 * q + e2;
+                                const int s2 = pairs ? idx % 2 : idx / NT, u = pairs ? idx / 2 : idx % NT;
+                                v[e2] = (u >= 7 ? 2.f : 1.f) * acc[s2][u];
+                            }
+                            go4[4 * q + part] = make_float4(v[0], v[1], v[2], v[3]);
+                        }
+                    };
+                    if (nets.g_pairs) put(std::true_type{});
+                    else put(std::false_type{});
                 }
             }
         }
