@@ -15,8 +15,9 @@
 // exponential (tanh.approx, accurate to about 11 bits, is not used here).
 //
 // Three launches per layer, as on the other network paths:
-//   forward (coefficient networks): x -> c^{t+1}; the derivative rows
-//     tanh'(z1), tanh'(z2) of every atom are written out for the backward;
+//   forward (coefficient networks): x -> c^{t+1}; the derivatives
+//     tanh'(z1), tanh'(z2) of every atom are written out for the backward
+//     (one column-major block per tile, so a warp's accesses are contiguous);
 //   energy: E_i and dE/dA of the last layer (forward and VJP in one pass);
 //   backward (coefficient networks): dE/dc^{t+1} -> dE/dA^t from the stored
 //     derivative rows -- three products, no recomputed forward.
@@ -94,22 +95,22 @@ struct T32Layout {
     static constexpr int bytes = SLOT + 16;
     static constexpr int RS = KPAD + 1;                 // stride of staged output rows (odd)
     static_assert(TM * RS * 4 <= SE, "output rows fit the activation planes");
+    static_assert(2 * X_PLANE + TM * RS * 4 <= SE, "raw input rows fit beside the input planes");
     static_assert(GROUP_BYTES % 16 == 0 && GRP % 16 == 0, "16-byte aligned operand planes");
     // TMEM columns of a group (base 256 g)
     static constexpr int C_A = 0, C_B = 64, C_C = 128;
 };
 
-// this thread's 32 derivative values of one layer: row i, columns 32 h .. + 31
-__device__ __forceinline__ void store32(float *dst, const float (&v)[32]) {
+// this thread's 32 derivative values of one layer (its row, columns 32 h ..
+// + 31), stored column-major inside the tile: column c of the tile's rows at
+// c * rows, so a warp's 32 rows of one column are 32 consecutive floats
+__device__ __forceinline__ void store_cols(float *dst, int stride, const float (&v)[32]) {
 #pragma unroll
-    for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4 *>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+    for (int u = 0; u < 32; ++u) dst[(int64_t)u * stride] = v[u];
 }
-__device__ __forceinline__ void load32(const float *src, float (&v)[32]) {
+__device__ __forceinline__ void load_cols(const float *src, int stride, float (&v)[32]) {
 #pragma unroll
-    for (int u = 0; u < 32; u += 4) {
-        const float4 q = __ldg(reinterpret_cast<const float4 *>(src + u));
-        v[u] = q.x; v[u + 1] = q.y; v[u + 2] = q.z; v[u + 3] = q.w;
-    }
+    for (int u = 0; u < 32; ++u) v[u] = __ldg(src + (int64_t)u * stride);
 }
 
 template <int NP, int MODE>
@@ -228,12 +229,21 @@ __global__ void __launch_bounds__(T32_THREADS, 1)
         const int4 tile = tiles[ti];
         const int r0 = tile.y, rows = tile.z;
         const bool live = row < rows;
-        const int64_t atom = r0 + (live ? row : 0);
-        float *dt_row = Dt + atom * (2 * H) + 32 * h;   // tanh'(z1) at [0, H), tanh'(z2) at [H, 2H)
+        // the tile's derivative block [2H][rows] at Dt + r0 2H: tanh'(z1) in columns
+        // [0, H), tanh'(z2) in [H, 2H); this thread's first column 32 h
+        float *dt_col = Dt + (int64_t)r0 * (2 * H) + (int64_t)(32 * h) * rows + row;
         if (MODE != TC_FWD && gt == 0) prefetch_l2(A + (int64_t)r0 * NA, (uint32_t)(rows * NA * 4));
-        // input: this thread's 16 features (x standardised, or dY), split tf32
+        // input: the tile's contiguous raw rows (x, or dY in the backward) in
+        // element order into padded rows in the free half of the activation
+        // planes, then this thread's 16 features (x standardised), split tf32
         {
-            const float *src = MODE == TC_BWD ? dY + atom * D : X + atom * D;
+            float *xs = reinterpret_cast<float *>(gs + L::ACT + 2 * L::X_PLANE);
+            const float *src = (MODE == TC_BWD ? dY : X) + (int64_t)r0 * D;
+            for (int k = gt; k < rows * D; k += T32_GROUP) {
+                const int rk = k / D, f = k - rk * D;
+                xs[rk * L::RS + f] = src[k];
+            }
+            grp_sync(g);
 #pragma unroll
             for (int c4 = 0; c4 < 16; c4 += 4) {
                 float v[4];
@@ -241,7 +251,8 @@ __global__ void __launch_bounds__(T32_THREADS, 1)
                 for (int u = 0; u < 4; ++u) {
                     const int f = 16 * h + c4 + u;
                     const bool ok = live && f < D;
-                    v[u] = !ok ? 0.f : (MODE == TC_BWD ? src[f] : (src[f] - sshift[f]) / sscale[f]);
+                    const float x = ok ? xs[row * L::RS + f] : 0.f;
+                    v[u] = !ok ? 0.f : (MODE == TC_BWD ? x : (x - sshift[f]) / sscale[f]);
                 }
                 st_chunk4_tf32(x_hi, x_lo, TM, row, 16 * h + c4, v);
             }
@@ -252,8 +263,8 @@ __global__ void __launch_bounds__(T32_THREADS, 1)
         if (MODE == TC_BWD) {
             // u = dY W3 into A, then g2 = u tanh'(z2) (stored by the forward)
             float d2[32];
-            if (live) load32(dt_row + H, d2);
-            if (live) load32(dt_row, d1);
+            if (live) load_cols(dt_col + H * rows, rows, d2);
+            if (live) load_cols(dt_col, rows, d1);
             if (!product(L::C_A, [&](uint32_t d) { gemm3_tf32<H, KPAD>(d, sa(x_hi), sa(x_lo), hi_of(L::W3T),
                                                                          hi_of(L::W3T + L::SQ)); })) {
                 failed = true;
@@ -279,7 +290,7 @@ __global__ void __launch_bounds__(T32_THREADS, 1)
                 v[u] = tanh_f32(v[u] + sb1[32 * h + u]);
                 d1[u] = 1.f - v[u] * v[u];
             }
-            if (MODE == TC_FWD && live) store32(dt_row, d1);
+            if (MODE == TC_FWD && live) store_cols(dt_col, rows, d1);
 #pragma unroll
             for (int u = 0; u < 32; u += 4) st_chunk4_tf32(act_hi, act_lo, TM, row, 32 * h + u, &v[u]);
             handoff();
@@ -306,7 +317,7 @@ __global__ void __launch_bounds__(T32_THREADS, 1)
                 float d2[32];
 #pragma unroll
                 for (int u = 0; u < 32; ++u) d2[u] = 1.f - v[u] * v[u];
-                store32(dt_row + H, d2);
+                store_cols(dt_col + H * rows, rows, d2);
             }
 #pragma unroll
             for (int u = 0; u < 32; u += 4) st_chunk4_tf32(act_hi, act_lo, TM, row, 32 * h + u, &v[u]);
@@ -456,7 +467,8 @@ bool tc32_supported(const reann_ctx *c) {
     return c->H1 == H && c->H2 == H && (c->NP == 8 || c->NP == 10) && c->DR == c->D;
 }
 
-// tanh' rows of coefficient network t: [n][2H] at d_tanhd + t n 2H
+// tanh' of coefficient network t: n 2H values at d_tanhd + t n 2H, one
+// column-major [2H][rows] block per 128-row tile at the tile's first row x 2H
 static float *tanhd_rows(reann_ctx *c, int t) { return c->d_tanhd + (int64_t)t * c->n * (2 * H); }
 
 cudaError_t launch_mlp_tc32_coef_fwd(reann_ctx *c, int t, cudaStream_t s) {
