@@ -24,9 +24,9 @@
 // MMA-completion mbarrier and named barrier, so one group's epilogue overlaps
 // the other's products.  In a group, warp w reads TMEM lanes 32 (w % 4) .. + 31
 // and half (w / 4) % 2 takes 64 columns of every 128-wide accumulator.  The
-// epilogue is bound by the tanh unit: bf16 rounding of the split operands is
-// done with integer instructions so that the special-function pipe only
-// evaluates tanh.  The coefficient backward recomputes the first layer's
+// epilogues keep the special-function unit (tanh) and the issue slots busy
+// while they run: bf16 rounding of the split operands is done with integer
+// instructions so that the special-function pipe only evaluates tanh.  The coefficient backward recomputes the first layer's
 // pre-activation (one small product) instead of keeping it, to fit 256 columns.
 //
 // Global traffic: the forward and energy networks' raw input rows arrive by
