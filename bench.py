@@ -394,6 +394,10 @@ def roofline(prof, active_pairs, NP, T, n_atoms, sm_count, pk, pk_kind, clk, net
     r["traffic"] = traffic
     r["traffic_note"] = EDGE_BWD_TRAFFIC_NOTE if traffic is not None else \
         "no DRAM capture of the current source of this kernel on this model"
+    if dominant in ("edge_bwd", "density"):
+        # what ncu shows binding the edge passes (the FP32 peak is the arithmetic roofline only)
+        r["limiter_note"] = ("ncu: the L1 data pipe at 72-78 % of its wavefront rate and the register "
+                             "writeback at 61-67 % (neighbour-row gathers); FP32 pipes about half busy")
     return r
 
 
