@@ -90,6 +90,25 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert time.perf_counter() - t0 < 60
 
 
+def test_reference_arm_prints_the_contract_line():
+    # one process (N = 1): the oracle's JSON line carries the metric of the GPU arm, a CPU
+    # baseline describing this run and an end-to-end entry with no host-device traffic
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "ag256",
+                        "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"],
+                       env=dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0"),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "atom-steps/s" and d["higher_is_better"] is True
+    assert d["metric"].startswith("atom-steps/s") and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["dtype"] == "f64" and d["data"] == "synthetic" and d["config"]["workload"].startswith("ag256")
+
+
 def test_roofline_arithmetic():
     import bench
     # 10 launches of 3 ms each of the edge backward; T = 3, N_phi = 8
