@@ -1,7 +1,8 @@
 // tcgen05 building blocks shared by the tensor-core network kernels
-// (mlp_tc.cu, mlp_tc_pair.cu): shared-memory and instruction descriptors, the
-// split-bf16 GEMM issued by one thread, MMA completion on an mbarrier with a
-// bounded wait, TMEM loads, and the hi/lo bf16 operand stores.
+// (mlp_tc.cu, mlp_tc_pair.cu, mlp_tc32.cu): shared-memory and instruction
+// descriptors, the split-bf16 and three-pass tf32 GEMMs issued by one thread,
+// MMA completion on an mbarrier with a bounded wait, TMEM loads, the L2
+// prefetch of global ranges, and the hi/lo operand stores.
 //
 // Shared-memory operand layout (K-major, no swizzle): an R x K bf16 tile keeps
 // element (r, k) at byte (k/8) R 16 + (r/8) 128 + (r%8) 16 + (k%8) 2, i.e.
